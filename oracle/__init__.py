@@ -1,0 +1,123 @@
+"""Python access to the fp64 CPU oracle (oracle/sfa_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: tests/, __graft_entry__.smoke() and bench.py's CPU
+baseline leg use it.  The product path (sparse_flashattention_b200) never
+imports it.  It takes the numpy arrays made by sfa_workloads and returns float64
+results.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sfa_oracle.c")
+_LIB = os.path.join(_HERE, "libsfa_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (plain C, -O2, pthreads)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-D_POSIX_C_SOURCE=200809L", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.sfa_oracle_fwd.restype = ctypes.c_int64
+        lib.sfa_oracle_fwd.argtypes = [P, P, P, P, P, I, I, I, I, P, I, I, I, I, I, ctypes.c_double,
+                                       P, ctypes.c_int64, P, P, I]
+        lib.sfa_oracle_fwd_index.restype = ctypes.c_int64
+        lib.sfa_oracle_fwd_index.argtypes = [P, P, I, I, P, I, I, I, I, I, P, P]
+        lib.sfa_oracle_decode.restype = None
+        lib.sfa_oracle_decode.argtypes = [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, ctypes.c_double,
+                                          P, P, I, P]
+        lib.sfa_oracle_decode_index.restype = ctypes.c_int64
+        lib.sfa_oracle_decode_index.argtypes = [P, P, I, I, I, I, P, P]
+        _lib = lib
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def default_threads():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+
+
+def fwd(case, rows=None, nthreads=None, sel=None):
+    """Prefill oracle.  rows=None: out (total_q, Hq, d), lse (Hq, total_q).
+    rows = int64 flat ids t*Hq+h: out (n, d), lse (n,).  Returns (out, lse, bad_ids)."""
+    lib = _load()
+    q, k, v = _c(case.q, np.uint16), _c(case.k, np.uint16), _c(case.v, np.uint16)
+    cu_q, cu_k = _c(case.cu_q, np.int32), _c(case.cu_k, np.int32)
+    sel = _c(case.sel if sel is None else sel, np.int32)
+    if rows is None:
+        out = np.zeros((case.total_q, case.Hq, case.d), np.float64)
+        lse = np.zeros((case.Hq, case.total_q), np.float64)
+        r, n = None, 0
+    else:
+        r = _c(rows, np.int64)
+        n = r.size
+        out = np.zeros((n, case.d), np.float64)
+        lse = np.zeros((n,), np.float64)
+    bad = lib.sfa_oracle_fwd(_p(q), _p(k), _p(v), _p(cu_q), _p(cu_k), case.batch, case.Hq, case.Hkv, case.d,
+                             _p(sel), sel.shape[-1], case.bs, case.causal, case.wl, case.wr, float(case.scale),
+                             _p(r), n, _p(out), _p(lse), nthreads or default_threads())
+    return out, lse, int(bad)
+
+
+def fwd_index(case, sel=None):
+    """Canonical (sel_c, cnt, bad_ids) of every (token, kv head)."""
+    lib = _load()
+    sel = _c(case.sel if sel is None else sel, np.int32)
+    topk = sel.shape[-1]
+    sel_c = np.zeros((case.total_q, case.Hkv, topk), np.int32)
+    cnt = np.zeros((case.total_q, case.Hkv), np.int32)
+    bad = lib.sfa_oracle_fwd_index(_p(_c(case.cu_q, np.int32)), _p(_c(case.cu_k, np.int32)), case.batch, case.Hkv,
+                                   _p(sel), topk, case.bs, case.causal, case.wl, case.wr, _p(sel_c), _p(cnt))
+    return sel_c, cnt, int(bad)
+
+
+def decode(case, nthreads=None, sel=None, block_table=None):
+    """Decode oracle: out (B, Hq, d), lse (B, Hq), bad = [bad token ids, bad pages]."""
+    lib = _load()
+    sel = _c(case.sel if sel is None else sel, np.int32)
+    bt = _c(case.block_table if block_table is None else block_table, np.int32)
+    out = np.zeros((case.B, case.Hq, case.d), np.float64)
+    lse = np.zeros((case.B, case.Hq), np.float64)
+    bad = np.zeros(2, np.int64)
+    lib.sfa_oracle_decode(_p(_c(case.q, np.uint16)), _p(_c(case.k_cache, np.uint16)),
+                          _p(_c(case.v_cache, np.uint16)), _p(bt), bt.shape[1], case.num_pages, case.page,
+                          _p(_c(case.cache_seqlens, np.int32)), _p(sel), sel.shape[-1], case.B, case.Hq,
+                          case.Hkv, case.d, case.wl, float(case.scale), _p(out), _p(lse),
+                          nthreads or default_threads(), _p(bad))
+    return out, lse, bad
+
+
+def decode_index(case, sel=None):
+    lib = _load()
+    sel = _c(case.sel if sel is None else sel, np.int32)
+    topk = sel.shape[-1]
+    tok_c = np.zeros((case.B, case.Hkv, topk), np.int32)
+    cnt = np.zeros((case.B, case.Hkv), np.int32)
+    bad = lib.sfa_oracle_decode_index(_p(_c(case.cache_seqlens, np.int32)), _p(sel), topk, case.B, case.Hkv,
+                                      case.wl, _p(tok_c), _p(cnt))
+    return tok_c, cnt, int(bad)

@@ -1,0 +1,351 @@
+"""Seeded synthetic inputs for top-k sparse FlashAttention (prefill and paged decode).
+
+This module only draws inputs. It holds none of the attention arithmetic: no
+masking, no softmax, no index canonicalisation. Both the fp64 CPU oracle and the
+CUDA path consume exactly the arrays produced here.
+
+Value recipe: q/k/v ~ N(0, 1) drawn in float32 by numpy's PCG64 and rounded to
+bfloat16 with round-to-nearest-even; the bf16 bit patterns are kept as uint16.
+
+Selection recipe (NSA block selection, as parameterised on the
+"Relaxed-System-Lab/Flash-Sparse-Attention" project page, quick-start example:
+block_size, topk, init_blocks, local_blocks): for a query at position p of a
+sequence (causal, equal q/k lengths), its own block is b = p // bs; the causally
+valid blocks are {0..b}.  Always selected: the first `init_blocks` blocks and the
+`local_blocks` blocks ending at b ({b, b-1, ...} clipped to >= 0).  The remaining
+min(topk, b+1) - |forced| slots are drawn uniformly without replacement from the
+other valid blocks.  The row of `topk` slots is -1 padded and then shuffled, so
+padding and order are arbitrary.  One selection per (token, kv head), shared by
+the G query heads of that kv head.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Sequence
+
+import numpy as np
+
+INVALID = -1
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round float32 to bfloat16 (round to nearest, ties to even); return uint16 bits."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    lsb = (u >> 16) & 1
+    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
+    return r
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def _normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    step = 1 << 24
+    for s in range(0, n, step):
+        e = min(n, s + step)
+        out[s:e] = f32_to_bf16_bits(rng.standard_normal(e - s, dtype=np.float32))
+    return out.reshape(shape)
+
+
+def _normal_bf16_parallel(seed_seq: np.random.SeedSequence, shape, chunk=1 << 24, threads=None) -> np.ndarray:
+    """Large N(0,1) bf16 arrays: one child stream per fixed-size chunk (result independent of thread count)."""
+    import concurrent.futures as cf
+    import os
+
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.uint16)
+    nchunks = (n + chunk - 1) // chunk
+    kids = seed_seq.spawn(nchunks)
+
+    def work(i):
+        s = i * chunk
+        e = min(n, s + chunk)
+        g = np.random.Generator(np.random.PCG64(kids[i]))
+        out[s:e] = f32_to_bf16_bits(g.standard_normal(e - s, dtype=np.float32))
+
+    threads = threads or min(32, os.cpu_count() or 1)
+    with cf.ThreadPoolExecutor(threads) as ex:
+        list(ex.map(work, range(nchunks)))
+    return out.reshape(shape)
+
+
+def _shuffle_rows(rng: np.random.Generator, a: np.ndarray) -> np.ndarray:
+    keys = rng.random(a.shape)
+    order = np.argsort(keys, axis=1, kind="stable")
+    return np.take_along_axis(a, order, axis=1)
+
+
+def nsa_block_selection(rng: np.random.Generator, seqlens: Sequence[int], hkv: int, bs: int, topk: int,
+                        init_blocks: int, local_blocks: int) -> np.ndarray:
+    """(total, hkv, topk) int32 block ids, -1 padded, shuffled per row."""
+    total = int(sum(seqlens))
+    sel = np.full((total, hkv, topk), INVALID, dtype=np.int32)
+    base = 0
+    for L in seqlens:
+        nb = (L + bs - 1) // bs
+        for b in range(nb):
+            t0, t1 = base + b * bs, base + min(L, (b + 1) * bs)
+            rows = (t1 - t0) * hkv
+            forced = sorted(set(range(min(init_blocks, b + 1))) |
+                            set(x for x in range(b - local_blocks + 1, b + 1) if x >= 0))
+            forced = forced[:topk]
+            nsel = min(topk, b + 1)
+            nrand = nsel - len(forced)
+            block = np.full((rows, topk), INVALID, dtype=np.int32)
+            block[:, :len(forced)] = np.asarray(forced, dtype=np.int32)
+            if nrand > 0:
+                cand = np.asarray([x for x in range(b + 1) if x not in set(forced)], dtype=np.int32)
+                keys = rng.random((rows, cand.size))
+                pick = np.argpartition(keys, nrand - 1, axis=1)[:, :nrand]
+                block[:, len(forced):nsel] = cand[pick]
+            block = _shuffle_rows(rng, block)
+            sel[t0:t1] = block.reshape(t1 - t0, hkv, topk)
+        base += L
+    return sel
+
+
+def window_block_selection(rng: np.random.Generator, sq: int, sk: int, batch: int, hkv: int, bs: int,
+                           causal: bool, wl: int, wr: int, topk: Optional[int] = None) -> np.ndarray:
+    """Every block touching a query's key window [i+sk-sq-wl, i+sk-sq+wr] (clipped to [0, sk)); shuffled.
+
+    This lists blocks by the window arithmetic alone, so it is an input recipe, not the
+    kernel's mask: the kernel still applies the mask inside each block."""
+    delta = sk - sq
+    lo = np.arange(sq) + delta - (wl if wl >= 0 else 10 ** 9)
+    hi = np.arange(sq) + delta + (wr if wr >= 0 else 10 ** 9)
+    if causal:
+        hi = np.minimum(hi, np.arange(sq) + delta)
+    lo = np.clip(lo, 0, sk - 1)
+    hi = np.clip(hi, -1, sk - 1)
+    nmax = int(((hi // bs) - (lo // bs) + 1).max()) if sq else 0
+    topk = topk or max(nmax, 1)
+    rows = np.full((sq, topk), INVALID, dtype=np.int32)
+    for i in range(sq):
+        if hi[i] < lo[i]:
+            continue
+        blocks = np.arange(lo[i] // bs, hi[i] // bs + 1, dtype=np.int32)[:topk]
+        rows[i, :blocks.size] = blocks
+    sel = np.broadcast_to(rows[None, :, None, :], (batch, sq, hkv, topk)).reshape(batch * sq, hkv, topk).copy()
+    flat = sel.reshape(-1, topk)
+    return _shuffle_rows(rng, flat).reshape(sel.shape).astype(np.int32)
+
+
+@dataclasses.dataclass
+class PrefillCase:
+    name: str
+    q: np.ndarray            # uint16 bf16 bits (total_q, Hq, d)
+    k: np.ndarray            # uint16 (total_k, Hkv, d)
+    v: np.ndarray            # uint16 (total_k, Hkv, d)
+    cu_q: np.ndarray         # int32 (batch+1)
+    cu_k: np.ndarray         # int32 (batch+1)
+    sel: np.ndarray          # int32 (total_q, Hkv, topk)
+    Hq: int
+    Hkv: int
+    d: int
+    bs: int
+    topk: int
+    causal: int = 1
+    wl: int = -1
+    wr: int = -1
+    scale: float = 0.0       # <= 0 means 1/sqrt(d)
+
+    @property
+    def batch(self):
+        return int(self.cu_q.size - 1)
+
+    @property
+    def total_q(self):
+        return int(self.cu_q[-1])
+
+    @property
+    def total_k(self):
+        return int(self.cu_k[-1])
+
+    @property
+    def max_sq(self):
+        return int(np.diff(self.cu_q).max()) if self.batch else 0
+
+    @property
+    def max_sk(self):
+        return int(np.diff(self.cu_k).max()) if self.batch else 0
+
+    @property
+    def softmax_scale(self):
+        return self.scale if self.scale > 0 else 1.0 / np.sqrt(self.d)
+
+
+@dataclasses.dataclass
+class DecodeCase:
+    name: str
+    q: np.ndarray            # uint16 (B, Hq, d)
+    k_cache: np.ndarray      # uint16 (num_pages, page, Hkv, d)
+    v_cache: np.ndarray
+    block_table: np.ndarray  # int32 (B, max_pages)
+    cache_seqlens: np.ndarray  # int32 (B,)
+    sel: np.ndarray          # int32 (B, Hkv, topk_tok)
+    Hq: int
+    Hkv: int
+    d: int
+    page: int
+    wl: int = -1
+    scale: float = 0.0
+
+    @property
+    def B(self):
+        return int(self.q.shape[0])
+
+    @property
+    def num_pages(self):
+        return int(self.k_cache.shape[0])
+
+    @property
+    def max_pages(self):
+        return int(self.block_table.shape[1])
+
+    @property
+    def topk(self):
+        return int(self.sel.shape[2])
+
+    @property
+    def softmax_scale(self):
+        return self.scale if self.scale > 0 else 1.0 / np.sqrt(self.d)
+
+
+def _cu(lens):
+    return np.concatenate([[0], np.cumsum(np.asarray(lens, dtype=np.int64))]).astype(np.int32)
+
+
+def make_nsa_prefill(seed: int, seqlens, Hq, Hkv, d, bs, topk, init_blocks, local_blocks, name="nsa",
+                     parallel_values=False) -> PrefillCase:
+    ss = np.random.SeedSequence(seed)
+    s_q, s_k, s_v, s_sel = ss.spawn(4)
+    total = int(sum(seqlens))
+    if parallel_values:
+        q = _normal_bf16_parallel(s_q, (total, Hq, d))
+        k = _normal_bf16_parallel(s_k, (total, Hkv, d))
+        v = _normal_bf16_parallel(s_v, (total, Hkv, d))
+    else:
+        q = _normal_bf16(np.random.Generator(np.random.PCG64(s_q)), (total, Hq, d))
+        k = _normal_bf16(np.random.Generator(np.random.PCG64(s_k)), (total, Hkv, d))
+        v = _normal_bf16(np.random.Generator(np.random.PCG64(s_v)), (total, Hkv, d))
+    sel = nsa_block_selection(np.random.Generator(np.random.PCG64(s_sel)), seqlens, Hkv, bs, topk,
+                              init_blocks, local_blocks)
+    cu = _cu(seqlens)
+    return PrefillCase(name, q, k, v, cu, cu.copy(), sel, Hq, Hkv, d, bs, topk, causal=1)
+
+
+def make_window_prefill(seed: int, batch, sq, sk, Hq, Hkv, d, bs, wl, wr, causal=1, name="window") -> PrefillCase:
+    ss = np.random.SeedSequence(seed)
+    s_q, s_k, s_v, s_sel = ss.spawn(4)
+    q = _normal_bf16(np.random.Generator(np.random.PCG64(s_q)), (batch * sq, Hq, d))
+    k = _normal_bf16(np.random.Generator(np.random.PCG64(s_k)), (batch * sk, Hkv, d))
+    v = _normal_bf16(np.random.Generator(np.random.PCG64(s_v)), (batch * sk, Hkv, d))
+    sel = window_block_selection(np.random.Generator(np.random.PCG64(s_sel)), sq, sk, batch, Hkv, bs,
+                                 bool(causal), wl, wr)
+    return PrefillCase(name, q, k, v, _cu([sq] * batch), _cu([sk] * batch), sel, Hq, Hkv, d, bs,
+                       int(sel.shape[2]), causal=causal, wl=wl, wr=wr)
+
+
+def make_decode(seed: int, B, Hq, Hkv, d, page, len_lo, len_hi, topk_tok, n_last, name="decode",
+                parallel_values=False, max_len=None) -> DecodeCase:
+    """Paged top-k decode inputs.  cache_seqlens ~ U[len_lo, len_hi] (inclusive); pages are placed
+    through a seeded permutation; each (b, kv head) selects the last `n_last` positions plus
+    topk_tok - n_last positions drawn without replacement from [0, L - n_last), shuffled."""
+    ss = np.random.SeedSequence(seed)
+    s_len, s_perm, s_q, s_k, s_v, s_sel = ss.spawn(6)
+    g_len = np.random.Generator(np.random.PCG64(s_len))
+    L = g_len.integers(len_lo, len_hi + 1, size=B).astype(np.int32)
+    max_len = max_len or len_hi
+    max_pages = (max_len + page - 1) // page
+    npages_b = (L + page - 1) // page
+    num_pages = int(npages_b.sum())
+    perm = np.random.Generator(np.random.PCG64(s_perm)).permutation(num_pages).astype(np.int32)
+    bt = np.full((B, max_pages), INVALID, dtype=np.int32)
+    off = 0
+    for b in range(B):
+        bt[b, :npages_b[b]] = perm[off:off + npages_b[b]]
+        off += npages_b[b]
+    q = _normal_bf16(np.random.Generator(np.random.PCG64(s_q)), (B, Hq, d))
+    shape = (num_pages, page, Hkv, d)
+    if parallel_values:
+        kc = _normal_bf16_parallel(s_k, shape)
+        vc = _normal_bf16_parallel(s_v, shape)
+    else:
+        kc = _normal_bf16(np.random.Generator(np.random.PCG64(s_k)), shape)
+        vc = _normal_bf16(np.random.Generator(np.random.PCG64(s_v)), shape)
+    g_sel = np.random.Generator(np.random.PCG64(s_sel))
+    sel = np.full((B, Hkv, topk_tok), INVALID, dtype=np.int32)
+    for b in range(B):
+        Lb = int(L[b])
+        nl = min(n_last, Lb, topk_tok)
+        last = np.arange(Lb - nl, Lb, dtype=np.int32)
+        nr = min(topk_tok - nl, Lb - nl)
+        for h in range(Hkv):
+            rest = g_sel.choice(Lb - nl, size=nr, replace=False).astype(np.int32) if nr > 0 else \
+                np.zeros(0, np.int32)
+            row = np.concatenate([last, rest])
+            g_sel.shuffle(row)
+            sel[b, h, :row.size] = row
+    return DecodeCase(name, q, kc, vc, bt, L, sel, Hq, Hkv, d, page)
+
+
+# ---------------------------------------------------------------------------------------------
+# The five named workloads and their oracle-sized variants.
+# ---------------------------------------------------------------------------------------------
+
+def config1():
+    """Tiny selected attention: 1 x 256 tokens, Hq4/Hkv1, d64, bs32, topk4 (block 0 + own block forced)."""
+    return make_nsa_prefill(1, [256], 4, 1, 64, 32, 4, init_blocks=1, local_blocks=1, name="tiny_256_d64")
+
+
+def config2(parallel_values=False):
+    """Varlen NSA: lengths [8192, 4096, 2048, 2048], Hq16/Hkv4, d128, bs64, topk16, init 1, local 2."""
+    return make_nsa_prefill(2, [8192, 4096, 2048, 2048], 16, 4, 128, 64, 16, 1, 2, name="nsa_varlen_16k",
+                            parallel_values=parallel_values)
+
+
+def config3():
+    """Dense limit: B2, sq1024, sk4096, Hq32/Hkv8, d128, causal, window (1024, 0), every touched 64-block."""
+    return make_window_prefill(3, 2, 1024, 4096, 32, 8, 128, 64, 1024, 0, causal=1, name="dense_window_1k_4k")
+
+
+def config4(parallel_values=False):
+    """Long context: lengths [65536, 32768], Hq=Hkv=4, d128, bs64, topk16, init 1, local 2."""
+    return make_nsa_prefill(4, [65536, 32768], 4, 4, 128, 64, 16, 1, 2, name="nsa_long_96k",
+                            parallel_values=parallel_values)
+
+
+def config5(parallel_values=True):
+    """Paged top-k decode: B32, Hq32/Hkv8, d128, L ~ U[16384, 131072], page 256, 2048 tokens (last 128 forced)."""
+    return make_decode(5, 32, 32, 8, 128, 256, 16384, 131072, 2048, 128, name="paged_topk_decode_b32",
+                       parallel_values=parallel_values)
+
+
+def small_config(n: int):
+    """Oracle-sized variants of the five workloads (several tiles, ragged tails)."""
+    if n == 1:
+        return config1()
+    if n == 2:
+        return make_nsa_prefill(12, [1024, 517, 300, 77], 16, 4, 128, 64, 16, 1, 2, name="nsa_varlen_small")
+    if n == 3:
+        return make_window_prefill(13, 2, 200, 700, 32, 8, 128, 64, 256, 0, causal=1, name="dense_window_small")
+    if n == 4:
+        return make_nsa_prefill(14, [2048, 1000], 4, 4, 128, 64, 16, 1, 2, name="nsa_long_small")
+    if n == 5:
+        return make_decode(15, 4, 32, 8, 128, 256, 700, 3000, 256, 32, name="decode_small")
+    raise ValueError(n)
+
+
+def kept_pairs_nsa(seqlens, bs, topk):
+    """Closed form of kept (query, key) pairs per query head for the NSA recipe with causal mask:
+    a query at p with b = p // bs keeps (min(topk, b+1) - 1) * bs + (p % bs + 1) keys."""
+    tot = 0
+    for L in seqlens:
+        p = np.arange(L)
+        b = p // bs
+        tot += int(((np.minimum(topk, b + 1) - 1) * bs + (p % bs + 1)).sum())
+    return tot
