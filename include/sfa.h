@@ -1,0 +1,197 @@
+/*
+ * sfa.h — C ABI of libsfa.so: top-k sparse FlashAttention forward on NVIDIA B200 (sm_100a).
+ *
+ * Two operations, each also available as its separate stages:
+ *
+ *   sfa_fwd     varlen prefill.  Every query token attends only to the key blocks its
+ *               (token, kv head) selection lists, shared by the G = Hq/Hkv query heads of
+ *               that kv head.  Sources: the Ascend "Sparse FlashAttention" article (ggplus
+ *               blog post), section "这到底是个啥？Sparse FlashAttention架构初探" — gather the
+ *               K/V rows named by the top-k indices into a compact sub-matrix and run plain
+ *               attention on those entries only; the "Relaxed-System-Lab/Flash-Sparse-Attention"
+ *               project page, quick-start (block_size / topk / init_blocks / local_blocks NSA
+ *               selection, cu_seqlens varlen input); flash-attention-npu "FlashAttention v2"
+ *               docstrings of flash_attn_varlen_func (layouts, bottom-right causal mask, window,
+ *               GQA mapping, softmax_lse).
+ *   sfa_decode  paged top-k decode, one query token per sequence.  Sources: the
+ *               Flash-Sparse-Attention README (gitcode mirror), feature list ("Top-k gather
+ *               KV-cache decode", "Split-KV", "Paged Attention"); flash-attention-npu
+ *               flash_attn_with_kvcache docstrings (paged cache + block_table, cache_seqlens,
+ *               num_splits with 0 = automatic, softmax_lse).
+ *
+ * Semantics common to both (the plain reading of those pages):
+ *   - q head h reads kv head h / (Hq/Hkv); Hq must be a multiple of Hkv.
+ *   - For a query at local position i of a sequence with lengths (sq, sk), delta = sk - sq.
+ *     Key j is kept iff it is selected and  causal => j <= i+delta;  window_left >= 0 =>
+ *     j >= i+delta-window_left;  window_right >= 0 => j <= i+delta+window_right.
+ *   - Softmax over the kept keys of  scale * q.k ; scale <= 0 means 1/sqrt(d).
+ *   - A row with no kept key outputs exactly 0 and lse = -inf.
+ *   - lse is the natural-log logsumexp of scale*q.k over the kept keys.
+ *   - A selection is a set: -1 slots are padding, duplicates and order do not matter.
+ *
+ * Conventions of this ABI:
+ *   - Every pointer argument except the workspace size queries is a DEVICE pointer of the
+ *     current CUDA device, owned by the caller.  The library allocates no device memory,
+ *     never synchronises the host and launches everything on `stream` (cudaStream_t; NULL is
+ *     the legacy default stream), so the calls can be captured in a CUDA graph.
+ *   - bf16 tensors are contiguous row-major with the last dimension contiguous, 16-byte
+ *     aligned base addresses.
+ *   - Return value: a synchronous sfa_status.  Argument errors are detected on the host
+ *     before anything is launched.  SFA_ERR_CUDA means a launch failed (the CUDA error is
+ *     left for the caller's next runtime call to report).
+ *   - Data errors found on the device are OR-ed into *status_dev (int32, may be NULL) as
+ *     SFA_DEV_* bits and the offending entry is ignored: an out-of-range block/token id,
+ *     a block_table entry outside [0, num_pages), a sequence longer than the bound given,
+ *     or a pipeline wait that exceeded its time limit (the kernel then stops early; its
+ *     outputs are undefined).  Kernels never trap.
+ *   - Calls on one workspace must not overlap in time (use one workspace per stream).
+ */
+#ifndef SFA_H_
+#define SFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *sfa_stream_t; /* same type as cudaStream_t */
+
+typedef enum sfa_status {
+    SFA_OK = 0,
+    SFA_ERR_INVALID_ARG = 1,         /* NULL pointer, negative size, Hq % Hkv != 0, misaligned base */
+    SFA_ERR_UNSUPPORTED = 2,         /* valid but outside this build: see the limits below */
+    SFA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the matching *_workspace_size() */
+    SFA_ERR_CUDA = 4                 /* a CUDA launch or driver call failed */
+} sfa_status;
+
+enum {
+    SFA_DEV_BAD_INDEX = 1,  /* a block / token id neither -1 nor inside its sequence: ignored */
+    SFA_DEV_BAD_PAGE = 2,   /* a block_table entry outside [0, num_pages): its tokens are dropped */
+    SFA_DEV_TIMEOUT = 4,    /* a pipeline wait passed its time limit: outputs undefined */
+    SFA_DEV_BAD_SEQLEN = 8  /* a sequence longer than max_seqlen_q/k (or than the block table): the
+                               excess is not computed / its ids are treated as out of range */
+};
+
+/* Supported in this build: bf16 inputs; d in {64, 128}; prefill block_size in {32, 64},
+ * 1 <= topk <= 128, G = Hq/Hkv <= 128, ceil(max_seqlen_k / block_size) <= 65536;
+ * decode G <= 16, page_size >= 1, 1 <= topk_tok <= 65536, max_pages_per_seq*page_size
+ * <= 2^20.  Anything else returns SFA_ERR_UNSUPPORTED. */
+
+/* ----------------------------------------------------------------------------------------
+ * Prefill
+ * -------------------------------------------------------------------------------------- */
+
+/* Bytes of device workspace sfa_fwd / sfa_fwd_prep / sfa_fwd_attend need for these sizes
+ * (0 only when total_q == 0).  max_seqlen_q / max_seqlen_k bound every sequence's length. */
+size_t sfa_fwd_workspace_size(int batch, int max_seqlen_q, int max_seqlen_k, int total_q,
+                              int Hq, int Hkv, int d, int topk, int block_size);
+
+/* Byte offsets, inside that workspace, of the canonical selection written by sfa_fwd_prep:
+ * sel_c int32 (total_q, Hkv, topk) — per (token, kv head) the ascending distinct block ids
+ * that are blocks of the sequence and hold at least one key the mask keeps, then -1 — and
+ * cnt int32 (total_q, Hkv) — how many.  Returns SFA_OK or SFA_ERR_INVALID_ARG. */
+int sfa_fwd_workspace_offsets(int batch, int max_seqlen_q, int max_seqlen_k, int total_q,
+                              int Hq, int Hkv, int d, int topk, int block_size,
+                              size_t *off_sel_c, size_t *off_cnt);
+
+/* Full prefill forward = sfa_fwd_prep followed by sfa_fwd_attend on the same workspace.
+ *   q            bf16 (total_q, Hq, d)
+ *   k, v         bf16 (total_k, Hkv, d)
+ *   cu_seqlens_q int32 (batch+1), prefix sums from 0; cu_seqlens_k likewise, or NULL for
+ *                "same as q" (then total_k must equal total_q)
+ *   sel_idx      int32 (total_q, Hkv, topk): block ids of the sequence's own K coordinates,
+ *                block s = keys [s*block_size, min((s+1)*block_size, sk)); -1 = unused slot
+ *   out          bf16 (total_q, Hq, d);  lse  fp32 (Hq, total_q)
+ * max_seqlen_q/k are host-side bounds used to size the grid (no device->host read). */
+int sfa_fwd(const void *q, const void *k, const void *v,
+            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+            int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+            int Hq, int Hkv, int d,
+            const int32_t *sel_idx, int topk, int block_size,
+            int causal, int window_left, int window_right, float scale,
+            void *workspace, size_t workspace_bytes, int32_t *status_dev,
+            void *out, float *lse, sfa_stream_t stream);
+
+/* Stage 1 alone: canonicalise the selection (validate, drop padding / out-of-range ids /
+ * blocks with no kept key, dedupe, sort ascending, count) and build, per query tile, the
+ * ascending union of its rows' blocks.  Writes only the workspace. */
+int sfa_fwd_prep(const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                 int batch, int max_seqlen_q, int max_seqlen_k, int total_q,
+                 int Hq, int Hkv, int d, const int32_t *sel_idx, int topk, int block_size,
+                 int causal, int window_left, int window_right,
+                 void *workspace, size_t workspace_bytes, int32_t *status_dev, sfa_stream_t stream);
+
+/* Stage 2 alone: the attention kernel (TMA gather of K/V blocks, tcgen05 QK^T and PV with
+ * TMEM accumulators, masked online softmax, epilogue) on a workspace filled by
+ * sfa_fwd_prep with the same arguments. */
+int sfa_fwd_attend(const void *q, const void *k, const void *v,
+                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                   int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                   int Hq, int Hkv, int d, int topk, int block_size,
+                   int causal, int window_left, int window_right, float scale,
+                   void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                   void *out, float *lse, sfa_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
+ * Paged top-k decode
+ * -------------------------------------------------------------------------------------- */
+
+/* The split count sfa_decode uses for num_splits (0 = automatic choice). */
+int sfa_decode_num_splits(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits);
+
+/* Bytes of device workspace for sfa_decode with these sizes; num_splits as passed there. */
+size_t sfa_decode_workspace_size(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits);
+
+/* Byte offsets inside the decode workspace of the canonical token sets written by
+ * sfa_decode_prep: tok_c int32 (B, Hkv, topk_tok) ascending distinct positions in
+ * [0, cache_seqlens[b]) (and >= L-1-window_left when window_left >= 0), then -1; and
+ * cnt int32 (B, Hkv). */
+int sfa_decode_workspace_offsets(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits,
+                                 size_t *off_tok_c, size_t *off_cnt);
+
+/* Paged top-k decode = prep, split-KV attention, LSE combine.
+ *   q             bf16 (B, Hq, d): the new token of each sequence, at position L_b - 1
+ *   k_cache,
+ *   v_cache       bf16 (num_pages, page_size, Hkv, d)
+ *   block_table   int32 (B, max_pages_per_seq): logical page p of sequence b lives in
+ *                 physical page block_table[b][p]
+ *   cache_seqlens int32 (B): L_b, tokens in the cache (the new token included)
+ *   sel_tok_idx   int32 (B, Hkv, topk_tok): logical token positions, -1 = unused slot
+ *   window_left   -1 = unbounded, else keep positions >= L_b - 1 - window_left
+ *   num_splits    0 = automatic, else the number of key chunks per (b, kv head)
+ *   out           bf16 (B, Hq, d);  lse  fp32 (B, Hq) */
+int sfa_decode(const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
+               const int32_t *cache_seqlens, const int32_t *sel_tok_idx, int topk_tok,
+               int B, int Hq, int Hkv, int d, int window_left, float scale, int num_splits,
+               void *workspace, size_t workspace_bytes, int32_t *status_dev,
+               void *out, float *lse, sfa_stream_t stream);
+
+/* Stage 1 alone: canonical token sets into the workspace. */
+int sfa_decode_prep(const int32_t *cache_seqlens, const int32_t *sel_tok_idx, int topk_tok,
+                    int max_pages_per_seq, int page_size, int B, int Hq, int Hkv, int d,
+                    int window_left, int num_splits,
+                    void *workspace, size_t workspace_bytes, int32_t *status_dev, sfa_stream_t stream);
+
+/* Stages 2+3 alone: per-split partial attention (gather through block_table) and the
+ * LSE combine, on a workspace filled by sfa_decode_prep with the same arguments. */
+int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache,
+                      const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
+                      int topk_tok, int B, int Hq, int Hkv, int d, float scale, int num_splits,
+                      void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                      void *out, float *lse, sfa_stream_t stream);
+
+/* Human-readable name of an sfa_status value (static string). */
+const char *sfa_status_string(int status);
+
+/* Number of kernel launches the last successful call on this host thread made (prefill:
+ * 2, decode: 3, a single stage: its own count). */
+int sfa_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFA_H_ */

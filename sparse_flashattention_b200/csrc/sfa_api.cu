@@ -1,0 +1,506 @@
+// Host side of libsfa.so: argument validation, workspace layout, TMA descriptor encoding and
+// kernel launches for the C ABI declared in include/sfa.h.  Nothing here allocates device
+// memory or synchronises with the device.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+
+#include "sfa_internal.h"
+
+using namespace sfa;
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x)
+{
+    return (x + kAlign - 1) / kAlign * kAlign;
+}
+
+bool aligned16(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// ----------------------------------------------------------------------------------------
+// Prefill geometry
+// ----------------------------------------------------------------------------------------
+int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv, int d, int topk, int bs,
+                 FwdGeom &g)
+{
+    if (batch < 0 || max_sq < 0 || max_sk < 0 || total_q < 0 || Hq <= 0 || Hkv <= 0 || topk <= 0 || bs <= 0)
+        return SFA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return SFA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SFA_ERR_UNSUPPORTED;
+    if (bs != 32 && bs != 64) return SFA_ERR_UNSUPPORTED;
+    if (topk > 128) return SFA_ERR_UNSUPPORTED;
+    const int G = Hq / Hkv;
+    if (G > 128) return SFA_ERR_UNSUPPORTED;
+    const int64_t nblk_max = ((int64_t)max_sk + bs - 1) / bs;
+    if (nblk_max > 65536) return SFA_ERR_UNSUPPORTED;
+    g = FwdGeom{};
+    g.batch = batch;
+    g.max_sq = max_sq;
+    g.max_sk = max_sk;
+    g.total_q = total_q;
+    g.Hq = Hq;
+    g.Hkv = Hkv;
+    g.d = d;
+    g.topk = topk;
+    g.bs = bs;
+    g.G = G;
+    g.Tq = 128 / G;
+    g.nqt = (max_sq + g.Tq - 1) / g.Tq;
+    const int64_t tiles = (int64_t)g.nqt * batch * Hkv;
+    if (tiles > (1ll << 31) - 1) return SFA_ERR_UNSUPPORTED;
+    g.tiles = (int)tiles;
+    g.nblk_max = (int)std::max<int64_t>(nblk_max, 1);
+    g.umax = (int)std::max<int64_t>(1, std::min<int64_t>(nblk_max, (int64_t)g.Tq * topk));
+    size_t off = 0;
+    g.off_sel_c = off;
+    off = align_up(off + (size_t)total_q * Hkv * topk * 4);
+    g.off_cnt = off;
+    off = align_up(off + (size_t)total_q * Hkv * 4);
+    g.off_ucnt = off;
+    off = align_up(off + (size_t)g.tiles * 4);
+    g.off_union = off;
+    off = align_up(off + (size_t)g.tiles * g.umax * 4);
+    g.bytes = total_q == 0 ? 0 : off;
+    return SFA_OK;
+}
+
+// ----------------------------------------------------------------------------------------
+// TMA descriptors
+// ----------------------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A (rows, heads, d) bf16 tensor viewed as 3-D {d, heads, rows}; box {64, box_heads, box_rows},
+// 128-byte swizzle (matches the UMMA K-major / MN-major SWIZZLE_128B canonical layouts).
+bool encode_3d(CUtensorMap &m, const void *base, int d, int heads, int64_t rows, int box_heads, int box_rows)
+{
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_heads, (cuuint32_t)box_rows};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int check_window(int causal, int wl, int wr)
+{
+    if (causal != 0 && causal != 1) return SFA_ERR_INVALID_ARG;
+    if (wl < -1 || wr < -1) return SFA_ERR_INVALID_ARG;
+    return SFA_OK;
+}
+
+int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, const int32_t *sel, int causal, int wl,
+                  int wr, void *ws, int32_t *status, cudaStream_t st)
+{
+    FwdPrepParams p{};
+    p.cu_q = cu_q;
+    p.cu_k = cu_k ? cu_k : cu_q;
+    p.sel = sel;
+    p.batch = g.batch;
+    p.Hkv = g.Hkv;
+    p.topk = g.topk;
+    p.bs = g.bs;
+    p.causal = causal;
+    p.wl = wl;
+    p.wr = wr;
+    p.Tq = g.Tq;
+    p.nqt = g.nqt;
+    p.umax = g.umax;
+    p.max_sq = g.max_sq;
+    p.nblk_max = g.nblk_max;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    p.sel_c = reinterpret_cast<int32_t *>(w + g.off_sel_c);
+    p.cnt = reinterpret_cast<int32_t *>(w + g.off_cnt);
+    p.ucnt = reinterpret_cast<int32_t *>(w + g.off_ucnt);
+    p.uni = reinterpret_cast<int32_t *>(w + g.off_union);
+    p.status = status;
+    return launch_fwd_prep(g, p, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+}
+
+int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *v, const int32_t *cu_q,
+                    const int32_t *cu_k, int total_k, int causal, int wl, int wr, float scale, void *ws,
+                    int32_t *status, void *out, float *lse, cudaStream_t st)
+{
+    if (fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    CUtensorMap tq, tk, tv;
+    if (!encode_3d(tq, q, g.d, g.Hq, g.total_q, g.G, g.Tq)) return SFA_ERR_CUDA;
+    if (!encode_3d(tk, k, g.d, g.Hkv, total_k, 1, g.bs)) return SFA_ERR_CUDA;
+    if (!encode_3d(tv, v, g.d, g.Hkv, total_k, 1, g.bs)) return SFA_ERR_CUDA;
+    FwdAttendParams p{};
+    p.cu_q = cu_q;
+    p.cu_k = cu_k ? cu_k : cu_q;
+    const uint8_t *w = static_cast<const uint8_t *>(ws);
+    p.sel_c = reinterpret_cast<const int32_t *>(w + g.off_sel_c);
+    p.cnt = reinterpret_cast<const int32_t *>(w + g.off_cnt);
+    p.ucnt = reinterpret_cast<const int32_t *>(w + g.off_ucnt);
+    p.uni = reinterpret_cast<const int32_t *>(w + g.off_union);
+    p.batch = g.batch;
+    p.total_q = g.total_q;
+    p.Hq = g.Hq;
+    p.Hkv = g.Hkv;
+    p.G = g.G;
+    p.Tq = g.Tq;
+    p.nqt = g.nqt;
+    p.topk = g.topk;
+    p.umax = g.umax;
+    p.causal = causal;
+    p.wl = wl;
+    p.wr = wr;
+    const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)g.d);
+    p.scale_log2 = (float)(sc * 1.4426950408889634);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    p.status = status;
+    return launch_fwd_attend(g, p, tq, tk, tv, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+}
+
+int fwd_common_checks(const int32_t *cu_q, const int32_t *cu_k, int total_q, int total_k, int max_sq, int max_sk,
+                      int causal, int wl, int wr)
+{
+    if (!cu_q) return SFA_ERR_INVALID_ARG;
+    if (total_k < 0) return SFA_ERR_INVALID_ARG;
+    if (!cu_k && total_k != total_q) return SFA_ERR_INVALID_ARG;
+    if (!cu_k && max_sk != max_sq) return SFA_ERR_INVALID_ARG;
+    return check_window(causal, wl, wr);
+}
+
+// ----------------------------------------------------------------------------------------
+// Decode geometry
+// ----------------------------------------------------------------------------------------
+int num_sms()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+// Split count: the smallest S whose last wave of CTAs is the fullest (CTAs = B*Hkv*S over
+// num_SMs * CTAs-per-SM slots), with at least 128 tokens per split.
+int choose_splits(int B, int Hkv, int d, int topk)
+{
+    const int units = B * Hkv;
+    const int slots = num_sms() * decode_split_blocks_per_sm(d);
+    const int smax = std::max(1, std::min(64, (topk + 127) / 128));
+    int best = 1;
+    double best_eff = -1.0;
+    for (int S = 1; S <= smax; ++S) {
+        const double waves = (double)units * S / slots;
+        const double eff = waves / std::ceil(waves);
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = S;
+        }
+    }
+    return best;
+}
+
+int dec_geometry(int B, int Hq, int Hkv, int d, int topk, int num_splits, DecGeom &g)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || topk <= 0 || num_splits < 0) return SFA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return SFA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SFA_ERR_UNSUPPORTED;
+    if (Hq / Hkv > 16) return SFA_ERR_UNSUPPORTED;
+    if (topk > 65536) return SFA_ERR_UNSUPPORTED;
+    g = DecGeom{};
+    g.B = B;
+    g.Hq = Hq;
+    g.Hkv = Hkv;
+    g.d = d;
+    g.topk = topk;
+    g.G = Hq / Hkv;
+    g.S = num_splits > 0 ? std::min(num_splits, topk) : choose_splits(B, Hkv, d, topk);
+    size_t off = 0;
+    g.off_tok = off;
+    off = align_up(off + (size_t)B * Hkv * topk * 4);
+    g.off_cnt = off;
+    off = align_up(off + (size_t)B * Hkv * 4);
+    g.off_po = off;
+    off = align_up(off + (size_t)B * Hq * g.S * d * 4);
+    g.off_plse = off;
+    off = align_up(off + (size_t)B * Hq * g.S * 4);
+    g.bytes = B == 0 ? 0 : off;
+    return SFA_OK;
+}
+
+int dec_prep_impl(const DecGeom &g, const int32_t *seqlens, const int32_t *sel, int max_pages, int page, int wl,
+                  void *ws, int32_t *status, cudaStream_t st)
+{
+    const int64_t max_len = (int64_t)max_pages * page;
+    if (max_len > (1 << 20)) return SFA_ERR_UNSUPPORTED;
+    DecPrepParams p{};
+    p.seqlens = seqlens;
+    p.sel = sel;
+    p.topk = g.topk;
+    p.max_len = (int)max_len;
+    p.Hkv = g.Hkv;
+    p.wl = wl;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    p.tok_c = reinterpret_cast<int32_t *>(w + g.off_tok);
+    p.cnt = reinterpret_cast<int32_t *>(w + g.off_cnt);
+    p.status = status;
+    return launch_decode_prep(g, p, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+}
+
+int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void *vc, const int32_t *bt, int max_pages,
+                    int num_pages, int page, float scale, void *ws, int32_t *status, void *out, float *lse,
+                    cudaStream_t st)
+{
+    if ((int64_t)num_pages * page * g.Hkv > (int64_t)INT32_MAX) return SFA_ERR_UNSUPPORTED;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    DecSplitParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.kc = static_cast<const __nv_bfloat16 *>(kc);
+    p.vc = static_cast<const __nv_bfloat16 *>(vc);
+    p.bt = bt;
+    p.tok_c = reinterpret_cast<const int32_t *>(w + g.off_tok);
+    p.cnt = reinterpret_cast<const int32_t *>(w + g.off_cnt);
+    p.max_pages = max_pages;
+    p.num_pages = num_pages;
+    p.page = page;
+    p.Hq = g.Hq;
+    p.Hkv = g.Hkv;
+    p.G = g.G;
+    p.topk = g.topk;
+    p.S = g.S;
+    const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)g.d);
+    p.scale_log2 = (float)(sc * 1.4426950408889634);
+    p.po = reinterpret_cast<float *>(w + g.off_po);
+    p.plse = reinterpret_cast<float *>(w + g.off_plse);
+    p.status = status;
+    if (launch_decode_split(g, p, st) != cudaSuccess) return SFA_ERR_CUDA;
+    DecCombineParams c{};
+    c.po = p.po;
+    c.plse = p.plse;
+    c.Hq = g.Hq;
+    c.S = g.S;
+    c.out = static_cast<__nv_bfloat16 *>(out);
+    c.lse = lse;
+    return launch_decode_combine(g, c, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sfa_fwd_workspace_size(int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int Hq, int Hkv, int d,
+                              int topk, int block_size)
+{
+    FwdGeom g;
+    if (fwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size, g) != SFA_OK) return 0;
+    return g.bytes;
+}
+
+int sfa_fwd_workspace_offsets(int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int Hq, int Hkv, int d,
+                              int topk, int block_size, size_t *off_sel_c, size_t *off_cnt)
+{
+    FwdGeom g;
+    const int rc = fwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size, g);
+    if (rc != SFA_OK) return rc;
+    if (off_sel_c) *off_sel_c = g.off_sel_c;
+    if (off_cnt) *off_cnt = g.off_cnt;
+    return SFA_OK;
+}
+
+int sfa_fwd_prep(const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int batch, int max_seqlen_q,
+                 int max_seqlen_k, int total_q, int Hq, int Hkv, int d, const int32_t *sel_idx, int topk,
+                 int block_size, int causal, int window_left, int window_right, void *workspace,
+                 size_t workspace_bytes, int32_t *status_dev, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    FwdGeom g;
+    int rc = fwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size, g);
+    if (rc != SFA_OK) return rc;
+    if (!cu_seqlens_q || (total_q > 0 && !sel_idx)) return SFA_ERR_INVALID_ARG;
+    if ((rc = check_window(causal, window_left, window_right)) != SFA_OK) return rc;
+    if (total_q == 0 || batch == 0) return SFA_OK;
+    if (!workspace) return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    rc = fwd_prep_impl(g, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
+                       status_dev, stream);
+    if (rc == SFA_OK) g_last_launches = 1;
+    return rc;
+}
+
+int sfa_fwd_attend(const void *q, const void *k, const void *v, const int32_t *cu_seqlens_q,
+                   const int32_t *cu_seqlens_k, int batch, int max_seqlen_q, int max_seqlen_k, int total_q,
+                   int total_k, int Hq, int Hkv, int d, int topk, int block_size, int causal, int window_left,
+                   int window_right, float scale, void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                   void *out, float *lse, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    FwdGeom g;
+    int rc = fwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size, g);
+    if (rc != SFA_OK) return rc;
+    if ((rc = fwd_common_checks(cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k, causal,
+                                window_left, window_right)) != SFA_OK)
+        return rc;
+    if (total_q == 0 || batch == 0) return SFA_OK;
+    if (!q || !k || !v || !out || !lse || !workspace) return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
+    if (total_k == 0) return SFA_ERR_UNSUPPORTED;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right, scale,
+                         workspace, status_dev, out, lse, stream);
+    if (rc == SFA_OK) g_last_launches = 1;
+    return rc;
+}
+
+int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+            int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int d,
+            const int32_t *sel_idx, int topk, int block_size, int causal, int window_left, int window_right,
+            float scale, void *workspace, size_t workspace_bytes, int32_t *status_dev, void *out, float *lse,
+            sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    FwdGeom g;
+    int rc = fwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size, g);
+    if (rc != SFA_OK) return rc;
+    if ((rc = fwd_common_checks(cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k, causal,
+                                window_left, window_right)) != SFA_OK)
+        return rc;
+    if (total_q == 0 || batch == 0) return SFA_OK;
+    if (!q || !k || !v || !out || !lse || !workspace || !sel_idx) return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
+    if (total_k == 0) return SFA_ERR_UNSUPPORTED;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    rc = fwd_prep_impl(g, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
+                       status_dev, stream);
+    if (rc != SFA_OK) return rc;
+    rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right, scale,
+                         workspace, status_dev, out, lse, stream);
+    if (rc == SFA_OK) g_last_launches = 2;
+    return rc;
+}
+
+int sfa_decode_num_splits(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits)
+{
+    DecGeom g;
+    if (dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g) != SFA_OK) return 0;
+    return g.S;
+}
+
+size_t sfa_decode_workspace_size(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits)
+{
+    DecGeom g;
+    if (dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g) != SFA_OK) return 0;
+    return g.bytes;
+}
+
+int sfa_decode_workspace_offsets(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits, size_t *off_tok_c,
+                                 size_t *off_cnt)
+{
+    DecGeom g;
+    const int rc = dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g);
+    if (rc != SFA_OK) return rc;
+    if (off_tok_c) *off_tok_c = g.off_tok;
+    if (off_cnt) *off_cnt = g.off_cnt;
+    return SFA_OK;
+}
+
+int sfa_decode_prep(const int32_t *cache_seqlens, const int32_t *sel_tok_idx, int topk_tok, int max_pages_per_seq,
+                    int page_size, int B, int Hq, int Hkv, int d, int window_left, int num_splits, void *workspace,
+                    size_t workspace_bytes, int32_t *status_dev, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    DecGeom g;
+    int rc = dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g);
+    if (rc != SFA_OK) return rc;
+    if (page_size <= 0 || max_pages_per_seq <= 0 || window_left < -1) return SFA_ERR_INVALID_ARG;
+    if (B == 0) return SFA_OK;
+    if (!cache_seqlens || !sel_tok_idx || !workspace) return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    rc = dec_prep_impl(g, cache_seqlens, sel_tok_idx, max_pages_per_seq, page_size, window_left, workspace, status_dev,
+                       stream);
+    if (rc == SFA_OK) g_last_launches = 1;
+    return rc;
+}
+
+int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                      int max_pages_per_seq, int num_pages, int page_size, int topk_tok, int B, int Hq, int Hkv, int d,
+                      float scale, int num_splits, void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                      void *out, float *lse, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    DecGeom g;
+    int rc = dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g);
+    if (rc != SFA_OK) return rc;
+    if (page_size <= 0 || max_pages_per_seq <= 0 || num_pages < 0) return SFA_ERR_INVALID_ARG;
+    if (B == 0) return SFA_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !workspace || !out || !lse) return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, scale,
+                         workspace, status_dev, out, lse, stream);
+    if (rc == SFA_OK) g_last_launches = 2;
+    return rc;
+}
+
+int sfa_decode(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+               int max_pages_per_seq, int num_pages, int page_size, const int32_t *cache_seqlens,
+               const int32_t *sel_tok_idx, int topk_tok, int B, int Hq, int Hkv, int d, int window_left, float scale,
+               int num_splits, void *workspace, size_t workspace_bytes, int32_t *status_dev, void *out, float *lse,
+               sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    DecGeom g;
+    int rc = dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g);
+    if (rc != SFA_OK) return rc;
+    if (page_size <= 0 || max_pages_per_seq <= 0 || num_pages < 0 || window_left < -1) return SFA_ERR_INVALID_ARG;
+    if (B == 0) return SFA_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !cache_seqlens || !sel_tok_idx || !workspace || !out || !lse)
+        return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    rc = dec_prep_impl(g, cache_seqlens, sel_tok_idx, max_pages_per_seq, page_size, window_left, workspace, status_dev,
+                       stream);
+    if (rc != SFA_OK) return rc;
+    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, scale,
+                         workspace, status_dev, out, lse, stream);
+    if (rc == SFA_OK) g_last_launches = 3;
+    return rc;
+}
+
+const char *sfa_status_string(int status)
+{
+    switch (status) {
+    case SFA_OK: return "SFA_OK";
+    case SFA_ERR_INVALID_ARG: return "SFA_ERR_INVALID_ARG: invalid argument";
+    case SFA_ERR_UNSUPPORTED: return "SFA_ERR_UNSUPPORTED: valid but not supported by this build";
+    case SFA_ERR_WORKSPACE_TOO_SMALL: return "SFA_ERR_WORKSPACE_TOO_SMALL: workspace below the required size";
+    case SFA_ERR_CUDA: return "SFA_ERR_CUDA: a CUDA launch or driver call failed";
+    default: return "unknown sfa_status";
+    }
+}
+
+int sfa_last_launch_count(void)
+{
+    return g_last_launches;
+}
+
+}  // extern "C"

@@ -1,0 +1,400 @@
+// Prefill attention kernel for top-k sparse FlashAttention on sm_100a.
+//
+// One CTA computes one query tile: Tq consecutive tokens of one sequence times the G query
+// heads that share one kv head (and therefore one block selection), Tq*G <= 128 rows — the
+// GQA heads are packed into the M dimension of the tensor-core tile.  The CTA walks the
+// ascending union of its rows' selected blocks (built by the prep kernel).  Per block s:
+//
+//   producer warp   TMA-loads K and V rows [s*bs, s*bs+bs) of the kv head into a 3-stage
+//                   shared-memory ring (128-byte swizzle), signalling an mbarrier.
+//   MMA warp        one thread issues tcgen05.mma: S = Q K^T into one of two TMEM score
+//                   buffers, and O += P V into the TMEM output accumulator.
+//   softmax warps   4 warps, one thread per row: read S from TMEM, apply the row's mask
+//                   (block not selected by this row, bottom-right causal limit, window,
+//                   sequence end), keep the running max and sum in fp32 (base-2 domain),
+//                   write P = 2^(s*scale*log2e - m) as bf16 into shared memory for the MMA,
+//                   rescale O in TMEM when the running max grows by more than 2^8.
+//
+// The epilogue divides O by the running sum, writes bf16 out and the natural-log LSE.
+// The method is the FlashAttention tiling with online softmax applied to the gathered blocks
+// only, as the Ascend "Sparse FlashAttention" article describes the fused SFA operator
+// (gather the top-k K/V, then QK^T, softmax and PV tile by tile in one kernel); the
+// mask/GQA/LSE semantics are those of the flash-attention-npu FlashAttention v2 docstrings.
+//
+// Every mbarrier wait is bounded (sfa_device.cuh): on a timeout the CTA records
+// SFA_DEV_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and exits.
+#include "sfa_device.cuh"
+
+namespace sfa {
+
+namespace {
+
+constexpr int kThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 softmax/epilogue
+constexpr int kStages = 3;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
+constexpr float kLn2 = 0.6931471805599453f;
+
+template <int D, int BS>
+struct Cfg {
+    static constexpr int kQBytes = 128 * D * 2;
+    static constexpr int kKVBytes = BS * D * 2;  // one K (or V) block
+    static constexpr int kPBytes = 128 * 128;    // 128 rows x 64 bf16 (128-byte swizzle rows)
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kStages * kKVBytes;
+    static constexpr int kOffP = kOffV + kStages * kKVBytes;
+    static constexpr int kOffMeta = kOffP + 2 * kPBytes;
+    static constexpr int kTmemCols = (2 * BS + D <= 128) ? 128 : 256;
+    static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
+    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+};
+
+struct Meta {
+    uint64_t q_full;
+    uint64_t kv_full[kStages];
+    uint64_t kv_empty[kStages];
+    uint64_t s_full[2];
+    uint64_t s_free[2];
+    uint64_t p_full[2];
+    uint64_t pv_done[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int ntok;
+    int nU;
+};
+
+__device__ __forceinline__ int warp_all(bool v)
+{
+    return __all_sync(0xffffffffu, v);
+}
+
+template <int D, int BS>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_attend_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                      const __grid_constant__ CUtensorMap tmv, const FwdAttendParams p)
+{
+    using C = Cfg<D, BS>;
+    extern __shared__ uint8_t fwd_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(fwd_smem_raw) + 1023) & ~uintptr_t(1023));
+    Meta *meta = reinterpret_cast<Meta *>(smem + C::kOffMeta);
+    int *s_union = reinterpret_cast<int *>(smem + C::kOffMeta + sizeof(Meta));
+    int *s_lists = s_union + p.umax;             // [Tq][topk]
+    int *s_cnt = s_lists + p.Tq * p.topk;        // [Tq]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tile = blockIdx.x;
+    const int hk = tile % p.Hkv;
+    const int rest = tile / p.Hkv;
+    const int b = rest % p.batch;
+    const int qt = p.nqt - 1 - rest / p.batch;
+    const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+    const int k0 = p.cu_k[b], sk = p.cu_k[b + 1] - k0;
+    const int tok0 = qt * p.Tq;
+    const int ntok = min(p.Tq, sq - tok0);
+    if (ntok <= 0) return;  // tile beyond this sequence's end (uniform for the CTA)
+    const int nU = p.ucnt[tile];
+
+    if (threadIdx.x == 0) {
+        mbar_init(&meta->q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&meta->kv_full[s], 1);
+            mbar_init(&meta->kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&meta->s_full[s], 1);
+            mbar_init(&meta->s_free[s], 128);
+            mbar_init(&meta->p_full[s], 128);
+            mbar_init(&meta->pv_done[s], 1);
+        }
+        mbar_init(&meta->drain, 1);
+        meta->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&meta->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    // Tile metadata into shared memory: the union of blocks, and each token's sorted list.
+    {
+        const int *gu = p.uni + (int64_t)tile * p.umax;
+        for (int j = threadIdx.x; j < nU; j += kThreads) s_union[j] = gu[j];
+        for (int e = threadIdx.x; e < ntok * p.topk; e += kThreads) {
+            const int tt = e / p.topk, slot = e % p.topk;
+            s_lists[e] = p.sel_c[((int64_t)(q0 + tok0 + tt) * p.Hkv + hk) * p.topk + slot];
+        }
+        for (int tt = threadIdx.x; tt < ntok; tt += kThreads) s_cnt[tt] = p.cnt[(int64_t)(q0 + tok0 + tt) * p.Hkv + hk];
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = meta->tmem_base;
+    volatile int *abort_flag = &meta->abort_flag;
+
+    uint8_t *sQ = smem + C::kOffQ;
+    uint8_t *sK = smem + C::kOffK;
+    uint8_t *sV = smem + C::kOffV;
+    uint8_t *sP = smem + C::kOffP;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0 && nU > 0) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+            const uint32_t qbytes = (uint32_t)(D / 64) * 64u * (uint32_t)(p.G * p.Tq) * 2u;
+            mbar_arrive_expect_tx(&meta->q_full, qbytes);
+            for (int c = 0; c < D / 64; ++c)
+                tma_load_3d(&tmq, &meta->q_full, sQ + c * (128 * 128), c * 64, hk * p.G, q0 + tok0);
+            int issued[kStages] = {};
+            bool ok = true;
+            for (int j = 0; j < nU && ok; ++j) {
+                const int st = j % kStages;
+                if (j >= kStages) ok = mbar_wait(&meta->kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                const int row = k0 + s_union[j] * BS;
+                mbar_arrive_expect_tx(&meta->kv_full[st], 2u * (uint32_t)C::kKVBytes);
+                for (int c = 0; c < D / 64; ++c) {
+                    tma_load_3d(&tmk, &meta->kv_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                    tma_load_3d(&tmv, &meta->kv_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                }
+                issued[st]++;
+            }
+            if (*abort_flag) {  // wind down: let every copy this thread started land
+                mbar_drain(&meta->q_full, 0);
+                for (int st = 0; st < kStages; ++st)
+                    if (issued[st] > 0) mbar_drain(&meta->kv_full[st], (issued[st] - 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0 && nU > 0) {
+            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+            const uint32_t tO = tmem + 2 * BS;
+            bool ok = mbar_wait(&meta->q_full, 0, abort_flag, p.status);
+            auto issue_pv = [&](int i) -> bool {
+                if (!mbar_wait(&meta->p_full[i & 1], (i >> 1) & 1, abort_flag, p.status)) return false;
+                tc_fence_after();
+                const int st = i % kStages;
+#pragma unroll
+                for (int ks = 0; ks < BS / 16; ++ks) {
+                    const uint64_t a = sdesc_sw128(sPa + (i & 1) * C::kPBytes + ks * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(sVa + st * C::kKVBytes + ks * 16 * 128, BS * 128, 1024);
+                    umma_bf16(tO, a, bd, C::kIdescPV, (i > 0 || ks > 0) ? 1u : 0u);
+                }
+                umma_commit(&meta->pv_done[i & 1]);
+                umma_commit(&meta->kv_empty[st]);
+                return true;
+            };
+            for (int j = 0; j < nU && ok; ++j) {
+                const int st = j % kStages;
+                ok = mbar_wait(&meta->kv_full[st], (j / kStages) & 1, abort_flag, p.status);
+                if (ok && j >= 2) ok = mbar_wait(&meta->s_free[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t tS = tmem + (j & 1) * BS;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t a = sdesc_sw128(sQa + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd =
+                        sdesc_sw128(sKa + st * C::kKVBytes + (ks >> 2) * (BS * 128) + (ks & 3) * 32, 16, 1024);
+                    umma_bf16(tS, a, bd, C::kIdescS, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&meta->s_full[j & 1]);
+                if (j >= 1) ok = issue_pv(j - 1);
+            }
+            if (ok) ok = issue_pv(nU - 1);
+            if (!ok) {  // wind down: wait for the MMAs already issued
+                umma_commit(&meta->drain);
+                mbar_drain(&meta->drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ softmax + epilogue
+        const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;
+        const int tok = r / p.G, g = r % p.G;
+        const bool row_valid = (tok < ntok);  // r < Tq*G is implied by tok < ntok <= Tq
+        const int i = tok0 + tok;
+        const int delta = sk - sq;
+        int lo = 0, hi = sk - 1;
+        if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
+        if (p.causal) hi = min(hi, i + delta);
+        if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
+        const int *mylist = s_lists + (row_valid ? tok : 0) * p.topk;
+        const int mycnt = row_valid ? s_cnt[tok] : 0;
+        int ptr = 0;
+        float m_run = -INFINITY;  // running max of s*scale*log2e
+        float l_run = 0.f;
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t tO = lane_base + 2 * BS;
+        uint8_t *prow_base = sP + (r >> 3) * 1024 + (r & 7) * 128;
+        bool ok = true;
+
+        for (int j = 0; j < nU; ++j) {
+            const int s = s_union[j];
+            const bool selected = ptr < mycnt && mylist[ptr] == s;
+            if (selected) ++ptr;
+            ok = warp_all(mbar_wait(&meta->s_full[j & 1], (j >> 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            float x[BS];
+            {
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < BS / 32; ++c) {
+                    tmem_ld32(lane_base + (j & 1) * BS + c * 32, raw);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[e]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&meta->s_free[j & 1]);
+
+            const int kb = s * BS;
+            const bool full = selected && kb >= lo && kb + BS - 1 <= hi;
+            if (!full) {
+#pragma unroll
+                for (int c = 0; c < BS; ++c) {
+                    const int key = kb + c;
+                    const bool keep = selected && key >= lo && key <= hi;
+                    x[c] = keep ? x[c] : -INFINITY;
+                }
+            }
+            float mx = x[0];
+#pragma unroll
+            for (int c = 1; c < BS; ++c) mx = fmaxf(mx, x[c]);
+            const float m_new = mx * p.scale_log2;
+            const bool need = m_new > m_run + kRescaleLog2;
+            if (__any_sync(0xffffffffu, need)) {
+                float factor = 1.f;
+                if (need) {
+                    factor = ex2(m_run - m_new);
+                    m_run = m_new;
+                    l_run *= factor;
+                }
+                if (j > 0) {
+                    ok = warp_all(mbar_wait(&meta->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.status));
+                    if (!ok) break;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + c * 32, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+                        tmem_st32(tO + c * 32, o);
+                    }
+                    tmem_wait_st();
+                }
+            } else if (j >= 2) {
+                ok = warp_all(mbar_wait(&meta->pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.status));
+                if (!ok) break;
+            }
+            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+            float rowsum = 0.f;
+            uint32_t packed[BS / 2];
+#pragma unroll
+            for (int c = 0; c < BS; c += 2) {
+                const float p0 = ex2(fmaf(x[c], p.scale_log2, -m_use));
+                const float p1 = ex2(fmaf(x[c + 1], p.scale_log2, -m_use));
+                rowsum += p0 + p1;
+                packed[c / 2] = pack_bf16x2(p0, p1);
+            }
+            l_run += rowsum;
+            uint8_t *prow = prow_base + (j & 1) * C::kPBytes;
+#pragma unroll
+            for (int cc = 0; cc < BS / 8; ++cc) {
+                const int phys = cc ^ (r & 7);
+                *reinterpret_cast<uint4 *>(prow + phys * 16) =
+                    make_uint4(packed[cc * 4 + 0], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&meta->p_full[j & 1]);
+        }
+
+        // ---------------------------------------------------------------- epilogue
+        if (ok && nU > 0) {
+            ok = warp_all(mbar_wait(&meta->pv_done[(nU - 1) & 1], ((nU - 1) >> 1) & 1, abort_flag, p.status));
+            tc_fence_after();
+        }
+        if (ok) {
+            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+            const int64_t t = (int64_t)q0 + i;
+            const int h = hk * p.G + g;
+            __nv_bfloat16 *orow = p.out + (t * p.Hq + h) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                if (nU > 0) {
+                    tmem_ld32(tO + c * 32, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                }
+                if (row_valid) {
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                }
+            }
+            if (row_valid)
+                p.lse[(int64_t)h * p.total_q + t] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <int D, int BS>
+size_t smem_bytes_for(const FwdGeom &g)
+{
+    using C = Cfg<D, BS>;
+    return 1024 + C::kOffMeta + sizeof(Meta) + (size_t)g.umax * 4 + (size_t)g.Tq * g.topk * 4 + (size_t)g.Tq * 4;
+}
+
+template <int D, int BS>
+cudaError_t launch_t(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                     const CUtensorMap &tv, cudaStream_t st)
+{
+    const size_t smem = smem_bytes_for<D, BS>(g);
+    static int configured = 0;
+    if ((int)smem > configured) {
+        cudaError_t e =
+            cudaFuncSetAttribute(fwd_attend_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = (int)smem;
+    }
+    fwd_attend_kernel<D, BS><<<g.tiles, kThreads, smem, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t fwd_attend_smem_bytes(const FwdGeom &g)
+{
+    if (g.d == 64) return g.bs == 32 ? smem_bytes_for<64, 32>(g) : smem_bytes_for<64, 64>(g);
+    return g.bs == 32 ? smem_bytes_for<128, 32>(g) : smem_bytes_for<128, 64>(g);
+}
+
+cudaError_t launch_fwd_attend(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
+                              const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
+{
+    if (g.d == 64) return g.bs == 32 ? launch_t<64, 32>(g, p, tq, tk, tv, st) : launch_t<64, 64>(g, p, tq, tk, tv, st);
+    return g.bs == 32 ? launch_t<128, 32>(g, p, tq, tk, tv, st) : launch_t<128, 64>(g, p, tq, tk, tv, st);
+}
+
+}  // namespace sfa

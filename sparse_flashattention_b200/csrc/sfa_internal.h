@@ -1,0 +1,87 @@
+// Internal interfaces between the C-ABI host layer (sfa_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/sfa.h"
+
+namespace sfa {
+
+// ---------------------------------------------------------------------------------------
+// Prefill
+// ---------------------------------------------------------------------------------------
+// A query tile is Tq consecutive tokens of one sequence times the G query heads of one kv
+// head: Tq * G <= 128 rows, the M dimension of one tcgen05 MMA.  Tiles are numbered
+// tile = (qt_rev * batch + b) * Hkv + hk with qt = nqt - 1 - qt_rev, so the tiles deepest
+// into their sequences (the ones with the most blocks under a causal mask) start first.
+struct FwdGeom {
+    int batch, max_sq, max_sk, total_q, Hq, Hkv, d, topk, bs;
+    int G, Tq, nqt, tiles, nblk_max, umax;
+    size_t off_sel_c, off_cnt, off_ucnt, off_union, bytes;
+};
+
+struct FwdPrepParams {
+    const int32_t *cu_q, *cu_k, *sel;
+    int batch, Hkv, topk, bs, causal, wl, wr, Tq, nqt, umax, max_sq, nblk_max;
+    int32_t *sel_c, *cnt, *ucnt, *uni;
+    int32_t *status;
+};
+
+struct FwdAttendParams {
+    const int32_t *cu_q, *cu_k;
+    const int32_t *sel_c, *cnt, *ucnt, *uni;
+    int batch, total_q, Hq, Hkv, G, Tq, nqt, topk, umax;
+    int causal, wl, wr;
+    float scale_log2;  // softmax scale * log2(e)
+    __nv_bfloat16 *out;
+    float *lse;
+    int32_t *status;
+};
+
+// ---------------------------------------------------------------------------------------
+// Decode
+// ---------------------------------------------------------------------------------------
+struct DecGeom {
+    int B, Hq, Hkv, d, topk, S, G;
+    size_t off_tok, off_cnt, off_po, off_plse, bytes;
+};
+
+struct DecPrepParams {
+    const int32_t *seqlens, *sel;
+    int topk, max_len, Hkv, wl;
+    int32_t *tok_c, *cnt;
+    int32_t *status;
+};
+
+struct DecSplitParams {
+    const __nv_bfloat16 *q, *kc, *vc;
+    const int32_t *bt, *tok_c, *cnt;
+    int max_pages, num_pages, page, Hq, Hkv, G, topk, S;
+    float scale_log2;
+    float *po, *plse;  // partial outputs (B, Hq, S, d) and natural-log lse (B, Hq, S)
+    int32_t *status;
+};
+
+struct DecCombineParams {
+    const float *po, *plse;
+    int Hq, S;
+    __nv_bfloat16 *out;
+    float *lse;
+};
+
+// Launchers (return the launch's cudaError_t).
+cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream_t st);
+cudaError_t launch_fwd_attend(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
+                              const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
+size_t fwd_attend_smem_bytes(const FwdGeom &g);
+
+cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStream_t st);
+cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaStream_t st);
+cudaError_t launch_decode_combine(const DecGeom &g, const DecCombineParams &p, cudaStream_t st);
+int decode_split_blocks_per_sm(int d);
+
+}  // namespace sfa

@@ -1,0 +1,104 @@
+"""The C ABI without a GPU: the library loads, exports every function include/sfa.h declares,
+and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sfa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from sparse_flashattention_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sfa_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "sfa_fwd" in names and "sfa_decode" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/sfa.h but not exported"
+
+
+def test_status_strings(lib):
+    lib.sfa_status_string.restype = ctypes.c_char_p
+    for code in range(5):
+        assert lib.sfa_status_string(code).decode().startswith("SFA_")
+
+
+P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+FAKE = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def _fwd(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, cu_q=FAKE, cu_k=None, batch=1, max_sq=128, max_sk=128, total_q=128,
+             total_k=128, Hq=4, Hkv=1, d=64, sel=FAKE, topk=4, bs=32, causal=1, wl=-1, wr=-1, scale=0.0,
+             ws=FAKE, ws_bytes=0, status=None, out=FAKE, lse=FAKE, stream=None)
+    a.update(over)
+    lib.sfa_fwd.restype = I
+    lib.sfa_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, P, I, I, I, I, I, F, P, Z, P, P, P, P]
+    return lib.sfa_fwd(*a.values())
+
+
+def test_fwd_host_validation(lib):
+    lib.sfa_fwd_workspace_size.restype = Z
+    lib.sfa_fwd_workspace_size.argtypes = [I] * 9
+    need = lib.sfa_fwd_workspace_size(1, 128, 128, 128, 4, 1, 64, 4, 32)
+    assert need > 0
+    assert lib.sfa_fwd_workspace_size(1, 0, 0, 0, 4, 1, 64, 4, 32) == 0
+    assert _fwd(lib, Hq=6, Hkv=4) == 1          # Hq % Hkv != 0 -> SFA_ERR_INVALID_ARG
+    assert _fwd(lib, d=96) == 2                  # unsupported head dim
+    assert _fwd(lib, bs=48) == 2                 # unsupported block size
+    assert _fwd(lib, topk=0) == 1
+    assert _fwd(lib, topk=129) == 2
+    assert _fwd(lib, causal=2) == 1
+    assert _fwd(lib, wl=-2) == 1
+    assert _fwd(lib, q=ctypes.c_void_p((1 << 20) + 8)) == 1   # misaligned base
+    assert _fwd(lib, sel=None) == 1
+    assert _fwd(lib, total_k=100) == 1           # cu_k NULL but total_k != total_q
+    assert _fwd(lib, ws_bytes=need - 1) == 3     # SFA_ERR_WORKSPACE_TOO_SMALL
+    assert _fwd(lib, total_q=0, total_k=0) == 0   # nothing to do: OK without launching
+
+
+def test_decode_host_validation(lib):
+    lib.sfa_decode.restype = I
+    lib.sfa_decode.argtypes = [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]
+    lib.sfa_decode_workspace_size.restype = Z
+    lib.sfa_decode_workspace_size.argtypes = [I] * 6
+
+    def call(**over):
+        a = dict(q=FAKE, kc=FAKE, vc=FAKE, bt=FAKE, maxp=4, npages=8, page=256, lens=FAKE, sel=FAKE, topk=64, B=2,
+                 Hq=8, Hkv=2, d=128, wl=-1, scale=0.0, splits=0, ws=FAKE, ws_bytes=0, status=None, out=FAKE,
+                 lse=FAKE, stream=None)
+        a.update(over)
+        return lib.sfa_decode(*a.values())
+
+    need = lib.sfa_decode_workspace_size(2, 8, 2, 128, 64, 0)
+    assert need > 0
+    assert call(Hq=8, Hkv=3) == 1
+    assert call(Hq=64, Hkv=2) == 2               # G = 32 > 16 unsupported
+    assert call(d=80) == 2
+    assert call(page=0) == 1
+    assert call(bt=None) == 1
+    assert call(wl=-5) == 1
+    assert call(ws_bytes=need - 1) == 3
+    assert call(B=0) == 0
+
+
+def test_decode_split_heuristic(lib):
+    lib.sfa_decode_num_splits.restype = I
+    lib.sfa_decode_num_splits.argtypes = [I] * 6
+    assert lib.sfa_decode_num_splits(32, 32, 8, 128, 2048, 5) == 5
+    s = lib.sfa_decode_num_splits(32, 32, 8, 128, 2048, 0)
+    assert 1 <= s <= 16
+    assert lib.sfa_decode_num_splits(1, 8, 8, 128, 100, 0) == 1

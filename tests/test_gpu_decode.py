@@ -1,0 +1,137 @@
+"""GPU parity of the paged top-k decode path (sfa_decode through the C ABI) against the oracle."""
+import numpy as np
+import pytest
+
+import sfa_workloads as W
+from tests.parity import assert_empty_rows_exact, assert_lse_close, assert_out_close, dev_tensor, run_decode, upload_decode
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sfa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_flashattention_b200 as m
+    return m
+
+
+def _parity(sfa, oracle_lib, c, status_expect=0, **kw):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = run_decode(sfa, c, status=status, **kw)
+    ro, rl, _ = oracle_lib.decode(c)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    assert int(status.item()) == status_expect
+    return out, lse
+
+
+def test_small_decode_parity(sfa, oracle_lib):
+    _parity(sfa, oracle_lib, W.small_config(5))
+
+
+def test_decode_prep_bit_exact(sfa, oracle_lib):
+    c = W.small_config(5)
+    d = upload_decode(c)
+    _, tok_c, cnt = sfa.decode_prep(d["cache_seqlens"], d["sel"], Hq=c.Hq, d=c.d, max_pages_per_seq=c.max_pages,
+                                    page_size=c.page)
+    rt, rc, _ = oracle_lib.decode_index(c)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
+    np.testing.assert_array_equal(tok_c.cpu().numpy(), rt)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 4, 8, 16])
+def test_split_count_invariance(sfa, oracle_lib, splits):
+    """Any number of key chunks merged through their LSEs gives the unsplit result."""
+    c = W.small_config(5)
+    out, lse = _parity(sfa, oracle_lib, c, num_splits=splits)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,d,page,lo,hi,topk,last", [(3, 8, 8, 128, 64, 10, 900, 200, 16),
+                                                              (5, 16, 2, 64, 16, 1, 333, 100, 8),
+                                                              (2, 16, 1, 128, 256, 3000, 5000, 1000, 64),
+                                                              (4, 4, 4, 64, 1, 5, 300, 64, 4)])
+def test_decode_shapes(sfa, oracle_lib, B, Hq, Hkv, d, page, lo, hi, topk, last):
+    c = W.make_decode(B * 7 + d + page, B, Hq, Hkv, d, page, lo, hi, topk, last)
+    _parity(sfa, oracle_lib, c)
+
+
+def test_decode_window(sfa, oracle_lib):
+    c = W.small_config(5)
+    c = W.DecodeCase(**{**c.__dict__, "wl": 500})
+    _parity(sfa, oracle_lib, c)
+
+
+def test_paging_invariance_bitwise(sfa):
+    """The seeded permuted block table over the permuted pool == the identity table over
+    contiguous pages, bit for bit."""
+    c = W.small_config(5)
+    out, lse = run_decode(sfa, c)
+    npg = c.max_pages
+    kc = np.zeros((c.B * npg, c.page, c.Hkv, c.d), np.uint16)
+    vc = np.zeros_like(kc)
+    bt = np.full((c.B, npg), -1, np.int32)
+    for b in range(c.B):
+        for p in range(npg):
+            if c.block_table[b, p] >= 0:
+                kc[b * npg + p] = c.k_cache[c.block_table[b, p]]
+                vc[b * npg + p] = c.v_cache[c.block_table[b, p]]
+                bt[b, p] = b * npg + p
+    c2 = W.DecodeCase(**{**c.__dict__, "k_cache": kc, "v_cache": vc, "block_table": bt})
+    o2, l2 = run_decode(sfa, c2)
+    assert torch.equal(out, o2) and torch.equal(lse, l2)
+
+
+def test_bad_page_and_bad_ids(sfa, oracle_lib):
+    c = W.small_config(5)
+    bt = c.block_table.copy()
+    bt[1, 0] = c.num_pages + 3
+    c2 = W.DecodeCase(**{**c.__dict__, "block_table": bt})
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = run_decode(sfa, c2, status=status)
+    ro, rl, bad = oracle_lib.decode(c2)
+    assert bad[1] > 0 and int(status.item()) & 2  # SFA_DEV_BAD_PAGE
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    sel = c.sel.copy()
+    sel[0, 0, 0] = c.cache_seqlens[0] + 5
+    sel[2, 1, 3] = -9
+    c3 = W.DecodeCase(**{**c.__dict__, "sel": sel})
+    status.zero_()
+    out, lse = run_decode(sfa, c3, status=status)
+    ro, rl, bad = oracle_lib.decode(c3)
+    assert bad[0] == 2 and int(status.item()) & 1
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+
+
+def test_all_padding_decode(sfa):
+    c = W.small_config(5)
+    out, lse = run_decode(sfa, c, sel=dev_tensor(np.full_like(c.sel, -1)))
+    assert_empty_rows_exact(out, lse)
+
+
+def test_decode_launch_count(sfa):
+    c = W.small_config(5)
+    run_decode(sfa, c)
+    assert sfa.last_launch_count() == 3
+
+
+def test_full_size_decode(sfa, oracle_lib):
+    """The paged decode workload at full size (B32, Hq32/Hkv8, L up to 131072, 2048 tokens per
+    (sequence, kv head)), in the launch configuration the benchmark times: every output row
+    against the oracle, and the canonical token sets bit-exact."""
+    c = W.config5()
+    d = upload_decode(c)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = run_decode(sfa, c, d=d, status=status)
+    ro, rl, _ = oracle_lib.decode(c)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    assert int(status.item()) == 0
+    _, tok_c, cnt = sfa.decode_prep(d["cache_seqlens"], d["sel"], Hq=c.Hq, d=c.d, max_pages_per_seq=c.max_pages,
+                                    page_size=c.page)
+    rt, rc, _ = oracle_lib.decode_index(c)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
+    np.testing.assert_array_equal(tok_c.cpu().numpy(), rt)

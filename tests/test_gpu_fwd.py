@@ -1,0 +1,210 @@
+"""GPU parity of the prefill path (sfa_fwd through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+
+import sfa_workloads as W
+from tests.parity import (assert_empty_rows_exact, assert_lse_close, assert_out_close, dev_tensor, run_fwd,
+                          upload_prefill)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def sfa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import sparse_flashattention_b200 as m
+    return m
+
+
+def _case(seqlens_q, seqlens_k, Hq, Hkv, d, bs, sel, seed, causal=1, wl=-1, wr=-1, scale=0.0):
+    rng = np.random.default_rng(seed)
+    tq, tk = int(sum(seqlens_q)), int(sum(seqlens_k))
+    q = W.f32_to_bf16_bits(rng.standard_normal((tq, Hq, d), dtype=np.float32))
+    k = W.f32_to_bf16_bits(rng.standard_normal((tk, Hkv, d), dtype=np.float32))
+    v = W.f32_to_bf16_bits(rng.standard_normal((tk, Hkv, d), dtype=np.float32))
+    return W.PrefillCase("t", q, k, v, W._cu(seqlens_q), W._cu(seqlens_k), np.asarray(sel, np.int32), Hq, Hkv, d, bs,
+                         sel.shape[-1], causal, wl, wr, scale)
+
+
+def _all_blocks(total_q, Hkv, nblk, rng=None):
+    s = np.broadcast_to(np.arange(nblk, dtype=np.int32), (total_q, Hkv, nblk)).copy()
+    if rng is not None:
+        s = W._shuffle_rows(rng, s.reshape(-1, nblk)).reshape(s.shape)
+    return s
+
+
+def _full_parity(sfa, oracle_lib, c, status_expect=0):
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = run_fwd(sfa, c, status=status)
+    ro, rl, _ = oracle_lib.fwd(c)
+    assert_out_close(out, ro)
+    assert_lse_close(lse, rl)
+    ninf = np.isneginf(rl)  # (Hq, total_q)
+    if ninf.any():
+        h, t = np.where(ninf)
+        assert_empty_rows_exact(out[torch.as_tensor(t), torch.as_tensor(h)], lse[torch.as_tensor(h), torch.as_tensor(t)])
+    assert int(status.item()) == status_expect
+    return out, lse
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4])
+def test_small_configs_full_parity(sfa, oracle_lib, n):
+    """Oracle-sized versions of the four prefill workloads: every output element."""
+    _full_parity(sfa, oracle_lib, W.small_config(n))
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4])
+def test_index_prep_bit_exact(sfa, oracle_lib, n):
+    c = W.small_config(n)
+    d = upload_prefill(c)
+    _, sel_c, cnt = sfa.fwd_prep(d["cu_q"], d["sel"], Hq=c.Hq, d=c.d, block_size=c.bs, cu_seqlens_k=d["cu_k"],
+                                 max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk, causal=bool(c.causal),
+                                 window=(c.wl, c.wr))
+    rs, rc, _ = oracle_lib.fwd_index(c)
+    np.testing.assert_array_equal(sel_c.cpu().numpy(), rs)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
+
+
+def _sample_rows(c, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.integers(0, c.total_q * c.Hq, size=n).tolist())
+    for b in range(c.batch):  # first and last token of every sequence, every head
+        for t in (c.cu_q[b], c.cu_q[b + 1] - 1):
+            rows.update(int(t) * c.Hq + h for h in range(c.Hq))
+    return np.asarray(sorted(rows), np.int64)
+
+
+FULL = {1: W.config1, 2: W.config2, 3: W.config3, 4: W.config4}
+
+
+@pytest.mark.parametrize("n", [1, 2, 3, 4])
+def test_full_size_configs_sampled(sfa, oracle_lib, n):
+    """The four prefill workloads at full size, in the launch configuration the benchmark
+    times: every row computed on the GPU, a sample of rows (plus every sequence's first and
+    last token) checked against the oracle; the whole canonical index set bit-exact."""
+    c = FULL[n]()
+    d = upload_prefill(c)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = run_fwd(sfa, c, d=d, status=status)
+    rows = _sample_rows(c, 3000, n)
+    ro, rl, _ = oracle_lib.fwd(c, rows=rows)
+    t, h = rows // c.Hq, rows % c.Hq
+    assert_out_close(out.view(-1, c.d)[torch.as_tensor(rows, device="cuda")], ro)
+    assert_lse_close(lse[torch.as_tensor(h, device="cuda"), torch.as_tensor(t, device="cuda")], rl)
+    assert int(status.item()) == 0
+    _, sel_c, cnt = sfa.fwd_prep(d["cu_q"], d["sel"], Hq=c.Hq, d=c.d, block_size=c.bs, cu_seqlens_k=d["cu_k"],
+                                 max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk, causal=bool(c.causal),
+                                 window=(c.wl, c.wr))
+    rs, rc, _ = oracle_lib.fwd_index(c)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
+    np.testing.assert_array_equal(sel_c.cpu().numpy(), rs)
+    o = out.float()
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("sq,sk", [(2, 5), (5, 2), (70, 200), (200, 70)])
+def test_bottom_right_causal_and_empty_rows(sfa, oracle_lib, sq, sk):
+    """Unequal lengths (the printed 2x5 and 5x2 examples and larger ones): rows whose causal
+    limit is below key 0 output exactly 0 with lse -inf."""
+    bs = 32
+    nblk = -(-sk // bs)
+    c = _case([sq, sq], [sk, sk], 4, 2, 64, bs, _all_blocks(2 * sq, 2, nblk, np.random.default_rng(0)), 3)
+    _full_parity(sfa, oracle_lib, c)
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,bs", [(6, 2, 64, 32), (6, 2, 128, 64), (8, 8, 128, 64), (16, 2, 64, 64),
+                                         (32, 2, 128, 32), (1, 1, 64, 64), (128, 1, 64, 32)])
+def test_gqa_groups_and_shapes(sfa, oracle_lib, Hq, Hkv, d, bs):
+    """GQA groups G = 3 (the 6->2 example), 1, 8, 16, 128 with d 64/128 and block 32/64, on
+    ragged sequences with an NSA selection."""
+    lens = [300, 1, 77, 129]
+    c = W.make_nsa_prefill(Hq * 100 + Hkv + d + bs, lens, Hq, Hkv, d, bs, 6, 1, 2)
+    _full_parity(sfa, oracle_lib, c)
+
+
+@pytest.mark.parametrize("causal,wl,wr", [(0, -1, -1), (0, 40, 30), (1, 100, 0), (0, 0, 0), (1, 0, -1)])
+def test_windows(sfa, oracle_lib, causal, wl, wr):
+    sq, sk, bs = 150, 260, 64
+    nblk = -(-sk // bs)
+    c = _case([sq, 90], [sk, 100], 8, 2, 128, bs, _all_blocks(sq + 90, 2, nblk, np.random.default_rng(1)), 5,
+              causal=causal, wl=wl, wr=wr)
+    _full_parity(sfa, oracle_lib, c)
+
+
+def test_window_minus1_0_equals_causal_bitwise(sfa):
+    c = W.small_config(2)
+    a, la = run_fwd(sfa, c)
+    c2 = W.PrefillCase(**{**c.__dict__, "causal": 0, "wl": -1, "wr": 0})
+    b, lb = run_fwd(sfa, c2)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_selection_is_a_set_bitwise(sfa, oracle_lib):
+    """Permuted and duplicated slots give bit-identical outputs (the kernel sees only the
+    canonical set)."""
+    c = W.small_config(4)
+    base, lbase = run_fwd(sfa, c)
+    rng = np.random.default_rng(3)
+    sel = W._shuffle_rows(rng, c.sel.reshape(-1, c.topk)).reshape(c.sel.shape).copy()
+    flat = sel.reshape(-1, c.topk)
+    for r in range(flat.shape[0]):
+        valid = flat[r][flat[r] >= 0]
+        pads = np.where(flat[r] < 0)[0]
+        if valid.size and pads.size:
+            flat[r, pads] = rng.choice(valid, size=pads.size)
+    out, lse = run_fwd(sfa, c, sel=dev_tensor(sel))
+    assert torch.equal(out, base) and torch.equal(lse, lbase)
+
+
+def test_bad_ids_flagged_and_ignored(sfa, oracle_lib):
+    c = W.small_config(2)
+    base, lbase = run_fwd(sfa, c)
+    sel = c.sel.copy()
+    idx = np.argwhere(sel == -1)[:50]
+    sel[idx[:, 0], idx[:, 1], idx[:, 2]] = np.where(np.arange(len(idx)) % 2 == 0, 10 ** 6, -7)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = run_fwd(sfa, c, sel=dev_tensor(sel), status=status)
+    assert int(status.item()) & 1  # SFA_DEV_BAD_INDEX
+    assert torch.equal(out, base) and torch.equal(lse, lbase)
+
+
+def test_all_padding_rows(sfa):
+    """A selection of only -1 slots: every row is empty."""
+    c = W.small_config(2)
+    sel = np.full_like(c.sel, -1)
+    out, lse = run_fwd(sfa, c, sel=dev_tensor(sel))
+    assert_empty_rows_exact(out, lse)
+
+
+def test_rows_sum_to_one(sfa):
+    """v == 1: every non-empty row outputs 1 within the bf16 tolerance."""
+    c = W.small_config(4)
+    c = W.PrefillCase(**{**c.__dict__, "v": np.full_like(c.v, 0x3F80)})
+    out, _ = run_fwd(sfa, c)
+    assert_out_close(out, np.ones(out.shape))
+
+
+def test_empty_batch_and_explicit_scale(sfa, oracle_lib):
+    c = W.small_config(1)
+    c = W.PrefillCase(**{**c.__dict__, "scale": 0.3})
+    _full_parity(sfa, oracle_lib, c)
+    q = torch.empty((0, 4, 64), dtype=torch.bfloat16, device="cuda")
+    cu = torch.zeros(2, dtype=torch.int32, device="cuda")
+    sel = torch.empty((0, 1, 4), dtype=torch.int32, device="cuda")
+    out, lse = sfa.fwd(q, q[:, :1], q[:, :1], cu, sel, 32, max_seqlen_q=0, max_seqlen_k=0)
+    assert out.shape == (0, 4, 64) and lse.shape == (4, 0)
+
+
+def test_launch_count_and_stages(sfa, oracle_lib):
+    """sfa_fwd = prep + attend: two launches; the split-stage calls give the same result."""
+    c = W.small_config(2)
+    d = upload_prefill(c)
+    out, lse = run_fwd(sfa, c, d=d)
+    assert sfa.last_launch_count() == 2
+    ws, _, _ = sfa.fwd_prep(d["cu_q"], d["sel"], Hq=c.Hq, d=c.d, block_size=c.bs, cu_seqlens_k=d["cu_k"],
+                            max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk)
+    o2, l2 = sfa.fwd_attend(d["q"], d["k"], d["v"], d["cu_q"], ws, topk=c.topk, block_size=c.bs,
+                            cu_seqlens_k=d["cu_k"], max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk)
+    assert torch.equal(out, o2) and torch.equal(lse, l2)
