@@ -183,6 +183,25 @@ int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache,
                       void *workspace, size_t workspace_bytes, int32_t *status_dev,
                       void *out, float *lse, sfa_stream_t stream);
 
+/* Paged top-k decode for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this call: it exists for callers such as serving engines whose device memory
+ * pool is fixed before serving and forbids later allocation, or plugin hooks that receive only
+ * input and output pointers.  Same arguments, semantics and kernels as sfa_decode, without the
+ * workspace: the scratch lives in a static device array of 8 MiB that every GPU loading this
+ * library keeps until the process exits.
+ *   - Returns SFA_ERR_WORKSPACE_TOO_SMALL when sfa_decode_workspace_size() of these arguments
+ *     exceeds 8 MiB (nothing is launched).  It calls no allocation routine of any kind.
+ *   - The first call on each device looks the array's address up on that device (with it
+ *     current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array, and each call rewrites every byte it reads
+ *     from it, so nothing carries over between calls; two calls that overlap on the GPU
+ *     (other streams, other host threads) race on it and give undefined results. */
+int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
+                       const int32_t *cache_seqlens, const int32_t *sel_tok_idx, int topk_tok,
+                       int B, int Hq, int Hkv, int d, int window_left, float scale, int num_splits,
+                       int32_t *status_dev, void *out, float *lse, sfa_stream_t stream);
+
 /* Human-readable name of an sfa_status value (static string). */
 const char *sfa_status_string(int status);
 

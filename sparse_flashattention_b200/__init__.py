@@ -19,7 +19,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["SfaError", "lib_path", "fwd", "fwd_prep", "fwd_attend", "fwd_workspace_size", "decode", "decode_prep",
-           "decode_attend", "decode_workspace_size", "decode_num_splits", "last_launch_count",
+           "decode_attend", "decode_noalloc", "decode_workspace_size", "decode_num_splits", "last_launch_count",
            "DEV_BAD_INDEX", "DEV_BAD_PAGE", "DEV_TIMEOUT"]
 
 DEV_BAD_INDEX, DEV_BAD_PAGE, DEV_TIMEOUT = 1, 2, 4
@@ -54,6 +54,7 @@ def _load():
         "sfa_decode": (I, [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]),
         "sfa_decode_prep": (I, [P, P, I, I, I, I, I, I, I, I, I, P, Z, P, P]),
         "sfa_decode_attend": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]),
+        "sfa_decode_noalloc": (I, [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, F, I, P, P, P, P]),
         "sfa_status_string": (ctypes.c_char_p, [I]),
         "sfa_last_launch_count": (I, []),
     }
@@ -310,5 +311,22 @@ def decode_attend(q, k_cache, v_cache, block_table, workspace, *, topk_tok: int,
                                 num_pages, page, int(topk_tok), B, Hq, Hkv, d, _scale(scale), int(num_splits),
                                 _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
                                 _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def decode_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx, *, window_left: int = -1,
+                   scale=None, num_splits: int = 0, out=None, lse=None, status=None, stream=None):
+    """sfa_decode_noalloc: the same decode without a workspace, for callers that may not
+    allocate device memory at call time.  Its scratch is a static 8 MiB device array shared by
+    every call on the device (calls must not overlap on the GPU); the first call on a device
+    should come before any stream capture.  Pass out/lse to avoid allocating them here."""
+    B, Hq, d, num_pages, page, Hkv = _dec_checks(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    rc = _lib.sfa_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table), block_table.shape[1],
+                                 num_pages, page, _ptr(cache_seqlens), _ptr(sel_tok_idx), sel_tok_idx.shape[2], B, Hq,
+                                 Hkv, d, int(window_left), _scale(scale), int(num_splits), _ptr(status), _ptr(out),
+                                 _ptr(lse), _stream(stream))
     _check(rc)
     return out, lse
