@@ -166,11 +166,15 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     hbm, tf_burst, tf_sust, peak_kind = peaks()
 
-    pc = W.config2()
+    pc = W.config2() if args.part != "decode-small" else W.small_config(2)
     P = upload_prefill(pc, dev)
     flops = prefill_flops(pc)
-    if args.part == "prefill":  # profiling aid: the prefill stages alone, without the 9.7 GB decode cache
+    # Profiling aids: 'prefill' skips the 9.7 GB decode cache (a tiny decode case stands in);
+    # 'decode-small' runs the decode shape with shorter caches (about 1.3 GB) for ncu captures.
+    if args.part == "prefill":
         dc = W.make_decode(5, 2, 32, 8, 128, 256, 1024, 2048, 256, 16)
+    elif args.part == "decode-small":
+        dc = W.make_decode(5, 32, 32, 8, 128, 256, 4096, 16384, 2048, 128, parallel_values=True)
     else:
         dc = W.config5(parallel_values=True)
     D = upload_decode(dc, dev)
@@ -349,7 +353,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--part", default="all", choices=["all", "prefill"],
+    ap.add_argument("--part", default="all", choices=["all", "prefill", "decode-small"],
                     help="'prefill' times only the prefill stages (a small decode case stands in); for profiling")
     ap.add_argument("--traffic", type=float, default=None,
                     help="dram bytes (read+write) per attend launch from an ncu capture of this kernel version")

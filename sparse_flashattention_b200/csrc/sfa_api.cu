@@ -199,20 +199,24 @@ int num_sms()
     return n > 0 ? n : 148;
 }
 
-// Split count: the smallest S whose last wave of CTAs is the fullest (CTAs = B*Hkv*S over
-// num_SMs * CTAs-per-SM slots), with at least 128 tokens per split.
+// Split count: each split is one warp's chunk of a (sequence, kv head) token list, and a CTA
+// runs decode_split_warps_per_block() of them.  Pick the S (at least 64 tokens per split)
+// whose last wave of CTAs over num_SMs * CTAs-per-SM slots is fullest, with a small charge per
+// extra split for its prologue and its partial output.
 int choose_splits(int B, int Hkv, int d, int topk)
 {
     const int units = B * Hkv;
+    const int wpb = decode_split_warps_per_block();
     const int slots = num_sms() * decode_split_blocks_per_sm(d);
-    const int smax = std::max(1, std::min(64, (topk + 127) / 128));
+    const int smax = std::max(1, std::min(64, topk / 64));
     int best = 1;
-    double best_eff = -1.0;
+    double best_score = -1e30;
     for (int S = 1; S <= smax; ++S) {
-        const double waves = (double)units * S / slots;
-        const double eff = waves / std::ceil(waves);
-        if (eff > best_eff + 1e-9) {
-            best_eff = eff;
+        const double ctas = std::ceil((double)units * S / wpb);
+        const double waves = ctas / slots;
+        const double score = waves / std::ceil(waves) - 0.002 * S;
+        if (score > best_score + 1e-9) {
+            best_score = score;
             best = S;
         }
     }
@@ -279,6 +283,7 @@ int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void 
     p.bt = bt;
     p.tok_c = reinterpret_cast<const int32_t *>(w + g.off_tok);
     p.cnt = reinterpret_cast<const int32_t *>(w + g.off_cnt);
+    p.B = g.B;
     p.max_pages = max_pages;
     p.num_pages = num_pages;
     p.page = page;

@@ -12,8 +12,12 @@
 //   softmax warps   4 warps, one thread per row: read S from TMEM, apply the row's mask
 //                   (block not selected by this row, bottom-right causal limit, window,
 //                   sequence end), keep the running max and sum in fp32 (base-2 domain),
-//                   write P = 2^(s*scale*log2e - m) as bf16 into shared memory for the MMA,
-//                   rescale O in TMEM when the running max grows by more than 2^8.
+//                   write P = 2^(s*scale*log2e - m) as bf16 back into TMEM over its own scores,
+//                   where the PV MMA reads it as the A operand, and rescale O in TMEM when the
+//                   running max grows by more than 2^8.
+//
+// A CTA needs about 100 KB of shared memory and 256 TMEM columns, so two CTAs share an SM and
+// one CTA's softmax overlaps the other's MMAs.
 //
 // The epilogue divides O by the running sum, writes bf16 out and the natural-log LSE.
 // The method is the FlashAttention tiling with online softmax applied to the gathered blocks
@@ -30,7 +34,7 @@ namespace sfa {
 namespace {
 
 constexpr int kThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 softmax/epilogue
-constexpr int kStages = 3;
+constexpr int kStages = 2;  // two 32 KB K/V stages keep the CTA near 100 KB: two CTAs per SM
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only when the max grows by more than 2^8
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -38,12 +42,10 @@ template <int D, int BS>
 struct Cfg {
     static constexpr int kQBytes = 128 * D * 2;
     static constexpr int kKVBytes = BS * D * 2;  // one K (or V) block
-    static constexpr int kPBytes = 128 * 128;    // 128 rows x 64 bf16 (128-byte swizzle rows)
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffP = kOffV + kStages * kKVBytes;
-    static constexpr int kOffMeta = kOffP + 2 * kPBytes;
+    static constexpr int kOffMeta = kOffV + kStages * kKVBytes;
     static constexpr int kTmemCols = (2 * BS + D <= 128) ? 128 : 256;
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
@@ -54,7 +56,6 @@ struct Meta {
     uint64_t kv_full[kStages];
     uint64_t kv_empty[kStages];
     uint64_t s_full[2];
-    uint64_t s_free[2];
     uint64_t p_full[2];
     uint64_t pv_done[2];
     uint64_t drain;
@@ -70,7 +71,7 @@ __device__ __forceinline__ int warp_all(bool v)
 }
 
 template <int D, int BS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     fwd_attend_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                       const __grid_constant__ CUtensorMap tmv, const FwdAttendParams p)
 {
@@ -103,7 +104,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&meta->s_full[s], 1);
-            mbar_init(&meta->s_free[s], 128);
             mbar_init(&meta->p_full[s], 128);
             mbar_init(&meta->pv_done[s], 1);
         }
@@ -134,7 +134,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
-    uint8_t *sP = smem + C::kOffP;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
@@ -169,7 +168,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0 && nU > 0) {
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV), sPa = smem_u32(sP);
+            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
             const uint32_t tO = tmem + 2 * BS;
             bool ok = mbar_wait(&meta->q_full, 0, abort_flag, p.status);
             auto issue_pv = [&](int i) -> bool {
@@ -178,9 +177,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int st = i % kStages;
 #pragma unroll
                 for (int ks = 0; ks < BS / 16; ++ks) {
-                    const uint64_t a = sdesc_sw128(sPa + (i & 1) * C::kPBytes + ks * 32, 16, 1024);
+                    // P_i (bf16) sits in the first BS/2 columns of score buffer i&1: 8 columns per K=16.
+                    const uint32_t a = tmem + (i & 1) * BS + ks * 8;
                     const uint64_t bd = sdesc_sw128(sVa + st * C::kKVBytes + ks * 16 * 128, BS * 128, 1024);
-                    umma_bf16(tO, a, bd, C::kIdescPV, (i > 0 || ks > 0) ? 1u : 0u);
+                    umma_bf16_tmem_a(tO, a, bd, C::kIdescPV, (i > 0 || ks > 0) ? 1u : 0u);
                 }
                 umma_commit(&meta->pv_done[i & 1]);
                 umma_commit(&meta->kv_empty[st]);
@@ -188,8 +188,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             for (int j = 0; j < nU && ok; ++j) {
                 const int st = j % kStages;
+                // Score buffer j&1 is free again: PV_{j-2}, which read P_{j-2} from it, was issued
+                // before this MMA (after softmax j-2 finished), and tcgen05 MMAs of one thread run in
+                // issue order.
                 ok = mbar_wait(&meta->kv_full[st], (j / kStages) & 1, abort_flag, p.status);
-                if (ok && j >= 2) ok = mbar_wait(&meta->s_free[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.status);
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t tS = tmem + (j & 1) * BS;
@@ -228,7 +230,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         float l_run = 0.f;
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t tO = lane_base + 2 * BS;
-        uint8_t *prow_base = sP + (r >> 3) * 1024 + (r & 7) * 128;
         bool ok = true;
 
         for (int j = 0; j < nU; ++j) {
@@ -249,8 +250,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[e]);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&meta->s_free[j & 1]);
 
             const int kb = s * BS;
             const bool full = selected && kb >= lo && kb + BS - 1 <= hi;
@@ -304,14 +303,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 packed[c / 2] = pack_bf16x2(p0, p1);
             }
             l_run += rowsum;
-            uint8_t *prow = prow_base + (j & 1) * C::kPBytes;
-#pragma unroll
-            for (int cc = 0; cc < BS / 8; ++cc) {
-                const int phys = cc ^ (r & 7);
-                *reinterpret_cast<uint4 *>(prow + phys * 16) =
-                    make_uint4(packed[cc * 4 + 0], packed[cc * 4 + 1], packed[cc * 4 + 2], packed[cc * 4 + 3]);
+            // P_j overwrites the first BS/2 columns of its own score buffer (already in registers).
+            if constexpr (BS == 64) {
+                tmem_st32(lane_base + (j & 1) * BS, packed);
+            } else {
+                tmem_st16(lane_base + (j & 1) * BS, packed);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&meta->p_full[j & 1]);
         }

@@ -60,7 +60,7 @@ struct DecPrepParams {
 struct DecSplitParams {
     const __nv_bfloat16 *q, *kc, *vc;
     const int32_t *bt, *tok_c, *cnt;
-    int max_pages, num_pages, page, Hq, Hkv, G, topk, S;
+    int B, max_pages, num_pages, page, Hq, Hkv, G, topk, S;
     float scale_log2;
     float *po, *plse;  // partial outputs (B, Hq, S, d) and natural-log lse (B, Hq, S)
     int32_t *status;
@@ -83,5 +83,6 @@ cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStr
 cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecGeom &g, const DecCombineParams &p, cudaStream_t st);
 int decode_split_blocks_per_sm(int d);
+int decode_split_warps_per_block();
 
 }  // namespace sfa

@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
     if (threadIdx.x == 0) p.ucnt[tile] = total;
 }
 
-constexpr int kDecPrepThreads = 256;
+constexpr int kDecPrepThreads = 512;
 
 __global__ void __launch_bounds__(kDecPrepThreads) decode_prep_kernel(DecPrepParams p)
 {
