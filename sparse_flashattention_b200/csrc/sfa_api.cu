@@ -61,6 +61,12 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     g.tiles = (int)tiles;
     g.nblk_max = (int)std::max<int64_t>(nblk_max, 1);
     g.umax = (int)std::max<int64_t>(1, std::min<int64_t>(nblk_max, (int64_t)g.Tq * topk));
+    // Block-major schedule for sparse windows: windows of 64 tiles; its block histogram lives in
+    // shared memory, and (token, slot) pairs pack the token into 24 bits.
+    g.W = g.Tq * 64;
+    g.nwin = (max_sq + g.W - 1) / g.W;
+    g.groups = g.nwin * batch * Hkv;
+    g.inv = (g.nblk_max <= 2048 && total_q < (1 << 24) && fwd_attend_inv_smem_bytes(g) <= 227 * 1024) ? 1 : 0;
     size_t off = 0;
     g.off_sel_c = off;
     off = align_up(off + (size_t)total_q * Hkv * topk * 4);
@@ -70,6 +76,19 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     off = align_up(off + (size_t)g.tiles * 4);
     g.off_union = off;
     off = align_up(off + (size_t)g.tiles * g.umax * 4);
+    if (g.inv) {
+        const size_t pairs = (size_t)total_q * Hkv * topk;
+        g.off_ctrl = off;
+        off = align_up(off + sizeof(InvCtrl));
+        g.off_pairs = off;
+        off = align_up(off + pairs * 4);
+        g.off_items = off;
+        off = align_up(off + pairs * 16);
+        g.off_pml = off;
+        off = align_up(off + (size_t)total_q * Hq * topk * 8);
+        g.off_po = off;
+        off = align_up(off + (size_t)total_q * Hq * topk * d * 2);
+    }
     g.bytes = total_q == 0 ? 0 : off;
     return SFA_OK;
 }
@@ -107,12 +126,30 @@ bool encode_3d(CUtensorMap &m, const void *base, int d, int heads, int64_t rows,
     return r == CUDA_SUCCESS;
 }
 
+// A (rows, d) bf16 matrix as a 2-D map {d, rows} with a {64, 1} box, 128-byte swizzle: the form
+// tile::gather4 loads use (four arbitrary rows per copy).
+bool encode_rows(CUtensorMap &m, const void *base, int d, int64_t rows)
+{
+    auto enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64u, 1u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = enc(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 int check_window(int causal, int wl, int wr)
 {
     if (causal != 0 && causal != 1) return SFA_ERR_INVALID_ARG;
     if (wl < -1 || wr < -1) return SFA_ERR_INVALID_ARG;
     return SFA_OK;
 }
+
+int fwd_invert_impl(const FwdGeom &g, const int32_t *cu_q, void *ws, cudaStream_t st);
 
 int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, const int32_t *sel, int causal, int wl,
                   int wr, void *ws, int32_t *status, cudaStream_t st)
@@ -138,8 +175,38 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     p.cnt = reinterpret_cast<int32_t *>(w + g.off_cnt);
     p.ucnt = reinterpret_cast<int32_t *>(w + g.off_ucnt);
     p.uni = reinterpret_cast<int32_t *>(w + g.off_union);
+    p.ctrl = g.inv ? reinterpret_cast<InvCtrl *>(w + g.off_ctrl) : nullptr;
     p.status = status;
-    return launch_fwd_prep(g, p, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+    if (launch_fwd_prep(g, p, st) != cudaSuccess) return SFA_ERR_CUDA;
+    return fwd_invert_impl(g, cu_q, ws, st);
+}
+
+// Second prep kernel: choose query-major or block-major per window and build the block-major
+// items.
+int fwd_invert_impl(const FwdGeom &g, const int32_t *cu_q, void *ws, cudaStream_t st)
+{
+    if (!g.inv) return SFA_OK;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    FwdInvertParams p{};
+    p.cu_q = cu_q;
+    p.cnt = reinterpret_cast<const int32_t *>(w + g.off_cnt);
+    p.sel_c = reinterpret_cast<const int32_t *>(w + g.off_sel_c);
+    p.ucnt = reinterpret_cast<int32_t *>(w + g.off_ucnt);
+    p.batch = g.batch;
+    p.Hq = g.Hq;
+    p.Hkv = g.Hkv;
+    p.G = g.G;
+    p.Tq = g.Tq;
+    p.nqt = g.nqt;
+    p.topk = g.topk;
+    p.W = g.W;
+    p.nwin = g.nwin;
+    p.total_q = g.total_q;
+    p.D = g.d;
+    p.pairs = reinterpret_cast<int32_t *>(w + g.off_pairs);
+    p.items = reinterpret_cast<int4 *>(w + g.off_items);
+    p.ctrl = reinterpret_cast<InvCtrl *>(w + g.off_ctrl);
+    return launch_fwd_invert(g, p, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
 }
 
 int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *v, const int32_t *cu_q,
@@ -176,7 +243,18 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.lse = lse;
     p.status = status;
-    return launch_fwd_attend(g, p, tq, tk, tv, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+    if (launch_fwd_attend(g, p, tq, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
+    if (!g.inv) return SFA_OK;
+    uint8_t *wm = static_cast<uint8_t *>(ws);
+    p.pairs = reinterpret_cast<const int32_t *>(wm + g.off_pairs);
+    p.items = reinterpret_cast<const int4 *>(wm + g.off_items);
+    p.ctrl = reinterpret_cast<InvCtrl *>(wm + g.off_ctrl);
+    p.po = reinterpret_cast<__nv_bfloat16 *>(wm + g.off_po);
+    p.pml = reinterpret_cast<float2 *>(wm + g.off_pml);
+    CUtensorMap tq2;  // q as (total_q * Hq) rows of d, one-row boxes for the 4-row gathers
+    if (!encode_rows(tq2, q, g.d, (int64_t)g.total_q * g.Hq)) return SFA_ERR_CUDA;
+    if (launch_fwd_attend_inv(g, p, tq2, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
+    return launch_fwd_merge(g, p, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
 }
 
 int fwd_common_checks(const int32_t *cu_q, const int32_t *cu_k, int total_q, int total_k, int max_sq, int max_sk,
@@ -347,7 +425,7 @@ int sfa_fwd_prep(const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int b
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
     rc = fwd_prep_impl(g, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
                        status_dev, stream);
-    if (rc == SFA_OK) g_last_launches = 1;
+    if (rc == SFA_OK) g_last_launches = 1 + g.inv;
     return rc;
 }
 
@@ -371,7 +449,7 @@ int sfa_fwd_attend(const void *q, const void *k, const void *v, const int32_t *c
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
     rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right, scale,
                          workspace, status_dev, out, lse, stream);
-    if (rc == SFA_OK) g_last_launches = 1;
+    if (rc == SFA_OK) g_last_launches = 1 + 2 * g.inv;
     return rc;
 }
 
@@ -399,7 +477,7 @@ int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqle
     if (rc != SFA_OK) return rc;
     rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right, scale,
                          workspace, status_dev, out, lse, stream);
-    if (rc == SFA_OK) g_last_launches = 2;
+    if (rc == SFA_OK) g_last_launches = 2 + 3 * g.inv;
     return rc;
 }
 

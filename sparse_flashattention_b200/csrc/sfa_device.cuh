@@ -84,6 +84,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     }
 }
 
+__device__ __forceinline__ bool warp_all_ok(bool v)
+{
+    return __all_sync(0xffffffffu, v) != 0;
+}
+
+// Barrier among the `count` threads that share an mbarrier initialised with that count; every
+// participant tracks the same use counter.  Bounded like mbar_wait (a plain bar.sync could
+// wait forever if a participant left after an abort).
+__device__ __forceinline__ bool group_sync(uint64_t *bar, int &uses, volatile int *abort_flag, int32_t *status_dev)
+{
+    mbar_arrive(bar);
+    const bool ok = mbar_wait(bar, (uint32_t)(uses & 1), abort_flag, status_dev);
+    ++uses;
+    return ok;
+}
+
 // Bounded wait used only while winding down after an abort (short limit, no flag checks).
 __device__ __forceinline__ void mbar_drain(uint64_t *bar, uint32_t parity)
 {
@@ -108,6 +124,18 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint64_t *ba
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Four rows (any row coordinates) of a 2-D tensor map whose box is {64 elements, 1 row}: the
+// rows land one after another (4 x 128 bytes) at dst, with the map's swizzle applied.
+__device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint64_t *bar, void *dst, int c0, int r0, int r1,
+                                            int r2, int r3)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
         : "memory");
 }
 

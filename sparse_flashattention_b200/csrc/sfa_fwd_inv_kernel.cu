@@ -1,0 +1,494 @@
+// Block-major prefill attention for sparse query windows, with the partial merge fused in.
+//
+// When a window's tokens select their blocks with little overlap (an NSA-style random top-k
+// over a long prefix), the union of a query tile's blocks is many times the selected work.
+// Here the loop is turned around, as the FSA project page describes for its selected-attention
+// kernel (key/value block outer, queries inner): an item is one selected K/V block of one kv
+// head plus up to Tq tokens of the window that selected it, Tq*G <= 128 query rows gathered
+// into one tensor-core tile.  Per item the CTA computes S = Q K^T (tcgen05, TMEM), the masked
+// softmax of that one block (max m, sum l, P = 2^(s*scale*log2e - m) in bf16 back into TMEM),
+// O = P V (tcgen05), and writes every row's normalised partial o/l (bf16) with (m, l).
+//
+// A separate merge kernel (the reduction step of FSA's kernel split) then combines each row's
+// partials: lse = log of the sum of l*2^m, out = the weighted mean of the partials.
+//
+// One persistent CTA per SM walks the item list with a fixed stride.  Warp 0 prefetches the
+// next item's record and token list, TMA-loads the K/V block and gathers the item's Q rows four
+// at a time with TMA tile::gather4 into a 128-byte-swizzled tile; warp 1 issues the MMAs; two
+// groups of four warps alternate over items (softmax and epilogue), so one group's softmax
+// overlaps the other group's MMAs.  All waits are bounded.
+#include "sfa_device.cuh"
+
+namespace sfa {
+
+namespace {
+
+constexpr int kInvThreadsAttn = 320;  // warp 0 producer, warp 1 MMA, warps 2-5 and 6-9: two softmax groups
+constexpr float kLn2i = 0.6931471805599453f;
+
+template <int D, int BS>
+struct InvCfg {
+    static constexpr int kQBytes = 128 * D * 2;
+    static constexpr int kKVBytes = BS * D * 2;
+    static constexpr int kOffQ = 0;                        // Q[2]
+    static constexpr int kOffK = 2 * kQBytes;              // K[2]
+    static constexpr int kOffV = kOffK + 2 * kKVBytes;     // V[2]
+    static constexpr int kOffMeta = kOffV + 2 * kKVBytes;
+    static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
+    static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+    static constexpr int kTmemCols = 512;  // S/P of group w at w*BS, O of group w at 128 + w*D
+};
+
+struct ItemSlot {
+    int4 rec;  // {b*Hkv + hk, block, first pair, tokens}; tokens < 0 ends the work
+    int tok[128];
+};
+
+struct InvMeta {
+    uint64_t item_full[2], item_free[2];
+    uint64_t q_full[2], q_empty[2];
+    uint64_t kv_full[2], kv_empty[2];
+    uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    ItemSlot slot[2];
+};
+
+template <int D, int BS>
+__global__ void __launch_bounds__(kInvThreadsAttn, 1)
+    fwd_attend_inv_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
+                          const __grid_constant__ CUtensorMap tmv, const FwdAttendParams p)
+{
+    using C = InvCfg<D, BS>;
+    extern __shared__ uint8_t inv_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(inv_smem_raw) + 1023) & ~uintptr_t(1023));
+    InvMeta *meta = reinterpret_cast<InvMeta *>(smem + C::kOffMeta);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&meta->item_full[s], 1);
+            mbar_init(&meta->item_free[s], 128);
+            mbar_init(&meta->q_full[s], 1);
+            mbar_init(&meta->q_empty[s], 1);
+            mbar_init(&meta->kv_full[s], 1);
+            mbar_init(&meta->kv_empty[s], 1);
+            mbar_init(&meta->s_full[s], 1);
+            mbar_init(&meta->p_full[s], 128);
+            mbar_init(&meta->pv_done[s], 1);
+            mbar_init(&meta->o_free[s], 128);
+        }
+        mbar_init(&meta->drain, 1);
+        meta->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&meta->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = meta->tmem_base;
+    volatile int *abort_flag = &meta->abort_flag;
+    uint8_t *sQ = smem + C::kOffQ;
+    uint8_t *sK = smem + C::kOffK;
+    uint8_t *sV = smem + C::kOffV;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- producer (all 32 lanes)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmq);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+        }
+        const int total = *reinterpret_cast<volatile int *>(&p.ctrl->item_total);
+        const int4 kEnd = make_int4(0, 0, 0, -1);
+        // Item j of this CTA is item blockIdx.x + j * gridDim.x; the next one's record and
+        // token list are fetched one item ahead.
+        int4 rec_next = (int)blockIdx.x < total ? __ldcg(&p.items[blockIdx.x]) : kEnd;
+        int tok_next[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = lane + 32 * u;
+            tok_next[u] = e < rec_next.w ? __ldcg(&p.pairs[rec_next.z + e]) : 0;
+        }
+        int issued[2] = {0, 0};
+        bool ok = true;
+        for (int j = 0; ok; ++j) {
+            const int sl = j & 1;
+            const uint32_t ph = ((j >> 1) - 1) & 1;  // phase of this slot's previous use
+            const int4 rec = rec_next;
+            int tok[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) tok[u] = tok_next[u];
+            const long long nidx = (long long)blockIdx.x + (long long)(j + 1) * gridDim.x;
+            rec_next = nidx < total ? __ldcg(&p.items[nidx]) : kEnd;
+            if (j >= 2) ok = warp_all_ok(mbar_wait(&meta->item_free[sl], ph, abort_flag, p.status));
+            if (!ok) break;
+            ItemSlot *slot = &meta->slot[sl];
+            if (rec.w < 0) {
+                // End of work: both slots get an end marker, so both softmax groups stop.
+                if (lane == 0) {
+                    slot->rec = kEnd;
+                    mbar_arrive(&meta->item_full[sl]);
+                }
+                const int j2 = j + 1, sl2 = j2 & 1;
+                if (j2 >= 2) ok = warp_all_ok(mbar_wait(&meta->item_free[sl2], ((j2 >> 1) - 1) & 1, abort_flag, p.status));
+                if (ok && lane == 0) {
+                    meta->slot[sl2].rec = kEnd;
+                    mbar_arrive(&meta->item_full[sl2]);
+                }
+                break;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (lane + 32 * u < rec.w) slot->tok[lane + 32 * u] = tok[u];
+            if (lane == 0) slot->rec = rec;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&meta->item_full[sl]);
+            const int hk = rec.x % p.Hkv, b = rec.x / p.Hkv;
+            // K/V block
+            if (j >= 2) ok = warp_all_ok(mbar_wait(&meta->kv_empty[sl], ph, abort_flag, p.status));
+            if (!ok) break;
+            if (lane == 0) {
+                const int row = p.cu_k[b] + rec.y * BS;
+                mbar_arrive_expect_tx(&meta->kv_full[sl], 2u * (uint32_t)C::kKVBytes);
+                for (int c = 0; c < D / 64; ++c) {
+                    tma_load_3d(&tmk, &meta->kv_full[sl], sK + sl * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                    tma_load_3d(&tmv, &meta->kv_full[sl], sV + sl * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                }
+                issued[sl]++;
+            }
+            // Q rows of the item's tokens, four rows per TMA gather into the swizzled K-major tile
+            // (row r = token * G + head; a last partial group repeats its last row).
+            if (j >= 2) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
+            if (!ok) break;
+            {
+                const int rows = rec.w * p.G;
+                const int ng = (rows + 3) >> 2;
+                if (lane == 0) mbar_arrive_expect_tx(&meta->q_full[sl], (uint32_t)(ng * (D / 64)) * 512u);
+                __syncwarp();
+                for (int gi = lane; gi < ng * (D / 64); gi += 32) {
+                    const int c = gi % (D / 64), g4 = gi / (D / 64);
+                    int grow[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int rr = min(4 * g4 + u, rows - 1);
+                        const int tk = rr / p.G, gg = rr - tk * p.G;
+                        grow[u] = (slot->tok[tk] >> 7) * p.Hq + hk * p.G + gg;
+                    }
+                    tma_gather4(&tmq, &meta->q_full[sl], sQ + sl * C::kQBytes + c * (128 * 128) + g4 * 512, c * 64,
+                                grow[0], grow[1], grow[2], grow[3]);
+                }
+            }
+            // The next item's token list (its record was requested above).
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = lane + 32 * u;
+                tok_next[u] = e < rec_next.w ? __ldcg(&p.pairs[rec_next.z + e]) : 0;
+            }
+        }
+        if (*abort_flag && lane == 0) {
+            for (int sl = 0; sl < 2; ++sl)
+                if (issued[sl] > 0) mbar_drain(&meta->kv_full[sl], (issued[sl] - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+            bool ok = true;
+            auto issue_pv = [&](int i) -> bool {
+                const int w = i & 1;
+                if (!mbar_wait(&meta->p_full[w], (i >> 1) & 1, abort_flag, p.status)) return false;
+                if (i >= 2 && !mbar_wait(&meta->o_free[w], ((i >> 1) - 1) & 1, abort_flag, p.status)) return false;
+                tc_fence_after();
+                const uint32_t tO = tmem + 128 + w * D;
+#pragma unroll
+                for (int ks = 0; ks < BS / 16; ++ks) {
+                    const uint32_t a = tmem + w * BS + ks * 8;
+                    const uint64_t bd = sdesc_sw128(sVa + w * C::kKVBytes + ks * 16 * 128, BS * 128, 1024);
+                    umma_bf16_tmem_a(tO, a, bd, C::kIdescPV, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&meta->pv_done[w]);
+                umma_commit(&meta->kv_empty[w]);
+                return true;
+            };
+            int j = 0;
+            for (;; ++j) {
+                const int sl = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                ok = mbar_wait(&meta->item_full[sl], ph, abort_flag, p.status);
+                if (!ok) break;
+                if (meta->slot[sl].rec.w < 0) break;
+                ok = mbar_wait(&meta->q_full[sl], ph, abort_flag, p.status) &&
+                     mbar_wait(&meta->kv_full[sl], ph, abort_flag, p.status);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t tS = tmem + sl * BS;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const uint64_t a =
+                        sdesc_sw128(sQa + sl * C::kQBytes + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
+                    const uint64_t bd =
+                        sdesc_sw128(sKa + sl * C::kKVBytes + (ks >> 2) * (BS * 128) + (ks & 3) * 32, 16, 1024);
+                    umma_bf16(tS, a, bd, C::kIdescS, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&meta->s_full[sl]);
+                umma_commit(&meta->q_empty[sl]);
+                if (j >= 1) {
+                    ok = issue_pv(j - 1);
+                    if (!ok) break;
+                }
+            }
+            if (ok && j >= 1) ok = issue_pv(j - 1);
+            if (!ok) {
+                umma_commit(&meta->drain);
+                mbar_drain(&meta->drain, 0);
+            }
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax groups
+        const int grp = (warp - 2) >> 2;        // 0: warps 2-5, 1: warps 6-9
+        const int quad = warp & 3;              // TMEM lane quadrant of this warp
+        const int r = quad * 32 + lane;         // tile row
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        const uint32_t tS = lane_base + grp * BS;
+        const uint32_t tO = lane_base + 128 + grp * D;
+        bool ok = true;
+        for (int j = grp; ok; j += 2) {
+            const uint32_t ph = (j >> 1) & 1;
+            ok = warp_all_ok(mbar_wait(&meta->item_full[grp], ph, abort_flag, p.status));
+            if (!ok) break;
+            const int4 rec = meta->slot[grp].rec;
+            if (rec.w < 0) break;
+            const int hk = rec.x % p.Hkv, b = rec.x / p.Hkv, s = rec.y, n = rec.w;
+            const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+            const int sk = p.cu_k[b + 1] - p.cu_k[b];
+            const int tok = r / p.G, gg = r - tok * p.G;
+            const bool valid = tok < n;
+            int64_t t = 0;
+            int kslot = 0, lo = 0, hi = -1;
+            if (valid) {
+                const int e = meta->slot[grp].tok[tok];
+                t = e >> 7;
+                kslot = e & 127;
+                const int i = (int)(t - q0), delta = sk - sq;
+                lo = 0;
+                hi = sk - 1;
+                if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
+                if (p.causal) hi = min(hi, i + delta);
+                if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
+            }
+            ok = warp_all_ok(mbar_wait(&meta->s_full[grp], ph, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            float x[BS];
+            {
+                uint32_t raw[32];
+#pragma unroll
+                for (int c = 0; c < BS / 32; ++c) {
+                    tmem_ld32(tS + c * 32, raw);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[e]);
+                }
+            }
+            const int kb = s * BS;
+            if (!(valid && kb >= lo && kb + BS - 1 <= hi)) {
+#pragma unroll
+                for (int c = 0; c < BS; ++c) {
+                    const int key = kb + c;
+                    x[c] = (valid && key >= lo && key <= hi) ? x[c] : -INFINITY;
+                }
+            }
+            float mx = x[0];
+#pragma unroll
+            for (int c = 1; c < BS; ++c) mx = fmaxf(mx, x[c]);
+            const float m = mx * p.scale_log2;
+            const float m_use = m == -INFINITY ? 0.f : m;
+            float l = 0.f;
+            uint32_t packed[BS / 2];
+#pragma unroll
+            for (int c = 0; c < BS; c += 2) {
+                const float p0 = ex2(fmaf(x[c], p.scale_log2, -m_use));
+                const float p1 = ex2(fmaf(x[c + 1], p.scale_log2, -m_use));
+                l += p0 + p1;
+                packed[c / 2] = pack_bf16x2(p0, p1);
+            }
+            if constexpr (BS == 64) {
+                tmem_st32(tS, packed);
+            } else {
+                tmem_st16(tS, packed);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&meta->p_full[grp]);
+
+            // Epilogue: the row's normalised partial and its (max, sum).
+            ok = warp_all_ok(mbar_wait(&meta->pv_done[grp], ph, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            const int h = hk * p.G + gg;
+            const int64_t pslot = (t * p.Hq + h) * p.topk + kslot;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tO + c * 32, o);
+                tmem_wait_ld();
+                if (valid) {
+                    uint32_t wv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.po + pslot * D + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&meta->o_free[grp]);
+            if (valid) p.pml[pslot] = make_float2(m, l);
+
+            mbar_arrive(&meta->item_free[grp]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// Merge of the block-major partials, one warp per (token, kv head) whose tile went block-major:
+// for each of the G heads, M = max m_k, L = sum l_k 2^(m_k - M), out = sum (l_k 2^(m_k - M) / L) o_k,
+// lse = (M + log2 L) ln 2.  Lanes cover the head dimension in 16-byte chunks and split the
+// partials between them, so every lane keeps several independent loads in flight.
+constexpr int kMergeWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kMergeWarps) fwd_merge_kernel(const FwdAttendParams p)
+{
+    constexpr int kChunks = D / 8;       // 16-byte chunks of a row
+    constexpr int kSplit = 32 / kChunks; // lanes sharing a chunk, each over every kSplit-th partial
+    const int lane = threadIdx.x & 31;
+    const int64_t u = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+    if (u >= (int64_t)p.total_q * p.Hkv) return;
+    const int cnt = p.cnt[u];
+    if (cnt == 0) return;  // written by the query-major kernel
+    const int64_t t = u / p.Hkv;
+    const int hk = (int)(u - t * p.Hkv);
+    int lo = 0, hi = p.batch - 1;
+    while (lo < hi) {  // batch entry of token t
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.cu_q[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const int b = lo;
+    const int qt = (int)(t - p.cu_q[b]) / p.Tq;
+    if (p.ucnt[((p.nqt - 1 - qt) * p.batch + b) * p.Hkv + hk] >= 0) return;  // query-major tile
+
+    const int c = lane % kChunks, kq = lane / kChunks;
+    for (int g = 0; g < p.G; ++g) {
+        const int h = hk * p.G + g;
+        const int64_t base = (t * p.Hq + h) * p.topk;
+        float M = -INFINITY;
+        for (int k = lane; k < cnt; k += 32) {
+            const float2 ml = __ldcg(&p.pml[base + k]);
+            if (ml.y > 0.f) M = fmaxf(M, ml.x);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int k = lane; k < cnt; k += 32) {
+            const float2 ml = __ldcg(&p.pml[base + k]);
+            if (ml.y > 0.f) L += ml.y * ex2(ml.x - M);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        const float invL = L > 0.f ? 1.f / L : 0.f;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll 4
+        for (int k = kq; k < cnt; k += kSplit) {
+            const float2 ml = __ldcg(&p.pml[base + k]);
+            const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(p.po + (base + k) * D) + c);
+            const float w = ml.y > 0.f ? ml.y * ex2(ml.x - M) * invL : 0.f;
+            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vv[e]));
+                acc[2 * e] += w * f.x;
+                acc[2 * e + 1] += w * f.y;
+            }
+        }
+#pragma unroll
+        for (int o = kChunks; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+        if (kq == 0) {
+            uint4 w4;
+            w4.x = pack_bf16x2(acc[0], acc[1]);
+            w4.y = pack_bf16x2(acc[2], acc[3]);
+            w4.z = pack_bf16x2(acc[4], acc[5]);
+            w4.w = pack_bf16x2(acc[6], acc[7]);
+            reinterpret_cast<uint4 *>(p.out + (t * p.Hq + h) * D)[c] = w4;
+        }
+        if (lane == 0) p.lse[(int64_t)h * p.total_q + t] = L > 0.f ? (M + log2f(L)) * kLn2i : -INFINITY;
+    }
+}
+
+template <int D, int BS>
+size_t inv_smem_bytes()
+{
+    return 1024 + InvCfg<D, BS>::kOffMeta + sizeof(InvMeta);
+}
+
+template <int D, int BS>
+cudaError_t launch_inv_t(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
+                         const CUtensorMap &tv, cudaStream_t st)
+{
+    const size_t smem = inv_smem_bytes<D, BS>();
+    static bool configured = false;
+    if (!configured) {
+        cudaError_t e =
+            cudaFuncSetAttribute(fwd_attend_inv_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured = true;
+    }
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    fwd_attend_inv_kernel<D, BS><<<sms, kInvThreadsAttn, smem, st>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t fwd_attend_inv_smem_bytes(const FwdGeom &g)
+{
+    if (g.d == 64) return g.bs == 32 ? inv_smem_bytes<64, 32>() : inv_smem_bytes<64, 64>();
+    return g.bs == 32 ? inv_smem_bytes<128, 32>() : inv_smem_bytes<128, 64>();
+}
+
+cudaError_t launch_fwd_merge(const FwdGeom &g, const FwdAttendParams &p, cudaStream_t st)
+{
+    const int64_t units = (int64_t)g.total_q * g.Hkv;
+    const unsigned grid = (unsigned)((units + kMergeWarps - 1) / kMergeWarps);
+    if (g.d == 64) fwd_merge_kernel<64><<<grid, 32 * kMergeWarps, 0, st>>>(p);
+    else fwd_merge_kernel<128><<<grid, 32 * kMergeWarps, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_attend_inv(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
+                                  const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
+{
+    if (g.d == 64) return g.bs == 32 ? launch_inv_t<64, 32>(g, p, tq, tk, tv, st) : launch_inv_t<64, 64>(g, p, tq, tk, tv, st);
+    return g.bs == 32 ? launch_inv_t<128, 32>(g, p, tq, tk, tv, st) : launch_inv_t<128, 64>(g, p, tq, tk, tv, st);
+}
+
+}  // namespace sfa

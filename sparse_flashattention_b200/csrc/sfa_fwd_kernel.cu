@@ -95,6 +95,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int ntok = min(p.Tq, sq - tok0);
     if (ntok <= 0) return;  // tile beyond this sequence's end (uniform for the CTA)
     const int nU = p.ucnt[tile];
+    if (nU < 0) {
+        // The block-major kernel computes this tile's rows; only rows that keep no key at all
+        // (no partial will ever arrive for them) are written here: output 0, lse -inf.
+        for (int e = threadIdx.x; e < ntok * p.G; e += kThreads) {
+            const int tt = e / p.G, gg = e - tt * p.G;
+            const int64_t t = (int64_t)q0 + tok0 + tt;
+            if (p.cnt[t * p.Hkv + hk] != 0) continue;
+            const int h = hk * p.G + gg;
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out + (t * p.Hq + h) * D);
+            for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+            p.lse[(int64_t)h * p.total_q + t] = -INFINITY;
+        }
+        return;
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(&meta->q_full, 1);

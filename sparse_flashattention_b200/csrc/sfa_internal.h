@@ -21,14 +21,39 @@ namespace sfa {
 struct FwdGeom {
     int batch, max_sq, max_sk, total_q, Hq, Hkv, d, topk, bs;
     int G, Tq, nqt, tiles, nblk_max, umax;
-    size_t off_sel_c, off_cnt, off_ucnt, off_union, bytes;
+    // Block-major schedule for sparse query windows (inv = 0 when this call cannot use it):
+    // a window is W consecutive tokens of one sequence; for one (window, sequence, kv head)
+    // group the prep lists, per selected block, the window's tokens that selected it, and cuts
+    // those lists into items of at most Tq tokens.
+    int inv, W, nwin, groups;
+    size_t off_sel_c, off_cnt, off_ucnt, off_union;
+    size_t off_ctrl, off_pairs, off_items, off_pml, off_po;
+    size_t bytes;
+};
+
+// Control words of the block-major schedule, reset by the prep kernel of every call.
+struct InvCtrl {
+    int item_total;    // items written by the invert kernel
+    int pair_total;    // (token, slot) entries written by the invert kernel
+    int work_counter;  // next item the attention kernel hands out
+    int pad;
 };
 
 struct FwdPrepParams {
     const int32_t *cu_q, *cu_k, *sel;
     int batch, Hkv, topk, bs, causal, wl, wr, Tq, nqt, umax, max_sq, nblk_max;
     int32_t *sel_c, *cnt, *ucnt, *uni;
+    InvCtrl *ctrl;     // nullptr when the block-major schedule is off
     int32_t *status;
+};
+
+struct FwdInvertParams {
+    const int32_t *cu_q, *cnt, *sel_c;
+    int32_t *ucnt;
+    int batch, Hq, Hkv, G, Tq, nqt, topk, W, nwin, total_q, D;
+    int32_t *pairs;   // (token << 7 | slot) per (token, selected block), grouped by block
+    int4 *items;      // {b * Hkv + hk, block, first pair, tokens}
+    InvCtrl *ctrl;
 };
 
 struct FwdAttendParams {
@@ -40,6 +65,12 @@ struct FwdAttendParams {
     __nv_bfloat16 *out;
     float *lse;
     int32_t *status;
+    // block-major schedule
+    const int32_t *pairs;
+    const int4 *items;
+    InvCtrl *ctrl;
+    __nv_bfloat16 *po;  // partial outputs, (total_q, Hq, topk, d) bf16, normalised
+    float2 *pml;        // partial (max, sum) in the base-2 scaled domain, (total_q, Hq, topk)
 };
 
 // ---------------------------------------------------------------------------------------
@@ -78,6 +109,11 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
 cudaError_t launch_fwd_attend(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
                               const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 size_t fwd_attend_smem_bytes(const FwdGeom &g);
+cudaError_t launch_fwd_invert(const FwdGeom &g, const FwdInvertParams &p, cudaStream_t st);
+cudaError_t launch_fwd_attend_inv(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
+                                  const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
+cudaError_t launch_fwd_merge(const FwdGeom &g, const FwdAttendParams &p, cudaStream_t st);
+size_t fwd_attend_inv_smem_bytes(const FwdGeom &g);
 
 cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStream_t st);
 cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaStream_t st);

@@ -68,10 +68,30 @@ __device__ int compact_bitmap(const uint32_t *bm, int words, int32_t *dst, int *
     return total;
 }
 
+// One warp-wide op on per-lane keys (-1 = no key): lanes holding the same key are counted
+// together and only the lowest of them touches shared memory.  Returns, for each lane, the
+// first value it may use (the leader's old value plus the lane's rank among equal keys).
+__device__ __forceinline__ int warp_aggregated_add(int *counters, int key)
+{
+    const int lane = threadIdx.x & 31;
+    const unsigned m = __match_any_sync(0xffffffffu, key);
+    const int leader = __ffs(m) - 1;
+    const int rank = __popc(m & ((1u << lane) - 1));
+    int base = 0;
+    if (lane == leader && key >= 0) base = atomicAdd(&counters[key], __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    return base + rank;
+}
+
 __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
 {
     extern __shared__ uint32_t prep_smem[];
     __shared__ int scan_scratch[32];
+    if (blockIdx.x == 0 && threadIdx.x == 0 && p.ctrl) {
+        p.ctrl->item_total = 0;
+        p.ctrl->pair_total = 0;
+        p.ctrl->work_counter = 0;
+    }
     const int tile = blockIdx.x;
     const int hk = tile % p.Hkv;
     const int rest = tile / p.Hkv;
@@ -79,39 +99,43 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
     const int qt = p.nqt - 1 - rest / p.batch;
 
     const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
-    const int k0 = p.cu_k[b], sk = p.cu_k[b + 1] - k0;
+    const int sk = p.cu_k[b + 1] - p.cu_k[b];
     const int tok0 = qt * p.Tq;
     const int ntok = min(p.Tq, sq - tok0);
     if (ntok <= 0) {
         if (threadIdx.x == 0) p.ucnt[tile] = 0;
         return;
     }
-    (void)k0;
     int nblk = (sk + p.bs - 1) / p.bs;
     if (sq > p.max_sq || nblk > p.nblk_max) {  // lengths beyond the caller's max_seqlen bounds
         if (threadIdx.x == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_SEQLEN);
         nblk = min(nblk, p.nblk_max);
     }
-    const int words = (nblk + 31) / 32;
+    const int words = (p.nblk_max + 31) / 32;
     uint32_t *bm = prep_smem;
-    int *lists = reinterpret_cast<int *>(prep_smem + words);  // [topk][kPrepThreads]
+    int *raw = reinterpret_cast<int *>(prep_smem + words);  // [Tq][topk] selections as given
+    int *lists = raw + p.Tq * p.topk;                         // [topk][kPrepThreads] canonical
     for (int w = threadIdx.x; w < words; w += kPrepThreads) bm[w] = 0;
+    const int64_t row0 = ((int64_t)(q0 + tok0) * p.Hkv + hk) * p.topk;
+    const int64_t tok_stride = (int64_t)p.Hkv * p.topk;
+    for (int e = threadIdx.x; e < ntok * p.topk; e += kPrepThreads) {
+        const int tt = e / p.topk;
+        raw[e] = p.sel[row0 + tt * tok_stride + (e - tt * p.topk)];
+    }
     __syncthreads();
 
     const int tt = threadIdx.x;
+    int n = 0;
     if (tt < ntok) {
         const int i = tok0 + tt;  // local query index
-        const int64_t t = (int64_t)q0 + i;
         const int delta = sk - sq;
         int lo = 0, hi = sk - 1;
         if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
         if (p.causal) hi = min(hi, i + delta);
         if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
-        const int32_t *row = p.sel + (t * p.Hkv + hk) * p.topk;
-        int n = 0;
         bool bad = false;
         for (int e = 0; e < p.topk; ++e) {
-            const int s = row[e];
+            const int s = raw[tt * p.topk + e];
             if (s == -1) continue;
             if (s < 0 || s >= nblk) {
                 bad = true;
@@ -127,18 +151,145 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
             lists[pos * kPrepThreads + tt] = s;
             ++n;
         }
-        int32_t *dst = p.sel_c + (t * p.Hkv + hk) * p.topk;
-        for (int e = 0; e < p.topk; ++e) {
-            const int s = e < n ? lists[e * kPrepThreads + tt] : -1;
-            dst[e] = s;
-            if (e < n) atomicOr(&bm[s >> 5], 1u << (s & 31));
-        }
+        const int64_t t = (int64_t)q0 + i;
         p.cnt[t * p.Hkv + hk] = n;
         if (bad && p.status) atomicOr(p.status, SFA_DEV_BAD_INDEX);
     }
+    // Union bitmap: lanes that hold the same block set its bit once.
+    {
+        const int maxn = __reduce_max_sync(0xffffffffu, n);
+        const int lane = threadIdx.x & 31;
+        for (int e = 0; e < maxn; ++e) {
+            const int s = e < n ? lists[e * kPrepThreads + tt] : -1;
+            const unsigned m = __match_any_sync(0xffffffffu, s);
+            if (s >= 0 && lane == __ffs(m) - 1) atomicOr(&bm[s >> 5], 1u << (s & 31));
+        }
+    }
+    __syncthreads();  // every thread is done reading raw
+    if (tt < ntok)
+        for (int e = 0; e < p.topk; ++e) raw[tt * p.topk + e] = e < n ? lists[e * kPrepThreads + tt] : -1;
     __syncthreads();
-    const int total = compact_bitmap<kPrepThreads>(bm, words, p.uni + (int64_t)tile * p.umax, scan_scratch);
+    for (int e = threadIdx.x; e < ntok * p.topk; e += kPrepThreads) {
+        const int t2 = e / p.topk;
+        p.sel_c[row0 + t2 * tok_stride + (e - t2 * p.topk)] = raw[e];
+    }
+    const int total = compact_bitmap<kPrepThreads>(bm, (nblk + 31) / 32, p.uni + (int64_t)tile * p.umax,
+                                                   scan_scratch);
     if (threadIdx.x == 0) p.ucnt[tile] = total;
+}
+
+constexpr int kInvThreads = 256;
+
+// Exclusive scan of v[0..n) in place (all threads); returns the total.
+__device__ int block_scan_array(int *v, int n, int *scratch)
+{
+    const int per = (n + kInvThreads - 1) / kInvThreads;
+    const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
+    int c = 0;
+    for (int i = i0; i < i1; ++i) c += v[i];
+    int pos;
+    const int total = block_exclusive_scan<kInvThreads>(c, scratch, pos);
+    for (int i = i0; i < i1; ++i) {
+        const int x = v[i];
+        v[i] = pos;
+        pos += x;
+    }
+    __syncthreads();
+    return total;
+}
+
+// Block-major schedule, one CTA per (window, sequence, kv head) group.  Decides whether the
+// window is better served by the query-major kernel (the union of its tiles' blocks is at most
+// 10 times the selected work) or block-major; for a block-major window it marks the window's
+// tiles as taken (ucnt = -1), lists for every selected block the window's (token, slot) pairs that selected it, and cuts each
+// list into items of at most Tq tokens.
+__global__ void __launch_bounds__(kInvThreads) fwd_invert_kernel(FwdInvertParams p, int nblk_max)
+{
+    extern __shared__ int inv_smem[];
+    __shared__ int scan_scratch[32];
+    __shared__ long long red_useful, red_union;
+    __shared__ int bases[2];
+    const int g = blockIdx.x;
+    const int hk = g % p.Hkv;
+    const int b = (g / p.Hkv) % p.batch;
+    const int w = g / (p.Hkv * p.batch);
+    const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+    const int t0 = w * p.W;
+    if (t0 >= sq) return;
+    const int nt = min(p.W, sq - t0);
+    if (threadIdx.x == 0) {
+        red_useful = 0;
+        red_union = 0;
+    }
+    __syncthreads();
+    long long useful = 0, uwork = 0;
+    for (int tt = threadIdx.x; tt < nt; tt += kInvThreads) useful += p.cnt[(int64_t)(q0 + t0 + tt) * p.Hkv + hk];
+    const int qt0 = t0 / p.Tq, qt1 = (t0 + nt - 1) / p.Tq;
+    auto tile_of = [&](int qt) { return ((p.nqt - 1 - qt) * p.batch + b) * p.Hkv + hk; };
+    for (int qt = qt0 + threadIdx.x; qt <= qt1; qt += kInvThreads)
+        uwork += (long long)max(p.ucnt[tile_of(qt)], 0) * min(p.Tq, sq - qt * p.Tq);
+    atomicAdd(reinterpret_cast<unsigned long long *>(&red_useful), (unsigned long long)useful);
+    atomicAdd(reinterpret_cast<unsigned long long *>(&red_union), (unsigned long long)uwork);
+    __syncthreads();
+    // A block-major item moves several times the memory of a query-major tile per selected
+    // row-block (its bf16 partial is written and read back, its Q rows gathered), so it pays only
+    // when the union wastes much more: the switch point is a union of 10x the selected work.
+    if (red_union <= 10 * red_useful) return;  // the query-major kernel keeps this window
+
+    // The window's tiles are taken; the query-major kernel only writes their rows that keep no key.
+    for (int qt = qt0 + threadIdx.x; qt <= qt1; qt += kInvThreads) p.ucnt[tile_of(qt)] = -1;
+
+    int *count = inv_smem;
+    int *cursor = count + nblk_max;
+    int *ioff = cursor + nblk_max;
+    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) count[s] = cursor[s] = 0;
+    __syncthreads();
+    // Histogram of selected blocks over the window's tokens.
+    for (int tb = 0; tb < nt; tb += kInvThreads) {
+        const int tt = tb + threadIdx.x;
+        const int64_t t = (int64_t)q0 + t0 + tt;
+        const int n = tt < nt ? p.cnt[t * p.Hkv + hk] : 0;
+        const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
+        const int maxn = __reduce_max_sync(0xffffffffu, n);
+        for (int e = 0; e < maxn; ++e) warp_aggregated_add(count, e < n ? row[e] : -1);
+    }
+    __syncthreads();
+    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) ioff[s] = (count[s] + p.Tq - 1) / p.Tq;
+    __syncthreads();
+    const int nitems = block_scan_array(ioff, nblk_max, scan_scratch);   // ioff = first item of block s
+    // count -> exclusive offsets of each block's pair list (count itself is rebuilt from cursor)
+    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) cursor[s] = count[s];
+    __syncthreads();
+    const int npairs = block_scan_array(count, nblk_max, scan_scratch);  // count = first pair of s
+    if (threadIdx.x == 0) {
+        bases[0] = atomicAdd(&p.ctrl->pair_total, npairs);
+        bases[1] = atomicAdd(&p.ctrl->item_total, nitems);
+    }
+    __syncthreads();
+    const int pair_base = bases[0], item_base = bases[1];
+    // Items: {b*Hkv + hk, block, first pair, tokens}.
+    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) {
+        const int c = cursor[s];
+        for (int i = 0; i * p.Tq < c; ++i)
+            p.items[item_base + ioff[s] + i] =
+                make_int4(b * p.Hkv + hk, s, pair_base + count[s] + i * p.Tq, min(p.Tq, c - i * p.Tq));
+    }
+    __syncthreads();
+    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) cursor[s] = 0;
+    __syncthreads();
+    // Scatter (token, slot) pairs into their blocks' lists.
+    for (int tb = 0; tb < nt; tb += kInvThreads) {
+        const int tt = tb + threadIdx.x;
+        const int64_t t = (int64_t)q0 + t0 + tt;
+        const int n = tt < nt ? p.cnt[t * p.Hkv + hk] : 0;
+        const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
+        const int maxn = __reduce_max_sync(0xffffffffu, n);
+        for (int e = 0; e < maxn; ++e) {
+            const int s = e < n ? row[e] : -1;
+            const int pos = warp_aggregated_add(cursor, s);
+            if (s >= 0) p.pairs[pair_base + count[s] + pos] = (int)(t << 7) | e;
+        }
+    }
 }
 
 constexpr int kDecPrepThreads = 512;
@@ -184,7 +335,7 @@ __global__ void __launch_bounds__(kDecPrepThreads) decode_prep_kernel(DecPrepPar
 cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream_t st)
 {
     const size_t words = (size_t)(g.nblk_max + 31) / 32;
-    const size_t smem = words * 4 + (size_t)g.topk * kPrepThreads * 4;
+    const size_t smem = words * 4 + (size_t)g.Tq * g.topk * 4 + (size_t)g.topk * kPrepThreads * 4;
     static int configured_bytes = 0;
     if ((int)smem > 48 * 1024 && (int)smem > configured_bytes) {
         cudaError_t e = cudaFuncSetAttribute(fwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -192,6 +343,20 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
         configured_bytes = (int)smem;
     }
     fwd_prep_kernel<<<g.tiles, kPrepThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_invert(const FwdGeom &g, const FwdInvertParams &p, cudaStream_t st)
+{
+    const size_t smem = (size_t)g.nblk_max * 3 * 4;
+    static int configured_bytes = 0;
+    if ((int)smem > 48 * 1024 && (int)smem > configured_bytes) {
+        cudaError_t e =
+            cudaFuncSetAttribute(fwd_invert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        configured_bytes = (int)smem;
+    }
+    fwd_invert_kernel<<<g.groups, kInvThreads, smem, st>>>(p, g.nblk_max);
     return cudaGetLastError();
 }
 
