@@ -206,7 +206,7 @@ int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
 const char *sfa_status_string(int status);
 
 /* Number of kernel launches the last successful call on this host thread made (prefill: 2,
- * or 5 when the call can use the block-major schedule; decode: 3; a stage: its own count). */
+ * or 6 when the call can use the block-major schedule; decode: 3; a stage: its own count). */
 int sfa_last_launch_count(void);
 
 #ifdef __cplusplus

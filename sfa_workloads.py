@@ -29,12 +29,15 @@ INVALID = -1
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round float32 to bfloat16 (round to nearest, ties to even); return uint16 bits."""
+    """Round finite float32 values to bfloat16 (round to nearest, ties to even); return uint16
+    bits.  For finite inputs u + 0x7FFF + lsb stays below 2^32, so uint32 arithmetic is exact."""
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    r = ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)
-    return r
+    u = x.view(np.uint32).copy()
+    lsb = (u >> 16) & np.uint32(1)
+    u += np.uint32(0x7FFF)
+    u += lsb
+    u >>= np.uint32(16)
+    return u.astype(np.uint16)
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -77,13 +77,22 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     g.off_union = off;
     off = align_up(off + (size_t)g.tiles * g.umax * 4);
     if (g.inv) {
-        const size_t pairs = (size_t)total_q * Hkv * topk;
+        const size_t gb = (size_t)g.groups * g.nblk_max;
+        g.cap_items = ((int64_t)total_q * Hkv * topk + g.Tq - 1) / g.Tq + (int64_t)gb;
+        g.off_zero = off;  // ctrl, group statistics, block histograms and cursors: cleared per call
         g.off_ctrl = off;
         off = align_up(off + sizeof(InvCtrl));
-        g.off_pairs = off;
-        off = align_up(off + pairs * 4);
+        g.off_gstat = off;
+        off = align_up(off + (size_t)g.groups * sizeof(GroupStat));
+        g.off_gcount = off;
+        off = align_up(off + gb * 4);
+        g.off_gcursor = off;
+        off = align_up(off + gb * 4);
+        g.zero_bytes = off - g.off_zero;
+        g.off_gfirst = off;
+        off = align_up(off + gb * 4);
         g.off_items = off;
-        off = align_up(off + pairs * 16);
+        off = align_up(off + (size_t)g.cap_items * sizeof(InvItem));
         g.off_pml = off;
         off = align_up(off + (size_t)total_q * Hq * topk * 8);
         g.off_po = off;
@@ -149,11 +158,11 @@ int check_window(int causal, int wl, int wr)
     return SFA_OK;
 }
 
-int fwd_invert_impl(const FwdGeom &g, const int32_t *cu_q, void *ws, cudaStream_t st);
-
 int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, const int32_t *sel, int causal, int wl,
                   int wr, void *ws, int32_t *status, cudaStream_t st)
 {
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    if (g.inv && cudaMemsetAsync(w + g.off_zero, 0, g.zero_bytes, st) != cudaSuccess) return SFA_ERR_CUDA;
     FwdPrepParams p{};
     p.cu_q = cu_q;
     p.cu_k = cu_k ? cu_k : cu_q;
@@ -170,43 +179,48 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     p.umax = g.umax;
     p.max_sq = g.max_sq;
     p.nblk_max = g.nblk_max;
-    uint8_t *w = static_cast<uint8_t *>(ws);
     p.sel_c = reinterpret_cast<int32_t *>(w + g.off_sel_c);
     p.cnt = reinterpret_cast<int32_t *>(w + g.off_cnt);
     p.ucnt = reinterpret_cast<int32_t *>(w + g.off_ucnt);
     p.uni = reinterpret_cast<int32_t *>(w + g.off_union);
-    p.ctrl = g.inv ? reinterpret_cast<InvCtrl *>(w + g.off_ctrl) : nullptr;
+    p.W = g.W;
+    p.gstat = g.inv ? reinterpret_cast<GroupStat *>(w + g.off_gstat) : nullptr;
+    p.gcount = g.inv ? reinterpret_cast<int32_t *>(w + g.off_gcount) : nullptr;
     p.status = status;
     if (launch_fwd_prep(g, p, st) != cudaSuccess) return SFA_ERR_CUDA;
-    return fwd_invert_impl(g, cu_q, ws, st);
-}
-
-// Second prep kernel: choose query-major or block-major per window and build the block-major
-// items.
-int fwd_invert_impl(const FwdGeom &g, const int32_t *cu_q, void *ws, cudaStream_t st)
-{
     if (!g.inv) return SFA_OK;
-    uint8_t *w = static_cast<uint8_t *>(ws);
-    FwdInvertParams p{};
-    p.cu_q = cu_q;
-    p.cnt = reinterpret_cast<const int32_t *>(w + g.off_cnt);
-    p.sel_c = reinterpret_cast<const int32_t *>(w + g.off_sel_c);
-    p.ucnt = reinterpret_cast<int32_t *>(w + g.off_ucnt);
-    p.batch = g.batch;
-    p.Hq = g.Hq;
-    p.Hkv = g.Hkv;
-    p.G = g.G;
-    p.Tq = g.Tq;
-    p.nqt = g.nqt;
-    p.topk = g.topk;
-    p.W = g.W;
-    p.nwin = g.nwin;
-    p.total_q = g.total_q;
-    p.D = g.d;
-    p.pairs = reinterpret_cast<int32_t *>(w + g.off_pairs);
-    p.items = reinterpret_cast<int4 *>(w + g.off_items);
-    p.ctrl = reinterpret_cast<InvCtrl *>(w + g.off_ctrl);
-    return launch_fwd_invert(g, p, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+    // Which windows go block-major, and their items.
+    FwdPlanParams pl{};
+    pl.ucnt = p.ucnt;
+    pl.gstat = p.gstat;
+    pl.gcount = p.gcount;
+    pl.gfirst = reinterpret_cast<int32_t *>(w + g.off_gfirst);
+    pl.batch = g.batch;
+    pl.Hkv = g.Hkv;
+    pl.Tq = g.Tq;
+    pl.nqt = g.nqt;
+    pl.W = g.W;
+    pl.nblk_max = g.nblk_max;
+    pl.cu_q = cu_q;
+    pl.items = reinterpret_cast<InvItem *>(w + g.off_items);
+    pl.ctrl = reinterpret_cast<InvCtrl *>(w + g.off_ctrl);
+    if (launch_fwd_plan(g, pl, st) != cudaSuccess) return SFA_ERR_CUDA;
+    FwdScatterParams sc{};
+    sc.cu_q = cu_q;
+    sc.sel_c = p.sel_c;
+    sc.cnt = p.cnt;
+    sc.ucnt = p.ucnt;
+    sc.gfirst = pl.gfirst;
+    sc.gcursor = reinterpret_cast<int32_t *>(w + g.off_gcursor);
+    sc.batch = g.batch;
+    sc.Hkv = g.Hkv;
+    sc.topk = g.topk;
+    sc.Tq = g.Tq;
+    sc.nqt = g.nqt;
+    sc.W = g.W;
+    sc.nblk_max = g.nblk_max;
+    sc.items = pl.items;
+    return launch_fwd_scatter(g, sc, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
 }
 
 int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *v, const int32_t *cu_q,
@@ -246,8 +260,7 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     if (launch_fwd_attend(g, p, tq, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
     uint8_t *wm = static_cast<uint8_t *>(ws);
-    p.pairs = reinterpret_cast<const int32_t *>(wm + g.off_pairs);
-    p.items = reinterpret_cast<const int4 *>(wm + g.off_items);
+    p.items = reinterpret_cast<const InvItem *>(wm + g.off_items);
     p.ctrl = reinterpret_cast<InvCtrl *>(wm + g.off_ctrl);
     p.po = reinterpret_cast<__nv_bfloat16 *>(wm + g.off_po);
     p.pml = reinterpret_cast<float2 *>(wm + g.off_pml);
@@ -425,7 +438,7 @@ int sfa_fwd_prep(const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int b
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
     rc = fwd_prep_impl(g, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
                        status_dev, stream);
-    if (rc == SFA_OK) g_last_launches = 1 + g.inv;
+    if (rc == SFA_OK) g_last_launches = 1 + 2 * g.inv;
     return rc;
 }
 
@@ -477,7 +490,7 @@ int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqle
     if (rc != SFA_OK) return rc;
     rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right, scale,
                          workspace, status_dev, out, lse, stream);
-    if (rc == SFA_OK) g_last_launches = 2 + 3 * g.inv;
+    if (rc == SFA_OK) g_last_launches = 2 + 4 * g.inv;
     return rc;
 }
 

@@ -127,6 +127,17 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint64_t *ba
         : "memory");
 }
 
+// Contiguous global -> shared copy through the TMA engine (16-byte aligned addresses, size a
+// multiple of 16), completing `bytes` on the mbarrier.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Four rows (any row coordinates) of a 2-D tensor map whose box is {64 elements, 1 row}: the
 // rows land one after another (4 x 128 bytes) at dst, with the map's swizzle applied.
 __device__ __forceinline__ void tma_gather4(const CUtensorMap *map, uint64_t *bar, void *dst, int c0, int r0, int r1,

@@ -25,34 +25,33 @@ namespace {
 
 constexpr int kInvThreadsAttn = 320;  // warp 0 producer, warp 1 MMA, warps 2-5 and 6-9: two softmax groups
 constexpr float kLn2i = 0.6931471805599453f;
+constexpr int kItemSlots = 8;   // item j lives in slot j % 8; softmax group j % 2 handles it
+constexpr int kFetchAhead = 4;  // item records are fetched this many items ahead
+constexpr int kLoadStages = 3;  // Q and K/V buffers: item j uses buffer j % 3
 
 template <int D, int BS>
 struct InvCfg {
     static constexpr int kQBytes = 128 * D * 2;
     static constexpr int kKVBytes = BS * D * 2;
-    static constexpr int kOffQ = 0;                        // Q[2]
-    static constexpr int kOffK = 2 * kQBytes;              // K[2]
-    static constexpr int kOffV = kOffK + 2 * kKVBytes;     // V[2]
-    static constexpr int kOffMeta = kOffV + 2 * kKVBytes;
+    static constexpr int kOffQ = 0;                                // Q[kLoadStages]
+    static constexpr int kOffK = kLoadStages * kQBytes;            // K[kLoadStages]
+    static constexpr int kOffV = kOffK + kLoadStages * kKVBytes;   // V[kLoadStages]
+    static constexpr int kOffMeta = kOffV + kLoadStages * kKVBytes;
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
     static constexpr int kTmemCols = 512;  // S/P of group w at w*BS, O of group w at 128 + w*D
 };
 
-struct ItemSlot {
-    int4 rec;  // {b*Hkv + hk, block, first pair, tokens}; tokens < 0 ends the work
-    int tok[128];
-};
 
 struct InvMeta {
-    uint64_t item_full[2], item_free[2];
-    uint64_t q_full[2], q_empty[2];
-    uint64_t kv_full[2], kv_empty[2];
+    uint64_t item_full[kItemSlots], item_free[kItemSlots];
+    uint64_t q_full[kLoadStages], q_empty[kLoadStages];
+    uint64_t kv_full[kLoadStages], kv_empty[kLoadStages];
     uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
-    ItemSlot slot[2];
+    InvItem slot[kItemSlots];
 };
 
 template <int D, int BS>
@@ -67,13 +66,17 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kItemSlots; ++s) {
             mbar_init(&meta->item_full[s], 1);
             mbar_init(&meta->item_free[s], 128);
+        }
+        for (int s = 0; s < kLoadStages; ++s) {
             mbar_init(&meta->q_full[s], 1);
             mbar_init(&meta->q_empty[s], 1);
             mbar_init(&meta->kv_full[s], 1);
             mbar_init(&meta->kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&meta->s_full[s], 1);
             mbar_init(&meta->p_full[s], 128);
             mbar_init(&meta->pv_done[s], 1);
@@ -98,62 +101,44 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- producer (all 32 lanes)
+        // Item j of this CTA is item blockIdx.x + j * gridDim.x.  Its record and token list are
+        // one 528-byte bulk copy into slot j % 8, issued four items ahead; past the last item the
+        // slot gets an end marker instead.
+        const int total = *reinterpret_cast<volatile int *>(&p.ctrl->item_total);
+        auto fetch = [&](int j) {  // lane 0 only
+            const int sl = j % kItemSlots;
+            const long long idx = (long long)blockIdx.x + (long long)j * gridDim.x;
+            if (idx < total) {
+                mbar_arrive_expect_tx(&meta->item_full[sl], (uint32_t)sizeof(InvItem));
+                bulk_load(&meta->slot[sl], &p.items[idx], (uint32_t)sizeof(InvItem), &meta->item_full[sl]);
+            } else {
+                meta->slot[sl].rec = make_int4(0, 0, 0, -1);
+                mbar_arrive(&meta->item_full[sl]);
+            }
+        };
         if (lane == 0) {
             tma_prefetch_desc(&tmq);
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
+            for (int f = 0; f < kFetchAhead; ++f) fetch(f);
         }
-        const int total = *reinterpret_cast<volatile int *>(&p.ctrl->item_total);
-        const int4 kEnd = make_int4(0, 0, 0, -1);
-        // Item j of this CTA is item blockIdx.x + j * gridDim.x; the next one's record and
-        // token list are fetched one item ahead.
-        int4 rec_next = (int)blockIdx.x < total ? __ldcg(&p.items[blockIdx.x]) : kEnd;
-        int tok_next[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = lane + 32 * u;
-            tok_next[u] = e < rec_next.w ? __ldcg(&p.pairs[rec_next.z + e]) : 0;
-        }
-        int issued[2] = {0, 0};
+        int issued[kLoadStages] = {};
         bool ok = true;
         for (int j = 0; ok; ++j) {
-            const int sl = j & 1;
-            const uint32_t ph = ((j >> 1) - 1) & 1;  // phase of this slot's previous use
-            const int4 rec = rec_next;
-            int tok[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) tok[u] = tok_next[u];
-            const long long nidx = (long long)blockIdx.x + (long long)(j + 1) * gridDim.x;
-            rec_next = nidx < total ? __ldcg(&p.items[nidx]) : kEnd;
-            if (j >= 2) ok = warp_all_ok(mbar_wait(&meta->item_free[sl], ph, abort_flag, p.status));
+            const int sl = j % kLoadStages;                  // K/V and Q buffers
+            const int it = j % kItemSlots;                   // item slot
+            const uint32_t ph = ((j / kLoadStages) - 1) & 1; // previous use of this K/V or Q buffer
+            ok = warp_all_ok(mbar_wait(&meta->item_full[it], (j / kItemSlots) & 1, abort_flag, p.status));
             if (!ok) break;
-            ItemSlot *slot = &meta->slot[sl];
-            if (rec.w < 0) {
-                // End of work: both slots get an end marker, so both softmax groups stop.
-                if (lane == 0) {
-                    slot->rec = kEnd;
-                    mbar_arrive(&meta->item_full[sl]);
-                }
-                const int j2 = j + 1, sl2 = j2 & 1;
-                if (j2 >= 2) ok = warp_all_ok(mbar_wait(&meta->item_free[sl2], ((j2 >> 1) - 1) & 1, abort_flag, p.status));
-                if (ok && lane == 0) {
-                    meta->slot[sl2].rec = kEnd;
-                    mbar_arrive(&meta->item_full[sl2]);
-                }
-                break;
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                if (lane + 32 * u < rec.w) slot->tok[lane + 32 * u] = tok[u];
-            if (lane == 0) slot->rec = rec;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&meta->item_full[sl]);
+            const InvItem *item = &meta->slot[it];
+            const int4 rec = item->rec;
+            if (rec.w < 0) break;  // item j+1 is past the end too, so both groups get a marker
             const int hk = rec.x % p.Hkv, b = rec.x / p.Hkv;
             // K/V block
-            if (j >= 2) ok = warp_all_ok(mbar_wait(&meta->kv_empty[sl], ph, abort_flag, p.status));
+            if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->kv_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
             if (lane == 0) {
-                const int row = p.cu_k[b] + rec.y * BS;
+                const int row = __ldg(&p.cu_k[b]) + rec.y * BS;
                 mbar_arrive_expect_tx(&meta->kv_full[sl], 2u * (uint32_t)C::kKVBytes);
                 for (int c = 0; c < D / 64; ++c) {
                     tma_load_3d(&tmk, &meta->kv_full[sl], sK + sl * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
@@ -163,7 +148,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             }
             // Q rows of the item's tokens, four rows per TMA gather into the swizzled K-major tile
             // (row r = token * G + head; a last partial group repeats its last row).
-            if (j >= 2) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
+            if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
             {
                 const int rows = rec.w * p.G;
@@ -177,72 +162,93 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                     for (int u = 0; u < 4; ++u) {
                         const int rr = min(4 * g4 + u, rows - 1);
                         const int tk = rr / p.G, gg = rr - tk * p.G;
-                        grow[u] = (slot->tok[tk] >> 7) * p.Hq + hk * p.G + gg;
+                        grow[u] = (item->tok[tk] >> 7) * p.Hq + hk * p.G + gg;
                     }
                     tma_gather4(&tmq, &meta->q_full[sl], sQ + sl * C::kQBytes + c * (128 * 128) + g4 * 512, c * 64,
                                 grow[0], grow[1], grow[2], grow[3]);
                 }
             }
-            // The next item's token list (its record was requested above).
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = lane + 32 * u;
-                tok_next[u] = e < rec_next.w ? __ldcg(&p.pairs[rec_next.z + e]) : 0;
-            }
+            // Item j+4 goes into the slot item j-4 used, once its softmax group is done with it.
+            if (j + kFetchAhead >= kItemSlots)
+                ok = warp_all_ok(mbar_wait(&meta->item_free[(j + kFetchAhead) % kItemSlots],
+                                           ((j + kFetchAhead - kItemSlots) / kItemSlots) & 1, abort_flag, p.status));
+            if (!ok) break;
+            if (lane == 0) fetch(j + kFetchAhead);
+            __syncwarp();
         }
         if (*abort_flag && lane == 0) {
-            for (int sl = 0; sl < 2; ++sl)
+            for (int sl = 0; sl < kLoadStages; ++sl)
                 if (issued[sl] > 0) mbar_drain(&meta->kv_full[sl], (issued[sl] - 1) & 1);
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
+        // Issues S_ns = Q K^T and PV_np = P V in whatever order their inputs become ready, so an
+        // item's PV never waits for the next item's loads.  Order constraints: PV_j after S_j;
+        // S_j after PV_{j-2} (its TMEM score buffer holds P_{j-2} until that MMA has read it;
+        // tcgen05 MMAs of one thread run in issue order).
         if (lane == 0) {
             const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            bool ok = true;
-            auto issue_pv = [&](int i) -> bool {
-                const int w = i & 1;
-                if (!mbar_wait(&meta->p_full[w], (i >> 1) & 1, abort_flag, p.status)) return false;
-                if (i >= 2 && !mbar_wait(&meta->o_free[w], ((i >> 1) - 1) & 1, abort_flag, p.status)) return false;
-                tc_fence_after();
-                const uint32_t tO = tmem + 128 + w * D;
+            int ns = 0, np = 0;
+            bool end_seen = false, ok = true;
+            uint64_t idle_since = global_timer_ns();
+            while (ok) {
+                bool progressed = false;
+                if (!end_seen && ns <= np + 1) {
+                    const int it = ns % kItemSlots, sl = ns % kLoadStages, sb = ns & 1;
+                    const uint32_t ph = (ns / kLoadStages) & 1;
+                    if (mbar_try_wait(smem_u32(&meta->item_full[it]), (ns / kItemSlots) & 1)) {
+                        if (meta->slot[it].rec.w < 0) {
+                            end_seen = true;
+                            progressed = true;
+                        } else if (mbar_try_wait(smem_u32(&meta->q_full[sl]), ph) &&
+                                   mbar_try_wait(smem_u32(&meta->kv_full[sl]), ph)) {
+                            tc_fence_after();
+                            const uint32_t tS = tmem + sb * BS;
 #pragma unroll
-                for (int ks = 0; ks < BS / 16; ++ks) {
-                    const uint32_t a = tmem + w * BS + ks * 8;
-                    const uint64_t bd = sdesc_sw128(sVa + w * C::kKVBytes + ks * 16 * 128, BS * 128, 1024);
-                    umma_bf16_tmem_a(tO, a, bd, C::kIdescPV, ks > 0 ? 1u : 0u);
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint64_t a = sdesc_sw128(
+                                    sQa + sl * C::kQBytes + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
+                                const uint64_t bd = sdesc_sw128(
+                                    sKa + sl * C::kKVBytes + (ks >> 2) * (BS * 128) + (ks & 3) * 32, 16, 1024);
+                                umma_bf16(tS, a, bd, C::kIdescS, ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&meta->s_full[sb]);
+                            umma_commit(&meta->q_empty[sl]);
+                            ++ns;
+                            progressed = true;
+                        }
+                    }
                 }
-                umma_commit(&meta->pv_done[w]);
-                umma_commit(&meta->kv_empty[w]);
-                return true;
-            };
-            int j = 0;
-            for (;; ++j) {
-                const int sl = j & 1;
-                const uint32_t ph = (j >> 1) & 1;
-                ok = mbar_wait(&meta->item_full[sl], ph, abort_flag, p.status);
-                if (!ok) break;
-                if (meta->slot[sl].rec.w < 0) break;
-                ok = mbar_wait(&meta->q_full[sl], ph, abort_flag, p.status) &&
-                     mbar_wait(&meta->kv_full[sl], ph, abort_flag, p.status);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t tS = tmem + sl * BS;
+                if (np < ns) {
+                    const int w = np & 1;
+                    if (mbar_try_wait(smem_u32(&meta->p_full[w]), (np >> 1) & 1) &&
+                        (np < 2 || mbar_try_wait(smem_u32(&meta->o_free[w]), ((np >> 1) - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t tO = tmem + 128 + w * D;
+                        const int vs = np % kLoadStages;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t a =
-                        sdesc_sw128(sQa + sl * C::kQBytes + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd =
-                        sdesc_sw128(sKa + sl * C::kKVBytes + (ks >> 2) * (BS * 128) + (ks & 3) * 32, 16, 1024);
-                    umma_bf16(tS, a, bd, C::kIdescS, ks > 0 ? 1u : 0u);
+                        for (int ks = 0; ks < BS / 16; ++ks) {
+                            const uint32_t a = tmem + w * BS + ks * 8;
+                            const uint64_t bd = sdesc_sw128(sVa + vs * C::kKVBytes + ks * 16 * 128, BS * 128, 1024);
+                            umma_bf16_tmem_a(tO, a, bd, C::kIdescPV, ks > 0 ? 1u : 0u);
+                        }
+                        umma_commit(&meta->pv_done[w]);
+                        umma_commit(&meta->kv_empty[vs]);
+                        ++np;
+                        progressed = true;
+                    }
                 }
-                umma_commit(&meta->s_full[sl]);
-                umma_commit(&meta->q_empty[sl]);
-                if (j >= 1) {
-                    ok = issue_pv(j - 1);
-                    if (!ok) break;
+                if (end_seen && np == ns) break;
+                if (progressed) {
+                    idle_since = global_timer_ns();
+                } else if (*abort_flag) {
+                    ok = false;
+                } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
+                    *abort_flag = 1;
+                    if (p.status) atomicOr(p.status, SFA_DEV_TIMEOUT);
+                    ok = false;
                 }
             }
-            if (ok && j >= 1) ok = issue_pv(j - 1);
             if (!ok) {
                 umma_commit(&meta->drain);
                 mbar_drain(&meta->drain, 0);
@@ -259,19 +265,20 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
         bool ok = true;
         for (int j = grp; ok; j += 2) {
             const uint32_t ph = (j >> 1) & 1;
-            ok = warp_all_ok(mbar_wait(&meta->item_full[grp], ph, abort_flag, p.status));
+            const int it = j % kItemSlots;
+            ok = warp_all_ok(mbar_wait(&meta->item_full[it], (j / kItemSlots) & 1, abort_flag, p.status));
             if (!ok) break;
-            const int4 rec = meta->slot[grp].rec;
+            const int4 rec = meta->slot[it].rec;
             if (rec.w < 0) break;
             const int hk = rec.x % p.Hkv, b = rec.x / p.Hkv, s = rec.y, n = rec.w;
-            const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
-            const int sk = p.cu_k[b + 1] - p.cu_k[b];
+            const int q0 = __ldg(&p.cu_q[b]), sq = __ldg(&p.cu_q[b + 1]) - q0;
+            const int sk = __ldg(&p.cu_k[b + 1]) - __ldg(&p.cu_k[b]);
             const int tok = r / p.G, gg = r - tok * p.G;
             const bool valid = tok < n;
             int64_t t = 0;
             int kslot = 0, lo = 0, hi = -1;
             if (valid) {
-                const int e = meta->slot[grp].tok[tok];
+                const int e = meta->slot[it].tok[tok];
                 t = e >> 7;
                 kslot = e & 127;
                 const int i = (int)(t - q0), delta = sk - sq;
@@ -352,7 +359,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             mbar_arrive(&meta->o_free[grp]);
             if (valid) p.pml[pslot] = make_float2(m, l);
 
-            mbar_arrive(&meta->item_free[grp]);
+            mbar_arrive(&meta->item_free[it]);
         }
     }
 

@@ -26,34 +26,57 @@ struct FwdGeom {
     // group the prep lists, per selected block, the window's tokens that selected it, and cuts
     // those lists into items of at most Tq tokens.
     int inv, W, nwin, groups;
+    int64_t cap_items;
     size_t off_sel_c, off_cnt, off_ucnt, off_union;
-    size_t off_ctrl, off_pairs, off_items, off_pml, off_po;
+    size_t off_zero, zero_bytes;  // the part of the workspace cleared before every prep
+    size_t off_ctrl, off_gstat, off_gcount, off_gcursor, off_gfirst, off_items, off_pml, off_po;
     size_t bytes;
 };
 
-// Control words of the block-major schedule, reset by the prep kernel of every call.
+// Control words of the block-major schedule (cleared before every prep).
 struct InvCtrl {
-    int item_total;    // items written by the invert kernel
-    int pair_total;    // (token, slot) entries written by the invert kernel
-    int work_counter;  // next item the attention kernel hands out
-    int pad;
+    int item_total;  // items planned so far
+    int pad[3];
+};
+
+// Per (window, sequence, kv head) group: selected row-blocks and union tile row-blocks.
+struct GroupStat {
+    unsigned long long useful, uni;
+};
+
+// One block-major item as stored in the workspace and copied whole into shared memory.
+struct InvItem {
+    int4 rec;      // {b * Hkv + hk, block, 0, tokens}; tokens < 0 marks the end of the work
+    int tok[128];  // (token << 7) | position of the block in the token's canonical list
 };
 
 struct FwdPrepParams {
     const int32_t *cu_q, *cu_k, *sel;
     int batch, Hkv, topk, bs, causal, wl, wr, Tq, nqt, umax, max_sq, nblk_max;
     int32_t *sel_c, *cnt, *ucnt, *uni;
-    InvCtrl *ctrl;     // nullptr when the block-major schedule is off
+    // block-major statistics (nullptr when the schedule is off)
+    int W;
+    GroupStat *gstat;
+    int32_t *gcount;
     int32_t *status;
 };
 
-struct FwdInvertParams {
-    const int32_t *cu_q, *cnt, *sel_c;
+struct FwdPlanParams {
     int32_t *ucnt;
-    int batch, Hq, Hkv, G, Tq, nqt, topk, W, nwin, total_q, D;
-    int32_t *pairs;   // (token << 7 | slot) per (token, selected block), grouped by block
-    int4 *items;      // {b * Hkv + hk, block, first pair, tokens}
+    const GroupStat *gstat;
+    const int32_t *gcount;
+    int32_t *gfirst;
+    int batch, Hkv, Tq, nqt, W, nblk_max;
+    const int32_t *cu_q;
+    InvItem *items;
     InvCtrl *ctrl;
+};
+
+struct FwdScatterParams {
+    const int32_t *cu_q, *sel_c, *cnt, *ucnt, *gfirst;
+    int32_t *gcursor;
+    int batch, Hkv, topk, Tq, nqt, W, nblk_max;
+    InvItem *items;
 };
 
 struct FwdAttendParams {
@@ -66,8 +89,7 @@ struct FwdAttendParams {
     float *lse;
     int32_t *status;
     // block-major schedule
-    const int32_t *pairs;
-    const int4 *items;
+    const InvItem *items;
     InvCtrl *ctrl;
     __nv_bfloat16 *po;  // partial outputs, (total_q, Hq, topk, d) bf16, normalised
     float2 *pml;        // partial (max, sum) in the base-2 scaled domain, (total_q, Hq, topk)
@@ -109,7 +131,8 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
 cudaError_t launch_fwd_attend(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
                               const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 size_t fwd_attend_smem_bytes(const FwdGeom &g);
-cudaError_t launch_fwd_invert(const FwdGeom &g, const FwdInvertParams &p, cudaStream_t st);
+cudaError_t launch_fwd_plan(const FwdGeom &g, const FwdPlanParams &p, cudaStream_t st);
+cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cudaStream_t st);
 cudaError_t launch_fwd_attend_inv(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
                                   const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 cudaError_t launch_fwd_merge(const FwdGeom &g, const FwdAttendParams &p, cudaStream_t st);

@@ -87,11 +87,6 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
 {
     extern __shared__ uint32_t prep_smem[];
     __shared__ int scan_scratch[32];
-    if (blockIdx.x == 0 && threadIdx.x == 0 && p.ctrl) {
-        p.ctrl->item_total = 0;
-        p.ctrl->pair_total = 0;
-        p.ctrl->work_counter = 0;
-    }
     const int tile = blockIdx.x;
     const int hk = tile % p.Hkv;
     const int rest = tile / p.Hkv;
@@ -155,14 +150,24 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
         p.cnt[t * p.Hkv + hk] = n;
         if (bad && p.status) atomicOr(p.status, SFA_DEV_BAD_INDEX);
     }
-    // Union bitmap: lanes that hold the same block set its bit once.
+    // Union bitmap: lanes that hold the same block set its bit once.  With the block-major
+    // schedule on, also count each block's selecting tokens for the window's group.
+    const int grp = p.gstat ? ((tok0 / p.W) * p.batch + b) * p.Hkv + hk : 0;
     {
         const int maxn = __reduce_max_sync(0xffffffffu, n);
         const int lane = threadIdx.x & 31;
+        int32_t *gc = p.gstat ? p.gcount + (int64_t)grp * p.nblk_max : nullptr;
         for (int e = 0; e < maxn; ++e) {
             const int s = e < n ? lists[e * kPrepThreads + tt] : -1;
             const unsigned m = __match_any_sync(0xffffffffu, s);
-            if (s >= 0 && lane == __ffs(m) - 1) atomicOr(&bm[s >> 5], 1u << (s & 31));
+            if (s >= 0 && lane == __ffs(m) - 1) {
+                atomicOr(&bm[s >> 5], 1u << (s & 31));
+                if (gc) atomicAdd(&gc[s], __popc(m));
+            }
+        }
+        if (p.gstat) {
+            const int wsum = __reduce_add_sync(0xffffffffu, n);
+            if (lane == 0 && wsum) atomicAdd(&p.gstat[grp].useful, (unsigned long long)wsum);
         }
     }
     __syncthreads();  // every thread is done reading raw
@@ -175,7 +180,10 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
     }
     const int total = compact_bitmap<kPrepThreads>(bm, (nblk + 31) / 32, p.uni + (int64_t)tile * p.umax,
                                                    scan_scratch);
-    if (threadIdx.x == 0) p.ucnt[tile] = total;
+    if (threadIdx.x == 0) {
+        p.ucnt[tile] = total;
+        if (p.gstat) atomicAdd(&p.gstat[grp].uni, (unsigned long long)total * ntok);
+    }
 }
 
 constexpr int kInvThreads = 256;
@@ -198,97 +206,76 @@ __device__ int block_scan_array(int *v, int n, int *scratch)
     return total;
 }
 
-// Block-major schedule, one CTA per (window, sequence, kv head) group.  Decides whether the
-// window is better served by the query-major kernel (the union of its tiles' blocks is at most
-// 10 times the selected work) or block-major; for a block-major window it marks the window's
-// tiles as taken (ucnt = -1), lists for every selected block the window's (token, slot) pairs that selected it, and cuts each
-// list into items of at most Tq tokens.
-__global__ void __launch_bounds__(kInvThreads) fwd_invert_kernel(FwdInvertParams p, int nblk_max)
+// Block-major plan, one CTA per (window, sequence, kv head) group.  The window stays with the
+// query-major kernel unless the union of its query tiles' blocks is over 10x its selected
+// blocks (a block-major item moves several times the memory of a query-major tile per selected
+// row-block: its bf16 partial is written and read back and its Q rows are gathered).  For a
+// block-major window: mark its tiles (ucnt = -1), cut each selected block's token list into
+// items of at most Tq tokens, reserve them, and write their records (tokens come from the
+// scatter kernel).
+__global__ void __launch_bounds__(kInvThreads) fwd_plan_kernel(FwdPlanParams p)
 {
-    extern __shared__ int inv_smem[];
+    extern __shared__ int plan_smem[];
     __shared__ int scan_scratch[32];
-    __shared__ long long red_useful, red_union;
-    __shared__ int bases[2];
+    __shared__ int item_base;
     const int g = blockIdx.x;
     const int hk = g % p.Hkv;
     const int b = (g / p.Hkv) % p.batch;
     const int w = g / (p.Hkv * p.batch);
-    const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+    const int sq = p.cu_q[b + 1] - p.cu_q[b];
     const int t0 = w * p.W;
     if (t0 >= sq) return;
+    const GroupStat st = p.gstat[g];
+    if (st.uni <= 10ull * st.useful) return;  // the query-major kernel keeps this window
     const int nt = min(p.W, sq - t0);
-    if (threadIdx.x == 0) {
-        red_useful = 0;
-        red_union = 0;
-    }
-    __syncthreads();
-    long long useful = 0, uwork = 0;
-    for (int tt = threadIdx.x; tt < nt; tt += kInvThreads) useful += p.cnt[(int64_t)(q0 + t0 + tt) * p.Hkv + hk];
     const int qt0 = t0 / p.Tq, qt1 = (t0 + nt - 1) / p.Tq;
-    auto tile_of = [&](int qt) { return ((p.nqt - 1 - qt) * p.batch + b) * p.Hkv + hk; };
     for (int qt = qt0 + threadIdx.x; qt <= qt1; qt += kInvThreads)
-        uwork += (long long)max(p.ucnt[tile_of(qt)], 0) * min(p.Tq, sq - qt * p.Tq);
-    atomicAdd(reinterpret_cast<unsigned long long *>(&red_useful), (unsigned long long)useful);
-    atomicAdd(reinterpret_cast<unsigned long long *>(&red_union), (unsigned long long)uwork);
-    __syncthreads();
-    // A block-major item moves several times the memory of a query-major tile per selected
-    // row-block (its bf16 partial is written and read back, its Q rows gathered), so it pays only
-    // when the union wastes much more: the switch point is a union of 10x the selected work.
-    if (red_union <= 10 * red_useful) return;  // the query-major kernel keeps this window
+        p.ucnt[((p.nqt - 1 - qt) * p.batch + b) * p.Hkv + hk] = -1;
 
-    // The window's tiles are taken; the query-major kernel only writes their rows that keep no key.
-    for (int qt = qt0 + threadIdx.x; qt <= qt1; qt += kInvThreads) p.ucnt[tile_of(qt)] = -1;
-
-    int *count = inv_smem;
-    int *cursor = count + nblk_max;
-    int *ioff = cursor + nblk_max;
-    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) count[s] = cursor[s] = 0;
+    const int32_t *count = p.gcount + (int64_t)g * p.nblk_max;
+    int *first = plan_smem;  // first item of each block, local to the group
+    for (int s = threadIdx.x; s < p.nblk_max; s += kInvThreads) first[s] = (count[s] + p.Tq - 1) / p.Tq;
     __syncthreads();
-    // Histogram of selected blocks over the window's tokens.
-    for (int tb = 0; tb < nt; tb += kInvThreads) {
-        const int tt = tb + threadIdx.x;
-        const int64_t t = (int64_t)q0 + t0 + tt;
-        const int n = tt < nt ? p.cnt[t * p.Hkv + hk] : 0;
-        const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
-        const int maxn = __reduce_max_sync(0xffffffffu, n);
-        for (int e = 0; e < maxn; ++e) warp_aggregated_add(count, e < n ? row[e] : -1);
-    }
+    const int nitems = block_scan_array(first, p.nblk_max, scan_scratch);
+    if (threadIdx.x == 0) item_base = atomicAdd(&p.ctrl->item_total, nitems);
     __syncthreads();
-    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) ioff[s] = (count[s] + p.Tq - 1) / p.Tq;
-    __syncthreads();
-    const int nitems = block_scan_array(ioff, nblk_max, scan_scratch);   // ioff = first item of block s
-    // count -> exclusive offsets of each block's pair list (count itself is rebuilt from cursor)
-    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) cursor[s] = count[s];
-    __syncthreads();
-    const int npairs = block_scan_array(count, nblk_max, scan_scratch);  // count = first pair of s
-    if (threadIdx.x == 0) {
-        bases[0] = atomicAdd(&p.ctrl->pair_total, npairs);
-        bases[1] = atomicAdd(&p.ctrl->item_total, nitems);
-    }
-    __syncthreads();
-    const int pair_base = bases[0], item_base = bases[1];
-    // Items: {b*Hkv + hk, block, first pair, tokens}.
-    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) {
-        const int c = cursor[s];
+    int32_t *gfirst = p.gfirst + (int64_t)g * p.nblk_max;
+    for (int s = threadIdx.x; s < p.nblk_max; s += kInvThreads) {
+        const int c = count[s];
+        const int i0 = item_base + first[s];
+        gfirst[s] = i0;
         for (int i = 0; i * p.Tq < c; ++i)
-            p.items[item_base + ioff[s] + i] =
-                make_int4(b * p.Hkv + hk, s, pair_base + count[s] + i * p.Tq, min(p.Tq, c - i * p.Tq));
+            p.items[i0 + i].rec = make_int4(b * p.Hkv + hk, s, 0, min(p.Tq, c - i * p.Tq));
     }
-    __syncthreads();
-    for (int s = threadIdx.x; s < nblk_max; s += kInvThreads) cursor[s] = 0;
-    __syncthreads();
-    // Scatter (token, slot) pairs into their blocks' lists.
-    for (int tb = 0; tb < nt; tb += kInvThreads) {
-        const int tt = tb + threadIdx.x;
-        const int64_t t = (int64_t)q0 + t0 + tt;
-        const int n = tt < nt ? p.cnt[t * p.Hkv + hk] : 0;
-        const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
-        const int maxn = __reduce_max_sync(0xffffffffu, n);
-        for (int e = 0; e < maxn; ++e) {
-            const int s = e < n ? row[e] : -1;
-            const int pos = warp_aggregated_add(cursor, s);
-            if (s >= 0) p.pairs[pair_base + count[s] + pos] = (int)(t << 7) | e;
-        }
+}
+
+// Block-major token lists, one CTA per query tile of a block-major window: every (token, block)
+// of the tile's canonical selections takes the next position in its block's list, which names
+// the item (position / Tq) and the slot in it.
+__global__ void __launch_bounds__(kPrepThreads) fwd_scatter_kernel(FwdScatterParams p)
+{
+    const int tile = blockIdx.x;
+    if (p.ucnt[tile] != -1) return;
+    const int hk = tile % p.Hkv;
+    const int rest = tile / p.Hkv;
+    const int b = rest % p.batch;
+    const int qt = p.nqt - 1 - rest / p.batch;
+    const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+    const int tok0 = qt * p.Tq;
+    const int ntok = min(p.Tq, sq - tok0);
+    const int grp = ((tok0 / p.W) * p.batch + b) * p.Hkv + hk;
+    int32_t *cursor = p.gcursor + (int64_t)grp * p.nblk_max;
+    const int32_t *first = p.gfirst + (int64_t)grp * p.nblk_max;
+    const int tt = threadIdx.x;
+    const int64_t t = (int64_t)q0 + tok0 + tt;
+    const int n = tt < ntok ? p.cnt[t * p.Hkv + hk] : 0;
+    const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
+    const int maxn = __reduce_max_sync(0xffffffffu, n);
+    for (int e = 0; e < maxn; ++e) {
+        const int s = e < n ? row[e] : -1;
+        // cursor is global here; warp_aggregated_add works on any address space
+        const int pos = warp_aggregated_add(cursor, s);
+        if (s >= 0) p.items[first[s] + pos / p.Tq].tok[pos % p.Tq] = (int)(t << 7) | e;
     }
 }
 
@@ -346,17 +333,16 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
     return cudaGetLastError();
 }
 
-cudaError_t launch_fwd_invert(const FwdGeom &g, const FwdInvertParams &p, cudaStream_t st)
+cudaError_t launch_fwd_plan(const FwdGeom &g, const FwdPlanParams &p, cudaStream_t st)
 {
-    const size_t smem = (size_t)g.nblk_max * 3 * 4;
-    static int configured_bytes = 0;
-    if ((int)smem > 48 * 1024 && (int)smem > configured_bytes) {
-        cudaError_t e =
-            cudaFuncSetAttribute(fwd_invert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured_bytes = (int)smem;
-    }
-    fwd_invert_kernel<<<g.groups, kInvThreads, smem, st>>>(p, g.nblk_max);
+    const size_t smem = (size_t)g.nblk_max * 4;
+    fwd_plan_kernel<<<g.groups, kInvThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cudaStream_t st)
+{
+    fwd_scatter_kernel<<<g.tiles, kPrepThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -199,12 +199,12 @@ def test_empty_batch_and_explicit_scale(sfa, oracle_lib):
 
 
 def test_launch_count_and_stages(sfa, oracle_lib):
-    """sfa_fwd = prep (1 kernel, or 2 with the block-major schedule) + attend (1 kernel, or 3:
+    """sfa_fwd = prep (1 kernel, or 3 with the block-major schedule) + attend (1 kernel, or 3:
     query-major, block-major, merge); the split-stage calls give the same result."""
     c = W.small_config(2)
     d = upload_prefill(c)
     out, lse = run_fwd(sfa, c, d=d)
-    assert sfa.last_launch_count() in (2, 5)
+    assert sfa.last_launch_count() in (2, 6)
     ws, _, _ = sfa.fwd_prep(d["cu_q"], d["sel"], Hq=c.Hq, d=c.d, block_size=c.bs, cu_seqlens_k=d["cu_k"],
                             max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk)
     o2, l2 = sfa.fwd_attend(d["q"], d["k"], d["v"], d["cu_q"], ws, topk=c.topk, block_size=c.bs,
@@ -212,16 +212,40 @@ def test_launch_count_and_stages(sfa, oracle_lib):
     assert torch.equal(out, o2) and torch.equal(lse, l2)
 
 
-@pytest.mark.parametrize("Hq,Hkv,d,bs,topk", [(16, 4, 128, 64, 6), (4, 4, 128, 64, 5), (8, 2, 64, 32, 7),
-                                              (6, 2, 128, 32, 6), (32, 2, 64, 64, 4)])
-def test_block_major_windows(sfa, oracle_lib, Hq, Hkv, d, bs, topk):
-    """Long sequences with a small random top-k: the union of a query tile's blocks is several
-    times the selected work, so the windows go to the block-major kernel (items of one block and
-    the tokens that selected it, bf16 partials, merge by the last writer).  Every element
-    against the oracle, ragged lengths included."""
-    lens = [3000, 2500, 70]
+def _block_major_windows(c, oracle_lib):
+    """How many (window, sequence, kv head) groups the prep will send to the block-major kernel:
+    the union of a window's query-tile block sets exceeds 10x the window's selected blocks."""
+    sel_c, cnt, _ = oracle_lib.fwd_index(c)
+    G = c.Hq // c.Hkv
+    Tq = 128 // G
+    W = Tq * 64
+    n = 0
+    for b in range(c.batch):
+        q0, sq = c.cu_q[b], c.cu_q[b + 1] - c.cu_q[b]
+        for hk in range(c.Hkv):
+            for w0 in range(0, sq, W):
+                useful = int(cnt[q0 + w0:q0 + min(sq, w0 + W), hk].sum())
+                union = 0
+                for t0 in range(w0, min(sq, w0 + W), Tq):
+                    t1 = min(sq, t0 + Tq)
+                    blocks = set(sel_c[q0 + t0:q0 + t1, hk].ravel().tolist()) - {-1}
+                    union += len(blocks) * (t1 - t0)
+                n += union > 10 * useful
+    return n
+
+
+@pytest.mark.parametrize("Hq,Hkv,d,bs,topk,lens", [(16, 4, 128, 64, 6, [12000, 300]),
+                                                   (2, 2, 64, 32, 6, [9000, 77]),
+                                                   (8, 2, 128, 32, 8, [8000]),
+                                                   (6, 2, 64, 64, 5, [10000, 1000])])
+def test_block_major_windows(sfa, oracle_lib, Hq, Hkv, d, bs, topk, lens):
+    """Long sequences with a small random top-k: late windows' query tiles select unions of
+    blocks over 10x their selected work, so those windows go to the block-major kernel (items of
+    one block and the tokens that selected it, bf16 partials, merge kernel) while early windows
+    stay query-major.  Every element against the oracle, ragged lengths included."""
     c = W.make_nsa_prefill(Hq + 7 * d + bs + topk, lens, Hq, Hkv, d, bs, topk, 1, 2)
+    assert _block_major_windows(c, oracle_lib) > 0
     _full_parity(sfa, oracle_lib, c)
     out, lse = run_fwd(sfa, c)
-    out2, lse2 = run_fwd(sfa, c)  # repeated call: same workspace state machine, same bits
+    out2, lse2 = run_fwd(sfa, c)  # a repeated call on fresh buffers gives the same bits
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
