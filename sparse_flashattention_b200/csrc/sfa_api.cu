@@ -76,6 +76,8 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     off = align_up(off + (size_t)g.tiles * 4);
     g.off_union = off;
     off = align_up(off + (size_t)g.tiles * g.umax * 4);
+    g.off_tilectr = off;
+    off = align_up(off + 4);
     if (g.inv) {
         const size_t gb = (size_t)g.groups * g.nblk_max;
         g.cap_items = ((int64_t)total_q * Hkv * topk + g.Tq - 1) / g.Tq + (int64_t)gb;
@@ -257,6 +259,9 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     p.out = static_cast<__nv_bfloat16 *>(out);
     p.lse = lse;
     p.status = status;
+    p.tiles = g.tiles;
+    p.tile_counter = reinterpret_cast<int32_t *>(const_cast<uint8_t *>(w) + g.off_tilectr);
+    if (cudaMemsetAsync(p.tile_counter, 0, 4, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (launch_fwd_attend(g, p, tq, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
     uint8_t *wm = static_cast<uint8_t *>(ws);

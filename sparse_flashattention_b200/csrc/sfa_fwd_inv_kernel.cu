@@ -293,37 +293,25 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             tc_fence_after();
             float x[BS];
             {
-                uint32_t raw[32];
+                uint32_t raw[BS];
+                tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(raw));
+                if constexpr (BS == 64) tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+                tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < BS / 32; ++c) {
-                    tmem_ld32(tS + c * 32, raw);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[e]);
-                }
+                for (int e = 0; e < BS; ++e) x[e] = __uint_as_float(raw[e]);
             }
             const int kb = s * BS;
-            if (!(valid && kb >= lo && kb + BS - 1 <= hi)) {
+            if (valid && !(kb >= lo && kb + BS - 1 <= hi)) {  // the block straddles the row's edge
 #pragma unroll
                 for (int c = 0; c < BS; ++c) {
                     const int key = kb + c;
-                    x[c] = (valid && key >= lo && key <= hi) ? x[c] : -INFINITY;
+                    x[c] = (key >= lo && key <= hi) ? x[c] : -INFINITY;
                 }
             }
-            float mx = x[0];
-#pragma unroll
-            for (int c = 1; c < BS; ++c) mx = fmaxf(mx, x[c]);
-            const float m = mx * p.scale_log2;
+            const float m = valid ? row_max3<BS>(x) * p.scale_log2 : -INFINITY;
             const float m_use = m == -INFINITY ? 0.f : m;
-            float l = 0.f;
             uint32_t packed[BS / 2];
-#pragma unroll
-            for (int c = 0; c < BS; c += 2) {
-                const float p0 = ex2(fmaf(x[c], p.scale_log2, -m_use));
-                const float p1 = ex2(fmaf(x[c + 1], p.scale_log2, -m_use));
-                l += p0 + p1;
-                packed[c / 2] = pack_bf16x2(p0, p1);
-            }
+            const float l = scores_to_p<BS>(x, valid ? p.scale_log2 : 0.f, valid ? -m_use : -INFINITY, packed);
             if constexpr (BS == 64) {
                 tmem_st32(tS, packed);
             } else {

@@ -61,8 +61,7 @@ struct Meta {
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
-    int ntok;
-    int nU;
+    int tile;  // the tile this CTA works on, broadcast by thread 0
 };
 
 __device__ __forceinline__ int warp_all(bool v)
@@ -70,6 +69,9 @@ __device__ __forceinline__ int warp_all(bool v)
     return __all_sync(0xffffffffu, v);
 }
 
+// Persistent CTAs (two per SM) take query tiles from a counter in the workspace, heaviest
+// tiles first.  Barrier phases run on a per-CTA count of processed blocks (jg), so the
+// pipeline state carries over from tile to tile; TMEM is allocated once.
 template <int D, int BS>
 __global__ void __launch_bounds__(kThreads, 2)
     fwd_attend_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
@@ -82,33 +84,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     int *s_union = reinterpret_cast<int *>(smem + C::kOffMeta + sizeof(Meta));
     int *s_lists = s_union + p.umax;             // [Tq][topk]
     int *s_cnt = s_lists + p.Tq * p.topk;        // [Tq]
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tile = blockIdx.x;
-    const int hk = tile % p.Hkv;
-    const int rest = tile / p.Hkv;
-    const int b = rest % p.batch;
-    const int qt = p.nqt - 1 - rest / p.batch;
-    const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
-    const int k0 = p.cu_k[b], sk = p.cu_k[b + 1] - k0;
-    const int tok0 = qt * p.Tq;
-    const int ntok = min(p.Tq, sq - tok0);
-    if (ntok <= 0) return;  // tile beyond this sequence's end (uniform for the CTA)
-    const int nU = p.ucnt[tile];
-    if (nU < 0) {
-        // The block-major kernel computes this tile's rows; only rows that keep no key at all
-        // (no partial will ever arrive for them) are written here: output 0, lse -inf.
-        for (int e = threadIdx.x; e < ntok * p.G; e += kThreads) {
-            const int tt = e / p.G, gg = e - tt * p.G;
-            const int64_t t = (int64_t)q0 + tok0 + tt;
-            if (p.cnt[t * p.Hkv + hk] != 0) continue;
-            const int h = hk * p.G + gg;
-            uint4 *dst = reinterpret_cast<uint4 *>(p.out + (t * p.Hq + h) * D);
-            for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-            p.lse[(int64_t)h * p.total_q + t] = -INFINITY;
-        }
-        return;
-    }
 
     if (threadIdx.x == 0) {
         mbar_init(&meta->q_full, 1);
@@ -129,240 +105,298 @@ __global__ void __launch_bounds__(kThreads, 2)
         tmem_alloc(&meta->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
-    // Tile metadata into shared memory: the union of blocks, and each token's sorted list.
-    {
-        const int *gu = p.uni + (int64_t)tile * p.umax;
-        for (int j = threadIdx.x; j < nU; j += kThreads) s_union[j] = gu[j];
-        for (int e = threadIdx.x; e < ntok * p.topk; e += kThreads) {
-            const int tt = e / p.topk, slot = e % p.topk;
-            s_lists[e] = p.sel_c[((int64_t)(q0 + tok0 + tt) * p.Hkv + hk) * p.topk + slot];
-        }
-        for (int tt = threadIdx.x; tt < ntok; tt += kThreads) s_cnt[tt] = p.cnt[(int64_t)(q0 + tok0 + tt) * p.Hkv + hk];
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = meta->tmem_base;
     volatile int *abort_flag = &meta->abort_flag;
-
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+    }
 
-    if (warp == 0) {
-        // ------------------------------------------------------------------ producer
-        if (lane == 0 && nU > 0) {
-            tma_prefetch_desc(&tmq);
-            tma_prefetch_desc(&tmk);
-            tma_prefetch_desc(&tmv);
-            const uint32_t qbytes = (uint32_t)(D / 64) * 64u * (uint32_t)(p.G * p.Tq) * 2u;
-            mbar_arrive_expect_tx(&meta->q_full, qbytes);
-            for (int c = 0; c < D / 64; ++c)
-                tma_load_3d(&tmq, &meta->q_full, sQ + c * (128 * 128), c * 64, hk * p.G, q0 + tok0);
-            int issued[kStages] = {};
-            bool ok = true;
-            for (int j = 0; j < nU && ok; ++j) {
-                const int st = j % kStages;
-                if (j >= kStages) ok = mbar_wait(&meta->kv_empty[st], ((j / kStages) - 1) & 1, abort_flag, p.status);
-                if (!ok) break;
-                const int row = k0 + s_union[j] * BS;
-                mbar_arrive_expect_tx(&meta->kv_full[st], 2u * (uint32_t)C::kKVBytes);
-                for (int c = 0; c < D / 64; ++c) {
-                    tma_load_3d(&tmk, &meta->kv_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
-                    tma_load_3d(&tmv, &meta->kv_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
-                }
-                issued[st]++;
-            }
-            if (*abort_flag) {  // wind down: let every copy this thread started land
-                mbar_drain(&meta->q_full, 0);
-                for (int st = 0; st < kStages; ++st)
-                    if (issued[st] > 0) mbar_drain(&meta->kv_full[st], (issued[st] - 1) & 1);
+    int jbase = 0;  // blocks this CTA processed in earlier tiles
+    int titer = 0;  // tiles this CTA computed (phase of q_full)
+    int last_jg[kStages];
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) last_jg[s] = -1;
+
+    while (true) {
+        if (threadIdx.x == 0) meta->tile = atomicAdd(p.tile_counter, 1);
+        __syncthreads();
+        const int tile = meta->tile;
+        if (tile >= p.tiles || *abort_flag) break;
+        const int hk = tile % p.Hkv;
+        const int rest = tile / p.Hkv;
+        const int b = rest % p.batch;
+        const int qt = p.nqt - 1 - rest / p.batch;
+        const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+        const int k0 = p.cu_k[b], sk = p.cu_k[b + 1] - k0;
+        const int tok0 = qt * p.Tq;
+        const int ntok = min(p.Tq, sq - tok0);
+        const int nU = ntok > 0 ? p.ucnt[tile] : 0;
+        if (ntok > 0 && nU < 0) {
+            // The block-major kernel computes this tile's rows; only rows that keep no key at all
+            // (no partial will ever arrive for them) are written here: output 0, lse -inf.
+            for (int e = threadIdx.x; e < ntok * p.G; e += kThreads) {
+                const int tt = e / p.G, gg = e - tt * p.G;
+                const int64_t t = (int64_t)q0 + tok0 + tt;
+                if (p.cnt[t * p.Hkv + hk] != 0) continue;
+                const int h = hk * p.G + gg;
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (t * p.Hq + h) * D);
+                for (int c = 0; c < D / 8; ++c) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+                p.lse[(int64_t)h * p.total_q + t] = -INFINITY;
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
-        if (lane == 0 && nU > 0) {
-            const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-            const uint32_t tO = tmem + 2 * BS;
-            bool ok = mbar_wait(&meta->q_full, 0, abort_flag, p.status);
-            auto issue_pv = [&](int i) -> bool {
-                if (!mbar_wait(&meta->p_full[i & 1], (i >> 1) & 1, abort_flag, p.status)) return false;
-                tc_fence_after();
-                const int st = i % kStages;
-#pragma unroll
-                for (int ks = 0; ks < BS / 16; ++ks) {
-                    // P_i (bf16) sits in the first BS/2 columns of score buffer i&1: 8 columns per K=16.
-                    const uint32_t a = tmem + (i & 1) * BS + ks * 8;
-                    const uint64_t bd = sdesc_sw128(sVa + st * C::kKVBytes + ks * 16 * 128, BS * 128, 1024);
-                    umma_bf16_tmem_a(tO, a, bd, C::kIdescPV, (i > 0 || ks > 0) ? 1u : 0u);
-                }
-                umma_commit(&meta->pv_done[i & 1]);
-                umma_commit(&meta->kv_empty[st]);
-                return true;
-            };
-            for (int j = 0; j < nU && ok; ++j) {
-                const int st = j % kStages;
-                // Score buffer j&1 is free again: PV_{j-2}, which read P_{j-2} from it, was issued
-                // before this MMA (after softmax j-2 finished), and tcgen05 MMAs of one thread run in
-                // issue order.
-                ok = mbar_wait(&meta->kv_full[st], (j / kStages) & 1, abort_flag, p.status);
-                if (!ok) break;
-                tc_fence_after();
-                const uint32_t tS = tmem + (j & 1) * BS;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const uint64_t a = sdesc_sw128(sQa + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd =
-                        sdesc_sw128(sKa + st * C::kKVBytes + (ks >> 2) * (BS * 128) + (ks & 3) * 32, 16, 1024);
-                    umma_bf16(tS, a, bd, C::kIdescS, ks > 0 ? 1u : 0u);
-                }
-                umma_commit(&meta->s_full[j & 1]);
-                if (j >= 1) ok = issue_pv(j - 1);
+        if (ntok > 0 && nU >= 0) {
+            // Tile metadata into shared memory: the union of blocks, and each token's sorted list.
+            const int *gu = p.uni + (int64_t)tile * p.umax;
+            for (int j = threadIdx.x; j < nU; j += kThreads) s_union[j] = gu[j];
+            for (int e = threadIdx.x; e < ntok * p.topk; e += kThreads) {
+                const int tt = e / p.topk, slot = e - tt * p.topk;
+                s_lists[e] = p.sel_c[((int64_t)(q0 + tok0 + tt) * p.Hkv + hk) * p.topk + slot];
             }
-            if (ok) ok = issue_pv(nU - 1);
-            if (!ok) {  // wind down: wait for the MMAs already issued
-                umma_commit(&meta->drain);
-                mbar_drain(&meta->drain, 0);
-            }
-        }
-    } else {
-        // ------------------------------------------------------------------ softmax + epilogue
-        const int quad = warp & 3;  // TMEM lane quadrant this warp may access
-        const int r = quad * 32 + lane;
-        const int tok = r / p.G, g = r % p.G;
-        const bool row_valid = (tok < ntok);  // r < Tq*G is implied by tok < ntok <= Tq
-        const int i = tok0 + tok;
-        const int delta = sk - sq;
-        int lo = 0, hi = sk - 1;
-        if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
-        if (p.causal) hi = min(hi, i + delta);
-        if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
-        const int *mylist = s_lists + (row_valid ? tok : 0) * p.topk;
-        const int mycnt = row_valid ? s_cnt[tok] : 0;
-        int ptr = 0;
-        float m_run = -INFINITY;  // running max of s*scale*log2e
-        float l_run = 0.f;
-        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        const uint32_t tO = lane_base + 2 * BS;
-        bool ok = true;
+            for (int tt = threadIdx.x; tt < ntok; tt += kThreads)
+                s_cnt[tt] = p.cnt[(int64_t)(q0 + tok0 + tt) * p.Hkv + hk];
+            __syncthreads();
 
-        for (int j = 0; j < nU; ++j) {
-            const int s = s_union[j];
-            const bool selected = ptr < mycnt && mylist[ptr] == s;
-            if (selected) ++ptr;
-            ok = warp_all(mbar_wait(&meta->s_full[j & 1], (j >> 1) & 1, abort_flag, p.status));
-            if (!ok) break;
-            tc_fence_after();
-            float x[BS];
-            {
-                uint32_t raw[32];
-#pragma unroll
-                for (int c = 0; c < BS / 32; ++c) {
-                    tmem_ld32(lane_base + (j & 1) * BS + c * 32, raw);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(raw[e]);
+            if (warp == 0) {
+                // -------------------------------------------------------------- producer
+                if (lane == 0 && nU > 0) {
+                    const uint32_t qbytes = (uint32_t)(D / 64) * 64u * (uint32_t)(p.G * p.Tq) * 2u;
+                    mbar_arrive_expect_tx(&meta->q_full, qbytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(&tmq, &meta->q_full, sQ + c * (128 * 128), c * 64, hk * p.G, q0 + tok0);
+                    for (int j = 0; j < nU; ++j) {
+                        const int jg = jbase + j, st = jg % kStages;
+                        if (jg >= kStages &&
+                            !mbar_wait(&meta->kv_empty[st], ((jg / kStages) - 1) & 1, abort_flag, p.status))
+                            break;
+                        const int row = k0 + s_union[j] * BS;
+                        mbar_arrive_expect_tx(&meta->kv_full[st], 2u * (uint32_t)C::kKVBytes);
+                        for (int c = 0; c < D / 64; ++c) {
+                            tma_load_3d(&tmk, &meta->kv_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64,
+                                        hk, row);
+                            tma_load_3d(&tmv, &meta->kv_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64,
+                                        hk, row);
+                        }
+                        last_jg[st] = jg;
+                    }
                 }
-            }
+            } else if (warp == 1) {
+                // -------------------------------------------------------------- MMA issuer
+                // Issues S_j = Q K_j^T and PV_j = P_j V_j in whatever order their inputs become
+                // ready, so PV_j never waits for block j+1's loads.  Order constraints: PV_j after
+                // S_j; S_j after PV_{j-2} (its TMEM score buffer holds P_{j-2} until that MMA has
+                // read it; tcgen05 MMAs of one thread run in issue order).
+                if (lane == 0 && nU > 0) {
+                    const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+                    const uint32_t tO = tmem + 2 * BS;
+                    bool ok = mbar_wait(&meta->q_full, titer & 1, abort_flag, p.status);
+                    int ns = 0, np = 0;
+                    uint64_t idle_since = global_timer_ns();
+                    while (ok && np < nU) {
+                        bool progressed = false;
+                        if (ns < nU && ns <= np + 1) {
+                            const int jg = jbase + ns, st = jg % kStages;
+                            if (mbar_try_wait(smem_u32(&meta->kv_full[st]), (jg / kStages) & 1)) {
+                                tc_fence_after();
+                                const uint32_t tS = tmem + (jg & 1) * BS;
+#pragma unroll
+                                for (int ks = 0; ks < D / 16; ++ks) {
+                                    const uint64_t a =
+                                        sdesc_sw128(sQa + (ks >> 2) * (128 * 128) + (ks & 3) * 32, 16, 1024);
+                                    const uint64_t bd = sdesc_sw128(
+                                        sKa + st * C::kKVBytes + (ks >> 2) * (BS * 128) + (ks & 3) * 32, 16, 1024);
+                                    umma_bf16(tS, a, bd, C::kIdescS, ks > 0 ? 1u : 0u);
+                                }
+                                umma_commit(&meta->s_full[jg & 1]);
+                                ++ns;
+                                progressed = true;
+                            }
+                        }
+                        if (np < ns) {
+                            const int ig = jbase + np, st = ig % kStages;
+                            if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1)) {
+                                tc_fence_after();
+#pragma unroll
+                                for (int ks = 0; ks < BS / 16; ++ks) {
+                                    // P (bf16) sits in the first BS/2 columns of its score buffer.
+                                    const uint32_t a = tmem + (ig & 1) * BS + ks * 8;
+                                    const uint64_t bd =
+                                        sdesc_sw128(sVa + st * C::kKVBytes + ks * 16 * 128, BS * 128, 1024);
+                                    umma_bf16_tmem_a(tO, a, bd, C::kIdescPV, (np > 0 || ks > 0) ? 1u : 0u);
+                                }
+                                umma_commit(&meta->pv_done[ig & 1]);
+                                umma_commit(&meta->kv_empty[st]);
+                                ++np;
+                                progressed = true;
+                            }
+                        }
+                        if (progressed) {
+                            idle_since = global_timer_ns();
+                        } else if (*abort_flag) {
+                            ok = false;
+                        } else if (global_timer_ns() - idle_since > kWaitLimitNs) {
+                            *abort_flag = 1;
+                            if (p.status) atomicOr(p.status, SFA_DEV_TIMEOUT);
+                            ok = false;
+                        }
+                    }
+                    if (!ok) {  // wind down: wait for the MMAs already issued
+                        umma_commit(&meta->drain);
+                        mbar_drain(&meta->drain, 0);
+                    }
+                }
+            } else {
+                // -------------------------------------------------------------- softmax + epilogue
+                const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+                const int r = quad * 32 + lane;
+                const int tok = r / p.G, g = r % p.G;
+                const bool row_valid = (tok < ntok);  // r < Tq*G is implied by tok < ntok <= Tq
+                const int i = tok0 + tok;
+                const int delta = sk - sq;
+                int lo = 0, hi = sk - 1;
+                if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
+                if (p.causal) hi = min(hi, i + delta);
+                if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
+                const int *mylist = s_lists + (row_valid ? tok : 0) * p.topk;
+                const int mycnt = row_valid ? s_cnt[tok] : 0;
+                int ptr = 0;
+                float m_run = -INFINITY;  // running max of s*scale*log2e
+                float l_run = 0.f;
+                const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+                const uint32_t tO = lane_base + 2 * BS;
+                bool ok = true;
 
-            const int kb = s * BS;
-            const bool full = selected && kb >= lo && kb + BS - 1 <= hi;
-            if (!full) {
-#pragma unroll
-                for (int c = 0; c < BS; ++c) {
-                    const int key = kb + c;
-                    const bool keep = selected && key >= lo && key <= hi;
-                    x[c] = keep ? x[c] : -INFINITY;
-                }
-            }
-            float mx = x[0];
-#pragma unroll
-            for (int c = 1; c < BS; ++c) mx = fmaxf(mx, x[c]);
-            const float m_new = mx * p.scale_log2;
-            const bool need = m_new > m_run + kRescaleLog2;
-            if (__any_sync(0xffffffffu, need)) {
-                float factor = 1.f;
-                if (need) {
-                    factor = ex2(m_run - m_new);
-                    m_run = m_new;
-                    l_run *= factor;
-                }
-                if (j > 0) {
-                    ok = warp_all(mbar_wait(&meta->pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.status));
+                for (int j = 0; j < nU; ++j) {
+                    const int jg = jbase + j;
+                    const int s = s_union[j];
+                    const bool selected = ptr < mycnt && mylist[ptr] == s;
+                    if (selected) ++ptr;
+                    ok = warp_all(mbar_wait(&meta->s_full[jg & 1], (jg >> 1) & 1, abort_flag, p.status));
                     if (!ok) break;
                     tc_fence_after();
+                    float x[BS];
+                    {
+                        uint32_t raw[BS];
+                        tmem_ld32(lane_base + (jg & 1) * BS, *reinterpret_cast<uint32_t(*)[32]>(raw));
+                        if constexpr (BS == 64)
+                            tmem_ld32(lane_base + (jg & 1) * BS + 32, *reinterpret_cast<uint32_t(*)[32]>(raw + 32));
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < BS; ++e) x[e] = __uint_as_float(raw[e]);
+                    }
+                    // Rows that did not select this block contribute nothing (handled arithmetically
+                    // below); selected rows are masked element by element only where the block
+                    // straddles their causal / window edge.
+                    const int kb = s * BS;
+                    if (selected && !(kb >= lo && kb + BS - 1 <= hi)) {
+#pragma unroll
+                        for (int c = 0; c < BS; ++c) {
+                            const int key = kb + c;
+                            x[c] = (key >= lo && key <= hi) ? x[c] : -INFINITY;
+                        }
+                    }
+                    const float mx = selected ? row_max3<BS>(x) : -INFINITY;
+                    const float m_new = mx * p.scale_log2;
+                    const bool need = m_new > m_run + kRescaleLog2;
+                    // O must be rescaled only for rows whose earlier blocks contributed (m_run
+                    // finite); a row's O is exactly 0 until its first kept key.
+                    const bool need_o = need && m_run != -INFINITY;
+                    float factor = 1.f;
+                    if (need) {
+                        factor = m_run == -INFINITY ? 0.f : ex2(m_run - m_new);
+                        m_run = m_new;
+                        l_run *= factor;
+                    }
+                    if (j > 0 && __any_sync(0xffffffffu, need_o)) {
+                        const int pg = jg - 1;
+                        ok = warp_all(mbar_wait(&meta->pv_done[pg & 1], (pg >> 1) & 1, abort_flag, p.status));
+                        if (!ok) break;
+                        tc_fence_after();
+                        if (!need_o) factor = 1.f;
+#pragma unroll 1
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t o[32];
+                            tmem_ld32(tO + c * 32, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+                            tmem_st32(tO + c * 32, o);
+                        }
+                        tmem_wait_st();
+                    }
+                    const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+                    uint32_t packed[BS / 2];
+                    l_run += scores_to_p<BS>(x, selected ? p.scale_log2 : 0.f, selected ? -m_use : -INFINITY, packed);
+                    // P overwrites the first BS/2 columns of its own score buffer (already in
+                    // registers).  S_{jg} completing implies PV_{jg-2}, which read the previous P
+                    // from this buffer, has completed too.
+                    if constexpr (BS == 64) {
+                        tmem_st32(lane_base + (jg & 1) * BS, packed);
+                    } else {
+                        tmem_st16(lane_base + (jg & 1) * BS, packed);
+                    }
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&meta->p_full[jg & 1]);
+                }
+
+                // ------------------------------------------------------------ epilogue
+                if (ok && nU > 0) {
+                    const int lg = jbase + nU - 1;
+                    ok = warp_all(mbar_wait(&meta->pv_done[lg & 1], (lg >> 1) & 1, abort_flag, p.status));
+                    tc_fence_after();
+                }
+                if (ok) {
+                    const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+                    const int64_t t = (int64_t)q0 + i;
+                    const int h = hk * p.G + g;
+                    __nv_bfloat16 *orow = p.out + (t * p.Hq + h) * D;
 #pragma unroll 1
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t o[32];
-                        tmem_ld32(tO + c * 32, o);
-                        tmem_wait_ld();
+                        if (nU > 0) {
+                            tmem_ld32(tO + c * 32, o);
+                            tmem_wait_ld();
+                        } else {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-                        tmem_st32(tO + c * 32, o);
+                            for (int e = 0; e < 32; ++e) o[e] = 0u;
+                        }
+                        if (row_valid) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l,
+                                                   __uint_as_float(o[2 * e + 1]) * inv_l);
+                            uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                        }
                     }
-                    tmem_wait_st();
-                }
-            } else if (j >= 2) {
-                ok = warp_all(mbar_wait(&meta->pv_done[j & 1], ((j - 2) >> 1) & 1, abort_flag, p.status));
-                if (!ok) break;
-            }
-            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-            float rowsum = 0.f;
-            uint32_t packed[BS / 2];
-#pragma unroll
-            for (int c = 0; c < BS; c += 2) {
-                const float p0 = ex2(fmaf(x[c], p.scale_log2, -m_use));
-                const float p1 = ex2(fmaf(x[c + 1], p.scale_log2, -m_use));
-                rowsum += p0 + p1;
-                packed[c / 2] = pack_bf16x2(p0, p1);
-            }
-            l_run += rowsum;
-            // P_j overwrites the first BS/2 columns of its own score buffer (already in registers).
-            if constexpr (BS == 64) {
-                tmem_st32(lane_base + (j & 1) * BS, packed);
-            } else {
-                tmem_st16(lane_base + (j & 1) * BS, packed);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            mbar_arrive(&meta->p_full[j & 1]);
-        }
-
-        // ---------------------------------------------------------------- epilogue
-        if (ok && nU > 0) {
-            ok = warp_all(mbar_wait(&meta->pv_done[(nU - 1) & 1], ((nU - 1) >> 1) & 1, abort_flag, p.status));
-            tc_fence_after();
-        }
-        if (ok) {
-            const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-            const int64_t t = (int64_t)q0 + i;
-            const int h = hk * p.G + g;
-            __nv_bfloat16 *orow = p.out + (t * p.Hq + h) * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                if (nU > 0) {
-                    tmem_ld32(tO + c * 32, o);
-                    tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = 0u;
-                }
-                if (row_valid) {
-                    uint32_t w[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv_l, __uint_as_float(o[2 * e + 1]) * inv_l);
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + c * 32);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+                    if (row_valid)
+                        p.lse[(int64_t)h * p.total_q + t] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
                 }
             }
-            if (row_valid)
-                p.lse[(int64_t)h * p.total_q + t] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+            jbase += nU;
+            titer += nU > 0 ? 1 : 0;
         }
+        tc_fence_before();
+        __syncthreads();  // the tile is done everywhere before the next one reuses its buffers
+        tc_fence_after();
     }
 
+    if (*abort_flag && warp == 0 && lane == 0) {  // wind down: let every copy this CTA started land
+        if (titer > 0) mbar_drain(&meta->q_full, (titer - 1) & 1);
+        for (int st = 0; st < kStages; ++st)
+            if (last_jg[st] >= 0) mbar_drain(&meta->kv_full[st], (last_jg[st] / kStages) & 1);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -390,7 +424,10 @@ cudaError_t launch_t(const FwdGeom &g, const FwdAttendParams &p, const CUtensorM
         if (e != cudaSuccess) return e;
         configured = (int)smem;
     }
-    fwd_attend_kernel<D, BS><<<g.tiles, kThreads, smem, st>>>(tq, tk, tv, p);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = g.tiles < 2 * sms ? g.tiles : 2 * sms;
+    fwd_attend_kernel<D, BS><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 

@@ -7,7 +7,7 @@
 #include <stddef.h>
 #include <stdint.h>
 
-#include "../../include/sfa.h"
+#include "sfa.h"  // include/ is on the include path
 
 namespace sfa {
 
@@ -27,7 +27,7 @@ struct FwdGeom {
     // those lists into items of at most Tq tokens.
     int inv, W, nwin, groups;
     int64_t cap_items;
-    size_t off_sel_c, off_cnt, off_ucnt, off_union;
+    size_t off_sel_c, off_cnt, off_ucnt, off_union, off_tilectr;
     size_t off_zero, zero_bytes;  // the part of the workspace cleared before every prep
     size_t off_ctrl, off_gstat, off_gcount, off_gcursor, off_gfirst, off_items, off_pml, off_po;
     size_t bytes;
@@ -82,7 +82,8 @@ struct FwdScatterParams {
 struct FwdAttendParams {
     const int32_t *cu_q, *cu_k;
     const int32_t *sel_c, *cnt, *ucnt, *uni;
-    int batch, total_q, Hq, Hkv, G, Tq, nqt, topk, umax;
+    int batch, total_q, Hq, Hkv, G, Tq, nqt, topk, umax, tiles;
+    int32_t *tile_counter;  // next query tile to hand out (cleared before the launch)
     int causal, wl, wr;
     float scale_log2;  // softmax scale * log2(e)
     __nv_bfloat16 *out;
