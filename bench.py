@@ -142,6 +142,26 @@ def physical_gpu_index(local_rank):
 
 
 # ---------------------------------------------------------------------------------------------
+# Multi-rank reductions (independent replicas: the only collectives are these timing reductions)
+# ---------------------------------------------------------------------------------------------
+def max_over_ranks(vals, world, device):
+    """Element-wise max of per-rank timings; every rank calls it the same number of times."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_rate(world, units_per_rank, ms):
+    """Whole-job throughput in units/s: each of `world` ranks processes `units_per_rank`, and the
+    job takes the slowest rank's `ms`."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
+# ---------------------------------------------------------------------------------------------
 # CPU oracle baseline (bounded sample)
 # ---------------------------------------------------------------------------------------------
 def cpu_oracle_rate(c, seconds, seed=0):
@@ -163,10 +183,13 @@ def cpu_oracle_rate(c, seconds, seed=0):
         return flops, time.perf_counter() - t0, n
 
     threads = oracle.default_threads()
-    f, t, n = run(64 * threads)
-    n2 = int(min(c.total_q * c.Hq, max(64, n * seconds / max(t, 1e-3))))
-    f, t, n = run(n2)
-    return f / t / 1e12, n, threads, t
+    cap = c.total_q * c.Hq
+    n = min(cap, 64 * threads)
+    while True:  # grow the sample until one run takes most of the requested time
+        f, t, n = run(n)
+        if t >= 0.6 * seconds or n >= cap:
+            return f / t / 1e12, n, threads, t
+        n = int(min(cap, max(n + 1, n * min(8.0, seconds / max(t, 1e-3)))))
 
 
 # ---------------------------------------------------------------------------------------------
@@ -278,17 +301,14 @@ def run_gpu(args, rank, world, local_rank):
     stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(len(stages))] for i in range(K)])
     region_ms = t_start.elapsed_time(t_end)
     mean = stage_ms.mean(axis=0)
-    tm = torch.tensor([region_ms, *mean.tolist()], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
-    region_ms, pp_ms, pa_ms, dp_ms, da_ms = tm.tolist()
+    region_ms, pp_ms, pa_ms, dp_ms, da_ms = max_over_ranks([region_ms, *mean.tolist()], world, dev)
     prefill_ms = pp_ms + pa_ms
     decode_ms = dp_ms + da_ms
     step_ms = prefill_ms + decode_ms
-    value = world * flops / (prefill_ms * 1e-3) / 1e12
-    attend_tflops = flops / (pa_ms * 1e-3) / 1e12
-    dec_gbs = world * gbytes / (decode_ms * 1e-3) / 1e9
-    dec_attend_gbs = gbytes / (da_ms * 1e-3) / 1e9
+    value = job_rate(world, flops, prefill_ms) / 1e12
+    attend_tflops = job_rate(1, flops, pa_ms) / 1e12
+    dec_gbs = job_rate(world, gbytes, decode_ms) / 1e9
+    dec_attend_gbs = job_rate(1, gbytes, da_ms) / 1e9
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
 
@@ -347,13 +367,10 @@ def run_gpu(args, rank, world, local_rank):
         T.cuda.synchronize()
         e_pre = float(np.mean([evs[i][0].elapsed_time(evs[i][1]) for i in range(Ke)]))
         e_dec = float(np.mean([evs[i][1].elapsed_time(evs[i][2]) for i in range(Ke)]))
-        te = torch.tensor([e_pre, e_dec], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e_pre, e_dec = te.tolist()
-        e2e = {"value": round(world * flops / (e_pre * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+        e_pre, e_dec = max_over_ranks([e_pre, e_dec], world, dev)
+        e2e = {"value": round(job_rate(world, flops, e_pre) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(h2d + dh2d), "d2h_bytes_per_step": int(d2h + dd2h),
-               "decode": {"value": round(world * gbytes / (e_dec * 1e-3) / 1e9, 1), "unit": "GB/s"},
+               "decode": {"value": round(job_rate(world, gbytes, e_dec) / 1e9, 1), "unit": "GB/s"},
                "note": "pinned host inputs copied in and outputs (out, lse) copied back every step; "
                        "the decode KV cache is resident state, its per-step inputs are q, block_table, "
                        "cache_seqlens, sel_tok_idx"}
