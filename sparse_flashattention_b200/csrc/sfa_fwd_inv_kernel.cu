@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(inv_smem_raw) + 1023) & ~uintptr_t(1023));
     InvMeta *meta = reinterpret_cast<InvMeta *>(smem + C::kOffMeta);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // No window went block-major: leave before any barrier or TMEM is set up (uniform exit).
+    if (__ldcg(&p.ctrl->item_total) == 0) return;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kItemSlots; ++s) {
@@ -373,6 +375,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) fwd_merge_kernel(const FwdAt
     const int lane = threadIdx.x & 31;
     const int64_t u = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
     if (u >= (int64_t)p.total_q * p.Hkv) return;
+    if (__ldcg(&p.ctrl->item_total) == 0) return;  // every row was written by the query-major kernel
     const int cnt = p.cnt[u];
     if (cnt == 0) return;  // written by the query-major kernel
     const int64_t t = u / p.Hkv;

@@ -53,8 +53,8 @@ struct Cfg {
 
 struct Meta {
     uint64_t q_full;
-    uint64_t kv_full[kStages];
-    uint64_t kv_empty[kStages];
+    uint64_t k_full[kStages], k_empty[kStages];  // K of a block is free once its S MMA is done,
+    uint64_t v_full[kStages], v_empty[kStages];  // V once its PV MMA is done
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t pv_done[2];
@@ -89,8 +89,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (threadIdx.x == 0) {
         mbar_init(&meta->q_full, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&meta->kv_full[s], 1);
-            mbar_init(&meta->kv_empty[s], 1);
+            mbar_init(&meta->k_full[s], 1);
+            mbar_init(&meta->k_empty[s], 1);
+            mbar_init(&meta->v_full[s], 1);
+            mbar_init(&meta->v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&meta->s_full[s], 1);
@@ -121,9 +123,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     int jbase = 0;  // blocks this CTA processed in earlier tiles
     int titer = 0;  // tiles this CTA computed (phase of q_full)
-    int last_jg[kStages];
+    int last_jg[kStages], last_k[kStages];  // last block whose V (K) load went into each stage
 #pragma unroll
-    for (int s = 0; s < kStages; ++s) last_jg[s] = -1;
+    for (int s = 0; s < kStages; ++s) last_jg[s] = last_k[s] = -1;
 
     while (true) {
         if (threadIdx.x == 0) meta->tile = atomicAdd(p.tile_counter, 1);
@@ -171,20 +173,40 @@ __global__ void __launch_bounds__(kThreads, 2)
                     mbar_arrive_expect_tx(&meta->q_full, qbytes);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(&tmq, &meta->q_full, sQ + c * (128 * 128), c * 64, hk * p.G, q0 + tok0);
-                    for (int j = 0; j < nU; ++j) {
-                        const int jg = jbase + j, st = jg % kStages;
+                    // K of block j+1 goes out as soon as S_{j-1} has freed its stage, ahead of V_j
+                    // (which waits for PV_{j-2}): S needs only K, so the loads S waits on are
+                    // issued a softmax step earlier than a joint K/V stage would allow.
+                    auto load_k = [&](int jg, int j) -> bool {
+                        const int st = jg % kStages;
                         if (jg >= kStages &&
-                            !mbar_wait(&meta->kv_empty[st], ((jg / kStages) - 1) & 1, abort_flag, p.status))
-                            break;
+                            !mbar_wait(&meta->k_empty[st], ((jg / kStages) - 1) & 1, abort_flag, p.status))
+                            return false;
                         const int row = k0 + s_union[j] * BS;
-                        mbar_arrive_expect_tx(&meta->kv_full[st], 2u * (uint32_t)C::kKVBytes);
-                        for (int c = 0; c < D / 64; ++c) {
-                            tma_load_3d(&tmk, &meta->kv_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64,
+                        mbar_arrive_expect_tx(&meta->k_full[st], (uint32_t)C::kKVBytes);
+                        for (int c = 0; c < D / 64; ++c)
+                            tma_load_3d(&tmk, &meta->k_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64,
                                         hk, row);
-                            tma_load_3d(&tmv, &meta->kv_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64,
+                        last_k[st] = jg;
+                        return true;
+                    };
+                    auto load_v = [&](int jg, int j) -> bool {
+                        const int st = jg % kStages;
+                        if (jg >= kStages &&
+                            !mbar_wait(&meta->v_empty[st], ((jg / kStages) - 1) & 1, abort_flag, p.status))
+                            return false;
+                        const int row = k0 + s_union[j] * BS;
+                        mbar_arrive_expect_tx(&meta->v_full[st], (uint32_t)C::kKVBytes);
+                        for (int c = 0; c < D / 64; ++c)
+                            tma_load_3d(&tmv, &meta->v_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64,
                                         hk, row);
-                        }
                         last_jg[st] = jg;
+                        return true;
+                    };
+                    if (load_k(jbase, 0)) {
+                        for (int j = 0; j < nU; ++j) {
+                            if (j + 1 < nU && !load_k(jbase + j + 1, j + 1)) break;
+                            if (!load_v(jbase + j, j)) break;
+                        }
                     }
                 }
             } else if (warp == 1) {
@@ -203,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         bool progressed = false;
                         if (ns < nU && ns <= np + 1) {
                             const int jg = jbase + ns, st = jg % kStages;
-                            if (mbar_try_wait(smem_u32(&meta->kv_full[st]), (jg / kStages) & 1)) {
+                            if (mbar_try_wait(smem_u32(&meta->k_full[st]), (jg / kStages) & 1)) {
                                 tc_fence_after();
                                 const uint32_t tS = tmem + (jg & 1) * BS;
 #pragma unroll
@@ -215,13 +237,15 @@ __global__ void __launch_bounds__(kThreads, 2)
                                     umma_bf16(tS, a, bd, C::kIdescS, ks > 0 ? 1u : 0u);
                                 }
                                 umma_commit(&meta->s_full[jg & 1]);
+                                umma_commit(&meta->k_empty[st]);
                                 ++ns;
                                 progressed = true;
                             }
                         }
                         if (np < ns) {
                             const int ig = jbase + np, st = ig % kStages;
-                            if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1)) {
+                            if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
+                                mbar_try_wait(smem_u32(&meta->v_full[st]), (ig / kStages) & 1)) {
                                 tc_fence_after();
 #pragma unroll
                                 for (int ks = 0; ks < BS / 16; ++ks) {
@@ -232,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                                     umma_bf16_tmem_a(tO, a, bd, C::kIdescPV, (np > 0 || ks > 0) ? 1u : 0u);
                                 }
                                 umma_commit(&meta->pv_done[ig & 1]);
-                                umma_commit(&meta->kv_empty[st]);
+                                umma_commit(&meta->v_empty[st]);
                                 ++np;
                                 progressed = true;
                             }
@@ -395,7 +419,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (*abort_flag && warp == 0 && lane == 0) {  // wind down: let every copy this CTA started land
         if (titer > 0) mbar_drain(&meta->q_full, (titer - 1) & 1);
         for (int st = 0; st < kStages; ++st)
-            if (last_jg[st] >= 0) mbar_drain(&meta->kv_full[st], (last_jg[st] / kStages) & 1);
+            if (last_jg[st] >= 0) mbar_drain(&meta->v_full[st], (last_jg[st] / kStages) & 1);
+        for (int st = 0; st < kStages; ++st)
+            if (last_k[st] >= 0) mbar_drain(&meta->k_full[st], (last_k[st] / kStages) & 1);
     }
     tc_fence_before();
     __syncthreads();
