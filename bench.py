@@ -39,6 +39,34 @@ PREFILL_NAME = "nsa_varlen_16k: lens [8192,4096,2048,2048], Hq16/Hkv4, d128, bs6
 DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], page256, 2048 tok/(b,hk)"
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant kernel of
+# each stage, from one `ncu --set full` capture (profiles/fwd_attend_kernel_nsa_varlen_16k.md and
+# profiles/decode_split_kernel_paged_topk_decode.md).  A figure holds only for the kernel sources it
+# was taken on: the digest of those files must match, else the bench reports null.
+TRAFFIC = {
+    "fwd_attend_kernel": {"files": ["sfa_fwd_kernel.cu", "sfa_device.cuh", "sfa_internal.h"],
+                          "sha256": "068f103d4e3be43aa78872ec491c3d70f6991bec07be93c43fa50e424bf7cd28",
+                          "bytes": 141967616},
+    "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh", "sfa_internal.h"],
+                            "sha256": "0e3110287e520ebb4120fbaa4f50ba10ef7cca2660fda43f63e84cc930dd5853",
+                            "bytes": 281162752},
+}
+
+
+def source_digest(files):
+    import hashlib
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "sparse_flashattention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def kernel_traffic(kernel):
+    t = TRAFFIC[kernel]
+    return t["bytes"] if source_digest(t["files"]) == t["sha256"] else None
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -378,7 +406,9 @@ def run_gpu(args, rank, world, local_rank):
                 dprep_ms=dp_ms, dattend_ms=da_ms, step_ms=step_ms, region_ms=region_ms, attend_tflops=attend_tflops,
                 dec_gbs=dec_gbs, dec_attend_gbs=dec_attend_gbs, flops=flops, gbytes=gbytes, clocks=clocks,
                 launches=n_launch, e2e=e2e, hbm=hbm, tf_burst=tf_burst, tf_sust=tf_sust, peak_kind=peak_kind,
-                pc=pc, dc=dc, traffic=args.traffic)
+                pc=pc, dc=dc,
+                traffic=args.traffic if args.traffic is not None else kernel_traffic("fwd_attend_kernel"),
+                dec_traffic=kernel_traffic("decode_split_kernel"))
 
 
 def main():
@@ -394,7 +424,7 @@ def main():
                     help="'prefill' times only the prefill stages (a small decode case stands in); for profiling")
     ap.add_argument("--prefill-config", type=int, default=2, choices=[1, 2, 3, 4],
                     help="prefill workload (default 2, the varlen NSA one the metric is quoted on)")
-    ap.add_argument("--traffic", type=float, default=None,
+    ap.add_argument("--traffic", type=int, default=None,
                     help="dram bytes (read+write) per attend launch from an ncu capture of this kernel version")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
@@ -445,11 +475,14 @@ def main():
                    "gathered_bytes": int(r["gbytes"]),
                    "roofline": {"bound": "hbm", "achieved": round(r["dec_attend_gbs"], 1), "peak": r["hbm"],
                                 "unit": "GB/s", "frac": round(r["dec_attend_gbs"] / r["hbm"], 4),
+                                "traffic": r["dec_traffic"], "traffic_unit": "B per decode_split_kernel launch",
                                 "kernel": "decode split + combine (sfa_decode_attend)",
                                 "peak_source": r["peak_kind"]}},
         "roofline": {"bound": "tensor", "achieved": round(r["attend_tflops"], 2), "peak": r["tf_burst"],
                      "unit": "TFLOP/s", "frac": round(r["attend_tflops"] / r["tf_burst"], 4),
-                     "traffic": r["traffic"], "kernel": "fwd_attend_kernel (sfa_fwd_attend)",
+                     "traffic": r["traffic"], "traffic_unit": "B per fwd_attend_kernel launch",
+                     "kernel": "fwd_attend_kernel (sfa_fwd_attend stage; its block-major kernels return at once "
+                               "on this workload)",
                      "peak_source": f"{r['peak_kind']} bf16 burst",
                      "frac_of_sustained": round(r["attend_tflops"] / r["tf_sust"], 4) if r["tf_sust"] else None},
         "gpu_launches": r["launches"],
