@@ -6,7 +6,8 @@ One step = one pass of the whole hot path on seeded synthetic inputs already res
 HBM: the varlen NSA prefill workload (lengths [8192, 4096, 2048, 2048], Hq16/Hkv4, d128,
 block 64, top-16 with init 1 / local 2; sfa_fwd_prep + sfa_fwd_attend) followed by the paged
 top-k decode workload (B32, Hq32/Hkv8, d128, L ~ U[16384, 131072], page 256, 2048 tokens per
-(sequence, kv head); sfa_decode_prep + sfa_decode_attend).  L2 is flushed (256 MiB write)
+(sequence, kv head); sfa_decode, which deduplicates the selections inside its split kernel).
+L2 is flushed (256 MiB write)
 before every step, outside the kernel events.
 
 The JSON line's value is prefill effective TFLOP/s (4*d flops per kept query-key pair per
@@ -275,14 +276,12 @@ def run_gpu(args, rank, world, local_rank):
                        status=status)
         launches[0] += sfa.last_launch_count()
 
-    def decode_prep():
-        sfa.decode_prep(D["cache_seqlens"], D["sel"], Hq=dc.Hq, d=dc.d, max_pages_per_seq=dc.max_pages,
-                        page_size=dc.page, workspace=dws, status=status)
-        launches[0] += sfa.last_launch_count()
+    def decode_prep():  # selections this short are deduplicated inside the split kernel: no stage
+        pass
 
     def decode_attend():
-        sfa.decode_attend(D["q"], D["k_cache"], D["v_cache"], D["block_table"], dws, topk_tok=dc.topk, out=dout,
-                          lse=dlse, status=status)
+        sfa.decode(D["q"], D["k_cache"], D["v_cache"], D["block_table"], D["cache_seqlens"], D["sel"], out=dout,
+                   lse=dlse, workspace=dws, status=status)
         launches[0] += sfa.last_launch_count()
 
     stages = [prefill_prep, prefill_attend, decode_prep, decode_attend]
@@ -476,7 +475,7 @@ def main():
                    "roofline": {"bound": "hbm", "achieved": round(r["dec_attend_gbs"], 1), "peak": r["hbm"],
                                 "unit": "GB/s", "frac": round(r["dec_attend_gbs"] / r["hbm"], 4),
                                 "traffic": r["dec_traffic"], "traffic_unit": "B per decode_split_kernel launch",
-                                "kernel": "decode split + combine (sfa_decode_attend)",
+                                "kernel": "decode split + combine (sfa_decode)",
                                 "peak_source": r["peak_kind"]}},
         "roofline": {"bound": "tensor", "achieved": round(r["attend_tflops"], 2), "peak": r["tf_burst"],
                      "unit": "TFLOP/s", "frac": round(r["attend_tflops"] / r["tf_burst"], 4),

@@ -151,7 +151,9 @@ size_t sfa_decode_workspace_size(int B, int Hq, int Hkv, int d, int topk_tok, in
 int sfa_decode_workspace_offsets(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits,
                                  size_t *off_tok_c, size_t *off_cnt);
 
-/* Paged top-k decode = prep, split-KV attention, LSE combine.
+/* Paged top-k decode = split-KV attention and LSE combine.  Each (sequence, kv head)'s
+ * selection is deduplicated and sorted inside the split kernel when topk_tok <= 2048 (two
+ * launches); longer selections first go through the prep kernel (three launches).
  *   q             bf16 (B, Hq, d): the new token of each sequence, at position L_b - 1
  *   k_cache,
  *   v_cache       bf16 (num_pages, page_size, Hkv, d)
@@ -206,7 +208,8 @@ int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
 const char *sfa_status_string(int status);
 
 /* Number of kernel launches the last successful call on this host thread made (prefill: 2,
- * or 6 when the call can use the block-major schedule; decode: 3; a stage: its own count). */
+ * or 6 when the call can use the block-major schedule; decode: 2, or 3 when topk_tok > 2048; a
+ * stage: its own count). */
 int sfa_last_launch_count(void);
 
 #ifdef __cplusplus

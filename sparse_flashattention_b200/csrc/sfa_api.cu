@@ -295,28 +295,17 @@ int num_sms()
     return n > 0 ? n : 148;
 }
 
-// Split count: each split is one warp's chunk of a (sequence, kv head) token list, and a CTA
-// runs decode_split_warps_per_block() of them.  Pick the S (at least 64 tokens per split)
-// whose last wave of CTAs over num_SMs * CTAs-per-SM slots is fullest, with a small charge per
-// extra split for its prologue and its partial output.
+// Split count: each split is one warp's chunk of a (sequence, kv head) token list; the splits of
+// one (sequence, kv head) run decode_split_warps_per_block() to a CTA, and each CTA first
+// deduplicates the whole selection.  Fill one wave of num_SMs * CTAs-per-SM slots: as many CTAs
+// per (sequence, kv head) as fit in that wave, at least one, with at least 64 tokens per split.
 int choose_splits(int B, int Hkv, int d, int topk)
 {
     const int units = B * Hkv;
     const int wpb = decode_split_warps_per_block();
     const int slots = num_sms() * decode_split_blocks_per_sm(d);
-    const int smax = std::max(1, std::min(64, topk / 64));
-    int best = 1;
-    double best_score = -1e30;
-    for (int S = 1; S <= smax; ++S) {
-        const double ctas = std::ceil((double)units * S / wpb);
-        const double waves = ctas / slots;
-        const double score = waves / std::ceil(waves) - 0.002 * S;
-        if (score > best_score + 1e-9) {
-            best_score = score;
-            best = S;
-        }
-    }
-    return best;
+    const int cps = std::max(1, std::min(slots / std::max(units, 1), topk / (wpb * 64)));
+    return std::max(1, std::min(cps * wpb, topk / 64));
 }
 
 int dec_geometry(int B, int Hq, int Hkv, int d, int topk, int num_splits, DecGeom &g)
@@ -366,9 +355,11 @@ int dec_prep_impl(const DecGeom &g, const int32_t *seqlens, const int32_t *sel, 
     return launch_decode_prep(g, p, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
 }
 
+// fused: the split kernel deduplicates sel itself (no prep launch); else it reads the prep kernel's
+// canonical sets from the workspace.
 int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void *vc, const int32_t *bt, int max_pages,
-                    int num_pages, int page, float scale, void *ws, int32_t *status, void *out, float *lse,
-                    cudaStream_t st)
+                    int num_pages, int page, const int32_t *seqlens, const int32_t *sel, int wl, bool fused,
+                    float scale, void *ws, int32_t *status, void *out, float *lse, cudaStream_t st)
 {
     if ((int64_t)num_pages * page * g.Hkv > (int64_t)INT32_MAX) return SFA_ERR_UNSUPPORTED;
     uint8_t *w = static_cast<uint8_t *>(ws);
@@ -379,6 +370,10 @@ int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void 
     p.bt = bt;
     p.tok_c = reinterpret_cast<const int32_t *>(w + g.off_tok);
     p.cnt = reinterpret_cast<const int32_t *>(w + g.off_cnt);
+    p.seqlens = seqlens;
+    p.sel = sel;
+    p.fused = fused ? 1 : 0;
+    p.wl = wl;
     p.B = g.B;
     p.max_pages = max_pages;
     p.num_pages = num_pages;
@@ -556,8 +551,8 @@ int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache, c
     if (!q || !k_cache || !v_cache || !block_table || !workspace || !out || !lse) return SFA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
-    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, scale,
-                         workspace, status_dev, out, lse, stream);
+    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, nullptr,
+                         nullptr, -1, false, scale, workspace, status_dev, out, lse, stream);
     if (rc == SFA_OK) g_last_launches = 2;
     return rc;
 }
@@ -578,12 +573,19 @@ int sfa_decode(const void *q, const void *k_cache, const void *v_cache, const in
         return SFA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
-    rc = dec_prep_impl(g, cache_seqlens, sel_tok_idx, max_pages_per_seq, page_size, window_left, workspace, status_dev,
-                       stream);
-    if (rc != SFA_OK) return rc;
-    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, scale,
-                         workspace, status_dev, out, lse, stream);
-    if (rc == SFA_OK) g_last_launches = 3;
+    // Selections of up to decode_fused_max_topk() positions are deduplicated inside the split
+    // kernel; longer ones go through the prep kernel first.
+    const bool fused = topk_tok <= decode_fused_max_topk();
+    if (!fused) {
+        rc = dec_prep_impl(g, cache_seqlens, sel_tok_idx, max_pages_per_seq, page_size, window_left, workspace,
+                           status_dev, stream);
+        if (rc != SFA_OK) return rc;
+    } else if ((int64_t)max_pages_per_seq * page_size > (1 << 20)) {
+        return SFA_ERR_UNSUPPORTED;
+    }
+    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, cache_seqlens,
+                         sel_tok_idx, window_left, fused, scale, workspace, status_dev, out, lse, stream);
+    if (rc == SFA_OK) g_last_launches = fused ? 2 : 3;
     return rc;
 }
 

@@ -1,6 +1,10 @@
 // Paged top-k decode: split-KV attention over gathered cache rows, then an LSE combine.
 //
-// Split kernel: every warp is an independent worker for one (sequence, kv head, split): it
+// Split kernel: the splits of one (sequence, kv head) run four to a CTA.  For selections of up to
+// 2048 positions the CTA first deduplicates its (sequence, kv head)'s selection itself: a bitmap
+// over the positions [0, L) in the (not yet used) pipeline rings, scanned into an ascending list
+// in shared memory — the same canonical list the prep kernel writes for longer selections.
+// Then every warp is an independent worker for one split: it
 // takes a contiguous chunk of the canonical (ascending) token list of its (sequence, kv head),
 // looks each token's physical row up through block_table, and streams the 256-byte K and V
 // rows of 16 tokens at a time through its own 3-stage cp.async ring in shared memory
@@ -27,6 +31,7 @@ constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kStageTok = 16;     // tokens per pipeline stage (one m16n8k16 K extent)
 constexpr int kDecStages = 3;     // per-warp ring depth
 constexpr int kWin = 256;         // tokens whose physical rows a warp looks up at a time
+constexpr int kFusedMaxTopk = 2048;  // the in-kernel dedupe keeps a (sequence, kv head)'s list in shared memory
 constexpr float kLn2d = 0.6931471805599453f;
 constexpr float kRescaleLog2d = 8.0f;
 
@@ -38,7 +43,9 @@ struct DecCfg {
     static constexpr int kStageBytes = 2 * kTileBytes;  // K then V
     static constexpr int kWarpRing = kDecStages * kStageBytes;
     static constexpr int kOffRows = kDecWarps * kWarpRing;
-    static constexpr int kBytes = kOffRows + kDecWarps * kWin * 4;
+    static constexpr int kOffList = kOffRows + kDecWarps * kWin * 4;  // deduplicated positions (fused)
+    static constexpr int kBytes = kOffList + kFusedMaxTopk * 4;
+    static constexpr int kBitmapWords = kOffRows / 4;  // the dedupe bitmap borrows the rings
 };
 
 // Byte offset of 16-byte chunk c of row r in a tile whose rows are D*2 bytes: the chunk index
@@ -54,24 +61,130 @@ __device__ __forceinline__ uint32_t ld_q2(const __nv_bfloat16 *p)
     return __ldg(reinterpret_cast<const uint32_t *>(p));
 }
 
+// Exclusive scan over the CTA's kDecThreads threads; returns the total (all threads call it).
+__device__ __forceinline__ int cta_exclusive_scan(int v, int *scratch, int &excl)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kDecWarps; ++w) {
+        const int t = scratch[w];
+        if (w < warp) before += t;
+        total += t;
+    }
+    __syncthreads();
+    excl = before + x - v;
+    return total;
+}
+
+// Ascending, duplicate-free positions of one (sequence, kv head)'s selection, each in [0, L) and
+// (window_left >= 0) >= L-1-window_left, into list[]; returns their number.  A bitmap over a
+// range of positions at a time lives in `bm` (the pipeline rings, not in use yet).  Ids that are
+// neither -1 nor in [0, L) set *bad.  All threads of the CTA call it.
+template <int D>
+__device__ int dedupe_positions(const int32_t *sel, int topk, int L, int wl, uint32_t *bm, int *list,
+                                int *scratch, bool &bad)
+{
+    using C = DecCfg<D>;
+    const bool vec = (topk & 3) == 0 && (reinterpret_cast<uintptr_t>(sel) & 15) == 0;
+    const int lo_pos = wl >= 0 ? max(0, L - 1 - wl) : 0;
+    int n = 0;
+    for (int c0 = 0; c0 < L; c0 += C::kBitmapWords * 32) {
+        const int c1 = min(L, c0 + C::kBitmapWords * 32);
+        const int nw = (c1 - c0 + 31) >> 5;
+        for (int w = threadIdx.x; w < nw; w += kDecThreads) bm[w] = 0u;
+        __syncthreads();
+        auto mark = [&](int j) {
+            if (j == -1) return;
+            if (j < 0 || j >= L) {
+                bad = true;
+                return;
+            }
+            if (j >= lo_pos && j >= c0 && j < c1) atomicOr(&bm[(j - c0) >> 5], 1u << ((j - c0) & 31));
+        };
+        if (vec) {
+            for (int e = threadIdx.x * 4; e < topk; e += kDecThreads * 4) {
+                const int4 v = __ldg(reinterpret_cast<const int4 *>(sel + e));
+                mark(v.x);
+                mark(v.y);
+                mark(v.z);
+                mark(v.w);
+            }
+        } else {
+            for (int e = threadIdx.x; e < topk; e += kDecThreads) mark(__ldg(&sel[e]));
+        }
+        __syncthreads();
+        // Thread t owns a run of words; a CTA scan gives its first output slot.
+        const int per = (nw + kDecThreads - 1) / kDecThreads;
+        const int w0 = min(nw, (int)threadIdx.x * per), w1 = min(nw, w0 + per);
+        int cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+        int pos;
+        const int total = cta_exclusive_scan(cnt, scratch, pos);
+        pos += n;
+        for (int w = w0; w < w1; ++w) {
+            uint32_t bits = bm[w];
+            while (bits) {
+                const int bt = __ffs(bits) - 1;
+                bits &= bits - 1;
+                list[pos++] = c0 + (w << 5) + bt;
+            }
+        }
+        n += total;
+        __syncthreads();  // the bitmap is read out before the next range clears it
+    }
+    return n;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSplitParams p)
 {
     using C = DecCfg<D>;
     extern __shared__ __align__(128) uint8_t dsm[];
+    __shared__ int scan_scratch[kDecWarps];
+    __shared__ int s_n;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * kDecWarps + warp;
-    if (gw >= p.B * p.Hkv * p.S) return;  // warp-uniform; the kernel has no CTA-wide barrier
-    const int split = gw % p.S;
-    const int bh = gw / p.S;  // b * Hkv + hk
+    const int cps = (p.S + kDecWarps - 1) / kDecWarps;  // CTAs per (sequence, kv head)
+    const int bh = blockIdx.x / cps;                     // b * Hkv + hk
+    const int split = (blockIdx.x - bh * cps) * kDecWarps + warp;
     const int hk = bh % p.Hkv, b = bh / p.Hkv;
-    const int n = p.cnt[bh];
+    const int32_t *toks;
+    int n;
+    if (p.fused) {
+        int L = p.seqlens[b];
+        if (L > p.max_pages * p.page) {  // more tokens than the block table can address
+            if (threadIdx.x == 0 && split == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_SEQLEN);
+            L = p.max_pages * p.page;
+        }
+        L = max(L, 0);
+        int *list = reinterpret_cast<int *>(dsm + C::kOffList);
+        bool bad = false;
+        const int nn = dedupe_positions<D>(p.sel + (int64_t)bh * p.topk, p.topk, L, p.wl,
+                                           reinterpret_cast<uint32_t *>(dsm), list, scan_scratch, bad);
+        if (bad && split == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_INDEX);
+        if (threadIdx.x == 0) s_n = nn;
+        __syncthreads();
+        n = s_n;
+        toks = list;
+    } else {
+        n = p.cnt[bh];
+        toks = p.tok_c + (int64_t)bh * p.topk;
+    }
+    if (split >= p.S) return;  // warp-uniform; no CTA-wide barrier follows
     const int chunk = (n + p.S - 1) / p.S;
     const int begin = min(n, split * chunk);
     const int ntok = min(n, begin + chunk) - begin;
+    toks += begin;
     const uint32_t ring = smem_u32(dsm) + warp * C::kWarpRing;
     int *rowoff = reinterpret_cast<int *>(dsm + C::kOffRows) + warp * kWin;
-    const int32_t *toks = p.tok_c + (int64_t)bh * p.topk + begin;
 
     // A fragments of the G query rows (rows >= G are zero), straight from global memory.
     uint32_t aq[D / 16][4];
@@ -265,8 +378,8 @@ cudaError_t launch_split_t(const DecGeom &g, const DecSplitParams &p, cudaStream
         if (e != cudaSuccess) return e;
         configured = true;
     }
-    const int warps = g.B * g.Hkv * g.S;
-    decode_split_kernel<D><<<(warps + kDecWarps - 1) / kDecWarps, kDecThreads, smem, st>>>(p);
+    const int cps = (g.S + kDecWarps - 1) / kDecWarps;
+    decode_split_kernel<D><<<g.B * g.Hkv * cps, kDecThreads, smem, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -282,6 +395,11 @@ int decode_split_blocks_per_sm(int d)
 int decode_split_warps_per_block()
 {
     return kDecWarps;
+}
+
+int decode_fused_max_topk()
+{
+    return kFusedMaxTopk;
 }
 
 cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaStream_t st)

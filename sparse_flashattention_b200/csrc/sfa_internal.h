@@ -113,8 +113,10 @@ struct DecPrepParams {
 
 struct DecSplitParams {
     const __nv_bfloat16 *q, *kc, *vc;
-    const int32_t *bt, *tok_c, *cnt;
-    int B, max_pages, num_pages, page, Hq, Hkv, G, topk, S;
+    const int32_t *bt, *tok_c, *cnt;  // canonical sets from the prep kernel (fused == 0)
+    const int32_t *seqlens, *sel;     // raw selections, deduplicated in the kernel (fused == 1)
+    int fused, wl;
+    int B, max_pages, num_pages, page, Hq, Hkv, G, topk, S;  // CTA c of (b, kv head) runs splits 4c..4c+3
     float scale_log2;
     float *po, *plse;  // partial outputs (B, Hq, S, d) and natural-log lse (B, Hq, S)
     int32_t *status;
@@ -144,5 +146,6 @@ cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaS
 cudaError_t launch_decode_combine(const DecGeom &g, const DecCombineParams &p, cudaStream_t st);
 int decode_split_blocks_per_sm(int d);
 int decode_split_warps_per_block();
+int decode_fused_max_topk();
 
 }  // namespace sfa

@@ -113,9 +113,35 @@ def test_all_padding_decode(sfa):
 
 
 def test_decode_launch_count(sfa):
-    c = W.small_config(5)
+    c = W.small_config(5)  # 256 positions per (sequence, kv head): deduplicated in the split kernel
     run_decode(sfa, c)
+    assert sfa.last_launch_count() == 2
+
+
+def test_long_selection_goes_through_prep(sfa, oracle_lib):
+    """More than 2048 selected positions per (sequence, kv head): prep kernel, then split + combine."""
+    c = W.make_decode(77, 2, 8, 2, 128, 64, 6000, 9000, 3000, 64)
+    _parity(sfa, oracle_lib, c)
     assert sfa.last_launch_count() == 3
+
+
+@pytest.mark.parametrize("splits", [0, 3, 8])
+def test_stages_equal_fused_call_bitwise(sfa, splits):
+    """sfa_decode_prep + sfa_decode_attend (canonical sets through the workspace) and sfa_decode
+    (deduplicated inside the split kernel) split the same sorted lists the same way: the outputs
+    are bit-identical."""
+    c = W.small_config(5)
+    d = upload_decode(c)
+    out1, lse1 = run_decode(sfa, c, d=d, num_splits=splits)
+    ws = torch.empty(sfa.decode_workspace_size(c.q.shape[0], c.Hq, c.Hkv, c.d, c.sel.shape[2], splits),
+                     dtype=torch.uint8, device="cuda")
+    sfa.decode_prep(d["cache_seqlens"], d["sel"], Hq=c.Hq, d=c.d, max_pages_per_seq=c.max_pages, page_size=c.page,
+                    window_left=c.wl, num_splits=splits, workspace=ws)
+    out2, lse2 = sfa.decode_attend(d["q"], d["k_cache"], d["v_cache"], d["block_table"], ws, topk_tok=c.sel.shape[2],
+                                   scale=c.scale if c.scale > 0 else None, num_splits=splits)
+    torch.cuda.synchronize()
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    assert torch.equal(lse1, lse2)
 
 
 def test_full_size_decode(sfa, oracle_lib):
