@@ -387,8 +387,11 @@ int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void 
     p.scale_log2 = (float)(sc * 1.4426950408889634);
     p.po = reinterpret_cast<float *>(w + g.off_po);
     p.plse = reinterpret_cast<float *>(w + g.off_plse);
+    p.out_direct = static_cast<__nv_bfloat16 *>(out);
+    p.lse_direct = lse;
     p.status = status;
     if (launch_decode_split(g, p, st) != cudaSuccess) return SFA_ERR_CUDA;
+    if (g.S <= decode_split_warps_per_block()) return SFA_OK;  // combined inside the split kernel
     DecCombineParams c{};
     c.po = p.po;
     c.plse = p.plse;
@@ -553,7 +556,7 @@ int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache, c
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
     rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, nullptr,
                          nullptr, -1, false, scale, workspace, status_dev, out, lse, stream);
-    if (rc == SFA_OK) g_last_launches = 2;
+    if (rc == SFA_OK) g_last_launches = g.S <= decode_split_warps_per_block() ? 1 : 2;
     return rc;
 }
 
@@ -585,7 +588,7 @@ int sfa_decode(const void *q, const void *k_cache, const void *v_cache, const in
     }
     rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, cache_seqlens,
                          sel_tok_idx, window_left, fused, scale, workspace, status_dev, out, lse, stream);
-    if (rc == SFA_OK) g_last_launches = fused ? 2 : 3;
+    if (rc == SFA_OK) g_last_launches = (fused ? 0 : 1) + (g.S <= decode_split_warps_per_block() ? 1 : 2);
     return rc;
 }
 

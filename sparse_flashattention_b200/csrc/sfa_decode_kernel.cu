@@ -178,10 +178,10 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
         n = p.cnt[bh];
         toks = p.tok_c + (int64_t)bh * p.topk;
     }
-    if (split >= p.S) return;  // warp-uniform; no CTA-wide barrier follows
+    const bool active = split < p.S;  // a CTA's last warps may have no split
     const int chunk = (n + p.S - 1) / p.S;
     const int begin = min(n, split * chunk);
-    const int ntok = min(n, begin + chunk) - begin;
+    const int ntok = active ? min(n, begin + chunk) - begin : 0;
     toks += begin;
     const uint32_t ring = smem_u32(dsm) + warp * C::kWarpRing;
     int *rowoff = reinterpret_cast<int *>(dsm + C::kOffRows) + warp * kWin;
@@ -324,23 +324,60 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
     }
     if (bad_page && p.status) atomicOr(p.status, SFA_DEV_BAD_PAGE);
 
-    // Normalised partial output and LSE of this split.
+    // Normalised partial output and LSE of this split: into global memory for the combine kernel,
+    // or, when the CTA holds every split of its (sequence, kv head), into this warp's own ring
+    // (its copies have all landed) for the combine below.
+    const bool cta_combine = cps == 1;
+    float *po_s = reinterpret_cast<float *>(dsm + warp * C::kWarpRing);  // [16][D] then lse[16]
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         float l = l_r[h];
         l += __shfl_xor_sync(0xffffffffu, l, 1);
         l += __shfl_xor_sync(0xffffffffu, l, 2);
         const int row = (lane >> 2) + 8 * h;
-        if (row < p.G) {
+        if (active && row < p.G) {
             const int hq = hk * p.G + row;
             const int64_t slot = ((int64_t)b * p.Hq + hq) * p.S + split;
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            float *dst = p.po + slot * D + 2 * (lane & 3);
+            float *dst = (cta_combine ? po_s + row * D : p.po + slot * D) + 2 * (lane & 3);
 #pragma unroll
             for (int nt = 0; nt < D / 8; ++nt)
                 *reinterpret_cast<float2 *>(dst + nt * 8) = make_float2(o[nt][2 * h] * inv, o[nt][2 * h + 1] * inv);
-            if ((lane & 3) == 0) p.plse[slot] = l > 0.f ? (m_r[h] + log2f(l)) * kLn2d : -INFINITY;
+            const float ls = l > 0.f ? (m_r[h] + log2f(l)) * kLn2d : -INFINITY;
+            if ((lane & 3) == 0) {
+                if (cta_combine) po_s[16 * D + row] = ls;
+                else p.plse[slot] = ls;
+            }
         }
+    }
+    if (!cta_combine) return;
+    // In-CTA LSE combine of the S <= 4 splits: lse = log sum_s e^{lse_s}; out = sum_s e^{lse_s - lse} o_s.
+    __syncthreads();
+    const int nsp = min(p.S, kDecWarps);
+    for (int e = threadIdx.x; e < p.G * D; e += kDecThreads) {
+        const int row = e / D, c = e - row * D;
+        float ls[kDecWarps];
+        float M = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp < kDecWarps; ++sp) {
+            ls[sp] = sp < nsp ? reinterpret_cast<const float *>(dsm + sp * C::kWarpRing)[16 * D + row] : -INFINITY;
+            M = fmaxf(M, ls[sp]);
+        }
+        float acc = 0.f, lse = -INFINITY;
+        if (M != -INFINITY) {
+            float Z = 0.f;
+#pragma unroll
+            for (int sp = 0; sp < kDecWarps; ++sp) Z += ls[sp] == -INFINITY ? 0.f : __expf(ls[sp] - M);
+            lse = M + __logf(Z);
+#pragma unroll
+            for (int sp = 0; sp < kDecWarps; ++sp)
+                if (ls[sp] != -INFINITY)
+                    acc += __expf(ls[sp] - lse) *
+                           reinterpret_cast<const float *>(dsm + sp * C::kWarpRing)[row * D + c];
+        }
+        const int64_t orow = (int64_t)b * p.Hq + hk * p.G + row;
+        p.out_direct[orow * D + c] = __float2bfloat16_rn(acc);
+        if (c == 0) p.lse_direct[orow] = lse;
     }
 }
 

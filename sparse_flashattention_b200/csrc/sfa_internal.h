@@ -119,6 +119,8 @@ struct DecSplitParams {
     int B, max_pages, num_pages, page, Hq, Hkv, G, topk, S;  // CTA c of (b, kv head) runs splits 4c..4c+3
     float scale_log2;
     float *po, *plse;  // partial outputs (B, Hq, S, d) and natural-log lse (B, Hq, S)
+    __nv_bfloat16 *out_direct;  // S <= 4: the CTA combines its splits and writes out / lse itself
+    float *lse_direct;
     int32_t *status;
 };
 

@@ -112,17 +112,24 @@ def test_all_padding_decode(sfa):
     assert_empty_rows_exact(out, lse)
 
 
-def test_decode_launch_count(sfa):
+def _split_launches(sfa, c, num_splits=0):
+    # split kernel, plus the combine kernel when the splits of a (sequence, kv head) span CTAs
+    S = sfa.decode_num_splits(c.q.shape[0], c.Hq, c.Hkv, c.d, c.sel.shape[2], num_splits)
+    return 1 if S <= 4 else 2
+
+
+@pytest.mark.parametrize("splits", [0, 4, 5, 16])
+def test_decode_launch_count(sfa, splits):
     c = W.small_config(5)  # 256 positions per (sequence, kv head): deduplicated in the split kernel
-    run_decode(sfa, c)
-    assert sfa.last_launch_count() == 2
+    run_decode(sfa, c, num_splits=splits)
+    assert sfa.last_launch_count() == _split_launches(sfa, c, splits)
 
 
 def test_long_selection_goes_through_prep(sfa, oracle_lib):
     """More than 2048 selected positions per (sequence, kv head): prep kernel, then split + combine."""
     c = W.make_decode(77, 2, 8, 2, 128, 64, 6000, 9000, 3000, 64)
     _parity(sfa, oracle_lib, c)
-    assert sfa.last_launch_count() == 3
+    assert sfa.last_launch_count() == 1 + _split_launches(sfa, c)
 
 
 @pytest.mark.parametrize("splits", [0, 3, 8])
