@@ -45,12 +45,12 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 # profiles/decode_split_kernel_paged_topk_decode.md).  A figure holds only for the kernel sources it
 # was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
-    "fwd_attend_kernel": {"files": ["sfa_fwd_kernel.cu", "sfa_device.cuh", "sfa_internal.h"],
-                          "sha256": "068f103d4e3be43aa78872ec491c3d70f6991bec07be93c43fa50e424bf7cd28",
+    "fwd_attend_kernel": {"files": ["sfa_fwd_kernel.cu", "sfa_device.cuh"],
+                          "sha256": "d1aa6475b8f3d0467ec50bf47ab49eac840d589f9c7c3616f0e9e18f4d058e35",
                           "bytes": 141967616},
-    "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh", "sfa_internal.h"],
-                            "sha256": "0e3110287e520ebb4120fbaa4f50ba10ef7cca2660fda43f63e84cc930dd5853",
-                            "bytes": 281162752},
+    "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
+                            "sha256": "7c4e1665908006ce7e9e774269d385ac3d367fa37cfbd3550339a23f3e1332c5",
+                            "bytes": 274851840},
 }
 
 
@@ -475,7 +475,7 @@ def main():
                    "roofline": {"bound": "hbm", "achieved": round(r["dec_attend_gbs"], 1), "peak": r["hbm"],
                                 "unit": "GB/s", "frac": round(r["dec_attend_gbs"] / r["hbm"], 4),
                                 "traffic": r["dec_traffic"], "traffic_unit": "B per decode_split_kernel launch",
-                                "kernel": "decode split + combine (sfa_decode)",
+                                "kernel": "decode_split_kernel (sfa_decode: one launch, splits merged in the CTA)",
                                 "peak_source": r["peak_kind"]}},
         "roofline": {"bound": "tensor", "achieved": round(r["attend_tflops"], 2), "peak": r["tf_burst"],
                      "unit": "TFLOP/s", "frac": round(r["attend_tflops"] / r["tf_burst"], 4),
