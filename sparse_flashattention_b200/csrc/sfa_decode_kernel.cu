@@ -97,49 +97,67 @@ __device__ int dedupe_positions(const int32_t *sel, int topk, int L, int wl, uin
     const bool vec = (topk & 3) == 0 && (reinterpret_cast<uintptr_t>(sel) & 15) == 0;
     const int lo_pos = wl >= 0 ? max(0, L - 1 - wl) : 0;
     int n = 0;
-    for (int c0 = 0; c0 < L; c0 += C::kBitmapWords * 32) {
-        const int c1 = min(L, c0 + C::kBitmapWords * 32);
+    // Positions [c0, c1) at a time.  Thread t owns the `per` consecutive bitmap words
+    // [t*per, (t+1)*per); word w is stored at (w % per) * kDecThreads + w / per, so when every
+    // thread walks its own words in order, the 32 lanes of a warp read 32 consecutive addresses.
+    // Beside the bitmap: wpref, the number of kept positions before each word.  A kept position j
+    // then goes straight to list[wpref[word] + (set bits below j in its word)] — duplicates write
+    // the same value to the same slot.
+    constexpr int kPer = C::kBitmapWords / 2 / kDecThreads;  // words per thread and range
+    constexpr int kRange = kPer * kDecThreads * 32;
+    int *wpref = reinterpret_cast<int *>(bm + kPer * kDecThreads);
+    for (int c0 = 0; c0 < L; c0 += kRange) {
+        const int c1 = min(L, c0 + kRange);
         const int nw = (c1 - c0 + 31) >> 5;
-        for (int w = threadIdx.x; w < nw; w += kDecThreads) bm[w] = 0u;
+        const int per = (nw + kDecThreads - 1) / kDecThreads;
+        for (int w = threadIdx.x; w < per * kDecThreads; w += kDecThreads) bm[w] = 0u;
         __syncthreads();
-        auto mark = [&](int j) {
+        // slot of word w of this range, or -1 when position j is not kept here
+        auto slot = [&](int j) -> int {
+            if (j < lo_pos || j < c0 || j >= c1) return -1;
+            const int w = (j - c0) >> 5;
+            return (w % per) * kDecThreads + w / per;
+        };
+        auto for_each_id = [&](auto &&f) {
+            if (vec) {
+                for (int e = threadIdx.x * 4; e < topk; e += kDecThreads * 4) {
+                    const int4 v = __ldg(reinterpret_cast<const int4 *>(sel + e));
+                    f(v.x);
+                    f(v.y);
+                    f(v.z);
+                    f(v.w);
+                }
+            } else {
+                for (int e = threadIdx.x; e < topk; e += kDecThreads) f(__ldg(&sel[e]));
+            }
+        };
+        for_each_id([&](int j) {
             if (j == -1) return;
             if (j < 0 || j >= L) {
                 bad = true;
                 return;
             }
-            if (j >= lo_pos && j >= c0 && j < c1) atomicOr(&bm[(j - c0) >> 5], 1u << ((j - c0) & 31));
-        };
-        if (vec) {
-            for (int e = threadIdx.x * 4; e < topk; e += kDecThreads * 4) {
-                const int4 v = __ldg(reinterpret_cast<const int4 *>(sel + e));
-                mark(v.x);
-                mark(v.y);
-                mark(v.z);
-                mark(v.w);
-            }
-        } else {
-            for (int e = threadIdx.x; e < topk; e += kDecThreads) mark(__ldg(&sel[e]));
-        }
+            const int sl = slot(j);
+            if (sl >= 0) atomicOr(&bm[sl], 1u << ((j - c0) & 31));
+        });
         __syncthreads();
-        // Thread t owns a run of words; a CTA scan gives its first output slot.
-        const int per = (nw + kDecThreads - 1) / kDecThreads;
-        const int w0 = min(nw, (int)threadIdx.x * per), w1 = min(nw, w0 + per);
         int cnt = 0;
-        for (int w = w0; w < w1; ++w) cnt += __popc(bm[w]);
+        for (int k = 0; k < per; ++k) cnt += __popc(bm[k * kDecThreads + threadIdx.x]);
         int pos;
         const int total = cta_exclusive_scan(cnt, scratch, pos);
         pos += n;
-        for (int w = w0; w < w1; ++w) {
-            uint32_t bits = bm[w];
-            while (bits) {
-                const int bt = __ffs(bits) - 1;
-                bits &= bits - 1;
-                list[pos++] = c0 + (w << 5) + bt;
-            }
+        for (int k = 0; k < per; ++k) {
+            wpref[k * kDecThreads + threadIdx.x] = pos;
+            pos += __popc(bm[k * kDecThreads + threadIdx.x]);
         }
+        __syncthreads();
+        for_each_id([&](int j) {
+            if (j < 0 || j >= L) return;
+            const int sl = slot(j);
+            if (sl >= 0) list[wpref[sl] + __popc(bm[sl] & ((1u << ((j - c0) & 31)) - 1u))] = j;
+        });
         n += total;
-        __syncthreads();  // the bitmap is read out before the next range clears it
+        __syncthreads();  // the list is complete and the bitmap read out before the next range
     }
     return n;
 }
