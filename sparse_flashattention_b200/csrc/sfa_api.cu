@@ -77,7 +77,7 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     g.off_union = off;
     off = align_up(off + (size_t)g.tiles * g.umax * 4);
     g.off_tilectr = off;
-    off = align_up(off + 4);
+    off = align_up(off + 8);
     if (g.inv) {
         const size_t gb = (size_t)g.groups * g.nblk_max;
         g.cap_items = ((int64_t)total_q * Hkv * topk + g.Tq - 1) / g.Tq + (int64_t)gb;
@@ -169,6 +169,7 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     p.cu_q = cu_q;
     p.cu_k = cu_k ? cu_k : cu_q;
     p.sel = sel;
+    p.tile_counter = reinterpret_cast<int32_t *>(w + g.off_tilectr);
     p.batch = g.batch;
     p.Hkv = g.Hkv;
     p.topk = g.topk;
@@ -261,7 +262,6 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     p.status = status;
     p.tiles = g.tiles;
     p.tile_counter = reinterpret_cast<int32_t *>(const_cast<uint8_t *>(w) + g.off_tilectr);
-    if (cudaMemsetAsync(p.tile_counter, 0, 4, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (launch_fwd_attend(g, p, tq, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
     uint8_t *wm = static_cast<uint8_t *>(ws);

@@ -127,6 +127,20 @@ __device__ __forceinline__ void tma_load_3d(const CUtensorMap *map, uint64_t *ba
         : "memory");
 }
 
+// Programmatic dependent launch.  grid_dep_wait: wait until the grids this one depends on have
+// completed and their memory is visible (a no-op when the launch did not ask for an early start).
+// grid_dep_launch: let the next grid in the stream start its prologue now (it still waits in
+// grid_dep_wait before it reads what this grid writes).
+__device__ __forceinline__ void grid_dep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dep_launch()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Contiguous global -> shared copy through the TMA engine (16-byte aligned addresses, size a
 // multiple of 16), completing `bytes` on the mbarrier.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar)

@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(inv_smem_raw) + 1023) & ~uintptr_t(1023));
     InvMeta *meta = reinterpret_cast<InvMeta *>(smem + C::kOffMeta);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dep_wait();
     // No window went block-major: leave before any barrier or TMEM is set up (uniform exit).
     if (__ldcg(&p.ctrl->item_total) == 0) return;
 
@@ -373,6 +374,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps) fwd_merge_kernel(const FwdAt
     constexpr int kChunks = D / 8;       // 16-byte chunks of a row
     constexpr int kSplit = 32 / kChunks; // lanes sharing a chunk, each over every kSplit-th partial
     const int lane = threadIdx.x & 31;
+    grid_dep_wait();
     const int64_t u = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
     if (u >= (int64_t)p.total_q * p.Hkv) return;
     if (__ldcg(&p.ctrl->item_total) == 0) return;  // every row was written by the query-major kernel
@@ -461,7 +463,9 @@ cudaError_t launch_inv_t(const FwdGeom &g, const FwdAttendParams &p, const CUten
     }
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    fwd_attend_inv_kernel<D, BS><<<sms, kInvThreadsAttn, smem, st>>>(tq, tk, tv, p);
+    const cudaError_t le =
+        launch_kernel(fwd_attend_inv_kernel<D, BS>, dim3(sms), dim3(kInvThreadsAttn), smem, st, true, tq, tk, tv, p);
+    if (le != cudaSuccess) return le;
     return cudaGetLastError();
 }
 
@@ -477,9 +481,8 @@ cudaError_t launch_fwd_merge(const FwdGeom &g, const FwdAttendParams &p, cudaStr
 {
     const int64_t units = (int64_t)g.total_q * g.Hkv;
     const unsigned grid = (unsigned)((units + kMergeWarps - 1) / kMergeWarps);
-    if (g.d == 64) fwd_merge_kernel<64><<<grid, 32 * kMergeWarps, 0, st>>>(p);
-    else fwd_merge_kernel<128><<<grid, 32 * kMergeWarps, 0, st>>>(p);
-    return cudaGetLastError();
+    if (g.d == 64) return launch_kernel(fwd_merge_kernel<64>, dim3(grid), dim3(32 * kMergeWarps), 0, st, true, p);
+    return launch_kernel(fwd_merge_kernel<128>, dim3(grid), dim3(32 * kMergeWarps), 0, st, true, p);
 }
 
 cudaError_t launch_fwd_attend_inv(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,

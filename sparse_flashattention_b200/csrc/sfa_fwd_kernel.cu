@@ -121,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tma_prefetch_desc(&tmv);
     }
 
+    grid_dep_wait();  // everything above ran while the prep kernels were finishing
     int jbase = 0;  // blocks this CTA processed in earlier tiles
     int titer = 0;  // tiles this CTA computed (phase of q_full)
     int last_jg[kStages], last_k[kStages];  // last block whose V (K) load went into each stage
@@ -425,6 +426,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0) {  // the last CTA out leaves the tile counters cleared for the next call
+        __threadfence();
+        if (atomicAdd(&p.tile_counter[1], 1) == (int)gridDim.x - 1) {
+            p.tile_counter[0] = 0;
+            p.tile_counter[1] = 0;
+        }
+    }
+    grid_dep_launch();
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
@@ -453,8 +462,7 @@ cudaError_t launch_t(const FwdGeom &g, const FwdAttendParams &p, const CUtensorM
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = g.tiles < 2 * sms ? g.tiles : 2 * sms;
-    fwd_attend_kernel<D, BS><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    return launch_kernel(fwd_attend_kernel<D, BS>, dim3(grid), dim3(kThreads), smem, st, true, tq, tk, tv, p);
 }
 
 }  // namespace

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "sfa.h"  // include/ is on the include path
 
 namespace sfa {
@@ -52,6 +54,7 @@ struct InvItem {
 
 struct FwdPrepParams {
     const int32_t *cu_q, *cu_k, *sel;
+    int32_t *tile_counter;  // cleared here (two ints) for the attend kernel
     int batch, Hkv, topk, bs, causal, wl, wr, Tq, nqt, umax, max_sq, nblk_max;
     int32_t *sel_c, *cnt, *ucnt, *uni;
     // block-major statistics (nullptr when the schedule is off)
@@ -83,7 +86,8 @@ struct FwdAttendParams {
     const int32_t *cu_q, *cu_k;
     const int32_t *sel_c, *cnt, *ucnt, *uni;
     int batch, total_q, Hq, Hkv, G, Tq, nqt, topk, umax, tiles;
-    int32_t *tile_counter;  // next query tile to hand out (cleared before the launch)
+    int32_t *tile_counter;  // next query tile to hand out; [1] counts CTAs done.  The prep kernel
+                            // clears both; the attend kernel's last CTA clears them again.
     int causal, wl, wr;
     float scale_log2;  // softmax scale * log2(e)
     __nv_bfloat16 *out;
@@ -132,6 +136,25 @@ struct DecCombineParams {
 };
 
 // Launchers (return the launch's cudaError_t).
+// Kernel launch on `st`; with pdl the kernel may start while the previous kernel in the stream is
+// finishing (it must call grid_dep_wait() before reading that kernel's results).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 bool pdl, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = pdl ? attr : nullptr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream_t st);
 cudaError_t launch_fwd_attend(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
                               const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);

@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
 {
     extern __shared__ uint32_t prep_smem[];
     __shared__ int scan_scratch[32];
+    if (blockIdx.x == 0 && threadIdx.x < 2 && p.tile_counter) p.tile_counter[threadIdx.x] = 0;
     const int tile = blockIdx.x;
     const int hk = tile % p.Hkv;
     const int rest = tile / p.Hkv;
@@ -240,6 +241,7 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
         p.ucnt[tile] = total;
         if (p.gstat) atomicAdd(&p.gstat[grp].uni, (unsigned long long)total * ntok);
     }
+    grid_dep_launch();
 }
 
 constexpr int kInvThreads = 256;
@@ -274,6 +276,7 @@ __global__ void __launch_bounds__(kInvThreads) fwd_plan_kernel(FwdPlanParams p)
     extern __shared__ int plan_smem[];
     __shared__ int scan_scratch[32];
     __shared__ int item_base;
+    grid_dep_wait();
     const int g = blockIdx.x;
     const int hk = g % p.Hkv;
     const int b = (g / p.Hkv) % p.batch;
@@ -310,6 +313,7 @@ __global__ void __launch_bounds__(kInvThreads) fwd_plan_kernel(FwdPlanParams p)
 // the item (position / Tq) and the slot in it.
 __global__ void __launch_bounds__(kPrepThreads) fwd_scatter_kernel(FwdScatterParams p)
 {
+    grid_dep_wait();
     const int tile = blockIdx.x;
     if (p.ucnt[tile] != -1) return;
     const int hk = tile % p.Hkv;
@@ -392,14 +396,12 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
 cudaError_t launch_fwd_plan(const FwdGeom &g, const FwdPlanParams &p, cudaStream_t st)
 {
     const size_t smem = (size_t)g.nblk_max * 4;
-    fwd_plan_kernel<<<g.groups, kInvThreads, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(fwd_plan_kernel, dim3(g.groups), dim3(kInvThreads), smem, st, true, p);
 }
 
 cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cudaStream_t st)
 {
-    fwd_scatter_kernel<<<g.tiles, kPrepThreads, 0, st>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(fwd_scatter_kernel, dim3(g.tiles), dim3(kPrepThreads), 0, st, true, p);
 }
 
 cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStream_t st)
