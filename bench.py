@@ -46,11 +46,11 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 # was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
     "fwd_attend_kernel": {"files": ["sfa_fwd_kernel.cu", "sfa_device.cuh"],
-                          "sha256": "d1aa6475b8f3d0467ec50bf47ab49eac840d589f9c7c3616f0e9e18f4d058e35",
-                          "bytes": 141967616},
+                          "sha256": "e4f766c95e05cfba6b56284861b117f474e3c861c67264646270591e1e7d4a12",
+                          "bytes": 141783296},
     "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
-                            "sha256": "7c4e1665908006ce7e9e774269d385ac3d367fa37cfbd3550339a23f3e1332c5",
-                            "bytes": 274851840},
+                            "sha256": "3390aa6e8d91bd87a314c4d02435dc778f96cf7de90cf462c2b70abdaedd7897",
+                            "bytes": 274700288},
 }
 
 
