@@ -168,3 +168,17 @@ def test_full_size_decode(sfa, oracle_lib):
     rt, rc, _ = oracle_lib.decode_index(c)
     np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
     np.testing.assert_array_equal(tok_c.cpu().numpy(), rt)
+
+
+@pytest.mark.parametrize("d,L", [(64, 900000), (128, 1000000)])
+def test_long_cache_dedupe_in_several_ranges(sfa, oracle_lib, d, L):
+    """Caches close to the 2^20-position limit: the split kernel deduplicates the selection one
+    position range at a time (several ranges at these lengths)."""
+    c = W.make_decode(d + 3, 1, 4, 1, d, 256, L, L, 2048, 64, parallel_values=True)
+    _parity(sfa, oracle_lib, c)
+
+
+def test_largest_selection(sfa, oracle_lib):
+    """topk_tok = 65536, the largest this build takes (prep kernel path)."""
+    c = W.make_decode(11, 1, 2, 1, 64, 128, 70000, 70000, 65536, 128, parallel_values=True)
+    _parity(sfa, oracle_lib, c)

@@ -249,3 +249,31 @@ def test_block_major_windows(sfa, oracle_lib, Hq, Hkv, d, bs, topk, lens):
     out, lse = run_fwd(sfa, c)
     out2, lse2 = run_fwd(sfa, c)  # a repeated call on fresh buffers gives the same bits
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+@pytest.mark.parametrize("topk,lens,bs,d", [(48, [3000, 700], 32, 64), (128, [5000], 32, 128)])
+def test_long_selections_sorted_in_shared_memory(sfa, oracle_lib, topk, lens, bs, d):
+    """topk above 32: the prep sorts each selection in shared memory instead of registers;
+    topk = 128 is the largest this build takes."""
+    c = W.make_nsa_prefill(topk + bs + d, lens, 8, 2, d, bs, topk, 1, 2)
+    _full_parity(sfa, oracle_lib, c)
+    rs, rc, _ = oracle_lib.fwd_index(c)
+    d_ = upload_prefill(c)
+    _, sel_c, cnt = sfa.fwd_prep(d_["cu_q"], d_["sel"], Hq=c.Hq, d=c.d, block_size=c.bs, cu_seqlens_k=d_["cu_k"],
+                                 max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk)
+    np.testing.assert_array_equal(sel_c.cpu().numpy(), rs)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
+
+
+def test_many_key_blocks_short_queries(sfa, oracle_lib):
+    """64 queries over 100000 keys (bs 32: 3125 blocks, more than the block-major schedule takes),
+    16 blocks drawn per (token, kv head) from the bottom-right causal range."""
+    sq, sk, bs, topk, Hkv = 64, 100000, 32, 16, 2
+    rng = np.random.default_rng(5)
+    sel = np.full((sq, Hkv, topk), -1, np.int32)
+    for i in range(sq):
+        nb = (i + sk - sq) // bs + 1
+        for h in range(Hkv):
+            sel[i, h] = rng.choice(nb, size=topk, replace=False)
+    c = _case([sq], [sk], 8, Hkv, 128, bs, sel, 6)
+    _full_parity(sfa, oracle_lib, c)
