@@ -153,8 +153,8 @@ int sfa_decode_workspace_offsets(int B, int Hq, int Hkv, int d, int topk_tok, in
 
 /* Paged top-k decode = split-KV attention and LSE combine.  Each (sequence, kv head)'s
  * selection is deduplicated and sorted inside the split kernel when topk_tok <= 2048; longer
- * selections first go through the prep kernel.  The splits of one (sequence, kv head) run four
- * to a CTA; with num_splits <= 4 the CTA also merges them (one launch), otherwise a combine
+ * selections first go through the prep kernel.  The splits of one (sequence, kv head) run six
+ * to a CTA; with num_splits <= 6 the CTA also merges them (one launch), otherwise a combine
  * kernel follows.
  *   q             bf16 (B, Hq, d): the new token of each sequence, at position L_b - 1
  *   k_cache,
@@ -210,7 +210,7 @@ int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
 const char *sfa_status_string(int status);
 
 /* Number of kernel launches the last successful call on this host thread made (prefill: 2,
- * or 6 when the call can use the block-major schedule; decode: 1 with at most 4 splits, else 2,
+ * or 6 when the call can use the block-major schedule; decode: 1 with at most 6 splits, else 2,
  * plus 1 when topk_tok > 2048; a stage: its own count). */
 int sfa_last_launch_count(void);
 

@@ -1,19 +1,19 @@
 // Paged top-k decode: split-KV attention over gathered cache rows, then an LSE combine.
 //
-// Split kernel: the splits of one (sequence, kv head) run four to a CTA.  For selections of up to
+// Split kernel: the splits of one (sequence, kv head) run six to a CTA.  For selections of up to
 // 2048 positions the CTA first deduplicates its (sequence, kv head)'s selection itself: a bitmap
 // over the positions [0, L) in the (not yet used) pipeline rings, scanned into an ascending list
 // in shared memory — the same canonical list the prep kernel writes for longer selections.
 // Then every warp is an independent worker for one split: it
 // takes a contiguous chunk of the canonical (ascending) token list of its (sequence, kv head),
 // looks each token's physical row up through block_table, and streams the 256-byte K and V
-// rows of 16 tokens at a time through its own 3-stage cp.async ring in shared memory
+// rows of 16 tokens at a time through its own 2-stage cp.async ring in shared memory
 // (16-byte chunks XOR-swizzled so ldmatrix reads are bank-conflict free).  The G query heads of
 // the kv head are the rows of a warp-level bf16 MMA (m16n8k16, fp32 accumulate): decode is
 // bound by HBM bandwidth on the gathered rows, and this keeps the arithmetic to a few
 // instructions per token.  The warp keeps its own online softmax (running max rescaled only
 // when it grows by more than 2^8) and writes a normalised partial output plus its natural-log
-// LSE; no shared state with other warps, so a CTA is just four workers sharing an SM.
+// LSE; no shared state with other warps, so a CTA is just six workers sharing an SM.
 //
 // Combine kernel, one CTA per (sequence, q head): lse = log sum_s e^{lse_s};
 // out = sum_s e^{lse_s - lse} o_s (the split-KV merge named by num_splits in the
@@ -26,10 +26,10 @@ namespace sfa {
 
 namespace {
 
-constexpr int kDecWarps = 4;
+constexpr int kDecWarps = 6;
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kStageTok = 16;     // tokens per pipeline stage (one m16n8k16 K extent)
-constexpr int kDecStages = 3;     // per-warp ring depth
+constexpr int kDecStages = 2;     // per-warp ring depth: one stage in flight while the other is consumed
 constexpr int kWin = 256;         // tokens whose physical rows a warp looks up at a time
 constexpr int kFusedMaxTopk = 2048;  // the in-kernel dedupe keeps a (sequence, kv head)'s list in shared memory
 constexpr float kLn2d = 0.6931471805599453f;
@@ -369,7 +369,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
         }
     }
     if (!cta_combine) return;
-    // In-CTA LSE combine of the S <= 4 splits: lse = log sum_s e^{lse_s}; out = sum_s e^{lse_s - lse} o_s.
+    // In-CTA LSE combine of the S <= 6 splits: lse = log sum_s e^{lse_s}; out = sum_s e^{lse_s - lse} o_s.
     __syncthreads();
     const int nsp = min(p.S, kDecWarps);
     for (int e = threadIdx.x; e < p.G * D; e += kDecThreads) {

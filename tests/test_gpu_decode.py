@@ -115,10 +115,10 @@ def test_all_padding_decode(sfa):
 def _split_launches(sfa, c, num_splits=0):
     # split kernel, plus the combine kernel when the splits of a (sequence, kv head) span CTAs
     S = sfa.decode_num_splits(c.q.shape[0], c.Hq, c.Hkv, c.d, c.sel.shape[2], num_splits)
-    return 1 if S <= 4 else 2
+    return 1 if S <= 6 else 2
 
 
-@pytest.mark.parametrize("splits", [0, 4, 5, 16])
+@pytest.mark.parametrize("splits", [0, 4, 6, 7, 16])
 def test_decode_launch_count(sfa, splits):
     c = W.small_config(5)  # 256 positions per (sequence, kv head): deduplicated in the split kernel
     run_decode(sfa, c, num_splits=splits)
