@@ -306,6 +306,22 @@ __global__ void __launch_bounds__(kThreads, 2)
                     ok = warp_all(mbar_wait(&meta->s_full[jg & 1], (jg >> 1) & 1, abort_flag, p.status));
                     if (!ok) break;
                     tc_fence_after();
+                    if (!__any_sync(0xffffffffu, selected)) {
+                        // None of this warp's 32 rows selected the block: their P is zero, their running
+                        // max and sum do not change, and the scores need not be read.
+                        uint32_t zero[BS / 2];
+#pragma unroll
+                        for (int e = 0; e < BS / 2; ++e) zero[e] = 0u;
+                        if constexpr (BS == 64) {
+                            tmem_st32(lane_base + (jg & 1) * BS, zero);
+                        } else {
+                            tmem_st16(lane_base + (jg & 1) * BS, zero);
+                        }
+                        tmem_wait_st();
+                        tc_fence_before();
+                        mbar_arrive(&meta->p_full[jg & 1]);
+                        continue;
+                    }
                     float x[BS];
                     {
                         uint32_t raw[BS];
