@@ -182,3 +182,44 @@ def test_largest_selection(sfa, oracle_lib):
     """topk_tok = 65536, the largest this build takes (prep kernel path)."""
     c = W.make_decode(11, 1, 2, 1, 64, 128, 70000, 70000, 65536, 128, parallel_values=True)
     _parity(sfa, oracle_lib, c)
+
+
+def test_decode_captured_in_cuda_graph(sfa):
+    """The decode call allocates nothing and never synchronises the host, so it can be captured in a
+    CUDA graph (as the Flash-Sparse-Attention README's decode example does) and replayed: the replay
+    gives the eager call's bits, also after the inputs change in place."""
+    c = W.small_config(5)
+    d = upload_decode(c)
+    B, Hq, dd = c.q.shape
+    ws = torch.empty(sfa.decode_workspace_size(B, Hq, c.Hkv, dd, c.sel.shape[2]), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+
+    def call():
+        sfa.decode(d["q"], d["k_cache"], d["v_cache"], d["block_table"], d["cache_seqlens"], d["sel"], out=out,
+                   lse=lse, workspace=ws, window_left=c.wl, scale=c.scale if c.scale > 0 else None)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            call()
+    torch.cuda.current_stream().wait_stream(s)
+    ref_out, ref_lse = out.clone(), lse.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    assert torch.equal(lse, ref_lse)
+    # new query values in place: the replay follows them
+    d["q"].copy_(torch.flip(d["q"], dims=[0]))
+    call()
+    torch.cuda.synchronize()
+    eager = out.clone()
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), eager.view(torch.int16))

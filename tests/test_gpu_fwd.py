@@ -277,3 +277,34 @@ def test_many_key_blocks_short_queries(sfa, oracle_lib):
             sel[i, h] = rng.choice(nb, size=topk, replace=False)
     c = _case([sq], [sk], 8, Hkv, 128, bs, sel, 6)
     _full_parity(sfa, oracle_lib, c)
+
+
+def test_prefill_captured_in_cuda_graph(sfa):
+    """sfa_fwd (prep, attend and, when eligible, the block-major kernels, chained with programmatic
+    dependent launch) captured in a CUDA graph and replayed gives the eager call's bits."""
+    c = W.small_config(2)
+    d = upload_prefill(c)
+    ws = torch.empty(sfa.fwd_workspace_size(c.batch, c.max_sq, c.max_sk, c.total_q, c.Hq, c.Hkv, c.d, c.topk, c.bs),
+                     dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(d["q"])
+    lse = torch.empty((c.Hq, c.total_q), dtype=torch.float32, device="cuda")
+
+    def call():
+        run_fwd(sfa, c, d=d, out=out, lse=lse, workspace=ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(2):
+            call()
+    torch.cuda.current_stream().wait_stream(s)
+    ref_out, ref_lse = out.clone(), lse.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        call()
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref_out.view(torch.int16))
+    assert torch.equal(lse, ref_lse)
