@@ -179,8 +179,9 @@ int sfa_decode_prep(const int32_t *cache_seqlens, const int32_t *sel_tok_idx, in
                     int window_left, int num_splits,
                     void *workspace, size_t workspace_bytes, int32_t *status_dev, sfa_stream_t stream);
 
-/* Stages 2+3 alone: per-split partial attention (gather through block_table) and the
- * LSE combine, on a workspace filled by sfa_decode_prep with the same arguments. */
+/* The attention stage alone, on the canonical sets sfa_decode_prep wrote into the workspace
+ * (same arguments): the split kernel, which gathers through block_table and, with at most six
+ * splits, also merges them; beyond six splits the LSE combine kernel follows. */
 int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache,
                       const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
                       int topk_tok, int B, int Hq, int Hkv, int d, float scale, int num_splits,

@@ -303,7 +303,8 @@ def decode_prep(cache_seqlens, sel_tok_idx, *, Hq: int, d: int, max_pages_per_se
 
 def decode_attend(q, k_cache, v_cache, block_table, workspace, *, topk_tok: int, scale=None, num_splits=0, out=None,
                   lse=None, status=None, stream=None):
-    """Stages 2+3 (sfa_decode_attend) on a workspace filled by decode_prep."""
+    """sfa_decode_attend: the split kernel (and, beyond six splits, the combine kernel) on the
+    canonical sets decode_prep wrote into the workspace."""
     B, Hq, d, num_pages, page, Hkv = _dec_checks(q, k_cache, v_cache, block_table, None, None)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
