@@ -265,6 +265,7 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     if (launch_fwd_attend(g, p, tq, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
     uint8_t *wm = static_cast<uint8_t *>(ws);
+    p.q = static_cast<const __nv_bfloat16 *>(q);
     p.items = reinterpret_cast<const InvItem *>(wm + g.off_items);
     p.ctrl = reinterpret_cast<InvCtrl *>(wm + g.off_ctrl);
     p.po = reinterpret_cast<__nv_bfloat16 *>(wm + g.off_po);

@@ -13,8 +13,8 @@
 // partials: lse = log of the sum of l*2^m, out = the weighted mean of the partials.
 //
 // One persistent CTA per SM walks the item list with a fixed stride.  Warp 0 prefetches the
-// next item's record and token list, TMA-loads the K/V block and gathers the item's Q rows four
-// at a time with TMA tile::gather4 into a 128-byte-swizzled tile; warp 1 issues the MMAs; two
+// next item's record and token list, TMA-loads the K/V block and gathers the item's Q rows with
+// 16-byte cp.async copies into a 128-byte-swizzled tile; warp 1 issues the MMAs; two
 // groups of four warps alternate over items (softmax and epilogue), so one group's softmax
 // overlaps the other group's MMAs.  All waits are bounded.
 #include "sfa_device.cuh"
@@ -74,7 +74,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             mbar_init(&meta->item_free[s], 128);
         }
         for (int s = 0; s < kLoadStages; ++s) {
-            mbar_init(&meta->q_full[s], 1);
+            mbar_init(&meta->q_full[s], 32);  // one cp.async arrival per producer lane
             mbar_init(&meta->q_empty[s], 1);
             mbar_init(&meta->kv_full[s], 1);
             mbar_init(&meta->kv_empty[s], 1);
@@ -149,27 +149,28 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 }
                 issued[sl]++;
             }
-            // Q rows of the item's tokens, four rows per TMA gather into the swizzled K-major tile
-            // (row r = token * G + head; a last partial group repeats its last row).
+            // Q rows of the item's tokens (row r = token * G + head) into the 128-byte-swizzled K-major
+            // tile the MMA reads: 16-byte cp.async copies, lane l taking rows l, l+32, l+64, l+96 (rows
+            // past the item are zero-filled).  Each lane's copies land on q_full through its own arrival.
             if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
             {
                 const int rows = rec.w * p.G;
-                const int ng = (rows + 3) >> 2;
-                if (lane == 0) mbar_arrive_expect_tx(&meta->q_full[sl], (uint32_t)(ng * (D / 64)) * 512u);
-                __syncwarp();
-                for (int gi = lane; gi < ng * (D / 64); gi += 32) {
-                    const int c = gi % (D / 64), g4 = gi / (D / 64);
-                    int grow[4];
+                const uint32_t qt = smem_u32(sQ + sl * C::kQBytes);
+#pragma unroll 1
+                for (int r = lane; r < 128; r += 32) {
+                    const bool live = r < rows;
+                    const int tk = live ? r / p.G : 0, gg = live ? r - tk * p.G : 0;
+                    const __nv_bfloat16 *src =
+                        p.q + ((int64_t)(live ? (item->tok[tk] >> 7) : 0) * p.Hq + hk * p.G + gg) * D;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int rr = min(4 * g4 + u, rows - 1);
-                        const int tk = rr / p.G, gg = rr - tk * p.G;
-                        grow[u] = (item->tok[tk] >> 7) * p.Hq + hk * p.G + gg;
-                    }
-                    tma_gather4(&tmq, &meta->q_full[sl], sQ + sl * C::kQBytes + c * (128 * 128) + g4 * 512, c * 64,
-                                grow[0], grow[1], grow[2], grow[3]);
+                    for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            cp_async16(qt + c * (128 * 128) + r * 128 + ((k ^ (r & 7)) << 4), src + c * 64 + k * 8,
+                                       live ? 16u : 0u);
                 }
+                cp_async_mbar_arrive(&meta->q_full[sl]);
             }
             // Item j+4 goes into the slot item j-4 used, once its softmax group is done with it.
             if (j + kFetchAhead >= kItemSlots)
@@ -179,6 +180,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             if (lane == 0) fetch(j + kFetchAhead);
             __syncwarp();
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's Q copies have all landed
         if (*abort_flag && lane == 0) {
             for (int sl = 0; sl < kLoadStages; ++sl)
                 if (issued[sl] > 0) mbar_drain(&meta->kv_full[sl], (issued[sl] - 1) & 1);

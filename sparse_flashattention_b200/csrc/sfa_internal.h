@@ -94,6 +94,7 @@ struct FwdAttendParams {
     float *lse;
     int32_t *status;
     // block-major schedule
+    const __nv_bfloat16 *q;  // (total_q, Hq, d): the block-major kernel gathers its rows with cp.async
     const InvItem *items;
     InvCtrl *ctrl;
     __nv_bfloat16 *po;  // partial outputs, (total_q, Hq, topk, d) bf16, normalised
