@@ -46,11 +46,11 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 # was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
     "fwd_attend_kernel": {"files": ["sfa_fwd_kernel.cu", "sfa_device.cuh"],
-                          "sha256": "e4f766c95e05cfba6b56284861b117f474e3c861c67264646270591e1e7d4a12",
-                          "bytes": 141783296},
+                          "sha256": "aa012f2036c9459160b60d5349443d3075e64ae9d88bffb12d6d73fc3d7a2b5d",
+                          "bytes": 141800192},
     "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
-                            "sha256": "3390aa6e8d91bd87a314c4d02435dc778f96cf7de90cf462c2b70abdaedd7897",
-                            "bytes": 274700288},
+                            "sha256": "97cdb157c5c8fdc2494f46485bb2cc932316e20e85b4dd914934997ad8f3e280",
+                            "bytes": 274500864},
 }
 
 
