@@ -66,7 +66,13 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     g.W = g.Tq * 64;
     g.nwin = (max_sq + g.W - 1) / g.W;
     g.groups = g.nwin * batch * Hkv;
-    g.inv = (g.nblk_max <= 2048 && total_q < (1 << 24) && fwd_attend_inv_smem_bytes(g) <= 227 * 1024) ? 1 : 0;
+    // A window goes block-major only when its tiles' unions hold over 10x its selected blocks; with at
+    // most 10*topk blocks per sequence that needs most selections padded away, so the schedule (and
+    // its planning kernels) is left off.
+    g.inv = (g.nblk_max <= 2048 && g.nblk_max > 10 * topk && total_q < (1 << 24) &&
+             fwd_attend_inv_smem_bytes(g) <= 227 * 1024)
+                ? 1
+                : 0;
     size_t off = 0;
     g.off_sel_c = off;
     off = align_up(off + (size_t)total_q * Hkv * topk * 4);
