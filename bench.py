@@ -523,8 +523,8 @@ def main():
         "roofline": {"bound": "tensor", "achieved": round(r["attend_tflops"], 2), "peak": r["tf_burst"],
                      "unit": "TFLOP/s", "frac": round(r["attend_tflops"] / r["tf_burst"], 4),
                      "traffic": r["traffic"], "traffic_unit": "B per fwd_attend_kernel launch",
-                     "kernel": "fwd_attend_kernel (sfa_fwd_attend stage; its block-major kernels return at once "
-                               "on this workload)",
+                     "kernel": "fwd_attend_kernel (the sfa_fwd_attend stage, which launches only this kernel on "
+                               "this workload)",
                      "peak_source": f"{r['peak_kind']} bf16 burst",
                      "frac_of_sustained": round(r["attend_tflops"] / r["tf_sust"], 4) if r["tf_sust"] else None},
         "gpu_launches": r["launches"],
