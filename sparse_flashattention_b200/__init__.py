@@ -38,7 +38,7 @@ def lib_path() -> str:
 
 def _load():
     if not os.path.exists(_LIB_PATH):
-        raise ImportError(f"{_LIB_PATH} is missing: build it with `python -m sparse_flashattention_b200.build` "
+        raise ImportError(f"{_LIB_PATH} is missing: build it with `python sparse_flashattention_b200/build.py` "
                           "(there is no fallback implementation)")
     lib = ctypes.CDLL(_LIB_PATH)
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t

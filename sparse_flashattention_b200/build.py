@@ -1,6 +1,8 @@
 """Build libsfa.so (the CUDA kernels + C ABI) in-tree with nvcc for sm_100a.
 
-    python -m sparse_flashattention_b200.build [--force] [--verbose]
+    python sparse_flashattention_b200/build.py [--force] [--verbose]
+
+(Run it as a script, not with -m: importing the package loads the library this builds.)
 
 Each csrc/*.cu compiles to an object in _build/ (parallel nvcc processes), then one shared
 library is linked next to this file.  The CUDA runtime is linked statically, so the library
