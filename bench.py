@@ -41,13 +41,13 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant kernel of
-# each stage, from one `ncu --set full` capture (profiles/fwd_attend_kernel_nsa_varlen_16k.md and
+# each stage, from one `ncu --set full` capture (profiles/fwd_attend_pipe_kernel_nsa_varlen_16k.md and
 # profiles/decode_split_kernel_paged_topk_decode.md).  A figure holds only for the kernel sources it
 # was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
-    "fwd_attend_kernel": {"files": ["sfa_fwd_kernel.cu", "sfa_device.cuh"],
-                          "sha256": "aa012f2036c9459160b60d5349443d3075e64ae9d88bffb12d6d73fc3d7a2b5d",
-                          "bytes": 141800192},
+    "fwd_attend_pipe_kernel": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
+                               "sha256": "",
+                               "bytes": None},
     "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
                             "sha256": "97cdb157c5c8fdc2494f46485bb2cc932316e20e85b4dd914934997ad8f3e280",
                             "bytes": 274500864},
@@ -449,7 +449,7 @@ def run_gpu(args, rank, world, local_rank):
                 dec_gbs=dec_gbs, dec_attend_gbs=dec_attend_gbs, flops=flops, gbytes=gbytes, clocks=clocks,
                 launches=n_launch, e2e=e2e, hbm=hbm, tf_burst=tf_burst, tf_sust=tf_sust, peak_kind=peak_kind,
                 pc=pc, dc=dc,
-                traffic=args.traffic if args.traffic is not None else kernel_traffic("fwd_attend_kernel"),
+                traffic=args.traffic if args.traffic is not None else kernel_traffic("fwd_attend_pipe_kernel"),
                 dec_traffic=kernel_traffic("decode_split_kernel"))
 
 
@@ -522,8 +522,8 @@ def main():
                                 "peak_source": r["peak_kind"]}},
         "roofline": {"bound": "tensor", "achieved": round(r["attend_tflops"], 2), "peak": r["tf_burst"],
                      "unit": "TFLOP/s", "frac": round(r["attend_tflops"] / r["tf_burst"], 4),
-                     "traffic": r["traffic"], "traffic_unit": "B per fwd_attend_kernel launch",
-                     "kernel": "fwd_attend_kernel (the sfa_fwd_attend stage, which launches only this kernel on "
+                     "traffic": r["traffic"], "traffic_unit": "B per fwd_attend_pipe_kernel launch",
+                     "kernel": "fwd_attend_pipe_kernel (the sfa_fwd_attend stage, which launches only this kernel on "
                                "this workload)",
                      "peak_source": f"{r['peak_kind']} bf16 burst",
                      "frac_of_sustained": round(r["attend_tflops"] / r["tf_sust"], 4) if r["tf_sust"] else None},

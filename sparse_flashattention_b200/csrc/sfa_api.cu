@@ -236,7 +236,8 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
                     const int32_t *cu_k, int total_k, int causal, int wl, int wr, float scale, void *ws,
                     int32_t *status, void *out, float *lse, cudaStream_t st)
 {
-    if (fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    const bool pipe = fwd_pipe_fits(g);
+    if (!pipe && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     CUtensorMap tq, tk, tv;
     if (!encode_3d(tq, q, g.d, g.Hq, g.total_q, g.G, g.Tq)) return SFA_ERR_CUDA;
     if (!encode_3d(tk, k, g.d, g.Hkv, total_k, 1, g.bs)) return SFA_ERR_CUDA;
@@ -268,7 +269,9 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     p.status = status;
     p.tiles = g.tiles;
     p.tile_counter = reinterpret_cast<int32_t *>(const_cast<uint8_t *>(w) + g.off_tilectr);
-    if (launch_fwd_attend(g, p, tq, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
+    if ((pipe ? launch_fwd_attend_pipe(g, p, tq, tk, tv, st) : launch_fwd_attend(g, p, tq, tk, tv, st)) !=
+        cudaSuccess)
+        return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
     uint8_t *wm = static_cast<uint8_t *>(ws);
     p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -494,7 +497,7 @@ int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqle
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
     if (total_k == 0) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
-    if (fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    if (!fwd_pipe_fits(g) && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     rc = fwd_prep_impl(g, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
                        status_dev, stream);
     if (rc != SFA_OK) return rc;

@@ -160,6 +160,12 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
 cudaError_t launch_fwd_attend(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
                               const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 size_t fwd_attend_smem_bytes(const FwdGeom &g);
+// Pipelined query-major kernel (tile switches overlapped with the previous tile's tail): whether
+// its shared memory (which holds two copies of a tile's union) fits two CTAs per SM for this
+// geometry; when it does not, fwd_attend_kernel runs instead.
+bool fwd_pipe_fits(const FwdGeom &g);
+cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
+                                   const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 cudaError_t launch_fwd_plan(const FwdGeom &g, const FwdPlanParams &p, cudaStream_t st);
 cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cudaStream_t st);
 cudaError_t launch_fwd_attend_inv(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,

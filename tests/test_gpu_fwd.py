@@ -265,17 +265,20 @@ def test_long_selections_sorted_in_shared_memory(sfa, oracle_lib, topk, lens, bs
     np.testing.assert_array_equal(cnt.cpu().numpy(), rc)
 
 
-def test_many_key_blocks_short_queries(sfa, oracle_lib):
+@pytest.mark.parametrize("sk,bs,topk,Hq,Hkv", [(100000, 32, 16, 8, 2), (131072, 64, 32, 2, 2)])
+def test_many_key_blocks_short_queries(sfa, oracle_lib, sk, bs, topk, Hq, Hkv):
     """64 queries over 100000 keys (bs 32: 3125 blocks, more than the block-major schedule takes),
-    16 blocks drawn per (token, kv head) from the bottom-right causal range."""
-    sq, sk, bs, topk, Hkv = 64, 100000, 32, 16, 2
+    blocks drawn per (token, kv head) from the bottom-right causal range.  The second case (one q
+    head per kv head, 128-token tiles, top-32 of 2048 blocks) gives tile unions of up to 2048 blocks,
+    too many for the pipelined query-major kernel's shared memory: the one-tile kernel runs it."""
+    sq = 64
     rng = np.random.default_rng(5)
     sel = np.full((sq, Hkv, topk), -1, np.int32)
     for i in range(sq):
         nb = (i + sk - sq) // bs + 1
         for h in range(Hkv):
             sel[i, h] = rng.choice(nb, size=topk, replace=False)
-    c = _case([sq], [sk], 8, Hkv, 128, bs, sel, 6)
+    c = _case([sq], [sk], Hq, Hkv, 128, bs, sel, 6)
     _full_parity(sfa, oracle_lib, c)
 
 
