@@ -264,16 +264,31 @@ def run_gpu(args, rank, world, local_rank):
                       device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     launches = [0]
+    # When the call needs no block-major plan, sfa_fwd is one kernel that canonicalizes the
+    # selections itself; time that whole call.  Otherwise time the prep and attention stages.
+    sfa.fwd(P["q"], P["k"], P["v"], P["cu_q"], P["sel"], pc.bs, cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq,
+            max_seqlen_k=pc.max_sk, causal=bool(pc.causal), window=(pc.wl, pc.wr), out=out, lse=lse, workspace=ws,
+            status=status)
+    fused = sfa.last_launch_count() == 1
 
-    def prefill_prep():
+    def prefill_prep():  # staged path only (the block-major schedule needs the prep kernel's plan)
+        if fused:
+            return
         sfa.fwd_prep(P["cu_q"], P["sel"], Hq=pc.Hq, d=pc.d, block_size=pc.bs, cu_seqlens_k=P["cu_k"],
-                     max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, workspace=ws, status=status)
+                     max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, causal=bool(pc.causal), window=(pc.wl, pc.wr),
+                     workspace=ws, status=status)
         launches[0] += sfa.last_launch_count()
 
     def prefill_attend():
+        if fused:  # the whole public call: one kernel canonicalizes the selections and attends
+            sfa.fwd(P["q"], P["k"], P["v"], P["cu_q"], P["sel"], pc.bs, cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq,
+                    max_seqlen_k=pc.max_sk, causal=bool(pc.causal), window=(pc.wl, pc.wr), out=out, lse=lse,
+                    workspace=ws, status=status)
+            launches[0] += sfa.last_launch_count()
+            return
         sfa.fwd_attend(P["q"], P["k"], P["v"], P["cu_q"], ws, topk=pc.topk, block_size=pc.bs,
-                       cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, out=out, lse=lse,
-                       status=status)
+                       cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, causal=bool(pc.causal),
+                       window=(pc.wl, pc.wr), out=out, lse=lse, status=status)
         launches[0] += sfa.last_launch_count()
 
     def decode_prep():  # selections this short are deduplicated inside the split kernel: no stage
@@ -444,7 +459,7 @@ def run_gpu(args, rank, world, local_rank):
                        "copies of neighbouring steps overlapping the compute on separate streams (two device "
                        "buffer sets); the decode KV cache is resident state, its per-step inputs are q, "
                        "block_table, cache_seqlens, sel_tok_idx"}
-    return dict(value=value, prefill_ms=prefill_ms, prep_ms=pp_ms, attend_ms=pa_ms, decode_ms=decode_ms,
+    return dict(value=value, fused=fused, prefill_ms=prefill_ms, prep_ms=pp_ms, attend_ms=pa_ms, decode_ms=decode_ms,
                 dprep_ms=dp_ms, dattend_ms=da_ms, step_ms=step_ms, region_ms=region_ms, attend_tflops=attend_tflops,
                 dec_gbs=dec_gbs, dec_attend_gbs=dec_attend_gbs, flops=flops, gbytes=gbytes, clocks=clocks,
                 launches=n_launch, e2e=e2e, hbm=hbm, tf_burst=tf_burst, tf_sust=tf_sust, peak_kind=peak_kind,
@@ -523,8 +538,10 @@ def main():
         "roofline": {"bound": "tensor", "achieved": round(r["attend_tflops"], 2), "peak": r["tf_burst"],
                      "unit": "TFLOP/s", "frac": round(r["attend_tflops"] / r["tf_burst"], 4),
                      "traffic": r["traffic"], "traffic_unit": "B per fwd_attend_pipe_kernel launch",
-                     "kernel": "fwd_attend_pipe_kernel (the sfa_fwd_attend stage, which launches only this kernel on "
-                               "this workload)",
+                     "kernel": ("fwd_attend_pipe_kernel (the whole sfa_fwd call: one launch canonicalizes the "
+                                "selections and attends)") if r["fused"] else
+                               ("fwd_attend_pipe_kernel (the sfa_fwd_attend stage, which launches only this kernel "
+                                "on this workload)"),
                      "peak_source": f"{r['peak_kind']} bf16 burst",
                      "frac_of_sustained": round(r["attend_tflops"] / r["tf_sust"], 4) if r["tf_sust"] else None},
         "gpu_launches": r["launches"],

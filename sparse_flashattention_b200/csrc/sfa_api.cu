@@ -232,11 +232,16 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     return launch_fwd_scatter(g, sc, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
 }
 
+// The attention stage.  sel == nullptr: the canonical sets come from the prep kernel's output in
+// the workspace.  sel != nullptr (fused, only without the block-major schedule): the pipelined
+// kernel canonicalizes the raw selections itself and the prep kernel does not run.
 int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *v, const int32_t *cu_q,
                     const int32_t *cu_k, int total_k, int causal, int wl, int wr, float scale, void *ws,
-                    int32_t *status, void *out, float *lse, cudaStream_t st)
+                    int32_t *status, void *out, float *lse, cudaStream_t st, const int32_t *sel = nullptr)
 {
-    const bool pipe = fwd_pipe_fits(g);
+    const bool fused = sel != nullptr;
+    const bool pipe = fwd_pipe_fits(g, fused);
+    if (fused && (!pipe || g.inv)) return SFA_ERR_UNSUPPORTED;
     if (!pipe && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     CUtensorMap tq, tk, tv;
     if (!encode_3d(tq, q, g.d, g.Hq, g.total_q, g.G, g.Tq)) return SFA_ERR_CUDA;
@@ -269,7 +274,12 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     p.status = status;
     p.tiles = g.tiles;
     p.tile_counter = reinterpret_cast<int32_t *>(const_cast<uint8_t *>(w) + g.off_tilectr);
-    if ((pipe ? launch_fwd_attend_pipe(g, p, tq, tk, tv, st) : launch_fwd_attend(g, p, tq, tk, tv, st)) !=
+    p.sel = sel;
+    p.bs = g.bs;
+    p.max_sq = g.max_sq;
+    p.nblk_max = g.nblk_max;
+    if (fused && cudaMemsetAsync(p.tile_counter, 0, 2 * sizeof(int32_t), st) != cudaSuccess) return SFA_ERR_CUDA;
+    if ((pipe ? launch_fwd_attend_pipe(g, p, fused, tq, tk, tv, st) : launch_fwd_attend(g, p, tq, tk, tv, st)) !=
         cudaSuccess)
         return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
@@ -497,7 +507,14 @@ int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqle
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
     if (total_k == 0) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
-    if (!fwd_pipe_fits(g) && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    if (!fwd_pipe_fits(g, false) && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    if (!g.inv && fwd_pipe_fits(g, true)) {
+        // One launch: the attention kernel canonicalizes each tile's selections itself.
+        rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right,
+                             scale, workspace, status_dev, out, lse, stream, sel_idx);
+        if (rc == SFA_OK) g_last_launches = 1;
+        return rc;
+    }
     rc = fwd_prep_impl(g, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
                        status_dev, stream);
     if (rc != SFA_OK) return rc;

@@ -411,6 +411,82 @@ __device__ __forceinline__ float scores_to_p(const float (&x)[BS], float sc, flo
 }
 
 // ---------------------------------------------------------------------------------------
+// Canonical block list of one (token, kv head) selection
+// ---------------------------------------------------------------------------------------
+// The kept ids of raw[0..topk) — not -1, inside [0, nblk), and naming a block [s*bs, s*bs+bs) ∩
+// [0, sk) that holds at least one key in [lo, hi] — ascending and without duplicates, written to
+// dst[0], dst[stride], ...; returns their number.  Ids that are neither -1 nor in [0, nblk) set
+// `bad`.  Register bitonic network for topk <= N (N a power of two).
+template <int N>
+__device__ __forceinline__ int canon_list_regs(const int *raw, int topk, int nblk, int bs, int sk, int lo, int hi,
+                                               int *dst, int stride, bool &bad)
+{
+    int v[N];
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+        const int s = e < topk ? raw[e] : -1;
+        int key = 0x7fffffff;
+        if (s != -1) {
+            if (s < 0 || s >= nblk) {
+                bad = true;
+            } else {
+                const int bl = s * bs, bh = min(bl + bs, sk) - 1;
+                if (max(bl, lo) <= min(bh, hi)) key = s;  // some key of this block survives the mask
+            }
+        }
+        v[e] = key;
+    }
+#pragma unroll
+    for (int k = 2; k <= N; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1)
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const int a = v[i], b = v[l];
+                    const bool up = (i & k) == 0;
+                    v[i] = up ? min(a, b) : max(a, b);
+                    v[l] = up ? max(a, b) : min(a, b);
+                }
+            }
+    int n = 0, prev = -1;
+#pragma unroll
+    for (int e = 0; e < N; ++e) {
+        if (v[e] != 0x7fffffff && v[e] != prev) {
+            dst[n * stride] = v[e];
+            ++n;
+        }
+        prev = v[e];
+    }
+    return n;
+}
+
+// Same result for any topk: insertion into the ascending list dst (which must be writable scratch).
+__device__ __forceinline__ int canon_list_insert(const int *raw, int topk, int nblk, int bs, int sk, int lo, int hi,
+                                                 int *dst, int stride, bool &bad)
+{
+    int n = 0;
+    for (int e = 0; e < topk; ++e) {
+        const int s = raw[e];
+        if (s == -1) continue;
+        if (s < 0 || s >= nblk) {
+            bad = true;
+            continue;
+        }
+        const int bl = s * bs, bh = min(bl + bs, sk) - 1;
+        if (max(bl, lo) > min(bh, hi)) continue;  // no key of this block survives the mask
+        int pos = n;
+        while (pos > 0 && dst[(pos - 1) * stride] > s) --pos;
+        if (pos > 0 && dst[(pos - 1) * stride] == s) continue;
+        for (int m = n; m > pos; --m) dst[m * stride] = dst[(m - 1) * stride];
+        dst[pos * stride] = s;
+        ++n;
+    }
+    return n;
+}
+
+// ---------------------------------------------------------------------------------------
 // Ampere-style async copy and warp-level MMA (used by the HBM-bound decode kernel)
 // ---------------------------------------------------------------------------------------
 // 16-byte global->shared copy; src_bytes = 0 writes zeros instead of reading.

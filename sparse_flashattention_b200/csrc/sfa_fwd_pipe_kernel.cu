@@ -35,7 +35,7 @@ namespace sfa {
 
 namespace {
 
-constexpr int kQThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2..5 softmax / epilogue
+constexpr int kQThreads = 224;  // warp 0 producer, warp 1 MMA, warps 2..5 softmax / epilogue, warp 6 index
 constexpr int kQStages = 2;     // K and V ring depth (two CTAs per SM bound the shared memory)
 constexpr float kQRescaleLog2 = 8.0f;
 constexpr float kQLn2 = 0.6931471805599453f;
@@ -73,13 +73,26 @@ struct QMeta {
     TileInfo info[2];
 };
 
-template <int D, int BS>
-__host__ __device__ constexpr size_t pipe_smem_bytes(int umax)
-{
-    return 1024 + QCfg<D, BS>::kOffMeta + ((sizeof(QMeta) + 15) & ~size_t(15)) + (size_t)2 * umax * 4;
-}
+// Shared memory after the Q tile and the K/V rings: the barriers, two copies of a tile's union
+// ([2][umax]) and, in the fused mode, two copies of the tile's canonical lists ([2][Tq][topk]),
+// their counts ([2][Tq]) and the union bitmap (one bit per key block).
+struct QLayout {
+    size_t off_union, off_lists, off_cnts, off_bm, bytes;
+};
 
 template <int D, int BS>
+__host__ __device__ inline QLayout pipe_layout(bool fused, int umax, int Tq, int topk, int nblk_max)
+{
+    QLayout l;
+    l.off_union = QCfg<D, BS>::kOffMeta + ((sizeof(QMeta) + 15) & ~size_t(15));
+    l.off_lists = l.off_union + (size_t)2 * umax * 4;
+    l.off_cnts = l.off_lists + (fused ? (size_t)2 * Tq * topk * 4 : 0);
+    l.off_bm = l.off_cnts + (fused ? (size_t)2 * Tq * 4 : 0);
+    l.bytes = l.off_bm + (fused ? (size_t)(nblk_max + 31) / 32 * 4 : 0);
+    return l;
+}
+
+template <int D, int BS, bool FUSED>
 __global__ void __launch_bounds__(kQThreads, 2)
     fwd_attend_pipe_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv, const FwdAttendParams p)
@@ -89,8 +102,12 @@ __global__ void __launch_bounds__(kQThreads, 2)
     uint8_t *smem =
         reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pipe_smem_raw) + 1023) & ~uintptr_t(1023));
     const int U = p.umax;
+    const QLayout L = pipe_layout<D, BS>(FUSED, U, p.Tq, p.topk, p.nblk_max);
     QMeta *meta = reinterpret_cast<QMeta *>(smem + C::kOffMeta);
-    int *s_union = reinterpret_cast<int *>(smem + C::kOffMeta + ((sizeof(QMeta) + 15) & ~size_t(15)));  // [2][U]
+    int *s_union = reinterpret_cast<int *>(smem + L.off_union);   // [2][U]
+    int *s_lists = reinterpret_cast<int *>(smem + L.off_lists);   // fused: [2][Tq][topk]
+    int *s_cnts = reinterpret_cast<int *>(smem + L.off_cnts);     // fused: [2][Tq]
+    uint32_t *s_bm = reinterpret_cast<uint32_t *>(smem + L.off_bm);  // fused: union bitmap
     uint8_t *sQ = smem;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
@@ -110,8 +127,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
             mbar_init(&meta->s_full[s], 1);
             mbar_init(&meta->p_full[s], 128);
             mbar_init(&meta->pv_done[s], 1);
-            mbar_init(&meta->meta_full[s], 32);  // every producer lane arrives after its writes
-            mbar_init(&meta->meta_empty[s], 5);  // the 4 softmax warps + the MMA thread
+            mbar_init(&meta->meta_full[s], 32);  // every index-warp lane arrives after its writes
+            mbar_init(&meta->meta_empty[s], 6);  // the 4 softmax warps, the MMA thread, the producer
         }
         mbar_init(&meta->o_free, 128);
         mbar_init(&meta->drain, 1);
@@ -136,10 +153,11 @@ __global__ void __launch_bounds__(kQThreads, 2)
 
     // Tile k uses metadata buffer k & 1; barrier phases of the rings run on a per-CTA count of
     // blocks (jg), so the pipeline carries over from tile to tile.
-    if (warp == 0) {
-        // ------------------------------------------------------------------ producer
-        int k_st = 0, k_ph = 0, nk = 0, v_st = 0, v_ph = 0, nv = 0;  // ring stage, phase, loads issued
-        int q_phases = 0;                                            // Q phases issued
+    if (warp == 6) {
+        // ------------------------------------------------------------------ index warp
+        // Runs a tile ahead of the producer: takes the next tile from the counter, builds (fused
+        // mode) or copies its block union and canonical lists into metadata buffer k & 1, and
+        // publishes them.
         int k = 0;
         bool ok = true;
         while (ok) {
@@ -173,9 +191,65 @@ __global__ void __launch_bounds__(kQThreads, 2)
             const int k0 = p.cu_k[b], sk = p.cu_k[b + 1] - k0;
             const int tok0 = qt * p.Tq;
             const int ntok = min(p.Tq, sq - tok0);
-            const int nU = p.ucnt[tile];
-            const int n = max(nU, 0);
-            for (int i = lane; i < n; i += 32) uni[i] = p.uni[(int64_t)tile * U + i];
+            int nU;
+            if constexpr (FUSED) {
+                // The tile's canonical lists (one token per lane at a time) and the ascending union
+                // of their blocks, built here instead of by a prep kernel.
+                int *lists = s_lists + m * p.Tq * p.topk;
+                int *cnts = s_cnts + m * p.Tq;
+                int nblk = (sk + BS - 1) / BS;
+                if (sq > p.max_sq || nblk > p.nblk_max) {  // lengths beyond the caller's max_seqlen bounds
+                    if (lane == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_SEQLEN);
+                    nblk = min(nblk, p.nblk_max);
+                }
+                const int words = (nblk + 31) >> 5;
+                for (int w = lane; w < words; w += 32) s_bm[w] = 0u;
+                __syncwarp();
+                bool bad = false;
+                const int delta = sk - sq;
+                for (int tt = lane; tt < ntok; tt += 32) {
+                    const int i = tok0 + tt;
+                    int lo = 0, hi = sk - 1;
+                    if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
+                    if (p.causal) hi = min(hi, i + delta);
+                    if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
+                    const int *raw = p.sel + ((int64_t)(q0 + i) * p.Hkv + hk) * p.topk;
+                    int *dst = lists + tt * p.topk;
+                    int cn;
+                    if (p.topk <= 16) cn = canon_list_regs<16>(raw, p.topk, nblk, BS, sk, lo, hi, dst, 1, bad);
+                    else if (p.topk <= 32) cn = canon_list_regs<32>(raw, p.topk, nblk, BS, sk, lo, hi, dst, 1, bad);
+                    else cn = canon_list_insert(raw, p.topk, nblk, BS, sk, lo, hi, dst, 1, bad);
+                    cnts[tt] = cn;
+                    for (int e = 0; e < cn; ++e) atomicOr(&s_bm[dst[e] >> 5], 1u << (dst[e] & 31));
+                }
+                if (__any_sync(full, bad) && lane == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_INDEX);
+                __syncwarp();
+                // Bitmap -> ascending ids: 32 words at a time, word w of a chunk to lane w, a warp scan
+                // of the bit counts places each word's ids.
+                int total = 0;
+                for (int c0 = 0; c0 < words; c0 += 32) {
+                    const int w = c0 + lane;
+                    uint32_t bits = w < words ? s_bm[w] : 0u;
+                    const int c = __popc(bits);
+                    int incl = c;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int y = __shfl_up_sync(full, incl, o);
+                        if (lane >= o) incl += y;
+                    }
+                    int pos = total + incl - c;
+                    while (bits) {
+                        const int bit = __ffs(bits) - 1;
+                        bits &= bits - 1;
+                        uni[pos++] = w * 32 + bit;
+                    }
+                    total += __shfl_sync(full, incl, 31);
+                }
+                nU = total;
+            } else {
+                nU = p.ucnt[tile];
+                for (int i = lane; i < nU; i += 32) uni[i] = p.uni[(int64_t)tile * U + i];
+            }
             if (lane == 0) {
                 ti.done = 0;
                 ti.nU = nU;
@@ -189,8 +263,23 @@ __global__ void __launch_bounds__(kQThreads, 2)
                 ti.ntok = ntok;
             }
             mbar_arrive(&meta->meta_full[m]);
-
-            if (lane == 0) {
+            ++k;
+        }
+    } else if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        int k_st = 0, k_ph = 0, nk = 0, v_st = 0, v_ph = 0, nv = 0;  // ring stage, phase, loads issued
+        int q_phases = 0;                                            // Q phases issued
+        if (lane == 0) {
+            int k = 0;
+            bool ok = true;
+            while (ok) {
+                const int m = k & 1;
+                ok = mbar_wait(&meta->meta_full[m], (k >> 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                const TileInfo &ti = meta->info[m];
+                if (ti.done) break;
+                const int *uni = s_union + m * U;
+                const int n = max(ti.nU, 0), hk = ti.hk, q0 = ti.q0, k0 = ti.k0, tok0 = ti.tok0;
                 // Q, once the previous tile's score MMAs no longer read it (a box of Tq tokens x
                 // G heads, Tq*G <= 128 rows).
                 if (k >= 1) ok = mbar_wait(&meta->q_empty, (k - 1) & 1, abort_flag, p.status);
@@ -240,9 +329,10 @@ __global__ void __launch_bounds__(kQThreads, 2)
                         else if (!load_v(u)) ok = false;
                     }
                 }
+                if (!ok) break;
+                mbar_arrive(&meta->meta_empty[m]);
+                ++k;
             }
-            ok = __shfl_sync(full, ok ? 1 : 0, 0) != 0;
-            ++k;
         }
         if (*abort_flag && lane == 0) {  // wind down: let every copy this CTA started land
             if (q_phases > 0) mbar_drain(&meta->q_full, (q_phases - 1) & 1);
@@ -390,12 +480,13 @@ __global__ void __launch_bounds__(kQThreads, 2)
             if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
             if (p.causal) hi = min(hi, i + delta);
             if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
-            // This row's canonical (ascending) block list, read from global memory one entry
-            // ahead of its use.
+            // This row's canonical (ascending) block list: in shared memory (fused mode), else read
+            // from the prep kernel's output in global memory one entry ahead of its use.
             const int64_t t = (int64_t)q0 + i;
-            const int32_t *gl = p.sel_c + (row_valid ? (t * p.Hkv + hk) * p.topk : 0);
-            const int mycnt = row_valid ? p.cnt[t * p.Hkv + hk] : 0;
-            int nxt = mycnt > 0 ? gl[0] : -1;
+            const int *mylist = s_lists + (m * p.Tq + (row_valid ? tok : 0)) * p.topk;
+            const int32_t *gl = p.sel_c + (row_valid && !FUSED ? (t * p.Hkv + hk) * p.topk : 0);
+            const int mycnt = !row_valid ? 0 : FUSED ? s_cnts[m * p.Tq + tok] : p.cnt[t * p.Hkv + hk];
+            int nxt = (!FUSED && mycnt > 0) ? gl[0] : -1;
             int ptr = 0;
             float m_run = -INFINITY;  // running max of s*scale*log2e
             float l_run = 0.f;
@@ -403,10 +494,16 @@ __global__ void __launch_bounds__(kQThreads, 2)
             for (int j = 0; j < n; ++j) {
                 const int jg = jg0 + j;
                 const int s = uni[j];
-                const bool selected = nxt == s;
-                if (selected) {
-                    ++ptr;
-                    nxt = ptr < mycnt ? gl[ptr] : -1;
+                bool selected;
+                if constexpr (FUSED) {
+                    selected = ptr < mycnt && mylist[ptr] == s;
+                    if (selected) ++ptr;
+                } else {
+                    selected = nxt == s;
+                    if (selected) {
+                        ++ptr;
+                        nxt = ptr < mycnt ? gl[ptr] : -1;
+                    }
                 }
                 ok = warp_all_ok(mbar_wait(&meta->s_full[jg & 1], (jg >> 1) & 1, abort_flag, p.status));
                 if (!ok) break;
@@ -552,14 +649,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
     }
 }
 
-template <int D, int BS>
-cudaError_t launch_pipe_t(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq, const CUtensorMap &tk,
-                          const CUtensorMap &tv, cudaStream_t st)
+template <int D, int BS, bool FUSED>
+cudaError_t launch_pipe_t(const FwdAttendParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                          cudaStream_t st)
 {
-    const size_t smem = pipe_smem_bytes<D, BS>(p.umax);
+    const size_t smem = 1024 + pipe_layout<D, BS>(FUSED, p.umax, p.Tq, p.topk, p.nblk_max).bytes;
     static int configured = 0;
     if ((int)smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_attend_pipe_kernel<D, BS>,
+        cudaError_t e = cudaFuncSetAttribute(fwd_attend_pipe_kernel<D, BS, FUSED>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         configured = (int)smem;
@@ -567,26 +664,38 @@ cudaError_t launch_pipe_t(const FwdGeom &g, const FwdAttendParams &p, const CUte
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = p.tiles < 2 * sms ? p.tiles : 2 * sms;
-    return launch_kernel(fwd_attend_pipe_kernel<D, BS>, dim3(grid > 0 ? grid : 1), dim3(kQThreads), smem, st, true,
-                         tq, tk, tv, p);
+    // The fused mode follows a memset of the tile counter, not a kernel: no early start.
+    return launch_kernel(fwd_attend_pipe_kernel<D, BS, FUSED>, dim3(grid > 0 ? grid : 1), dim3(kQThreads), smem, st,
+                         !FUSED, tq, tk, tv, p);
+}
+
+template <int D, int BS>
+cudaError_t launch_pipe_d(const FwdAttendParams &p, bool fused, const CUtensorMap &tq, const CUtensorMap &tk,
+                          const CUtensorMap &tv, cudaStream_t st)
+{
+    return fused ? launch_pipe_t<D, BS, true>(p, tq, tk, tv, st) : launch_pipe_t<D, BS, false>(p, tq, tk, tv, st);
 }
 
 }  // namespace
 
-bool fwd_pipe_fits(const FwdGeom &g)
+bool fwd_pipe_fits(const FwdGeom &g, bool fused)
 {
-    size_t b;
-    if (g.d == 64) b = g.bs == 32 ? pipe_smem_bytes<64, 32>(g.umax) : pipe_smem_bytes<64, 64>(g.umax);
-    else b = g.bs == 32 ? pipe_smem_bytes<128, 32>(g.umax) : pipe_smem_bytes<128, 64>(g.umax);
-    return b <= kQMaxSmem;
+    QLayout l;
+    if (g.d == 64)
+        l = g.bs == 32 ? pipe_layout<64, 32>(fused, g.umax, g.Tq, g.topk, g.nblk_max)
+                       : pipe_layout<64, 64>(fused, g.umax, g.Tq, g.topk, g.nblk_max);
+    else
+        l = g.bs == 32 ? pipe_layout<128, 32>(fused, g.umax, g.Tq, g.topk, g.nblk_max)
+                       : pipe_layout<128, 64>(fused, g.umax, g.Tq, g.topk, g.nblk_max);
+    return 1024 + l.bytes <= kQMaxSmem;
 }
 
-cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
+cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, bool fused, const CUtensorMap &tq,
                                    const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
 {
     if (g.d == 64)
-        return g.bs == 32 ? launch_pipe_t<64, 32>(g, p, tq, tk, tv, st) : launch_pipe_t<64, 64>(g, p, tq, tk, tv, st);
-    return g.bs == 32 ? launch_pipe_t<128, 32>(g, p, tq, tk, tv, st) : launch_pipe_t<128, 64>(g, p, tq, tk, tv, st);
+        return g.bs == 32 ? launch_pipe_d<64, 32>(p, fused, tq, tk, tv, st) : launch_pipe_d<64, 64>(p, fused, tq, tk, tv, st);
+    return g.bs == 32 ? launch_pipe_d<128, 32>(p, fused, tq, tk, tv, st) : launch_pipe_d<128, 64>(p, fused, tq, tk, tv, st);
 }
 
 }  // namespace sfa

@@ -86,6 +86,9 @@ struct FwdAttendParams {
     const int32_t *cu_q, *cu_k;
     const int32_t *sel_c, *cnt, *ucnt, *uni;
     int batch, total_q, Hq, Hkv, G, Tq, nqt, topk, umax, tiles;
+    // Selections as given (the pipelined kernel's fused mode canonicalizes them itself)
+    const int32_t *sel;
+    int bs, max_sq, nblk_max;
     int32_t *tile_counter;  // next query tile to hand out; [1] counts CTAs done.  The prep kernel
                             // clears both; the attend kernel's last CTA clears them again.
     int causal, wl, wr;
@@ -163,8 +166,10 @@ size_t fwd_attend_smem_bytes(const FwdGeom &g);
 // Pipelined query-major kernel (tile switches overlapped with the previous tile's tail): whether
 // its shared memory (which holds two copies of a tile's union) fits two CTAs per SM for this
 // geometry; when it does not, fwd_attend_kernel runs instead.
-bool fwd_pipe_fits(const FwdGeom &g);
-cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, const CUtensorMap &tq,
+// fused: the kernel builds each tile's canonical lists and union from the raw selections itself
+// (no prep kernel; the caller clears the tile counter), for calls without the block-major schedule.
+bool fwd_pipe_fits(const FwdGeom &g, bool fused);
+cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, bool fused, const CUtensorMap &tq,
                                    const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 cudaError_t launch_fwd_plan(const FwdGeom &g, const FwdPlanParams &p, cudaStream_t st);
 cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cudaStream_t st);

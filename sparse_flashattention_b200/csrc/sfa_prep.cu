@@ -85,54 +85,6 @@ __device__ __forceinline__ int warp_aggregated_add(int *counters, int key)
     return base + rank;
 }
 
-// Canonical list of one token's selection when topk <= N: the kept ids (others -> INT_MAX) are
-// sorted in registers by a bitonic network, duplicates dropped, and the result written to column
-// `col` of lists ([slot][kPrepThreads]).  Returns the count.
-template <int N>
-__device__ __forceinline__ int canon_in_registers(const int *raw, int topk, int nblk, int bs, int sk, int lo, int hi,
-                                                  int *lists, int col, bool &bad)
-{
-    int v[N];
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-        const int s = e < topk ? raw[e] : -1;
-        int key = INT_MAX;
-        if (s != -1) {
-            if (s < 0 || s >= nblk) {
-                bad = true;
-            } else {
-                const int bl = s * bs, bh = min(bl + bs, sk) - 1;
-                if (max(bl, lo) <= min(bh, hi)) key = s;  // some key of this block survives the mask
-            }
-        }
-        v[e] = key;
-    }
-#pragma unroll
-    for (int k = 2; k <= N; k <<= 1)
-#pragma unroll
-        for (int j = k >> 1; j > 0; j >>= 1)
-#pragma unroll
-            for (int i = 0; i < N; ++i) {
-                const int l = i ^ j;
-                if (l > i) {
-                    const int a = v[i], b = v[l];
-                    const bool up = (i & k) == 0;
-                    v[i] = up ? min(a, b) : max(a, b);
-                    v[l] = up ? max(a, b) : min(a, b);
-                }
-            }
-    int n = 0, prev = -1;
-#pragma unroll
-    for (int e = 0; e < N; ++e) {
-        if (v[e] != INT_MAX && v[e] != prev) {
-            lists[n * kPrepThreads + col] = v[e];
-            ++n;
-        }
-        prev = v[e];
-    }
-    return n;
-}
-
 __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
 {
     extern __shared__ uint32_t prep_smem[];
@@ -180,29 +132,11 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
         if (p.causal) hi = min(hi, i + delta);
         if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
         bool bad = false;
-        if (p.topk <= 16) {
-            n = canon_in_registers<16>(raw + tt * p.topk, p.topk, nblk, p.bs, sk, lo, hi, lists, tt, bad);
-        } else if (p.topk <= 32) {
-            n = canon_in_registers<32>(raw + tt * p.topk, p.topk, nblk, p.bs, sk, lo, hi, lists, tt, bad);
-        } else {
-        for (int e = 0; e < p.topk; ++e) {
-            const int s = raw[tt * p.topk + e];
-            if (s == -1) continue;
-            if (s < 0 || s >= nblk) {
-                bad = true;
-                continue;
-            }
-            const int bl = s * p.bs, bh = min(bl + p.bs, sk) - 1;
-            if (max(bl, lo) > min(bh, hi)) continue;  // no key of this block survives the mask
-            // Insert into the ascending list, skipping duplicates.
-            int pos = n;
-            while (pos > 0 && lists[(pos - 1) * kPrepThreads + tt] > s) --pos;
-            if (pos > 0 && lists[(pos - 1) * kPrepThreads + tt] == s) continue;
-            for (int m = n; m > pos; --m) lists[m * kPrepThreads + tt] = lists[(m - 1) * kPrepThreads + tt];
-            lists[pos * kPrepThreads + tt] = s;
-            ++n;
-        }
-        }
+        // canonical list into column tt of lists ([slot][kPrepThreads])
+        const int *r = raw + tt * p.topk;
+        if (p.topk <= 16) n = canon_list_regs<16>(r, p.topk, nblk, p.bs, sk, lo, hi, lists + tt, kPrepThreads, bad);
+        else if (p.topk <= 32) n = canon_list_regs<32>(r, p.topk, nblk, p.bs, sk, lo, hi, lists + tt, kPrepThreads, bad);
+        else n = canon_list_insert(r, p.topk, nblk, p.bs, sk, lo, hi, lists + tt, kPrepThreads, bad);
         const int64_t t = (int64_t)q0 + i;
         p.cnt[t * p.Hkv + hk] = n;
         if (bad && p.status) atomicOr(p.status, SFA_DEV_BAD_INDEX);

@@ -198,18 +198,25 @@ def test_empty_batch_and_explicit_scale(sfa, oracle_lib):
     assert out.shape == (0, 4, 64) and lse.shape == (4, 0)
 
 
-def test_launch_count_and_stages(sfa, oracle_lib):
-    """sfa_fwd = prep (1 kernel, or 3 with the block-major schedule) + attend (1 kernel, or 3:
-    query-major, block-major, merge); the split-stage calls give the same result."""
-    c = W.small_config(2)
+@pytest.mark.parametrize("n", [1, 2, 3])
+def test_launch_count_and_stages(sfa, oracle_lib, n):
+    """sfa_fwd without the block-major schedule is one kernel that canonicalizes the selections
+    itself; with it, prep (3 kernels) + attend (3: query-major, block-major, merge).  The split-stage
+    calls (prep kernel, then attention on its canonical sets) give bitwise the same result, and the
+    same status word."""
+    c = W.small_config(n)
     d = upload_prefill(c)
-    out, lse = run_fwd(sfa, c, d=d)
-    assert sfa.last_launch_count() in (2, 6)
-    ws, _, _ = sfa.fwd_prep(d["cu_q"], d["sel"], Hq=c.Hq, d=c.d, block_size=c.bs, cu_seqlens_k=d["cu_k"],
-                            max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk)
+    st1 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = run_fwd(sfa, c, d=d, status=st1)
+    assert sfa.last_launch_count() == 1  # these sequences hold at most 10*topk blocks: no block-major plan
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kw = dict(cu_seqlens_k=d["cu_k"], max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk, causal=bool(c.causal),
+              window=(c.wl, c.wr), status=st2)
+    ws, _, _ = sfa.fwd_prep(d["cu_q"], d["sel"], Hq=c.Hq, d=c.d, block_size=c.bs, **kw)
     o2, l2 = sfa.fwd_attend(d["q"], d["k"], d["v"], d["cu_q"], ws, topk=c.topk, block_size=c.bs,
-                            cu_seqlens_k=d["cu_k"], max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk)
+                            scale=c.scale if c.scale > 0 else None, **kw)
     assert torch.equal(out, o2) and torch.equal(lse, l2)
+    assert int(st1.item()) == int(st2.item())
 
 
 def _block_major_windows(c, oracle_lib):
