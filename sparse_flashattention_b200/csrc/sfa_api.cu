@@ -398,6 +398,9 @@ int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void 
     p.max_pages = max_pages;
     p.num_pages = num_pages;
     p.page = page;
+    p.page_shift = -1;
+    for (int sh = 0; sh < 31; ++sh)
+        if ((1 << sh) == page) p.page_shift = sh;
     p.Hq = g.Hq;
     p.Hkv = g.Hkv;
     p.G = g.G;

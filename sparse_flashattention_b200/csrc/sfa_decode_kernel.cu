@@ -30,8 +30,10 @@ constexpr int kDecWarps = 6;
 constexpr int kDecThreads = 32 * kDecWarps;
 constexpr int kStageTok = 16;     // tokens per pipeline stage (one m16n8k16 K extent)
 constexpr int kDecStages = 2;     // per-warp ring depth: one stage in flight while the other is consumed
-constexpr int kWin = 256;         // tokens whose physical rows a warp looks up at a time
 constexpr int kFusedMaxTopk = 2048;  // the in-kernel dedupe keeps a (sequence, kv head)'s list in shared memory
+// Without the in-kernel dedupe a warp stages its canonical positions from global memory this many
+// at a time, in its own slice of the list buffer.
+constexpr int kNfWin = (kFusedMaxTopk / kDecWarps) / kStageTok * kStageTok;
 constexpr float kLn2d = 0.6931471805599453f;
 constexpr float kRescaleLog2d = 8.0f;
 
@@ -43,7 +45,9 @@ struct DecCfg {
     static constexpr int kStageBytes = 2 * kTileBytes;  // K then V
     static constexpr int kWarpRing = kDecStages * kStageBytes;
     static constexpr int kOffRows = kDecWarps * kWarpRing;
-    static constexpr int kOffList = kOffRows + kDecWarps * kWin * 4;  // deduplicated positions (fused)
+    static constexpr int kBtMax = 1536;                   // block-table entries kept in shared memory
+    static constexpr int kOffBt = kOffRows;               // the sequence's block-table row
+    static constexpr int kOffList = kOffBt + kBtMax * 4;  // positions, then physical row offsets
     static constexpr int kBytes = kOffList + kFusedMaxTopk * 4;
     static constexpr int kBitmapWords = kOffRows / 4;  // the dedupe bitmap borrows the rings
 };
@@ -96,6 +100,26 @@ __device__ int dedupe_positions(const int32_t *sel, int topk, int L, int wl, uin
     using C = DecCfg<D>;
     const bool vec = (topk & 3) == 0 && (reinterpret_cast<uintptr_t>(sel) & 15) == 0;
     const int lo_pos = wl >= 0 ? max(0, L - 1 - wl) : 0;
+    // This thread's ids, read from global memory once for both passes (-1 past the end).
+    constexpr int kIdRegs = 4 * ((kFusedMaxTopk / 4 + kDecThreads - 1) / kDecThreads);
+    int ids[kIdRegs];
+    if (vec) {
+#pragma unroll
+        for (int k = 0; k < kIdRegs / 4; ++k) {
+            const int e = (threadIdx.x + k * kDecThreads) * 4;
+            const int4 v = e < topk ? __ldg(reinterpret_cast<const int4 *>(sel + e)) : make_int4(-1, -1, -1, -1);
+            ids[4 * k] = v.x;
+            ids[4 * k + 1] = v.y;
+            ids[4 * k + 2] = v.z;
+            ids[4 * k + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < kIdRegs; ++k) {
+            const int e = threadIdx.x + k * kDecThreads;
+            ids[k] = e < topk ? __ldg(&sel[e]) : -1;
+        }
+    }
     int n = 0;
     // Positions [c0, c1) at a time.  Thread t owns the `per` consecutive bitmap words
     // [t*per, (t+1)*per); word w is stored at (w % per) * kDecThreads + w / per, so when every
@@ -109,27 +133,21 @@ __device__ int dedupe_positions(const int32_t *sel, int topk, int L, int wl, uin
     for (int c0 = 0; c0 < L; c0 += kRange) {
         const int c1 = min(L, c0 + kRange);
         const int nw = (c1 - c0 + 31) >> 5;
-        const int per = (nw + kDecThreads - 1) / kDecThreads;
+        // words per thread, rounded up to a power of two so the slot arithmetic is shifts and masks
+        int per_shift = 0;
+        while ((kDecThreads << per_shift) < nw) ++per_shift;
+        const int per = 1 << per_shift;
         for (int w = threadIdx.x; w < per * kDecThreads; w += kDecThreads) bm[w] = 0u;
         __syncthreads();
         // slot of word w of this range, or -1 when position j is not kept here
         auto slot = [&](int j) -> int {
             if (j < lo_pos || j < c0 || j >= c1) return -1;
             const int w = (j - c0) >> 5;
-            return (w % per) * kDecThreads + w / per;
+            return (w & (per - 1)) * kDecThreads + (w >> per_shift);
         };
         auto for_each_id = [&](auto &&f) {
-            if (vec) {
-                for (int e = threadIdx.x * 4; e < topk; e += kDecThreads * 4) {
-                    const int4 v = __ldg(reinterpret_cast<const int4 *>(sel + e));
-                    f(v.x);
-                    f(v.y);
-                    f(v.z);
-                    f(v.w);
-                }
-            } else {
-                for (int e = threadIdx.x; e < topk; e += kDecThreads) f(__ldg(&sel[e]));
-            }
+#pragma unroll
+            for (int k = 0; k < kIdRegs; ++k) f(ids[k]);
         };
         for_each_id([&](int j) {
             if (j == -1) return;
@@ -174,6 +192,13 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
     const int bh = blockIdx.x / cps;                     // b * Hkv + hk
     const int split = (blockIdx.x - bh * cps) * kDecWarps + warp;
     const int hk = bh % p.Hkv, b = bh / p.Hkv;
+    // The sequence's block-table row into shared memory when it fits (read while the selection is
+    // deduplicated), so a token's physical row is found without a dependent global load.
+    int *bt_s = reinterpret_cast<int *>(dsm + C::kOffBt);
+    const int32_t *bt_g = p.bt + (int64_t)b * p.max_pages;
+    const bool bt_smem = p.max_pages <= C::kBtMax;
+    if (bt_smem)
+        for (int i = threadIdx.x; i < p.max_pages; i += kDecThreads) bt_s[i] = __ldg(&bt_g[i]);
     const int32_t *toks;
     int n;
     if (p.fused) {
@@ -195,6 +220,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
     } else {
         n = p.cnt[bh];
         toks = p.tok_c + (int64_t)bh * p.topk;
+        __syncthreads();  // the block-table row is in shared memory
     }
     const bool active = split < p.S;  // a CTA's last warps may have no split
     const int chunk = (n + p.S - 1) / p.S;
@@ -202,7 +228,11 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
     const int ntok = active ? min(n, begin + chunk) - begin : 0;
     toks += begin;
     const uint32_t ring = smem_u32(dsm) + warp * C::kWarpRing;
-    int *rowoff = reinterpret_cast<int *>(dsm + C::kOffRows) + warp * kWin;
+    // Physical row offsets of the warp's tokens: in place over its part of the deduplicated list
+    // (one pass), or, from the prep kernel's list, kNfWin at a time in the warp's slice of the buffer.
+    int *list_s = reinterpret_cast<int *>(dsm + C::kOffList);
+    int *rowoff = p.fused ? list_s + begin : list_s + warp * kNfWin;
+    const int wcap = p.fused ? max(ntok, 1) : kNfWin;
 
     // A fragments of the G query rows (rows >= G are zero), straight from global memory.
     uint32_t aq[D / 16][4];
@@ -225,17 +255,18 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
     float l_r[2] = {0.f, 0.f};              // this thread's share of the running sums
     bool bad_page = false;
 
-    for (int w0 = 0; w0 < ntok; w0 += kWin) {
-        const int wn = min(kWin, ntok - w0);
+    for (int w0 = 0; w0 < ntok; w0 += wcap) {
+        const int wn = min(wcap, ntok - w0);
         __syncwarp();
         for (int e = lane; e < wn; e += 32) {
-            const int pos = toks[w0 + e];
-            const int pg = p.bt[(int64_t)b * p.max_pages + pos / p.page];
+            const int pos = toks[w0 + e];  // (fused: the same shared-memory slot the offset goes to)
+            const int pi = p.page_shift >= 0 ? pos >> p.page_shift : pos / p.page;  // page of the position
+            const int pg = bt_smem ? bt_s[pi] : __ldg(&bt_g[pi]);
             if (pg < 0 || pg >= p.num_pages) {
                 rowoff[e] = -1;
                 bad_page = true;
             } else {
-                rowoff[e] = (pg * p.page + pos % p.page) * p.Hkv + hk;
+                rowoff[e] = (pg * p.page + (pos - pi * p.page)) * p.Hkv + hk;
             }
         }
         __syncwarp();

@@ -124,7 +124,8 @@ struct DecSplitParams {
     const int32_t *bt, *tok_c, *cnt;  // canonical sets from the prep kernel (fused == 0)
     const int32_t *seqlens, *sel;     // raw selections, deduplicated in the kernel (fused == 1)
     int fused, wl;
-    int B, max_pages, num_pages, page, Hq, Hkv, G, topk, S;  // CTA c of (b, kv head) runs splits 4c..4c+3
+    int B, max_pages, num_pages, page, Hq, Hkv, G, topk, S;  // CTA c of (b, kv head) runs splits 6c..6c+5
+    int page_shift;  // log2(page) when page is a power of two, else -1
     float scale_log2;
     float *po, *plse;  // partial outputs (B, Hq, S, d) and natural-log lse (B, Hq, S)
     __nv_bfloat16 *out_direct;  // S <= 4: the CTA combines its splits and writes out / lse itself
