@@ -23,7 +23,8 @@ namespace sfa {
 
 namespace {
 
-constexpr int kInvThreadsAttn = 320;  // warp 0 producer, warp 1 MMA, warps 2-5 and 6-9: two softmax groups
+constexpr int kInvThreadsAttn = 352;  // warp 0 producer, warp 1 MMA, warps 2-5 and 6-9: two softmax groups,
+                                      // warp 10: second half of each item's Q-row gather
 constexpr float kLn2i = 0.6931471805599453f;
 constexpr int kItemSlots = 8;   // item j lives in slot j % 8; softmax group j % 2 handles it
 constexpr int kFetchAhead = 4;  // item records are fetched this many items ahead
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             mbar_init(&meta->item_free[s], 128);
         }
         for (int s = 0; s < kLoadStages; ++s) {
-            mbar_init(&meta->q_full[s], 32);  // one cp.async arrival per producer lane
+            mbar_init(&meta->q_full[s], 64);  // one cp.async arrival per lane of the two gathering warps
             mbar_init(&meta->q_empty[s], 1);
             mbar_init(&meta->kv_full[s], 1);
             mbar_init(&meta->kv_empty[s], 1);
@@ -149,16 +150,17 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 }
                 issued[sl]++;
             }
-            // Q rows of the item's tokens (row r = token * G + head) into the 128-byte-swizzled K-major
-            // tile the MMA reads: 16-byte cp.async copies, lane l taking rows l, l+32, l+64, l+96 (rows
-            // past the item are zero-filled).  Each lane's copies land on q_full through its own arrival.
+            // Q rows 0..63 of the item's tokens (row r = token * G + head) into the 128-byte-swizzled
+            // K-major tile the MMA reads: 16-byte cp.async copies, lane l taking rows l and l+32 (rows
+            // past the item are zero-filled; warp 10 copies rows 64..127).  Each lane's copies land on
+            // q_full through its own arrival.
             if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
             {
                 const int rows = rec.w * p.G;
                 const uint32_t qt = smem_u32(sQ + sl * C::kQBytes);
 #pragma unroll 1
-                for (int r = lane; r < 128; r += 32) {
+                for (int r = lane; r < 64; r += 32) {
                     const bool live = r < rows;
                     const int tk = live ? r / p.G : 0, gg = live ? r - tk * p.G : 0;
                     const __nv_bfloat16 *src =
@@ -259,8 +261,41 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 mbar_drain(&meta->drain, 0);
             }
         }
+    } else if (warp == 10) {
+        // ---------------------------------------------------------------- Q-row gather, rows 64..127
+        // Follows the producer's item sequence: the item's slot stays valid until its softmax group
+        // frees it, which needs this warp's copies (q_full) first.
+        bool ok = true;
+        for (int j = 0; ok; ++j) {
+            const int sl = j % kLoadStages, it = j % kItemSlots;
+            const uint32_t ph = ((j / kLoadStages) - 1) & 1;
+            ok = warp_all_ok(mbar_wait(&meta->item_full[it], (j / kItemSlots) & 1, abort_flag, p.status));
+            if (!ok) break;
+            const InvItem *item = &meta->slot[it];
+            const int4 rec = item->rec;
+            if (rec.w < 0) break;
+            const int hk = rec.x % p.Hkv;
+            if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
+            if (!ok) break;
+            const int rows = rec.w * p.G;
+            const uint32_t qt = smem_u32(sQ + sl * C::kQBytes);
+#pragma unroll 1
+            for (int r = 64 + lane; r < 128; r += 32) {
+                const bool live = r < rows;
+                const int tk = live ? r / p.G : 0, gg = live ? r - tk * p.G : 0;
+                const __nv_bfloat16 *src = p.q + ((int64_t)(live ? (item->tok[tk] >> 7) : 0) * p.Hq + hk * p.G + gg) * D;
+#pragma unroll
+                for (int c = 0; c < D / 64; ++c)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        cp_async16(qt + c * (128 * 128) + r * 128 + ((k ^ (r & 7)) << 4), src + c * 64 + k * 8,
+                                   live ? 16u : 0u);
+            }
+            cp_async_mbar_arrive(&meta->q_full[sl]);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies have all landed
     } else {
-        // ---------------------------------------------------------------- softmax groups
+        // ---------------------------------------------------------------- softmax groups (warps 2-9)
         const int grp = (warp - 2) >> 2;        // 0: warps 2-5, 1: warps 6-9
         const int quad = warp & 3;              // TMEM lane quadrant of this warp
         const int r = quad * 32 + lane;         // tile row
