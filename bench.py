@@ -354,6 +354,58 @@ def run_gpu(args, rank, world, local_rank):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
 
+    # ---- the NSA branches beside the selected attention (not part of the step): the sliding-window
+    # branch (window 512 as in the NSA module example, causal) and the three-branch gated mix, on the
+    # prefill workload's tensors; L2 flushed before every repetition, CUDA events on the stream.
+    extras = None
+    if not args.no_extras and args.part != "decode-small":
+        wl = 512
+        seq = np.diff(pc.cu_q).tolist()
+        wpairs = sum(int(np.minimum(np.arange(L) + 1, wl + 1).sum()) for L in seq)
+        wflops = 4.0 * pc.d * pc.Hq * wpairs
+        wws = torch.empty(256, dtype=torch.uint8, device=dev)
+        wout = torch.empty_like(out)
+        wlse = torch.empty_like(lse)
+        gates = [torch.rand((pc.total_q, pc.Hq), dtype=torch.float32, device=dev) for _ in range(3)]
+        mix = torch.empty_like(out)
+
+        def run_window():
+            sfa.window_fwd(P["q"], P["k"], P["v"], P["cu_q"], cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq,
+                           max_seqlen_k=pc.max_sk, causal=True, window=(wl, 0), out=wout, lse=wlse, workspace=wws,
+                           status=status)
+
+        def run_mix():
+            sfa.gated_combine([(out, gates[0]), (wout, gates[1]), (P["q"], gates[2])], out=mix)
+
+        def timed(fn, reps=10):
+            for _ in range(3):
+                fn()
+            ts = []
+            for _ in range(reps):
+                flush.fill_(1)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                fn()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            return float(np.mean(ts))
+
+        w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
+        m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
+        mix_bytes = 4 * pc.total_q * pc.Hq * pc.d * 2 + 3 * pc.total_q * pc.Hq * 4
+        extras = {
+            "window_branch": {"workload": "the prefill workload's q/k/v, causal, window (512, 0), no selection",
+                              "ms": round(w_ms, 4), "effective_tflops": round(wflops / (w_ms * 1e-3) / 1e12, 2),
+                              "frac": round(wflops / (w_ms * 1e-3) / 1e12 / tf_burst, 4),
+                              "peak_source": f"{peak_kind} bf16 burst", "launches": 1},
+            "gated_combine": {"workload": "3 branches of (total_q, Hq, d) bf16 + fp32 gates -> bf16",
+                              "ms": round(m_ms, 4), "gbs": round(mix_bytes / (m_ms * 1e-3) / 1e9, 1),
+                              "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
+        }
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
+
     # ---- end to end through the public API with host buffers (pinned), copies inside the timing
     e2e = None
     if not args.no_e2e:
@@ -462,7 +514,8 @@ def run_gpu(args, rank, world, local_rank):
     return dict(value=value, fused=fused, prefill_ms=prefill_ms, prep_ms=pp_ms, attend_ms=pa_ms, decode_ms=decode_ms,
                 dprep_ms=dp_ms, dattend_ms=da_ms, step_ms=step_ms, region_ms=region_ms, attend_tflops=attend_tflops,
                 dec_gbs=dec_gbs, dec_attend_gbs=dec_attend_gbs, flops=flops, gbytes=gbytes, clocks=clocks,
-                launches=n_launch, e2e=e2e, hbm=hbm, tf_burst=tf_burst, tf_sust=tf_sust, peak_kind=peak_kind,
+                launches=n_launch, e2e=e2e, extras=extras, hbm=hbm, tf_burst=tf_burst, tf_sust=tf_sust,
+                peak_kind=peak_kind,
                 pc=pc, dc=dc,
                 traffic=args.traffic if args.traffic is not None else kernel_traffic("fwd_attend_pipe_kernel"),
                 dec_traffic=kernel_traffic("decode_split_kernel"))
@@ -475,6 +528,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sfa", choices=["sfa", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the NSA window-branch and gated-mix lines")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode-small"],
@@ -551,6 +605,8 @@ def main():
         line["clocks"] = r["clocks"]
     if r["e2e"]:
         line["e2e"] = r["e2e"]
+    if r["extras"]:
+        line["nsa_branches"] = r["extras"]
     if world == 1 and not args.no_cpu_baseline:
         v, n, thr, secs = cpu_oracle_rate(pc, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",

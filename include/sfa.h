@@ -96,7 +96,9 @@ int sfa_fwd_workspace_offsets(int batch, int max_seqlen_q, int max_seqlen_k, int
                               int Hq, int Hkv, int d, int topk, int block_size,
                               size_t *off_sel_c, size_t *off_cnt);
 
-/* Full prefill forward = sfa_fwd_prep followed by sfa_fwd_attend on the same workspace.
+/* Full prefill forward: the result of sfa_fwd_prep followed by sfa_fwd_attend on the same
+ * workspace (when the call needs no block-major plan it is one kernel that canonicalises each
+ * query tile's selections itself; the workspace then only carries its tile counter).
  *   q            bf16 (total_q, Hq, d)
  *   k, v         bf16 (total_k, Hkv, d)
  *   cu_seqlens_q int32 (batch+1), prefix sums from 0; cu_seqlens_k likewise, or NULL for
@@ -207,12 +209,42 @@ int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
                        int B, int Hq, int Hkv, int d, int window_left, float scale, int num_splits,
                        int32_t *status_dev, void *out, float *lse, sfa_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------
+ * NSA branches beside the selected attention (the "Relaxed-System-Lab/Flash-Sparse-Attention"
+ * project page, quick-start: window_size alongside block_size / topk; the Flash-Sparse-Attention
+ * README feature list: causal and local window attention, gated attention).
+ * --------------------------------------------------------------------------------------- */
+
+/* Bytes of device workspace sfa_window_fwd needs (a tile counter it clears itself). */
+size_t sfa_window_fwd_workspace_size(void);
+
+/* Sliding-window branch: every query attends to all keys its mask keeps — the common semantics
+ * above with every key selected (bottom-right causal limit when causal; window_left /
+ * window_right as in the flash-attention-npu docstrings, -1 = unbounded; a plain causal or full
+ * attention when no window is given).  Layouts, lengths, status word and errors as sfa_fwd;
+ * there is no selection.  out bf16 (total_q, Hq, d); lse fp32 (Hq, total_q).  One kernel. */
+int sfa_window_fwd(const void *q, const void *k, const void *v,
+                   const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                   int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                   int Hq, int Hkv, int d, int causal, int window_left, int window_right, float scale,
+                   void *workspace, size_t workspace_bytes, int32_t *status_dev,
+                   void *out, float *lse, sfa_stream_t stream);
+
+/* Gated mix of the branch outputs: out[t,h,:] = sum over the given branches c of
+ * g_c[t,h] * o_c[t,h,:] (fp32 arithmetic, bf16 round-to-nearest result).  Each o_c is bf16
+ * (total_q, Hq, d) and each g_c fp32 (total_q, Hq), e.g. the compressed, selected and window
+ * branches with the caller's gate values; a branch whose o or g pointer is NULL is left out (at
+ * least one must be given).  d in {64, 128}; 16-byte aligned bf16 tensors.  One kernel. */
+int sfa_gated_combine(const void *o_cmp, const float *g_cmp, const void *o_slc, const float *g_slc,
+                      const void *o_win, const float *g_win, int total_q, int Hq, int d, void *out,
+                      sfa_stream_t stream);
+
 /* Human-readable name of an sfa_status value (static string). */
 const char *sfa_status_string(int status);
 
-/* Number of kernel launches the last successful call on this host thread made (prefill: 2,
- * or 6 when the call can use the block-major schedule; decode: 1 with at most 6 splits, else 2,
- * plus 1 when topk_tok > 2048; a stage: its own count). */
+/* Number of kernel launches the last successful call on this host thread made (prefill: 1,
+ * or 6 when the call uses the block-major schedule; decode: 1 with at most 6 splits, else 2,
+ * plus 1 when topk_tok > 2048; a stage: its own count; window branch, gated mix: 1). */
 int sfa_last_launch_count(void);
 
 #ifdef __cplusplus

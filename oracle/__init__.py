@@ -121,3 +121,19 @@ def decode_index(case, sel=None):
     bad = lib.sfa_oracle_decode_index(_p(_c(case.cache_seqlens, np.int32)), _p(sel), topk, case.B, case.Hkv,
                                       case.wl, _p(tok_c), _p(cnt))
     return tok_c, cnt, int(bad)
+
+
+def gated_combine(branches):
+    """Gated mix of NSA branch outputs, in float64: out[t, h, :] = sum over the (o, g) pairs of
+    g[t, h] * o[t, h, :] — the Flash-Sparse-Attention module's combination of its compressed, selected
+    and sliding-window branches per token and head ("Relaxed-System-Lab/Flash-Sparse-Attention"
+    project page, quick-start; README feature list, "Gated attention").  o: bf16 bit patterns
+    (uint16) or floats, (total_q, Hq, d); g: floats (total_q, Hq)."""
+    out = None
+    for o, g in branches:
+        o = np.asarray(o)
+        of = (o.astype(np.uint32) << 16).view(np.float32).astype(np.float64) if o.dtype == np.uint16 else \
+            o.astype(np.float64)
+        term = np.asarray(g, np.float64)[..., None] * of
+        out = term if out is None else out + term
+    return out

@@ -18,7 +18,8 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["SfaError", "lib_path", "fwd", "fwd_prep", "fwd_attend", "fwd_workspace_size", "decode", "decode_prep",
+__all__ = ["SfaError", "lib_path", "fwd", "fwd_prep", "fwd_attend", "fwd_workspace_size", "window_fwd",
+           "gated_combine", "decode", "decode_prep",
            "decode_attend", "decode_noalloc", "decode_workspace_size", "decode_num_splits", "last_launch_count",
            "DEV_BAD_INDEX", "DEV_BAD_PAGE", "DEV_TIMEOUT"]
 
@@ -55,6 +56,9 @@ def _load():
         "sfa_decode_prep": (I, [P, P, I, I, I, I, I, I, I, I, I, P, Z, P, P]),
         "sfa_decode_attend": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]),
         "sfa_decode_noalloc": (I, [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, F, I, P, P, P, P]),
+        "sfa_window_fwd_workspace_size": (Z, []),
+        "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F, P, Z, P, P, P, P]),
+        "sfa_gated_combine": (I, [P, P, P, P, P, P, I, I, I, P, P]),
         "sfa_status_string": (ctypes.c_char_p, [I]),
         "sfa_last_launch_count": (I, []),
     }
@@ -185,6 +189,55 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.T
                       _stream(stream))
     _check(rc)
     return out, lse
+
+
+def window_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor, *,
+               cu_seqlens_k: Optional[torch.Tensor] = None, max_seqlen_q: Optional[int] = None,
+               max_seqlen_k: Optional[int] = None, causal: bool = True, window: Tuple[int, int] = (-1, -1),
+               scale: Optional[float] = None, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+               stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Sliding-window branch (sfa_window_fwd): every query attends to all keys its causal / window
+    mask keeps.  Layouts as fwd, no selection.  Returns out (total_q, Hq, d) bf16, lse (Hq, total_q)."""
+    a = _FwdArgs(q, k, v, cu_seqlens_q, None, 64, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, window, scale,
+                 topk=1)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((a.Hq, a.total_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    ws = _workspace(workspace, int(_lib.sfa_window_fwd_workspace_size()), q.device)
+    rc = _lib.sfa_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), a.batch, a.max_sq,
+                             a.max_sk, a.total_q, a.total_k, a.Hq, a.Hkv, a.d, a.causal, a.wl, a.wr, a.scale, _ptr(ws),
+                             ws.numel() * ws.element_size(), _ptr(status), _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+def gated_combine(branches, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Gated mix (sfa_gated_combine): out = sum over (o, g) in branches of g[..., None] * o, for up to
+    three (o, g) pairs in the order (compressed, selected, window); None entries are left out.
+    o bf16 (total_q, Hq, d), g fp32 (total_q, Hq)."""
+    pairs = list(branches) + [None] * (3 - len(branches))
+    if len(pairs) != 3:
+        raise ValueError("at most three branches")
+    ref = next((o for o, _ in (x for x in pairs if x is not None)), None)
+    if ref is None:
+        raise ValueError("no branch given")
+    _need(ref, "o", torch.bfloat16, 3)
+    total_q, Hq, d = ref.shape
+    args = []
+    for x in pairs:
+        if x is None:
+            args += [None, None]
+            continue
+        o, g = x
+        _need(o, "o", torch.bfloat16, 3)
+        _need(g, "g", torch.float32, 2)
+        if tuple(o.shape) != (total_q, Hq, d) or tuple(g.shape) != (total_q, Hq):
+            raise ValueError("branch shapes differ")
+        args += [o, g]
+    out = torch.empty_like(ref) if out is None else out
+    rc = _lib.sfa_gated_combine(*[_ptr(t) for t in args], total_q, Hq, d, _ptr(out), _stream(stream))
+    _check(rc)
+    return out
 
 
 def fwd_prep(cu_seqlens_q, sel_idx, *, Hq: int, d: int, block_size: int, cu_seqlens_k=None, max_seqlen_q=None,

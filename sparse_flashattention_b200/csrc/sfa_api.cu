@@ -240,7 +240,7 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
                     int32_t *status, void *out, float *lse, cudaStream_t st, const int32_t *sel = nullptr)
 {
     const bool fused = sel != nullptr;
-    const bool pipe = fwd_pipe_fits(g, fused);
+    const bool pipe = fwd_pipe_fits(g, fused ? kPipeFused : kPipePrep);
     if (fused && (!pipe || g.inv)) return SFA_ERR_UNSUPPORTED;
     if (!pipe && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     CUtensorMap tq, tk, tv;
@@ -279,7 +279,8 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     p.max_sq = g.max_sq;
     p.nblk_max = g.nblk_max;
     if (fused && cudaMemsetAsync(p.tile_counter, 0, 2 * sizeof(int32_t), st) != cudaSuccess) return SFA_ERR_CUDA;
-    if ((pipe ? launch_fwd_attend_pipe(g, p, fused, tq, tk, tv, st) : launch_fwd_attend(g, p, tq, tk, tv, st)) !=
+    if ((pipe ? launch_fwd_attend_pipe(g, p, fused ? kPipeFused : kPipePrep, tq, tk, tv, st)
+              : launch_fwd_attend(g, p, tq, tk, tv, st)) !=
         cudaSuccess)
         return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
@@ -510,8 +511,8 @@ int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqle
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
     if (total_k == 0) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
-    if (!fwd_pipe_fits(g, false) && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
-    if (!g.inv && fwd_pipe_fits(g, true)) {
+    if (!fwd_pipe_fits(g, kPipePrep) && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    if (!g.inv && fwd_pipe_fits(g, kPipeFused)) {
         // One launch: the attention kernel canonicalizes each tile's selections itself.
         rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right,
                              scale, workspace, status_dev, out, lse, stream, sel_idx);
@@ -620,6 +621,93 @@ int sfa_decode(const void *q, const void *k_cache, const void *v_cache, const in
                          sel_tok_idx, window_left, fused, scale, workspace, status_dev, out, lse, stream);
     if (rc == SFA_OK) g_last_launches = (fused ? 0 : 1) + (g.S <= decode_split_warps_per_block() ? 1 : 2);
     return rc;
+}
+
+size_t sfa_window_fwd_workspace_size(void)
+{
+    return 256;
+}
+
+int sfa_window_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens_q,
+                   const int32_t *cu_seqlens_k, int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                   int Hq, int Hkv, int d, int causal, int window_left, int window_right, float scale, void *workspace,
+                   size_t workspace_bytes, int32_t *status_dev, void *out, float *lse, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    // The window kernel tiles keys in 64-token blocks; no selection (topk 1 only sizes the geometry).
+    FwdGeom g;
+    int rc = fwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, 1, 64, g);
+    if (rc != SFA_OK) return rc;
+    if ((rc = fwd_common_checks(cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k, causal,
+                                window_left, window_right)) != SFA_OK)
+        return rc;
+    if (total_q == 0 || batch == 0) return SFA_OK;
+    if (!q || !k || !v || !out || !lse || !workspace) return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
+    if (total_k == 0) return SFA_ERR_UNSUPPORTED;
+    if (workspace_bytes < sfa_window_fwd_workspace_size()) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (!fwd_pipe_fits(g, kPipeWindow)) return SFA_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    CUtensorMap tq, tk, tv;
+    if (!encode_3d(tq, q, g.d, g.Hq, g.total_q, g.G, g.Tq)) return SFA_ERR_CUDA;
+    if (!encode_3d(tk, k, g.d, g.Hkv, total_k, 1, g.bs)) return SFA_ERR_CUDA;
+    if (!encode_3d(tv, v, g.d, g.Hkv, total_k, 1, g.bs)) return SFA_ERR_CUDA;
+    FwdAttendParams p{};
+    p.cu_q = cu_seqlens_q;
+    p.cu_k = cu_seqlens_k ? cu_seqlens_k : cu_seqlens_q;
+    p.batch = g.batch;
+    p.total_q = g.total_q;
+    p.Hq = g.Hq;
+    p.Hkv = g.Hkv;
+    p.G = g.G;
+    p.Tq = g.Tq;
+    p.nqt = g.nqt;
+    p.topk = g.topk;
+    p.umax = g.umax;
+    p.causal = causal;
+    p.wl = window_left;
+    p.wr = window_right;
+    const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)g.d);
+    p.scale_log2 = (float)(sc * 1.4426950408889634);
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.lse = lse;
+    p.status = status_dev;
+    p.tiles = g.tiles;
+    p.tile_counter = static_cast<int32_t *>(workspace);
+    p.bs = g.bs;
+    p.max_sq = g.max_sq;
+    p.nblk_max = g.nblk_max;
+    if (cudaMemsetAsync(p.tile_counter, 0, 2 * sizeof(int32_t), st) != cudaSuccess) return SFA_ERR_CUDA;
+    if (launch_fwd_attend_pipe(g, p, kPipeWindow, tq, tk, tv, st) != cudaSuccess) return SFA_ERR_CUDA;
+    g_last_launches = 1;
+    return SFA_OK;
+}
+
+int sfa_gated_combine(const void *o_cmp, const float *g_cmp, const void *o_slc, const float *g_slc, const void *o_win,
+                      const float *g_win, int total_q, int Hq, int d, void *out, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    if (total_q < 0 || Hq <= 0) return SFA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SFA_ERR_UNSUPPORTED;
+    CombineParams p{};
+    const void *os[3] = {o_cmp, o_slc, o_win};
+    const float *gs[3] = {g_cmp, g_slc, g_win};
+    int given = 0;
+    for (int b = 0; b < 3; ++b) {
+        if (!os[b] || !gs[b]) continue;
+        if (!aligned16(os[b])) return SFA_ERR_INVALID_ARG;
+        p.o[given] = static_cast<const __nv_bfloat16 *>(os[b]);
+        p.g[given] = gs[b];
+        ++given;
+    }
+    if (given == 0) return SFA_ERR_INVALID_ARG;
+    if (total_q == 0) return SFA_OK;
+    if (!out || !aligned16(out)) return SFA_ERR_INVALID_ARG;
+    p.out = static_cast<__nv_bfloat16 *>(out);
+    p.rows = (int64_t)total_q * Hq;
+    if (launch_gated_combine(p, d, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SFA_ERR_CUDA;
+    g_last_launches = 1;
+    return SFA_OK;
 }
 
 const char *sfa_status_string(int status)

@@ -58,7 +58,14 @@ struct TileInfo {
     int done;  // no tile left: every role leaves its loop
     int nU;    // union blocks (< 0: a block-major tile, whose rows another kernel computes)
     int b, hk, q0, sq, k0, sk, tok0, ntok;
+    int blo;   // window mode: the union is blocks blo, blo+1, ..., blo+nU-1
 };
+
+// How a tile's blocks and each row's selection are known (sfa_internal.h): kPipePrep, canonical
+// lists and union written by the prep kernel; kPipeFused, the index warp canonicalizes the raw
+// selections itself; kPipeWindow, dense attention under the causal / window mask (every block that
+// holds a key of the row's window is selected; no selection lists).
+constexpr int kModePrep = kPipePrep, kModeFused = kPipeFused, kModeWindow = kPipeWindow;
 
 struct QMeta {
     uint64_t q_full, q_empty;
@@ -81,28 +88,31 @@ struct QLayout {
 };
 
 template <int D, int BS>
-__host__ __device__ inline QLayout pipe_layout(bool fused, int umax, int Tq, int topk, int nblk_max)
+__host__ __device__ inline QLayout pipe_layout(int mode, int umax, int Tq, int topk, int nblk_max)
 {
     QLayout l;
+    const bool fused = mode == kModeFused;
     l.off_union = QCfg<D, BS>::kOffMeta + ((sizeof(QMeta) + 15) & ~size_t(15));
-    l.off_lists = l.off_union + (size_t)2 * umax * 4;
+    l.off_lists = l.off_union + (mode == kModeWindow ? 0 : (size_t)2 * umax * 4);
     l.off_cnts = l.off_lists + (fused ? (size_t)2 * Tq * topk * 4 : 0);
     l.off_bm = l.off_cnts + (fused ? (size_t)2 * Tq * 4 : 0);
     l.bytes = l.off_bm + (fused ? (size_t)(nblk_max + 31) / 32 * 4 : 0);
     return l;
 }
 
-template <int D, int BS, bool FUSED>
+template <int D, int BS, int MODE>
 __global__ void __launch_bounds__(kQThreads, 2)
     fwd_attend_pipe_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv, const FwdAttendParams p)
 {
     using C = QCfg<D, BS>;
+    constexpr bool FUSED = MODE == kModeFused;
+    constexpr bool WIN = MODE == kModeWindow;
     extern __shared__ uint8_t pipe_smem_raw[];
     uint8_t *smem =
         reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(pipe_smem_raw) + 1023) & ~uintptr_t(1023));
     const int U = p.umax;
-    const QLayout L = pipe_layout<D, BS>(FUSED, U, p.Tq, p.topk, p.nblk_max);
+    const QLayout L = pipe_layout<D, BS>(MODE, U, p.Tq, p.topk, p.nblk_max);
     QMeta *meta = reinterpret_cast<QMeta *>(smem + C::kOffMeta);
     int *s_union = reinterpret_cast<int *>(smem + L.off_union);   // [2][U]
     int *s_lists = reinterpret_cast<int *>(smem + L.off_lists);   // fused: [2][Tq][topk]
@@ -191,8 +201,23 @@ __global__ void __launch_bounds__(kQThreads, 2)
             const int k0 = p.cu_k[b], sk = p.cu_k[b + 1] - k0;
             const int tok0 = qt * p.Tq;
             const int ntok = min(p.Tq, sq - tok0);
-            int nU;
-            if constexpr (FUSED) {
+            int nU, blo = 0;
+            if constexpr (WIN) {
+                // Rows' key windows [lo(i), hi(i)] move right with i, so the tile's blocks are the
+                // contiguous range from the first row's lo to the last row's hi.
+                int nblk = (sk + BS - 1) / BS;
+                if (sq > p.max_sq || nblk > p.nblk_max) {  // lengths beyond the caller's max_seqlen bounds
+                    if (lane == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_SEQLEN);
+                    nblk = min(nblk, p.nblk_max);
+                }
+                const int delta = sk - sq, i0 = tok0, i1 = tok0 + ntok - 1;
+                int lo = 0, hi = min(sk, nblk * BS) - 1;
+                if (p.wl >= 0) lo = max(lo, i0 + delta - p.wl);
+                if (p.causal) hi = min(hi, i1 + delta);
+                if (p.wr >= 0) hi = min(hi, i1 + delta + p.wr);
+                blo = lo / BS;
+                nU = hi >= lo ? hi / BS - blo + 1 : 0;
+            } else if constexpr (FUSED) {
                 // The tile's canonical lists (one token per lane at a time) and the ascending union
                 // of their blocks, built here instead of by a prep kernel.
                 int *lists = s_lists + m * p.Tq * p.topk;
@@ -261,6 +286,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
                 ti.sk = sk;
                 ti.tok0 = tok0;
                 ti.ntok = ntok;
+                ti.blo = blo;
             }
             mbar_arrive(&meta->meta_full[m]);
             ++k;
@@ -279,7 +305,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
                 const TileInfo &ti = meta->info[m];
                 if (ti.done) break;
                 const int *uni = s_union + m * U;
-                const int n = max(ti.nU, 0), hk = ti.hk, q0 = ti.q0, k0 = ti.k0, tok0 = ti.tok0;
+                const int n = max(ti.nU, 0), hk = ti.hk, q0 = ti.q0, k0 = ti.k0, tok0 = ti.tok0, blo = ti.blo;
                 // Q, once the previous tile's score MMAs no longer read it (a box of Tq tokens x
                 // G heads, Tq*G <= 128 rows).
                 if (k >= 1) ok = mbar_wait(&meta->q_empty, (k - 1) & 1, abort_flag, p.status);
@@ -296,7 +322,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
                     const int st = k_st;
                     if (nk >= kQStages && !mbar_wait(&meta->k_empty[st], k_ph ^ 1, abort_flag, p.status))
                         return false;
-                    const int row = k0 + uni[u] * BS;
+                    const int row = k0 + (WIN ? blo + u : uni[u]) * BS;
                     mbar_arrive_expect_tx(&meta->k_full[st], (uint32_t)C::kKVBytes);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(&tmk, &meta->k_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
@@ -311,7 +337,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
                     const int st = v_st;
                     if (nv >= kQStages && !mbar_wait(&meta->v_empty[st], v_ph ^ 1, abort_flag, p.status))
                         return false;
-                    const int row = k0 + uni[u] * BS;
+                    const int row = k0 + (WIN ? blo + u : uni[u]) * BS;
                     mbar_arrive_expect_tx(&meta->v_full[st], (uint32_t)C::kKVBytes);
                     for (int c = 0; c < D / 64; ++c)
                         tma_load_3d(&tmv, &meta->v_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
@@ -484,18 +510,20 @@ __global__ void __launch_bounds__(kQThreads, 2)
             // from the prep kernel's output in global memory one entry ahead of its use.
             const int64_t t = (int64_t)q0 + i;
             const int *mylist = s_lists + (m * p.Tq + (row_valid ? tok : 0)) * p.topk;
-            const int32_t *gl = p.sel_c + (row_valid && !FUSED ? (t * p.Hkv + hk) * p.topk : 0);
-            const int mycnt = !row_valid ? 0 : FUSED ? s_cnts[m * p.Tq + tok] : p.cnt[t * p.Hkv + hk];
-            int nxt = (!FUSED && mycnt > 0) ? gl[0] : -1;
+            const int32_t *gl = p.sel_c + (row_valid && MODE == kModePrep ? (t * p.Hkv + hk) * p.topk : 0);
+            const int mycnt = !row_valid || WIN ? 0 : FUSED ? s_cnts[m * p.Tq + tok] : p.cnt[t * p.Hkv + hk];
+            int nxt = (MODE == kModePrep && mycnt > 0) ? gl[0] : -1;
             int ptr = 0;
             float m_run = -INFINITY;  // running max of s*scale*log2e
             float l_run = 0.f;
 
             for (int j = 0; j < n; ++j) {
                 const int jg = jg0 + j;
-                const int s = uni[j];
+                const int s = WIN ? ti.blo + j : uni[j];
                 bool selected;
-                if constexpr (FUSED) {
+                if constexpr (WIN) {
+                    selected = row_valid && s * BS <= hi && s * BS + BS - 1 >= lo;
+                } else if constexpr (FUSED) {
                     selected = ptr < mycnt && mylist[ptr] == s;
                     if (selected) ++ptr;
                 } else {
@@ -649,14 +677,14 @@ __global__ void __launch_bounds__(kQThreads, 2)
     }
 }
 
-template <int D, int BS, bool FUSED>
+template <int D, int BS, int MODE>
 cudaError_t launch_pipe_t(const FwdAttendParams &p, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                           cudaStream_t st)
 {
-    const size_t smem = 1024 + pipe_layout<D, BS>(FUSED, p.umax, p.Tq, p.topk, p.nblk_max).bytes;
+    const size_t smem = 1024 + pipe_layout<D, BS>(MODE, p.umax, p.Tq, p.topk, p.nblk_max).bytes;
     static int configured = 0;
     if ((int)smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_attend_pipe_kernel<D, BS, FUSED>,
+        cudaError_t e = cudaFuncSetAttribute(fwd_attend_pipe_kernel<D, BS, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         configured = (int)smem;
@@ -664,38 +692,40 @@ cudaError_t launch_pipe_t(const FwdAttendParams &p, const CUtensorMap &tq, const
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = p.tiles < 2 * sms ? p.tiles : 2 * sms;
-    // The fused mode follows a memset of the tile counter, not a kernel: no early start.
-    return launch_kernel(fwd_attend_pipe_kernel<D, BS, FUSED>, dim3(grid > 0 ? grid : 1), dim3(kQThreads), smem, st,
-                         !FUSED, tq, tk, tv, p);
+    // The fused and window modes follow a memset of the tile counter, not a kernel: no early start.
+    return launch_kernel(fwd_attend_pipe_kernel<D, BS, MODE>, dim3(grid > 0 ? grid : 1), dim3(kQThreads), smem, st,
+                         MODE == kModePrep, tq, tk, tv, p);
 }
 
 template <int D, int BS>
-cudaError_t launch_pipe_d(const FwdAttendParams &p, bool fused, const CUtensorMap &tq, const CUtensorMap &tk,
+cudaError_t launch_pipe_d(const FwdAttendParams &p, int mode, const CUtensorMap &tq, const CUtensorMap &tk,
                           const CUtensorMap &tv, cudaStream_t st)
 {
-    return fused ? launch_pipe_t<D, BS, true>(p, tq, tk, tv, st) : launch_pipe_t<D, BS, false>(p, tq, tk, tv, st);
+    if (mode == kModeWindow) return launch_pipe_t<D, BS, kModeWindow>(p, tq, tk, tv, st);
+    return mode == kModeFused ? launch_pipe_t<D, BS, kModeFused>(p, tq, tk, tv, st)
+                              : launch_pipe_t<D, BS, kModePrep>(p, tq, tk, tv, st);
 }
 
 }  // namespace
 
-bool fwd_pipe_fits(const FwdGeom &g, bool fused)
+bool fwd_pipe_fits(const FwdGeom &g, int mode)
 {
     QLayout l;
     if (g.d == 64)
-        l = g.bs == 32 ? pipe_layout<64, 32>(fused, g.umax, g.Tq, g.topk, g.nblk_max)
-                       : pipe_layout<64, 64>(fused, g.umax, g.Tq, g.topk, g.nblk_max);
+        l = g.bs == 32 ? pipe_layout<64, 32>(mode, g.umax, g.Tq, g.topk, g.nblk_max)
+                       : pipe_layout<64, 64>(mode, g.umax, g.Tq, g.topk, g.nblk_max);
     else
-        l = g.bs == 32 ? pipe_layout<128, 32>(fused, g.umax, g.Tq, g.topk, g.nblk_max)
-                       : pipe_layout<128, 64>(fused, g.umax, g.Tq, g.topk, g.nblk_max);
+        l = g.bs == 32 ? pipe_layout<128, 32>(mode, g.umax, g.Tq, g.topk, g.nblk_max)
+                       : pipe_layout<128, 64>(mode, g.umax, g.Tq, g.topk, g.nblk_max);
     return 1024 + l.bytes <= kQMaxSmem;
 }
 
-cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, bool fused, const CUtensorMap &tq,
+cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, int mode, const CUtensorMap &tq,
                                    const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
 {
     if (g.d == 64)
-        return g.bs == 32 ? launch_pipe_d<64, 32>(p, fused, tq, tk, tv, st) : launch_pipe_d<64, 64>(p, fused, tq, tk, tv, st);
-    return g.bs == 32 ? launch_pipe_d<128, 32>(p, fused, tq, tk, tv, st) : launch_pipe_d<128, 64>(p, fused, tq, tk, tv, st);
+        return g.bs == 32 ? launch_pipe_d<64, 32>(p, mode, tq, tk, tv, st) : launch_pipe_d<64, 64>(p, mode, tq, tk, tv, st);
+    return g.bs == 32 ? launch_pipe_d<128, 32>(p, mode, tq, tk, tv, st) : launch_pipe_d<128, 64>(p, mode, tq, tk, tv, st);
 }
 
 }  // namespace sfa

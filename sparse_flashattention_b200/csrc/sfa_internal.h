@@ -167,10 +167,13 @@ size_t fwd_attend_smem_bytes(const FwdGeom &g);
 // Pipelined query-major kernel (tile switches overlapped with the previous tile's tail): whether
 // its shared memory (which holds two copies of a tile's union) fits two CTAs per SM for this
 // geometry; when it does not, fwd_attend_kernel runs instead.
-// fused: the kernel builds each tile's canonical lists and union from the raw selections itself
-// (no prep kernel; the caller clears the tile counter), for calls without the block-major schedule.
-bool fwd_pipe_fits(const FwdGeom &g, bool fused);
-cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, bool fused, const CUtensorMap &tq,
+// mode 0: canonical lists and unions from the prep kernel; 1 (fused): the kernel builds each tile's
+// canonical lists and union from the raw selections itself (no prep kernel; the caller clears the
+// tile counter), for calls without the block-major schedule; 2 (window): dense attention under the
+// causal / window mask, every block holding a key of a row's window selected (no selection at all).
+constexpr int kPipePrep = 0, kPipeFused = 1, kPipeWindow = 2;
+bool fwd_pipe_fits(const FwdGeom &g, int mode);
+cudaError_t launch_fwd_attend_pipe(const FwdGeom &g, const FwdAttendParams &p, int mode, const CUtensorMap &tq,
                                    const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 cudaError_t launch_fwd_plan(const FwdGeom &g, const FwdPlanParams &p, cudaStream_t st);
 cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cudaStream_t st);
@@ -178,6 +181,15 @@ cudaError_t launch_fwd_attend_inv(const FwdGeom &g, const FwdAttendParams &p, co
                                   const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
 cudaError_t launch_fwd_merge(const FwdGeom &g, const FwdAttendParams &p, cudaStream_t st);
 size_t fwd_attend_inv_smem_bytes(const FwdGeom &g);
+
+// Gated mix of up to three branch outputs (o[b] == nullptr: branch absent).
+struct CombineParams {
+    const __nv_bfloat16 *o[3];
+    const float *g[3];
+    __nv_bfloat16 *out;
+    int64_t rows;  // total_q * Hq
+};
+cudaError_t launch_gated_combine(const CombineParams &p, int d, cudaStream_t st);
 
 cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStream_t st);
 cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaStream_t st);

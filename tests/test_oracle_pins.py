@@ -325,3 +325,20 @@ def test_workload_kept_pairs_closed_form():
     assert W.kept_pairs_nsa([256], 32, 4) == 22656
     assert W.kept_pairs_nsa([8192, 4096, 2048, 2048], 64, 16) == 14295040
     assert W.kept_pairs_nsa([65536, 32768], 64, 16) == 96583680
+
+
+def test_gated_combine_worked_example_and_gates():
+    """The gated mix out = sum_c g_c * o_c: a hand-computed value (0.25*4 + 0.75*8 = 7 and
+    0.25*(-2) + 0.75*2 = 1), a one-hot gate returning that branch unchanged, zero gates giving 0."""
+    import oracle
+    o1 = np.array([[[4.0, -2.0]]])
+    o2 = np.array([[[8.0, 2.0]]])
+    out = oracle.gated_combine([(o1, np.array([[0.25]])), (o2, np.array([[0.75]]))])
+    np.testing.assert_array_equal(out, [[[7.0, 1.0]]])
+    rng = np.random.default_rng(0)
+    bits = W.f32_to_bf16_bits(rng.standard_normal((3, 2, 8), dtype=np.float32))
+    other = W.f32_to_bf16_bits(rng.standard_normal((3, 2, 8), dtype=np.float32))
+    one, zero = np.ones((3, 2)), np.zeros((3, 2))
+    np.testing.assert_array_equal(oracle.gated_combine([(bits, one), (other, zero)]),
+                                  W.bf16_bits_to_f32(bits).astype(np.float64))
+    assert not oracle.gated_combine([(bits, zero), (other, zero)]).any()
