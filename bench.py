@@ -46,11 +46,11 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 # was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
     "fwd_attend_pipe_kernel": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
-                               "sha256": "58da5e8e1b953ea7b7c0e15b109ae9188a80b17f2d2fa08d32499b953f8acce4",
-                               "bytes": 138887680},
+                               "sha256": "c0bfe6e5fd6809d644e486b85999b49ba7c92229e2cc744a83dc0cf192bbb7ad",
+                               "bytes": 136768256},
     "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
-                            "sha256": "97cdb157c5c8fdc2494f46485bb2cc932316e20e85b4dd914934997ad8f3e280",
-                            "bytes": 274500864},
+                            "sha256": "0b3c75fd09b59df6d32629609ae9f9caec91a4576e50ef43e1aba16360f25f22",
+                            "bytes": 274462976},
 }
 
 

@@ -221,12 +221,16 @@ size_t sfa_window_fwd_workspace_size(void);
 /* Sliding-window branch: every query attends to all keys its mask keeps — the common semantics
  * above with every key selected (bottom-right causal limit when causal; window_left /
  * window_right as in the flash-attention-npu docstrings, -1 = unbounded; a plain causal or full
- * attention when no window is given).  Layouts, lengths, status word and errors as sfa_fwd;
- * there is no selection.  out bf16 (total_q, Hq, d); lse fp32 (Hq, total_q).  One kernel. */
+ * attention when no window is given).  window_left_per_head / window_right_per_head: int32 (Hq)
+ * device arrays or NULL; when given, q head h uses element h instead of window_left /
+ * window_right (negative = unbounded) — per-head windows as in the Flash-Sparse-Attention README
+ * ("Flex Local Window Attention").  Layouts, lengths, status word and errors as sfa_fwd; there is
+ * no selection.  out bf16 (total_q, Hq, d); lse fp32 (Hq, total_q).  One kernel. */
 int sfa_window_fwd(const void *q, const void *k, const void *v,
                    const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
                    int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
-                   int Hq, int Hkv, int d, int causal, int window_left, int window_right, float scale,
+                   int Hq, int Hkv, int d, int causal, int window_left, int window_right,
+                   const int32_t *window_left_per_head, const int32_t *window_right_per_head, float scale,
                    void *workspace, size_t workspace_bytes, int32_t *status_dev,
                    void *out, float *lse, sfa_stream_t stream);
 

@@ -57,7 +57,7 @@ def _load():
         "sfa_decode_attend": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]),
         "sfa_decode_noalloc": (I, [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, F, I, P, P, P, P]),
         "sfa_window_fwd_workspace_size": (Z, []),
-        "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, F, P, Z, P, P, P, P]),
+        "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P, F, P, Z, P, P, P, P]),
         "sfa_gated_combine": (I, [P, P, P, P, P, P, I, I, I, P, P]),
         "sfa_status_string": (ctypes.c_char_p, [I]),
         "sfa_last_launch_count": (I, []),
@@ -194,19 +194,29 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.T
 def window_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor, *,
                cu_seqlens_k: Optional[torch.Tensor] = None, max_seqlen_q: Optional[int] = None,
                max_seqlen_k: Optional[int] = None, causal: bool = True, window: Tuple[int, int] = (-1, -1),
+               window_per_head: Optional[Tuple[Optional[torch.Tensor], Optional[torch.Tensor]]] = None,
                scale: Optional[float] = None, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Sliding-window branch (sfa_window_fwd): every query attends to all keys its causal / window
-    mask keeps.  Layouts as fwd, no selection.  Returns out (total_q, Hq, d) bf16, lse (Hq, total_q)."""
+    mask keeps.  Layouts as fwd, no selection.  window_per_head: optional (left, right) int32 (Hq)
+    device tensors (either may be None) overriding `window` per query head.  Returns out
+    (total_q, Hq, d) bf16, lse (Hq, total_q)."""
     a = _FwdArgs(q, k, v, cu_seqlens_q, None, 64, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, window, scale,
                  topk=1)
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((a.Hq, a.total_q), dtype=torch.float32, device=q.device) if lse is None else lse
     ws = _workspace(workspace, int(_lib.sfa_window_fwd_workspace_size()), q.device)
+    wlh, wrh = window_per_head if window_per_head is not None else (None, None)
+    for t, name in ((wlh, "window_left_per_head"), (wrh, "window_right_per_head")):
+        if t is not None:
+            _need(t, name, torch.int32, 1)
+            if t.numel() != a.Hq:
+                raise ValueError(f"{name} must have Hq = {a.Hq} elements")
     rc = _lib.sfa_window_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), a.batch, a.max_sq,
-                             a.max_sk, a.total_q, a.total_k, a.Hq, a.Hkv, a.d, a.causal, a.wl, a.wr, a.scale, _ptr(ws),
-                             ws.numel() * ws.element_size(), _ptr(status), _ptr(out), _ptr(lse), _stream(stream))
+                             a.max_sk, a.total_q, a.total_k, a.Hq, a.Hkv, a.d, a.causal, a.wl, a.wr, _ptr(wlh),
+                             _ptr(wrh), a.scale, _ptr(ws), ws.numel() * ws.element_size(), _ptr(status), _ptr(out),
+                             _ptr(lse), _stream(stream))
     _check(rc)
     return out, lse
 

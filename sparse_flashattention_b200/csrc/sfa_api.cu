@@ -630,8 +630,10 @@ size_t sfa_window_fwd_workspace_size(void)
 
 int sfa_window_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqlens_q,
                    const int32_t *cu_seqlens_k, int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
-                   int Hq, int Hkv, int d, int causal, int window_left, int window_right, float scale, void *workspace,
-                   size_t workspace_bytes, int32_t *status_dev, void *out, float *lse, sfa_stream_t stream)
+                   int Hq, int Hkv, int d, int causal, int window_left, int window_right,
+                   const int32_t *window_left_per_head, const int32_t *window_right_per_head, float scale,
+                   void *workspace, size_t workspace_bytes, int32_t *status_dev, void *out, float *lse,
+                   sfa_stream_t stream)
 {
     g_last_launches = 0;
     // The window kernel tiles keys in 64-token blocks; no selection (topk 1 only sizes the geometry).
@@ -667,6 +669,8 @@ int sfa_window_fwd(const void *q, const void *k, const void *v, const int32_t *c
     p.causal = causal;
     p.wl = window_left;
     p.wr = window_right;
+    p.wl_head = window_left_per_head;
+    p.wr_head = window_right_per_head;
     const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)g.d);
     p.scale_log2 = (float)(sc * 1.4426950408889634);
     p.out = static_cast<__nv_bfloat16 *>(out);

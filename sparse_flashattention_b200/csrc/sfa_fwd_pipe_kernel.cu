@@ -210,12 +210,31 @@ __global__ void __launch_bounds__(kQThreads, 2)
                     if (lane == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_SEQLEN);
                     nblk = min(nblk, p.nblk_max);
                 }
+                // With per-head windows, the range covers every head's window of the kv head
+                // (all of them hold the last row's diagonal key, so their union has no gap).
                 const int delta = sk - sq, i0 = tok0, i1 = tok0 + ntok - 1;
-                int lo = 0, hi = min(sk, nblk * BS) - 1;
-                if (p.wl >= 0) lo = max(lo, i0 + delta - p.wl);
-                if (p.causal) hi = min(hi, i1 + delta);
-                if (p.wr >= 0) hi = min(hi, i1 + delta + p.wr);
-                blo = lo / BS;
+                const int cap = min(sk, nblk * BS) - 1;
+                int lo = 0x7fffffff, hi = -1;
+                const int nh = (p.wl_head || p.wr_head) ? p.G : 1;
+                for (int g = lane; g < nh; g += 32) {
+                    const int h = hk * p.G + g;
+                    const int wl = p.wl_head ? __ldg(&p.wl_head[h]) : p.wl;
+                    const int wr = p.wr_head ? __ldg(&p.wr_head[h]) : p.wr;
+                    int l = 0, r = cap;
+                    if (wl >= 0) l = max(l, i0 + delta - wl);
+                    if (p.causal) r = min(r, i1 + delta);
+                    if (wr >= 0) r = min(r, i1 + delta + wr);
+                    if (r >= l) {
+                        lo = min(lo, l);
+                        hi = max(hi, r);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    lo = min(lo, __shfl_xor_sync(full, lo, o));
+                    hi = max(hi, __shfl_xor_sync(full, hi, o));
+                }
+                blo = hi >= lo ? lo / BS : 0;
                 nU = hi >= lo ? hi / BS - blo + 1 : 0;
             } else if constexpr (FUSED) {
                 // The tile's canonical lists (one token per lane at a time) and the ascending union
@@ -502,10 +521,13 @@ __global__ void __launch_bounds__(kQThreads, 2)
             const bool row_valid = nU >= 0 && tok < ntok;
             const int i = tok0 + tok;
             const int delta = sk - sq;
+            // the row's window (per query head in the window mode when the caller gives per-head windows)
+            const int wl = WIN && p.wl_head ? __ldg(&p.wl_head[hk * p.G + g]) : p.wl;
+            const int wr = WIN && p.wr_head ? __ldg(&p.wr_head[hk * p.G + g]) : p.wr;
             int lo = 0, hi = sk - 1;
-            if (p.wl >= 0) lo = max(lo, i + delta - p.wl);
+            if (wl >= 0) lo = max(lo, i + delta - wl);
             if (p.causal) hi = min(hi, i + delta);
-            if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
+            if (wr >= 0) hi = min(hi, i + delta + wr);
             // This row's canonical (ascending) block list: in shared memory (fused mode), else read
             // from the prep kernel's output in global memory one entry ahead of its use.
             const int64_t t = (int64_t)q0 + i;

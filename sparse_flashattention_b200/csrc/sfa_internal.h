@@ -92,6 +92,7 @@ struct FwdAttendParams {
     int32_t *tile_counter;  // next query tile to hand out; [1] counts CTAs done.  The prep kernel
                             // clears both; the attend kernel's last CTA clears them again.
     int causal, wl, wr;
+    const int32_t *wl_head, *wr_head;  // window mode: per-q-head windows (nullptr: wl / wr for all heads)
     float scale_log2;  // softmax scale * log2(e)
     __nv_bfloat16 *out;
     float *lse;

@@ -2,6 +2,8 @@
 branch (sfa_window_fwd) against the fp64 oracle given every block of the sequence (the oracle then
 computes plain attention under the causal / window mask), and bitwise against sfa_fwd on that same
 all-blocks selection; the gated mix (sfa_gated_combine) against the oracle's float64 sum."""
+import dataclasses
+
 import numpy as np
 import pytest
 
@@ -96,3 +98,42 @@ def test_gated_combine_one_hot_is_the_branch(sfa):
     one = torch.ones((total_q, Hq), dtype=torch.float32, device="cuda")
     out = sfa.gated_combine([(os_[0], zero), (os_[1], one), (os_[2], zero)])
     assert torch.equal(out, os_[1])
+
+
+FLEX_CASES = [
+    # lengths q, lengths k, Hq, Hkv, d, causal, per-head left windows, per-head right windows (None: scalar -1)
+    ([700, 130, 64], [700, 130, 64], 8, 2, 128, 1, [0, 16, 64, 512, -1, 100, 7, 300], None),
+    ([257, 90], [400, 90], 6, 2, 64, 0, [0, 33, -1, 64, 5, 128], [0, 5, -1, 70, 64, 1]),
+    ([300], [300], 4, 4, 128, 0, None, [0, 64, 200, -1]),
+]
+
+
+@pytest.mark.parametrize("lq,lk,Hq,Hkv,d,causal,wlh,wrh", FLEX_CASES)
+def test_window_fwd_per_head_windows(sfa, oracle_lib, lq, lk, Hq, Hkv, d, causal, wlh, wrh):
+    """Flex local windows: each query head takes its own window; head h must equal the oracle run
+    with head h's window for every head."""
+    c = _case(lq, lk, Hq, Hkv, d, causal, -1, -1, seed=sum(lq) + Hq + 7)
+    dd = upload_prefill(c)
+    wl = torch.tensor(wlh, dtype=torch.int32, device="cuda") if wlh is not None else None
+    wr = torch.tensor(wrh, dtype=torch.int32, device="cuda") if wrh is not None else None
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = sfa.window_fwd(dd["q"], dd["k"], dd["v"], dd["cu_q"], cu_seqlens_k=dd["cu_k"], max_seqlen_q=max(lq),
+                              max_seqlen_k=max(lk), causal=bool(causal), window_per_head=(wl, wr), status=status)
+    assert int(status.item()) == 0
+    for h in range(Hq):
+        ch = dataclasses.replace(c, wl=wlh[h] if wlh is not None else -1, wr=wrh[h] if wrh is not None else -1)
+        ro, rl, _ = oracle_lib.fwd(ch)
+        assert_out_close(out[:, h:h + 1], ro[:, h:h + 1])
+        assert_lse_close(lse[h:h + 1], rl[h:h + 1])
+
+
+def test_window_fwd_uniform_per_head_equals_scalar(sfa):
+    """Per-head arrays holding one value for every head give the scalar-window result bit for bit."""
+    c = _case([600, 77], [600, 77], 8, 2, 128, 1, 256, 0, seed=11)
+    dd = upload_prefill(c)
+    kw = dict(cu_seqlens_k=dd["cu_k"], max_seqlen_q=600, max_seqlen_k=600, causal=True)
+    o1, l1 = sfa.window_fwd(dd["q"], dd["k"], dd["v"], dd["cu_q"], window=(256, 0), **kw)
+    wl = torch.full((8,), 256, dtype=torch.int32, device="cuda")
+    wr = torch.zeros(8, dtype=torch.int32, device="cuda")
+    o2, l2 = sfa.window_fwd(dd["q"], dd["k"], dd["v"], dd["cu_q"], window_per_head=(wl, wr), **kw)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
