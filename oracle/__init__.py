@@ -41,6 +41,9 @@ def _load():
                                        P, ctypes.c_int64, P, P, I]
         lib.sfa_oracle_fwd_index.restype = ctypes.c_int64
         lib.sfa_oracle_fwd_index.argtypes = [P, P, I, I, P, I, I, I, I, I, P, P]
+        lib.sfa_oracle_bwd.restype = ctypes.c_int64
+        lib.sfa_oracle_bwd.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, I, I, I, I, ctypes.c_double,
+                                       P, P, P, I]
         lib.sfa_oracle_decode.restype = None
         lib.sfa_oracle_decode.argtypes = [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, ctypes.c_double,
                                           P, P, I, P]
@@ -82,6 +85,24 @@ def fwd(case, rows=None, nthreads=None, sel=None):
                              _p(sel), sel.shape[-1], case.bs, case.causal, case.wl, case.wr, float(case.scale),
                              _p(r), n, _p(out), _p(lse), nthreads or default_threads())
     return out, lse, int(bad)
+
+
+def bwd(case, dout, nthreads=None, sel=None):
+    """Prefill backward oracle: gradients of sum(dout * out) through the selected attention.
+    dout: bf16 bit patterns (uint16), (total_q, Hq, d).  Returns (dq (total_q, Hq, d),
+    dk (total_k, Hkv, d), dv (total_k, Hkv, d), bad_ids), float64."""
+    lib = _load()
+    q, k, v = _c(case.q, np.uint16), _c(case.k, np.uint16), _c(case.v, np.uint16)
+    do = _c(dout, np.uint16)
+    cu_q, cu_k = _c(case.cu_q, np.int32), _c(case.cu_k, np.int32)
+    sel = _c(case.sel if sel is None else sel, np.int32)
+    dq = np.zeros((case.total_q, case.Hq, case.d), np.float64)
+    dk = np.zeros((case.total_k, case.Hkv, case.d), np.float64)
+    dv = np.zeros((case.total_k, case.Hkv, case.d), np.float64)
+    bad = lib.sfa_oracle_bwd(_p(q), _p(k), _p(v), _p(do), _p(cu_q), _p(cu_k), case.batch, case.Hq, case.Hkv,
+                             case.d, _p(sel), sel.shape[-1], case.bs, case.causal, case.wl, case.wr,
+                             float(case.scale), _p(dq), _p(dk), _p(dv), nthreads or default_threads())
+    return dq, dk, dv, int(bad)
 
 
 def fwd_index(case, sel=None):

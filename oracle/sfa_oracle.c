@@ -289,6 +289,144 @@ int64_t sfa_oracle_fwd_index(const int32_t *cu_q, const int32_t *cu_k, int batch
 }
 
 /* ---------------------------------------------------------------------------------------------
+ * Prefill backward: gradients of the selected attention with respect to q, k and v
+ * -------------------------------------------------------------------------------------------
+ * Sources: "Sparse FlashAttention" on Ascend (ggplus blog post), FlashAttentionScoreGrad case
+ * study at the end of the post: recompute the probabilities P, then dP = dO V^T, dS = P o (dP -
+ * rowsum(dO o O)), dQ = (dS K) * scale; the flash-sparse-attention README, "反向" (backward)
+ * example: gradients of the selected attention flow to query, key and value.  The pages stop at
+ * dQ; dK = scale * dS^T Q and dV = P^T dO are the same chain rule applied to the other two
+ * operands (the plainest reading).  Per row (query t, head h) over its kept keys a — the same
+ * key set as the forward:
+ *   p_a  = exp(s_a - lse),  s_a = scale * q . k_a
+ *   dp_a = dO . v_a;  D = sum_a p_a dp_a  (= dO . o);  ds_a = p_a (dp_a - D)
+ *   dq   = scale * sum_a ds_a k_a;   dk_a += scale * ds_a q;   dv_a += p_a dO
+ * A row with no kept key contributes nothing and has dq = 0.  Every key that no row keeps has
+ * dk = dv = 0.  Work is split by (sequence, kv head): the rows of one split are the only writers of
+ * its keys' dk / dv, so the sums need no locks and run in a fixed order. */
+
+typedef struct {
+    fwd_job F;              /* the forward's inputs and key-set rules */
+    const uint16_t *dout;   /* (total_q, Hq, d) bf16 bits */
+    double *dq, *dk, *dv;   /* (total_q, Hq, d), (total_k, Hkv, d), (total_k, Hkv, d) */
+} bwd_job;
+
+typedef struct {
+    const bwd_job *J;
+    int tid;
+    int64_t bad;
+} bwd_thread;
+
+static void *bwd_worker(void *arg)
+{
+    bwd_thread *th = (bwd_thread *)arg;
+    const bwd_job *J = th->J;
+    const fwd_job *F = &J->F;
+    const int G = F->Hq / F->Hkv, d = F->d;
+    const int cap = F->max_sk > 0 ? F->max_sk : 1;
+    unsigned char *mark = (unsigned char *)calloc((size_t)cap, 1);
+    int *keys = (int *)malloc(sizeof(int) * (size_t)cap);
+    double *p = (double *)malloc(sizeof(double) * (size_t)cap);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)cap);
+    double *qv = (double *)malloc(sizeof(double) * (size_t)d);
+    double *gv = (double *)malloc(sizeof(double) * (size_t)d);
+    int64_t bad = 0;
+    for (int job = th->tid; job < F->batch * F->Hkv; job += F->nthreads) {
+        const int b = job / F->Hkv, hk = job % F->Hkv;
+        for (int64_t t = F->cu_q[b]; t < F->cu_q[b + 1]; ++t) {
+            int64_t bad_row = 0;
+            const int n = fwd_keyset(F, t, hk, mark, keys, &bad_row);
+            bad += bad_row;
+            for (int g = 0; g < G; ++g) {
+                const int h = hk * G + g;
+                const int64_t flat = t * F->Hq + h;
+                double *dqrow = J->dq + flat * d;
+                for (int c = 0; c < d; ++c) dqrow[c] = 0.0;
+                if (n == 0) continue;
+                for (int c = 0; c < d; ++c) {
+                    qv[c] = bf16_value(F->q[flat * d + c]);
+                    gv[c] = bf16_value(J->dout[flat * d + c]);
+                }
+                /* probabilities, by the forward's definition (max-shifted for range) */
+                double m = -INFINITY;
+                for (int a = 0; a < n; ++a) {
+                    const uint16_t *kr = F->k + (((int64_t)F->cu_k[b] + keys[a]) * F->Hkv + hk) * d;
+                    double s = 0.0;
+                    for (int c = 0; c < d; ++c) s += qv[c] * bf16_value(kr[c]);
+                    p[a] = s * F->scale;
+                    if (p[a] > m) m = p[a];
+                }
+                double z = 0.0;
+                for (int a = 0; a < n; ++a) {
+                    p[a] = exp(p[a] - m);
+                    z += p[a];
+                }
+                double D = 0.0;
+                for (int a = 0; a < n; ++a) {
+                    p[a] /= z;
+                    const uint16_t *vr = F->v + (((int64_t)F->cu_k[b] + keys[a]) * F->Hkv + hk) * d;
+                    double x = 0.0;
+                    for (int c = 0; c < d; ++c) x += gv[c] * bf16_value(vr[c]);
+                    dp[a] = x;
+                    D += p[a] * x;
+                }
+                for (int a = 0; a < n; ++a) {
+                    const int64_t krow = ((int64_t)F->cu_k[b] + keys[a]) * F->Hkv + hk;
+                    const uint16_t *kr = F->k + krow * d;
+                    const double ds = p[a] * (dp[a] - D);
+                    double *dkrow = J->dk + krow * d, *dvrow = J->dv + krow * d;
+                    for (int c = 0; c < d; ++c) {
+                        dqrow[c] += F->scale * ds * bf16_value(kr[c]);
+                        dkrow[c] += F->scale * ds * qv[c];
+                        dvrow[c] += p[a] * gv[c];
+                    }
+                }
+            }
+        }
+    }
+    free(mark); free(keys); free(p); free(dp); free(qv); free(gv);
+    th->bad = bad;
+    return NULL;
+}
+
+/* Backward of sfa_oracle_fwd's attention (same arguments), given dout: dq (total_q, Hq, d) and
+ * dk, dv (total_k, Hkv, d), all written in full.  Returns the number of out-of-range block ids
+ * (each (token, kv head) slot once). */
+int64_t sfa_oracle_bwd(const uint16_t *q, const uint16_t *k, const uint16_t *v, const uint16_t *dout,
+                       const int32_t *cu_q, const int32_t *cu_k, int batch, int Hq, int Hkv, int d,
+                       const int32_t *sel, int topk, int bs, int causal, int wl, int wr, double scale,
+                       double *dq, double *dk, double *dv, int nthreads)
+{
+    bwd_job J;
+    memset(&J, 0, sizeof J);
+    J.F.q = q; J.F.k = k; J.F.v = v; J.F.cu_q = cu_q; J.F.cu_k = cu_k ? cu_k : cu_q;
+    J.F.batch = batch; J.F.Hq = Hq; J.F.Hkv = Hkv; J.F.d = d; J.F.sel = sel; J.F.topk = topk; J.F.bs = bs;
+    J.F.causal = causal; J.F.wl = wl; J.F.wr = wr;
+    J.F.scale = scale > 0 ? scale : 1.0 / sqrt((double)d);
+    J.F.nthreads = nthreads < 1 ? 1 : nthreads;
+    J.F.max_sk = max_len(J.F.cu_k, batch);
+    J.dout = dout; J.dq = dq; J.dk = dk; J.dv = dv;
+    const int64_t total_k = J.F.cu_k[batch];
+    memset(dk, 0, sizeof(double) * (size_t)(total_k * Hkv * d));
+    memset(dv, 0, sizeof(double) * (size_t)(total_k * Hkv * d));
+    pthread_t *ids = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)J.F.nthreads);
+    bwd_thread *ths = (bwd_thread *)calloc((size_t)J.F.nthreads, sizeof(bwd_thread));
+    for (int i = 0; i < J.F.nthreads; ++i) {
+        ths[i].J = &J;
+        ths[i].tid = i;
+        pthread_create(&ids[i], NULL, bwd_worker, &ths[i]);
+    }
+    int64_t bad = 0;
+    for (int i = 0; i < J.F.nthreads; ++i) {
+        pthread_join(ids[i], NULL);
+        bad += ths[i].bad;
+    }
+    free(ids);
+    free(ths);
+    return bad;
+}
+
+/* ---------------------------------------------------------------------------------------------
  * Paged decode (one new query token per sequence, at logical position L-1)
  * ------------------------------------------------------------------------------------------- */
 
