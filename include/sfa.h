@@ -137,6 +137,38 @@ int sfa_fwd_attend(const void *q, const void *k, const void *v,
                    void *out, float *lse, sfa_stream_t stream);
 
 /* ----------------------------------------------------------------------------------------
+ * Prefill backward
+ * The gradients of sfa_fwd's attention: with P the probabilities recomputed from the forward's
+ * lse, dP = dO V^T, dS = P o (dP - rowsum(dO o O)), dQ = scale dS K, dK = scale dS^T Q and
+ * dV = P^T dO, every product restricted to the keys each row selected and its mask keeps (the
+ * FlashAttentionScoreGrad case study of the Ascend "Sparse FlashAttention" article for P, dP, dS
+ * and dQ; dK and dV by the same chain rule; the flash-sparse-attention README's backward example
+ * for what is differentiated).
+ * -------------------------------------------------------------------------------------- */
+
+/* Bytes of device workspace sfa_bwd needs (0 when total_q == 0 or the sizes are unsupported).
+ * It grows with batch * Hkv * ceil(max_seqlen_k / block_size) * ceil(max_seqlen_q / 32) (the
+ * token bitmaps that invert the selection) and with total_q * Hkv * topk. */
+size_t sfa_bwd_workspace_size(int batch, int max_seqlen_q, int max_seqlen_k, int total_q,
+                              int Hq, int Hkv, int d, int topk, int block_size);
+
+/* Backward of sfa_fwd.  Inputs are sfa_fwd's (same layouts, selection, mask, scale) plus:
+ *   out   bf16 (total_q, Hq, d), the forward's output;  lse fp32 (Hq, total_q), its LSE
+ *   dout  bf16 (total_q, Hq, d), the gradient of the loss with respect to out
+ * Outputs (written in full; the caller owns them): dq bf16 (total_q, Hq, d), dk and dv bf16
+ * (total_k, Hkv, d).  A key no row keeps gets dk = dv = 0; a row that keeps no key gets dq = 0.
+ * This build: d = 128, block_size = 64 (else SFA_ERR_UNSUPPORTED).  Deterministic: the sums run
+ * in a fixed order whatever the timing.  Seven kernels and one memset on `stream`; status bits as
+ * sfa_fwd (SFA_DEV_BAD_SEQLEN also when a token of a sequence is past max_seqlen_q). */
+int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,
+            const float *lse, const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+            int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+            int Hq, int Hkv, int d, const int32_t *sel_idx, int topk, int block_size,
+            int causal, int window_left, int window_right, float scale,
+            void *workspace, size_t workspace_bytes, int32_t *status_dev,
+            void *dq, void *dk, void *dv, sfa_stream_t stream);
+
+/* ----------------------------------------------------------------------------------------
  * Paged top-k decode
  * -------------------------------------------------------------------------------------- */
 
@@ -248,7 +280,7 @@ const char *sfa_status_string(int status);
 
 /* Number of kernel launches the last successful call on this host thread made (prefill: 1,
  * or 6 when the call uses the block-major schedule; decode: 1 with at most 6 splits, else 2,
- * plus 1 when topk_tok > 2048; a stage: its own count; window branch, gated mix: 1). */
+ * plus 1 when topk_tok > 2048; a stage: its own count; window branch, gated mix: 1; backward: 7). */
 int sfa_last_launch_count(void);
 
 #ifdef __cplusplus

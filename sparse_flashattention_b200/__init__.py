@@ -59,6 +59,8 @@ def _load():
         "sfa_window_fwd_workspace_size": (Z, []),
         "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P, F, P, Z, P, P, P, P]),
         "sfa_gated_combine": (I, [P, P, P, P, P, P, I, I, I, P, P]),
+        "sfa_bwd_workspace_size": (Z, [I, I, I, I, I, I, I, I, I]),
+        "sfa_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, I, I, I, I, I, F, P, Z, P, P, P, P, P]),
         "sfa_status_string": (ctypes.c_char_p, [I]),
         "sfa_last_launch_count": (I, []),
     }
@@ -189,6 +191,41 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.T
                       _stream(stream))
     _check(rc)
     return out, lse
+
+
+def bwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size) -> int:
+    return int(_lib.sfa_bwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk,
+                                           block_size))
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
+        lse: torch.Tensor, cu_seqlens_q: torch.Tensor, sel_idx: torch.Tensor, block_size: int, *,
+        cu_seqlens_k: Optional[torch.Tensor] = None, max_seqlen_q: Optional[int] = None,
+        max_seqlen_k: Optional[int] = None, causal: bool = True, window: Tuple[int, int] = (-1, -1),
+        scale: Optional[float] = None, dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+        dv: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+        status: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Backward of fwd (sfa_bwd): given the forward's out and lse and the gradient dout of the loss
+    with respect to out, returns dq (total_q, Hq, d), dk and dv (total_k, Hkv, d), bf16.  The other
+    arguments are fwd's."""
+    a = _FwdArgs(q, k, v, cu_seqlens_q, sel_idx, block_size, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal,
+                 window, scale)
+    for t, name in ((out, "out"), (dout, "dout")):
+        _need(t, name, torch.bfloat16, 3)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} must have q's shape {tuple(q.shape)}")
+    _need(lse, "lse", torch.float32, 2)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    nbytes = bwd_workspace_size(*a.geom())
+    ws = _workspace(workspace, nbytes, q.device)
+    rc = _lib.sfa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(cu_seqlens_q),
+                      _ptr(cu_seqlens_k), a.batch, a.max_sq, a.max_sk, a.total_q, a.total_k, a.Hq, a.Hkv, a.d,
+                      _ptr(sel_idx), a.topk, a.bs, a.causal, a.wl, a.wr, a.scale, _ptr(ws),
+                      ws.numel() * ws.element_size(), _ptr(status), _ptr(dq), _ptr(dk), _ptr(dv), _stream(stream))
+    _check(rc)
+    return dq, dk, dv
 
 
 def window_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor, *,

@@ -307,6 +307,54 @@ int fwd_common_checks(const int32_t *cu_q, const int32_t *cu_k, int total_q, int
 }
 
 // ----------------------------------------------------------------------------------------
+// Backward geometry: the forward's prep region (canonical lists, unions, tile counter) followed by
+// the backward's own arrays.
+// ----------------------------------------------------------------------------------------
+int bwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv, int d, int topk, int bs,
+                 BwdGeom &g)
+{
+    int rc = fwd_geometry(batch, max_sq, max_sk, total_q, Hq, Hkv, d, topk, bs, g.f);
+    if (rc != SFA_OK) return rc;
+    if (d != 128 || bs != 64) return SFA_ERR_UNSUPPORTED;
+    g.f.inv = 0;  // the backward walks the query tiles; no block-major forward schedule
+    const int64_t total_sel = (int64_t)total_q * Hkv * topk;
+    if ((int64_t)total_q * Hq >= (1ll << 31) || total_sel >= (1ll << 31)) return SFA_ERR_UNSUPPORTED;
+    const int64_t R = (int64_t)batch * Hkv * g.f.nblk_max;
+    const int64_t words = std::max<int64_t>(1, ((int64_t)max_sq + 31) / 32);
+    if (R >= (1ll << 31) || R * words >= (1ll << 40)) return SFA_ERR_UNSUPPORTED;
+    g.R = (int)R;
+    g.words = (int)words;
+    const int64_t per_piece = (int64_t)kBwdPieceChunks * g.f.Tq;
+    // A row of c tokens makes ceil(c / per_piece) pieces; only rows of more than per_piece tokens
+    // need a running partial.
+    g.max_pieces = total_sel / per_piece + std::min(R, total_sel) + 1;
+    g.max_slots = total_sel / (per_piece + 1) + 1;
+    size_t off = align_up(g.f.off_tilectr + 8);
+    g.off_delta = off;
+    off = align_up(off + (size_t)total_q * Hq * 4);
+    g.off_zero = off;
+    g.off_bits = off;
+    off = align_up(off + (size_t)R * words * 4);
+    g.off_rowcnt = off;
+    off = align_up(off + (size_t)R * 4);
+    g.off_flags = off;
+    off = align_up(off + (size_t)g.max_slots * 4);
+    g.zero_bytes = off - g.off_zero;
+    g.off_ctrl = off;
+    off = align_up(off + sizeof(BwdCtrl));
+    g.off_rowoff = off;
+    off = align_up(off + (size_t)R * 4);
+    g.off_toks = off;
+    off = align_up(off + (size_t)total_sel * 4);
+    g.off_pieces = off;
+    off = align_up(off + (size_t)g.max_pieces * sizeof(BwdPiece));
+    g.off_part = off;
+    off = align_up(off + (size_t)g.max_slots * 2 * bs * d * 4);
+    g.bytes = total_q == 0 ? 0 : off;
+    return SFA_OK;
+}
+
+// ----------------------------------------------------------------------------------------
 // Decode geometry
 // ----------------------------------------------------------------------------------------
 int num_sms()
@@ -526,6 +574,107 @@ int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqle
                          workspace, status_dev, out, lse, stream);
     if (rc == SFA_OK) g_last_launches = 2 + 4 * g.inv;
     return rc;
+}
+
+size_t sfa_bwd_workspace_size(int batch, int max_seqlen_q, int max_seqlen_k, int total_q, int Hq, int Hkv, int d,
+                              int topk, int block_size)
+{
+    BwdGeom g;
+    if (bwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size, g) != SFA_OK) return 0;
+    return g.bytes;
+}
+
+int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout, const float *lse,
+            const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int batch, int max_seqlen_q, int max_seqlen_k,
+            int total_q, int total_k, int Hq, int Hkv, int d, const int32_t *sel_idx, int topk, int block_size,
+            int causal, int window_left, int window_right, float scale, void *workspace, size_t workspace_bytes,
+            int32_t *status_dev, void *dq, void *dk, void *dv, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    BwdGeom g;
+    int rc = bwd_geometry(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size, g);
+    if (rc != SFA_OK) return rc;
+    if ((rc = fwd_common_checks(cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k, causal,
+                                window_left, window_right)) != SFA_OK)
+        return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (total_k > 0 && (!dk || !dv || !aligned16(dk) || !aligned16(dv))) return SFA_ERR_INVALID_ARG;
+    if (total_q == 0 || batch == 0) {  // no query: every key's gradient is zero
+        if (total_k > 0) {
+            const size_t bytes = (size_t)total_k * Hkv * d * 2;
+            if (cudaMemsetAsync(dk, 0, bytes, st) != cudaSuccess || cudaMemsetAsync(dv, 0, bytes, st) != cudaSuccess)
+                return SFA_ERR_CUDA;
+        }
+        return SFA_OK;
+    }
+    if (!q || !k || !v || !out || !dout || !lse || !workspace || !sel_idx || !dq) return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq))
+        return SFA_ERR_INVALID_ARG;
+    if (total_k == 0) return SFA_ERR_UNSUPPORTED;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t *w = static_cast<uint8_t *>(workspace);
+    if (cudaMemsetAsync(w + g.off_zero, 0, g.zero_bytes, st) != cudaSuccess) return SFA_ERR_CUDA;
+    rc = fwd_prep_impl(g.f, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
+                       status_dev, st);
+    if (rc != SFA_OK) return rc;
+    CUtensorMap tq, tdo, tk, tv, tqr, tdor;
+    if (!encode_3d(tq, q, d, Hq, total_q, g.f.G, g.f.Tq) || !encode_3d(tdo, dout, d, Hq, total_q, g.f.G, g.f.Tq) ||
+        !encode_3d(tk, k, d, Hkv, total_k, 1, block_size) || !encode_3d(tv, v, d, Hkv, total_k, 1, block_size) ||
+        !encode_rows(tqr, q, d, (int64_t)total_q * Hq) || !encode_rows(tdor, dout, d, (int64_t)total_q * Hq))
+        return SFA_ERR_CUDA;
+    BwdParams p{};
+    p.out = static_cast<const __nv_bfloat16 *>(out);
+    p.dout = static_cast<const __nv_bfloat16 *>(dout);
+    p.lse = lse;
+    p.cu_q = cu_seqlens_q;
+    p.cu_k = cu_seqlens_k ? cu_seqlens_k : cu_seqlens_q;
+    p.sel_c = reinterpret_cast<const int32_t *>(w + g.f.off_sel_c);
+    p.cnt = reinterpret_cast<const int32_t *>(w + g.f.off_cnt);
+    p.ucnt = reinterpret_cast<const int32_t *>(w + g.f.off_ucnt);
+    p.uni = reinterpret_cast<const int32_t *>(w + g.f.off_union);
+    p.batch = batch;
+    p.total_q = total_q;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = g.f.G;
+    p.Tq = g.f.Tq;
+    p.nqt = g.f.nqt;
+    p.topk = topk;
+    p.umax = g.f.umax;
+    p.tiles = g.f.tiles;
+    p.nblk_max = g.f.nblk_max;
+    p.max_sq = max_seqlen_q;
+    p.words = g.words;
+    p.R = g.R;
+    p.causal = causal;
+    p.wl = window_left;
+    p.wr = window_right;
+    const double sc = scale > 0.f ? (double)scale : 1.0 / std::sqrt((double)d);
+    p.scale = (float)sc;
+    p.scale_log2 = (float)(sc * 1.4426950408889634);
+    p.delta = reinterpret_cast<float *>(w + g.off_delta);
+    p.bits = reinterpret_cast<uint32_t *>(w + g.off_bits);
+    p.rowcnt = reinterpret_cast<int32_t *>(w + g.off_rowcnt);
+    p.rowoff = reinterpret_cast<int32_t *>(w + g.off_rowoff);
+    p.toks = reinterpret_cast<int32_t *>(w + g.off_toks);
+    p.pieces = reinterpret_cast<BwdPiece *>(w + g.off_pieces);
+    p.ctrl = reinterpret_cast<BwdCtrl *>(w + g.off_ctrl);
+    p.flags = reinterpret_cast<int32_t *>(w + g.off_flags);
+    p.part = reinterpret_cast<float *>(w + g.off_part);
+    p.max_pieces = g.max_pieces;
+    p.max_slots = g.max_slots;
+    p.tile_counter = reinterpret_cast<int32_t *>(w + g.f.off_tilectr);
+    p.dq = static_cast<__nv_bfloat16 *>(dq);
+    p.dk = static_cast<__nv_bfloat16 *>(dk);
+    p.dv = static_cast<__nv_bfloat16 *>(dv);
+    p.status = status_dev;
+    if (launch_bwd_delta(g, p, st) != cudaSuccess || launch_bwd_index(g, p, st) != cudaSuccess ||
+        launch_bwd_plan(g, p, st) != cudaSuccess || launch_bwd_fill(g, p, st) != cudaSuccess ||
+        launch_bwd_dq(g, p, tq, tdo, tk, tv, st) != cudaSuccess ||
+        launch_bwd_dkdv(g, p, tqr, tdor, tk, tv, st) != cudaSuccess)
+        return SFA_ERR_CUDA;
+    g_last_launches = 7;
+    return SFA_OK;
 }
 
 int sfa_decode_num_splits(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits)

@@ -1,0 +1,963 @@
+// Prefill backward attention kernels (sm_100a): gradients of the selected attention.
+//
+// The chain rule through the softmax (the FlashAttentionScoreGrad case study of the Ascend
+// "Sparse FlashAttention" article): recompute P = exp(S - lse) from the forward's LSE, dP = dO V^T,
+// dS = P o (dP - D) with D = rowsum(dO o O), then dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO —
+// all restricted, like the forward, to the keys a row selected and its mask keeps.
+//
+// bwd_dq_kernel (query-major, one CTA per SM, persistent): the forward's tiles (Tq tokens x G heads
+//   = 128 rows of one kv head) walk the ascending union of their rows' blocks.  Per block the MMA
+//   thread issues S = Q K^T and dP = dO V^T into double-buffered TMEM, four softmax warps turn
+//   them into dS (bf16, written over the block's S columns), and dQ += dS K accumulates in TMEM
+//   (A operand from TMEM, K read MN-major).  TMEM: 2 x S, 2 x dP, dQ = 384 of 512 columns.
+//
+// bwd_dkdv_kernel (block-major, one CTA per SM, persistent): a piece is up to kBwdPieceChunks
+//   chunks of one (sequence, kv head, key block) row's token list.  K and V of the block stay in
+//   shared memory; each chunk's Q and dO rows (Tq tokens x G heads) are gathered four rows per TMA
+//   tile::gather4 copy into 128-byte-swizzled tiles.  Per chunk: S = Q K^T and dP = dO V^T (TMEM,
+//   double-buffered); the softmax warps write P and dS (bf16) into shared memory; then
+//   dV^T += dO^T P and dK^T += Q^T dS, with the gathered tiles read MN-major as the A operand
+//   (M = d = 128) and P / dS MN-major as B.  The accumulators live in TMEM across the piece; the
+//   epilogue writes bf16 dK / dV, or, for a row cut into several pieces, adds the row's fp32
+//   running partial in piece order (piece i waits until pieces 0..i-1 are in it), so the sums do
+//   not depend on timing.
+//
+// Every wait is bounded (sfa_device.cuh); on a timeout the CTA records SFA_DEV_TIMEOUT, lets its
+// copies and MMAs land, frees TMEM and exits.
+#include "sfa_device.cuh"
+
+namespace sfa {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// =========================================================================================
+// dQ
+// =========================================================================================
+constexpr int kDqThreads = 224;  // warp 0 producer, 1 MMA, 2..5 softmax / epilogue, 6 tile fetch
+constexpr int kDqStages = 3;     // K/V ring depth
+
+template <int D, int BS>
+struct DqCfg {
+    static constexpr int kTileBytes = 128 * D * 2;  // the tile's Q (or dO)
+    static constexpr int kKVBytes = BS * D * 2;     // one K (or V) block
+    static constexpr int kOffDO = kTileBytes;
+    static constexpr int kOffK = 2 * kTileBytes;
+    static constexpr int kOffV = kOffK + kDqStages * kKVBytes;
+    static constexpr int kOffMeta = kOffV + kDqStages * kKVBytes;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColDP = 2 * BS;
+    static constexpr int kColDQ = 4 * BS;
+    static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
+    static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, true);
+    static_assert(kColDQ + D <= kTmemCols, "TMEM columns");
+};
+
+struct DqTile {
+    int done, nU, hk, q0, sq, k0, sk, tok0, ntok;
+};
+
+struct DqMeta {
+    uint64_t q_full, q_empty;
+    uint64_t kv_full[kDqStages], kv_empty[kDqStages];
+    uint64_t s_full[2], p_full[2], dq_done[2];
+    uint64_t o_free;
+    uint64_t meta_full[2], meta_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    DqTile info[2];
+};
+
+template <int D, int BS>
+__host__ __device__ constexpr size_t dq_union_offset()
+{
+    return DqCfg<D, BS>::kOffMeta + ((sizeof(DqMeta) + 15) & ~size_t(15));
+}
+
+template <int D, int BS>
+__global__ void __launch_bounds__(kDqThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmdo,
+                  const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv, const BwdParams p)
+{
+    using C = DqCfg<D, BS>;
+    extern __shared__ uint8_t dq_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dq_smem_raw) + 1023) & ~uintptr_t(1023));
+    DqMeta *meta = reinterpret_cast<DqMeta *>(smem + C::kOffMeta);
+    const int U = p.umax;
+    int *s_union = reinterpret_cast<int *>(smem + dq_union_offset<D, BS>());  // [2][U]
+    uint8_t *sQ = smem, *sDO = smem + C::kOffDO, *sK = smem + C::kOffK, *sV = smem + C::kOffV;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const unsigned full = 0xffffffffu;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&meta->q_full, 1);
+        mbar_init(&meta->q_empty, 1);
+        for (int s = 0; s < kDqStages; ++s) {
+            mbar_init(&meta->kv_full[s], 1);
+            mbar_init(&meta->kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&meta->s_full[s], 1);
+            mbar_init(&meta->p_full[s], 128);
+            mbar_init(&meta->dq_done[s], 1);
+            mbar_init(&meta->meta_full[s], 32);
+            mbar_init(&meta->meta_empty[s], 6);  // producer, MMA thread, 4 softmax warps
+        }
+        mbar_init(&meta->o_free, 128);
+        mbar_init(&meta->drain, 1);
+        meta->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&meta->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = meta->tmem_base;
+    volatile int *abort_flag = &meta->abort_flag;
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmq);
+        tma_prefetch_desc(&tmdo);
+        tma_prefetch_desc(&tmk);
+        tma_prefetch_desc(&tmv);
+    }
+
+    if (warp == 6) {
+        // ------------------------------------------------------------------ tile fetch
+        int k = 0;
+        bool ok = true;
+        while (ok) {
+            const int m = k & 1;
+            if (k >= 2) ok = mbar_wait(&meta->meta_empty[m], ((k >> 1) - 1) & 1, abort_flag, p.status);
+            ok = __all_sync(full, ok);
+            if (!ok) break;
+            DqTile &ti = meta->info[m];
+            int *uni = s_union + m * U;
+            int tile, hk, b, qt, q0, sq;
+            while (true) {  // next tile that holds query rows
+                tile = 0;
+                if (lane == 0) tile = atomicAdd(p.tile_counter, 1);
+                tile = __shfl_sync(full, tile, 0);
+                if (tile >= p.tiles) break;
+                hk = tile % p.Hkv;
+                const int rest = tile / p.Hkv;
+                b = rest % p.batch;
+                qt = p.nqt - 1 - rest / p.batch;
+                q0 = p.cu_q[b];
+                sq = p.cu_q[b + 1] - q0;
+                if (qt * p.Tq < sq) break;
+            }
+            if (tile >= p.tiles) {
+                if (lane == 0) ti.done = 1;
+                mbar_arrive(&meta->meta_full[m]);
+                break;
+            }
+            const int nU = p.ucnt[tile];
+            for (int i = lane; i < nU; i += 32) uni[i] = p.uni[(int64_t)tile * U + i];
+            if (lane == 0) {
+                ti.done = 0;
+                ti.nU = nU;
+                ti.hk = hk;
+                ti.q0 = q0;
+                ti.sq = sq;
+                ti.k0 = p.cu_k[b];
+                ti.sk = p.cu_k[b + 1] - ti.k0;
+                ti.tok0 = qt * p.Tq;
+                ti.ntok = min(p.Tq, sq - ti.tok0);
+            }
+            mbar_arrive(&meta->meta_full[m]);
+            ++k;
+        }
+    } else if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        int kv_st = 0, kv_ph = 0, nkv = 0, q_phases = 0;
+        if (lane == 0) {
+            int k = 0;
+            bool ok = true;
+            while (ok) {
+                const int m = k & 1;
+                ok = mbar_wait(&meta->meta_full[m], (k >> 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                const DqTile &ti = meta->info[m];
+                if (ti.done) break;
+                const int *uni = s_union + m * U;
+                const int n = ti.nU, hk = ti.hk, k0 = ti.k0;
+                if (k >= 1) ok = mbar_wait(&meta->q_empty, (k - 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&meta->q_full, n > 0 ? 2u * D * (uint32_t)(p.G * p.Tq) * 2u : 0u);
+                if (n > 0)
+                    for (int c = 0; c < D / 64; ++c) {
+                        tma_load_3d(&tmq, &meta->q_full, sQ + c * (128 * 128), c * 64, hk * p.G, ti.q0 + ti.tok0);
+                        tma_load_3d(&tmdo, &meta->q_full, sDO + c * (128 * 128), c * 64, hk * p.G, ti.q0 + ti.tok0);
+                    }
+                q_phases = k + 1;
+                for (int u = 0; ok && u < n; ++u) {
+                    const int st = kv_st;
+                    if (nkv >= kDqStages && !mbar_wait(&meta->kv_empty[st], kv_ph ^ 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    const int row = k0 + uni[u] * BS;
+                    mbar_arrive_expect_tx(&meta->kv_full[st], 2u * (uint32_t)C::kKVBytes);
+                    for (int c = 0; c < D / 64; ++c) {
+                        tma_load_3d(&tmk, &meta->kv_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                        tma_load_3d(&tmv, &meta->kv_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                    }
+                    ++nkv;
+                    if (++kv_st == kDqStages) {
+                        kv_st = 0;
+                        kv_ph ^= 1;
+                    }
+                }
+                if (!ok) break;
+                mbar_arrive(&meta->meta_empty[m]);
+                ++k;
+            }
+            if (*abort_flag) {  // let every copy this CTA started land
+                if (q_phases > 0) mbar_drain(&meta->q_full, (q_phases - 1) & 1);
+                for (int st = 0; st < kDqStages; ++st) {
+                    const int c = nkv > st ? (nkv - st + kDqStages - 1) / kDqStages : 0;
+                    if (c > 0) mbar_drain(&meta->kv_full[st], (c - 1) & 1);
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint64_t dQd = sdesc_sw128(smem_u32(sQ), 16, 1024);
+            const uint64_t dDOd = sdesc_sw128(smem_u32(sDO), 16, 1024);
+            const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16, 1024);
+            const uint64_t dKmn0 = sdesc_sw128(smem_u32(sK), BS * 128, 1024);  // K as the MN-major B of dS K
+            int k = 0, jg0 = 0;
+            int s_st = 0, s_ph = 0, p_st = 0, p_ph = 0;
+            bool ok = true;
+            while (ok) {
+                const int m = k & 1;
+                ok = mbar_wait(&meta->meta_full[m], (k >> 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                const DqTile &ti = meta->info[m];
+                if (ti.done) break;
+                const int n = ti.nU;
+                ok = mbar_wait(&meta->q_full, k & 1, abort_flag, p.status);
+                if (!ok) break;
+                if (n == 0) umma_commit(&meta->q_empty);
+                // S/dP of block u once its K and V have landed and dQ u-2 was issued (S u overwrites
+                // the buffer whose dS that MMA reads); dQ u once dS u is written.  The tile's first
+                // dQ MMA overwrites the accumulator: it waits until the previous epilogue read it.
+                bool ofree = (k == 0);
+                int ns = 0, np = 0, spins = 0;
+                uint64_t idle_since = 0;
+                while (ok && np < n) {
+                    bool progressed = false;
+                    if (ns < n && ns <= np + 1) {
+                        const int jg = jg0 + ns, st = s_st;
+                        if (mbar_try_wait(smem_u32(&meta->kv_full[st]), s_ph)) {
+                            tc_fence_after();
+                            const uint32_t tS = tmem + (jg & 1) * BS, tDP = tmem + C::kColDP + (jg & 1) * BS;
+                            const uint32_t kvo = (uint32_t)st * C::kKVBytes;
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint64_t ao = (uint64_t)(((ks >> 2) * (128 * 128) + (ks & 3) * 32) >> 4);
+                                const uint64_t bo = (uint64_t)((kvo + (ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
+                                umma_bf16(tS, dQd + ao, dK0 + bo, C::kIdescS, ks > 0 ? 1u : 0u);
+                            }
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint64_t ao = (uint64_t)(((ks >> 2) * (128 * 128) + (ks & 3) * 32) >> 4);
+                                const uint64_t bo = (uint64_t)((kvo + (ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
+                                umma_bf16(tDP, dDOd + ao, dV0 + bo, C::kIdescS, ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&meta->s_full[jg & 1]);
+                            ++ns;
+                            if (++s_st == kDqStages) {
+                                s_st = 0;
+                                s_ph ^= 1;
+                            }
+                            if (ns == n) umma_commit(&meta->q_empty);
+                            progressed = true;
+                        }
+                    }
+                    if (np < ns) {
+                        const int ig = jg0 + np, st = p_st;
+                        if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
+                            (ofree || mbar_try_wait(smem_u32(&meta->o_free), (k - 1) & 1))) {
+                            ofree = true;
+                            tc_fence_after();
+#pragma unroll
+                            for (int ks = 0; ks < BS / 16; ++ks)  // dS (bf16) sits in the first BS/2 columns
+                                umma_bf16_tmem_a(tmem + C::kColDQ, tmem + (ig & 1) * BS + ks * 8,
+                                                 dKmn0 + (uint64_t)((st * C::kKVBytes + ks * 16 * 128) >> 4), C::kIdescDQ,
+                                                 (np > 0 || ks > 0) ? 1u : 0u);
+                            umma_commit(&meta->dq_done[ig & 1]);
+                            umma_commit(&meta->kv_empty[st]);
+                            ++np;
+                            if (++p_st == kDqStages) {
+                                p_st = 0;
+                                p_ph ^= 1;
+                            }
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        spins = 0;
+                    } else if (*abort_flag) {
+                        ok = false;
+                    } else if (spins++ == 0) {
+                        idle_since = global_timer_ns();
+                    } else if ((spins & 63) == 0 && global_timer_ns() - idle_since > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        if (p.status) atomicOr(p.status, SFA_DEV_TIMEOUT);
+                        ok = false;
+                    }
+                }
+                if (!ok) break;
+                mbar_arrive(&meta->meta_empty[m]);
+                jg0 += n;
+                ++k;
+            }
+            if (!ok) {
+                umma_commit(&meta->drain);
+                mbar_drain(&meta->drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ softmax + epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int tok = r / p.G, g = r - tok * p.G;
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        int k = 0, jg0 = 0;
+        bool ok = true;
+        while (ok) {
+            const int m = k & 1;
+            ok = warp_all_ok(mbar_wait(&meta->meta_full[m], (k >> 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+            const DqTile &ti = meta->info[m];
+            if (ti.done) break;
+            const int n = ti.nU, ntok = ti.ntok, hk = ti.hk;
+            const int *uni = s_union + m * U;
+            const bool row_valid = tok < ntok;
+            const int i = ti.tok0 + tok;
+            const int64_t t = (int64_t)ti.q0 + i;
+            const int h = hk * p.G + g;
+            const int delta_k = ti.sk - ti.sq;
+            int lo = 0, hi = ti.sk - 1;
+            if (p.wl >= 0) lo = max(lo, i + delta_k - p.wl);
+            if (p.causal) hi = min(hi, i + delta_k);
+            if (p.wr >= 0) hi = min(hi, i + delta_k + p.wr);
+            const int32_t *gl = p.sel_c + (row_valid ? (t * p.Hkv + hk) * p.topk : 0);
+            const int mycnt = row_valid ? p.cnt[t * p.Hkv + hk] : 0;
+            int nxt = mycnt > 0 ? gl[0] : -1, ptr = 0;
+            const float lse2 = row_valid ? p.lse[(int64_t)h * p.total_q + t] * kLog2e : 0.f;
+            const float dlt = row_valid ? p.delta[(int64_t)h * p.total_q + t] : 0.f;
+            for (int j = 0; j < n; ++j) {
+                const int jg = jg0 + j;
+                const int s = uni[j];
+                const bool selected = nxt == s;
+                if (selected) {
+                    ++ptr;
+                    nxt = ptr < mycnt ? gl[ptr] : -1;
+                }
+                ok = warp_all_ok(mbar_wait(&meta->s_full[jg & 1], (jg >> 1) & 1, abort_flag, p.status));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t tS = lane_base + (jg & 1) * BS, tDP = lane_base + C::kColDP + (jg & 1) * BS;
+                if (!__any_sync(full, selected)) {  // dS = 0 for all 32 rows: dQ unchanged
+                    uint32_t zero[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) zero[e] = 0u;
+#pragma unroll
+                    for (int hf = 0; hf < BS / 32; ++hf) tmem_st16(tS + hf * 16, zero);
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(&meta->p_full[jg & 1]);
+                    continue;
+                }
+                const int kb = s * BS;
+                const bool inner = kb >= lo && kb + BS - 1 <= hi;
+#pragma unroll
+                for (int hf = 0; hf < BS / 32; ++hf) {  // 32 keys at a time; dS half hf -> columns [16 hf, 16 hf + 16)
+                    uint32_t sr[32], dr[32], packed[16];
+                    tmem_ld32(tS + hf * 32, sr);
+                    tmem_ld32(tDP + hf * 32, dr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c0 = hf * 32 + 2 * e, c1 = c0 + 1;
+                        const bool k0v = selected && (inner || (kb + c0 >= lo && kb + c0 <= hi));
+                        const bool k1v = selected && (inner || (kb + c1 >= lo && kb + c1 <= hi));
+                        const float p0 = k0v ? ex2(fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -lse2)) : 0.f;
+                        const float p1 = k1v ? ex2(fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -lse2)) : 0.f;
+                        packed[e] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * e]) - dlt),
+                                                p1 * (__uint_as_float(dr[2 * e + 1]) - dlt));
+                    }
+                    tmem_st16(tS + hf * 16, packed);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&meta->p_full[jg & 1]);
+            }
+            if (!ok) break;
+            // ------------------------------------------------------------ epilogue: dq = scale * dS K
+            if (n > 0) {
+                const int lg = jg0 + n - 1;
+                ok = warp_all_ok(mbar_wait(&meta->dq_done[lg & 1], (lg >> 1) & 1, abort_flag, p.status));
+                if (!ok) break;
+                tc_fence_after();
+            }
+            __nv_bfloat16 *qrow = p.dq + (t * p.Hq + h) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                if (n > 0) {
+                    tmem_ld32(lane_base + C::kColDQ + c * 32, o);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0u;
+                }
+                if (row_valid) {
+                    uint32_t wv[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * p.scale, __uint_as_float(o[2 * e + 1]) * p.scale);
+                    uint4 *dst = reinterpret_cast<uint4 *>(qrow + c * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&meta->o_free);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&meta->meta_empty[m]);
+            jg0 += n;
+            ++k;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {  // the last CTA out leaves the tile counters cleared
+        __threadfence();
+        if (atomicAdd(&p.tile_counter[1], 1) == (int)gridDim.x - 1) {
+            p.tile_counter[0] = 0;
+            p.tile_counter[1] = 0;
+        }
+    }
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+// =========================================================================================
+// dK, dV
+// =========================================================================================
+constexpr int kKvThreads = 192;  // warp 0 loads, 1 MMA, 2..5 softmax / epilogue
+
+template <int D, int BS>
+struct KvCfg {
+    static_assert(D == 128, "the transposed products take d as the MMA's M dimension (128)");
+    static constexpr int kTileBytes = 128 * D * 2;  // 128 gathered rows of Q (or dO)
+    static constexpr int kKVBytes = BS * D * 2;
+    static constexpr int kPBytes = 128 * BS * 2;    // P (or dS): 128 rows x BS keys, bf16
+    static constexpr int kOffQ = 0;                 // [2] stages
+    static constexpr int kOffDO = 2 * kTileBytes;   // [2]
+    static constexpr int kOffK = 4 * kTileBytes;
+    static constexpr int kOffV = kOffK + kKVBytes;
+    static constexpr int kOffP = kOffV + kKVBytes;  // [2]
+    static constexpr int kOffDS = kOffP + 2 * kPBytes;
+    static constexpr int kOffMeta = kOffDS + 2 * kPBytes;
+    static constexpr int kTmemCols = 512;
+    static constexpr int kColDP = 2 * BS;
+    static constexpr int kColDV = 4 * BS;
+    static constexpr int kColDK = 5 * BS;
+    static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
+    static constexpr uint32_t kIdescT = idesc_bf16_f32_ab(128, BS, true, true);
+};
+
+struct PieceInfo {
+    int done, ntok, tok_begin, idx, npieces, slot, hk, s, q0, sq, k0, sk, rowoff, pad[3];
+};
+
+struct KvMeta {
+    uint64_t meta_full[2], meta_empty[2];
+    uint64_t kv_full, kv_empty;
+    uint64_t qd_full[2], qd_empty[2];
+    uint64_t s_full[2], p_full[2], p_free[2];
+    uint64_t acc_full, acc_free, epi_bar, drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    PieceInfo info[2];
+};
+
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t *ptr)
+{
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int32_t *ptr, int v)
+{
+    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+
+// Wait until *flag >= target (another CTA's piece of the same row is in the running partial).
+__device__ bool wait_flag(const int32_t *flag, int target, volatile int *abort_flag, int32_t *status)
+{
+    uint64_t t0 = 0;
+    int spins = 0;
+    while (ld_acquire_gpu(flag) < target) {
+        if (*abort_flag) return false;
+        if (spins++ == 0) {
+            t0 = global_timer_ns();
+        } else if ((spins & 255) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            if (status) atomicOr(status, SFA_DEV_TIMEOUT);
+            return false;
+        }
+        __nanosleep(128);
+    }
+    return true;
+}
+
+template <int D, int BS>
+__global__ void __launch_bounds__(kKvThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmqr, const __grid_constant__ CUtensorMap tmdor,
+                    const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv, const BwdParams p)
+{
+    using C = KvCfg<D, BS>;
+    extern __shared__ uint8_t kv_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(kv_smem_raw) + 1023) & ~uintptr_t(1023));
+    KvMeta *meta = reinterpret_cast<KvMeta *>(smem + C::kOffMeta);
+    uint8_t *sQ = smem + C::kOffQ, *sDO = smem + C::kOffDO, *sK = smem + C::kOffK, *sV = smem + C::kOffV;
+    uint8_t *sP = smem + C::kOffP, *sDS = smem + C::kOffDS;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // Rows of a chunk past its tokens are never loaded; they must hold finite values (they meet
+    // P = dS = 0 in the transposed products), so the gather tiles start out zeroed.
+    for (int e = threadIdx.x; e < 4 * C::kTileBytes / 16; e += kKvThreads)
+        reinterpret_cast<uint4 *>(smem)[e] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&meta->meta_full[s], 1);
+            mbar_init(&meta->meta_empty[s], 6);  // producer, MMA thread, 4 softmax warps
+            mbar_init(&meta->qd_full[s], 1);
+            mbar_init(&meta->qd_empty[s], 1);
+            mbar_init(&meta->s_full[s], 1);
+            mbar_init(&meta->p_full[s], 128);
+            mbar_init(&meta->p_free[s], 1);
+        }
+        mbar_init(&meta->kv_full, 1);
+        mbar_init(&meta->kv_empty, 1);
+        mbar_init(&meta->acc_full, 1);
+        mbar_init(&meta->acc_free, 128);
+        mbar_init(&meta->epi_bar, 128);
+        mbar_init(&meta->drain, 1);
+        meta->abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&meta->tmem_base, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = meta->tmem_base;
+    volatile int *abort_flag = &meta->abort_flag;
+    const int npieces_total = p.ctrl->npieces;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ loads
+        if (lane == 0) {
+            tma_prefetch_desc(&tmqr);
+            tma_prefetch_desc(&tmdor);
+            tma_prefetch_desc(&tmk);
+            tma_prefetch_desc(&tmv);
+        }
+        int kp = 0, cg = 0, kv_issued = 0;
+        bool ok = true;
+        while (ok) {
+            const int m = kp & 1;
+            if (kp >= 2) ok = warp_all_ok(mbar_wait(&meta->meta_empty[m], ((kp >> 1) - 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+            int piece = 0;
+            if (lane == 0) piece = atomicAdd(&p.ctrl->counter, 1);
+            piece = __shfl_sync(0xffffffffu, piece, 0);
+            PieceInfo &pi = meta->info[m];
+            if (piece >= npieces_total) {
+                if (lane == 0) {
+                    pi.done = 1;
+                    mbar_arrive(&meta->meta_full[m]);
+                }
+                break;
+            }
+            const BwdPiece pc = p.pieces[piece];
+            const int s = pc.row % p.nblk_max, bh = pc.row / p.nblk_max;
+            const int hk = bh % p.Hkv, b = bh / p.Hkv;
+            const int q0 = __ldg(&p.cu_q[b]), k0 = __ldg(&p.cu_k[b]);
+            const int rowoff = p.rowoff[pc.row];
+            if (lane == 0) {
+                pi.done = 0;
+                pi.ntok = pc.ntok;
+                pi.tok_begin = pc.tok_begin;
+                pi.idx = pc.idx;
+                pi.npieces = pc.npieces;
+                pi.slot = pc.slot;
+                pi.hk = hk;
+                pi.s = s;
+                pi.q0 = q0;
+                pi.sq = __ldg(&p.cu_q[b + 1]) - q0;
+                pi.k0 = k0;
+                pi.sk = __ldg(&p.cu_k[b + 1]) - k0;
+                pi.rowoff = rowoff;
+                mbar_arrive(&meta->meta_full[m]);
+            }
+            // K and V of the block, once the previous piece's MMAs are done with them.
+            if (kp >= 1) ok = warp_all_ok(mbar_wait(&meta->kv_empty, (kp - 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&meta->kv_full, 2u * (uint32_t)C::kKVBytes);
+                for (int c = 0; c < D / 64; ++c) {
+                    tma_load_3d(&tmk, &meta->kv_full, sK + c * (BS * 128), c * 64, hk, k0 + s * BS);
+                    tma_load_3d(&tmv, &meta->kv_full, sV + c * (BS * 128), c * 64, hk, k0 + s * BS);
+                }
+            }
+            ++kv_issued;
+            const int nch = (pc.ntok + p.Tq - 1) / p.Tq;
+            const int32_t *toks = p.toks + rowoff + pc.tok_begin;
+            for (int c = 0; c < nch; ++c) {
+                const int st = cg & 1;
+                if (cg >= 2) ok = warp_all_ok(mbar_wait(&meta->qd_empty[st], ((cg >> 1) - 1) & 1, abort_flag, p.status));
+                if (!ok) break;
+                const int ntc = min(p.Tq, pc.ntok - c * p.Tq), rows = ntc * p.G, n4 = (rows + 3) >> 2;
+                if (lane == 0) mbar_arrive_expect_tx(&meta->qd_full[st], (uint32_t)n4 * 512u * (D / 64) * 2u);
+                __syncwarp();
+                for (int g4 = lane; g4 < n4; g4 += 32) {
+                    int gr[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int rr = min(4 * g4 + e, rows - 1);  // a short last group repeats its last row
+                        const int tt = rr / p.G, gg = rr - tt * p.G;
+                        gr[e] = (q0 + toks[c * p.Tq + tt]) * p.Hq + hk * p.G + gg;
+                    }
+#pragma unroll
+                    for (int cc = 0; cc < D / 64; ++cc) {
+                        const int so = st * C::kTileBytes + cc * (128 * 128) + g4 * 512;
+                        tma_gather4(&tmqr, &meta->qd_full[st], sQ + so, cc * 64, gr[0], gr[1], gr[2], gr[3]);
+                        tma_gather4(&tmdor, &meta->qd_full[st], sDO + so, cc * 64, gr[0], gr[1], gr[2], gr[3]);
+                    }
+                }
+                ++cg;
+            }
+            if (!ok) break;
+            if (lane == 0) mbar_arrive(&meta->meta_empty[m]);
+            ++kp;
+        }
+        if (*abort_flag && lane == 0) {  // let every copy this CTA started land
+            if (kv_issued > 0) mbar_drain(&meta->kv_full, (uint32_t)((kv_issued - 1) & 1));
+            for (int st = 0; st < 2; ++st) {
+                const int c = cg > st ? (cg - st + 1) / 2 : 0;
+                if (c > 0) mbar_drain(&meta->qd_full[st], (c - 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint64_t dQ[2], dDO[2], dQt[2], dDOt[2], dP[2], dDS[2];
+            for (int b = 0; b < 2; ++b) {
+                dQ[b] = sdesc_sw128(smem_u32(sQ + b * C::kTileBytes), 16, 1024);
+                dDO[b] = sdesc_sw128(smem_u32(sDO + b * C::kTileBytes), 16, 1024);
+                dQt[b] = sdesc_sw128(smem_u32(sQ + b * C::kTileBytes), 128 * 128, 1024);   // M = d, MN-major
+                dDOt[b] = sdesc_sw128(smem_u32(sDO + b * C::kTileBytes), 128 * 128, 1024);
+                dP[b] = sdesc_sw128(smem_u32(sP + b * C::kPBytes), C::kPBytes, 1024);     // N = keys, MN-major
+                dDS[b] = sdesc_sw128(smem_u32(sDS + b * C::kPBytes), C::kPBytes, 1024);
+            }
+            const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);
+            const uint64_t dV = sdesc_sw128(smem_u32(sV), 16, 1024);
+            int kp = 0, cg0 = 0;
+            bool ok = true;
+            while (ok) {
+                const int m = kp & 1;
+                ok = mbar_wait(&meta->meta_full[m], (kp >> 1) & 1, abort_flag, p.status);
+                if (!ok) break;
+                const PieceInfo &pi = meta->info[m];
+                if (pi.done) break;
+                const int nch = (pi.ntok + p.Tq - 1) / p.Tq;
+                ok = mbar_wait(&meta->kv_full, kp & 1, abort_flag, p.status);
+                if (!ok) break;
+                // S/dP of chunk c once its rows have landed and the dK/dV products of chunk c-2 were
+                // issued (their softmax has read that TMEM buffer); dK/dV of chunk c once P and dS
+                // are written.  The piece's first dK/dV product overwrites the accumulators, so it
+                // waits until the previous piece's epilogue has read them.
+                bool accfree = (kp == 0);
+                int ns = 0, np = 0, spins = 0;
+                uint64_t idle_since = 0;
+                while (ok && np < nch) {
+                    bool progressed = false;
+                    if (ns < nch && ns <= np + 1) {
+                        const int cg = cg0 + ns, b = cg & 1;
+                        if (mbar_try_wait(smem_u32(&meta->qd_full[b]), (cg >> 1) & 1)) {
+                            tc_fence_after();
+                            const uint32_t tS = tmem + b * BS, tDP = tmem + C::kColDP + b * BS;
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint64_t ao = (uint64_t)(((ks >> 2) * (128 * 128) + (ks & 3) * 32) >> 4);
+                                const uint64_t bo = (uint64_t)(((ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
+                                umma_bf16(tS, dQ[b] + ao, dK + bo, C::kIdescS, ks > 0 ? 1u : 0u);
+                            }
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const uint64_t ao = (uint64_t)(((ks >> 2) * (128 * 128) + (ks & 3) * 32) >> 4);
+                                const uint64_t bo = (uint64_t)(((ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
+                                umma_bf16(tDP, dDO[b] + ao, dV + bo, C::kIdescS, ks > 0 ? 1u : 0u);
+                            }
+                            umma_commit(&meta->s_full[b]);
+                            ++ns;
+                            progressed = true;
+                        }
+                    }
+                    if (np < ns) {
+                        const int cg = cg0 + np, b = cg & 1;
+                        if (mbar_try_wait(smem_u32(&meta->p_full[b]), (cg >> 1) & 1) &&
+                            (accfree || mbar_try_wait(smem_u32(&meta->acc_free), (kp - 1) & 1))) {
+                            accfree = true;
+                            tc_fence_after();
+#pragma unroll
+                            for (int ks = 0; ks < 128 / 16; ++ks) {  // K dimension: the chunk's 128 rows
+                                const uint64_t o = (uint64_t)((ks * 16 * 128) >> 4);
+                                umma_bf16(tmem + C::kColDV, dDOt[b] + o, dP[b] + o, C::kIdescT, (np > 0 || ks > 0) ? 1u : 0u);
+                            }
+#pragma unroll
+                            for (int ks = 0; ks < 128 / 16; ++ks) {
+                                const uint64_t o = (uint64_t)((ks * 16 * 128) >> 4);
+                                umma_bf16(tmem + C::kColDK, dQt[b] + o, dDS[b] + o, C::kIdescT, (np > 0 || ks > 0) ? 1u : 0u);
+                            }
+                            umma_commit(&meta->qd_empty[b]);
+                            umma_commit(&meta->p_free[b]);
+                            ++np;
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        spins = 0;
+                    } else if (*abort_flag) {
+                        ok = false;
+                    } else if (spins++ == 0) {
+                        idle_since = global_timer_ns();
+                    } else if ((spins & 63) == 0 && global_timer_ns() - idle_since > kWaitLimitNs) {
+                        *abort_flag = 1;
+                        if (p.status) atomicOr(p.status, SFA_DEV_TIMEOUT);
+                        ok = false;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&meta->acc_full);
+                umma_commit(&meta->kv_empty);
+                mbar_arrive(&meta->meta_empty[m]);
+                cg0 += nch;
+                ++kp;
+            }
+            if (!ok) {
+                umma_commit(&meta->drain);
+                mbar_drain(&meta->drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ softmax + epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;  // a chunk row in the softmax, a d index in the epilogue
+        const int tl = r / p.G, g = r - tl * p.G;
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        int kp = 0, cg0 = 0, epi_uses = 0;
+        bool ok = true;
+        while (ok) {
+            const int m = kp & 1;
+            ok = warp_all_ok(mbar_wait(&meta->meta_full[m], (kp >> 1) & 1, abort_flag, p.status));
+            if (!ok) break;
+            const PieceInfo pi = meta->info[m];
+            if (pi.done) break;
+            const int nch = (pi.ntok + p.Tq - 1) / p.Tq;
+            const int kb = pi.s * BS, delta_k = pi.sk - pi.sq;
+            const int32_t *toks = p.toks + pi.rowoff + pi.tok_begin;
+            const int h = pi.hk * p.G + g;
+            for (int c = 0; c < nch; ++c) {
+                const int cg = cg0 + c, b = cg & 1;
+                const int ntc = min(p.Tq, pi.ntok - c * p.Tq);
+                const bool valid = tl < ntc;
+                const int i = valid ? toks[c * p.Tq + tl] : 0;
+                const int64_t t = (int64_t)pi.q0 + i;
+                const float lse2 = valid ? p.lse[(int64_t)h * p.total_q + t] * kLog2e : 0.f;
+                const float dlt = valid ? p.delta[(int64_t)h * p.total_q + t] : 0.f;
+                int lo = 0, hi = pi.sk - 1;
+                if (p.wl >= 0) lo = max(lo, i + delta_k - p.wl);
+                if (p.causal) hi = min(hi, i + delta_k);
+                if (p.wr >= 0) hi = min(hi, i + delta_k + p.wr);
+                if (!valid) hi = -1;  // keeps nothing
+                ok = warp_all_ok(mbar_wait(&meta->s_full[b], (cg >> 1) & 1, abort_flag, p.status));
+                if (ok && cg >= 2) ok = warp_all_ok(mbar_wait(&meta->p_free[b], ((cg >> 1) - 1) & 1, abort_flag, p.status));
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t tS = lane_base + b * BS, tDP = lane_base + C::kColDP + b * BS;
+                uint8_t *prow = sP + b * C::kPBytes + r * 128;
+                uint8_t *dsrow = sDS + b * C::kPBytes + r * 128;
+#pragma unroll
+                for (int hf = 0; hf < BS / 32; ++hf) {
+                    uint32_t sr[32], dr[32], pk[16], dk[16];
+                    tmem_ld32(tS + hf * 32, sr);
+                    tmem_ld32(tDP + hf * 32, dr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c0 = kb + hf * 32 + 2 * e;
+                        const float p0 = (c0 >= lo && c0 <= hi) ? ex2(fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -lse2)) : 0.f;
+                        const float p1 =
+                            (c0 + 1 >= lo && c0 + 1 <= hi) ? ex2(fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -lse2)) : 0.f;
+                        pk[e] = pack_bf16x2(p0, p1);
+                        dk[e] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * e]) - dlt), p1 * (__uint_as_float(dr[2 * e + 1]) - dlt));
+                    }
+                    // 16-byte pieces (8 keys) of the row, 128-byte swizzle: piece x at (x ^ (row & 7)) * 16.
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        const int piece = hf * 4 + x, so = ((piece ^ (r & 7)) << 4);
+                        *reinterpret_cast<uint4 *>(prow + so) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
+                        *reinterpret_cast<uint4 *>(dsrow + so) = make_uint4(dk[4 * x], dk[4 * x + 1], dk[4 * x + 2], dk[4 * x + 3]);
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&meta->p_full[b]);
+            }
+            if (!ok) break;
+            // ------------------------------------------------------------ epilogue (thread = d index r)
+            ok = warp_all_ok(mbar_wait(&meta->acc_full, kp & 1, abort_flag, p.status));
+            if (!ok) break;
+            tc_fence_after();
+            float dv[BS], dkk[BS];
+#pragma unroll
+            for (int hf = 0; hf < BS / 32; ++hf) {
+                uint32_t a[32], bq[32];
+                tmem_ld32(lane_base + C::kColDV + hf * 32, a);
+                tmem_ld32(lane_base + C::kColDK + hf * 32, bq);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    dv[hf * 32 + e] = __uint_as_float(a[e]);
+                    dkk[hf * 32 + e] = __uint_as_float(bq[e]) * p.scale;
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&meta->acc_free);  // the accumulators are in registers now
+            const int nk = min(BS, pi.sk - kb);
+            bool last = true;
+            if (pi.npieces > 1) {
+                float *pv = p.part + (size_t)pi.slot * 2 * BS * D, *pkk = pv + BS * D;
+                if (pi.idx > 0) {
+                    ok = warp_all_ok(wait_flag(p.flags + pi.slot, pi.idx, abort_flag, p.status));
+                    if (!ok) break;
+#pragma unroll
+                    for (int e = 0; e < BS; ++e) {
+                        dv[e] += pv[e * D + r];
+                        dkk[e] += pkk[e * D + r];
+                    }
+                }
+                last = pi.idx == pi.npieces - 1;
+                if (!last) {
+#pragma unroll
+                    for (int e = 0; e < BS; ++e) {
+                        pv[e * D + r] = dv[e];
+                        pkk[e * D + r] = dkk[e];
+                    }
+                    __threadfence();
+                    ok = group_sync(&meta->epi_bar, epi_uses, abort_flag, p.status);
+                    if (!ok) break;
+                    if (r == 0) st_release_gpu(p.flags + pi.slot, pi.idx + 1);
+                }
+            }
+            if (last) {
+                __nv_bfloat16 *dvo = p.dv + ((int64_t)(pi.k0 + kb) * p.Hkv + pi.hk) * D + r;
+                __nv_bfloat16 *dko = p.dk + ((int64_t)(pi.k0 + kb) * p.Hkv + pi.hk) * D + r;
+                const int64_t stride = (int64_t)p.Hkv * D;
+#pragma unroll
+                for (int e = 0; e < BS; ++e)
+                    if (e < nk) {
+                        dvo[e * stride] = __float2bfloat16_rn(dv[e]);
+                        dko[e * stride] = __float2bfloat16_rn(dkk[e]);
+                    }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&meta->meta_empty[m]);
+            cg0 += nch;
+            ++kp;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <typename K>
+cudaError_t set_smem(K kern, size_t bytes, int &configured)
+{
+    if ((int)bytes <= configured) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) configured = (int)bytes;
+    return e;
+}
+
+int sm_count()
+{
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+size_t bwd_dq_smem_bytes(const BwdGeom &g)
+{
+    return 1024 + dq_union_offset<128, 64>() + (size_t)2 * g.f.umax * 4;
+}
+
+size_t bwd_dkdv_smem_bytes()
+{
+    return 1024 + KvCfg<128, 64>::kOffMeta + sizeof(KvMeta);
+}
+
+cudaError_t launch_bwd_dq(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tdo,
+                          const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
+{
+    static int configured = 0;
+    const size_t smem = bwd_dq_smem_bytes(g);
+    cudaError_t e = set_smem(bwd_dq_kernel<128, 64>, smem, configured);
+    if (e != cudaSuccess) return e;
+    const int grid = std::max(1, std::min(p.tiles, sm_count()));
+    bwd_dq_kernel<128, 64><<<grid, kDqThreads, smem, st>>>(tq, tdo, tk, tv, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq_rows,
+                            const CUtensorMap &tdo_rows, const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
+{
+    (void)g;
+    static int configured = 0;
+    const size_t smem = bwd_dkdv_smem_bytes();
+    cudaError_t e = set_smem(bwd_dkdv_kernel<128, 64>, smem, configured);
+    if (e != cudaSuccess) return e;
+    bwd_dkdv_kernel<128, 64><<<sm_count(), kKvThreads, smem, st>>>(tq_rows, tdo_rows, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace sfa

@@ -106,6 +106,72 @@ struct FwdAttendParams {
 };
 
 // ---------------------------------------------------------------------------------------
+// Prefill backward
+// ---------------------------------------------------------------------------------------
+// dQ runs query-major over the forward's tiles and unions (the prep kernel's canonical lists);
+// dK / dV run block-major: for every (sequence, kv head, key block) "row" the ascending list of
+// the sequence's tokens that selected the block, cut into pieces of at most kBwdPieceChunks
+// chunks of Tq tokens.  A row longer than one piece is summed piece by piece in handout order
+// through an fp32 running partial, so the result does not depend on timing.
+constexpr int kBwdPieceChunks = 16;
+
+struct BwdPiece {
+    int row;        // (b * Hkv + hk) * nblk_max + block
+    int tok_begin;  // first entry of the row's token list this piece takes
+    int ntok;       // entries it takes
+    int idx, npieces;
+    int slot;       // running-partial slot of the row (-1: a one-piece row)
+    int pad[2];
+};
+
+struct BwdCtrl {
+    int npieces;  // pieces planned
+    int counter;  // next piece to hand out
+    int pad[2];
+};
+
+struct BwdGeom {
+    FwdGeom f;                 // query tiling, canonical lists and unions (block-major schedule off)
+    int R, words;              // rows = batch * Hkv * nblk_max; bitmap words per row = ceil(max_sq / 32)
+    int64_t max_pieces, max_slots;
+    size_t off_delta, off_bits, off_rowcnt, off_flags, off_ctrl, off_rowoff, off_toks, off_pieces, off_part;
+    size_t off_zero, zero_bytes;  // bitmap, row counts and partial flags: cleared before every call
+    size_t bytes;
+};
+
+struct BwdParams {
+    const __nv_bfloat16 *out, *dout;
+    const float *lse;     // (Hq, total_q), natural log
+    const int32_t *cu_q, *cu_k;
+    const int32_t *sel_c, *cnt, *ucnt, *uni;
+    int batch, total_q, Hq, Hkv, G, Tq, nqt, topk, umax, tiles, nblk_max, max_sq, words, R;
+    int causal, wl, wr;
+    float scale, scale_log2;
+    float *delta;         // (Hq, total_q): rowsum(dO o O)
+    uint32_t *bits;       // [R][words] token bitmaps
+    int32_t *rowcnt, *rowoff, *toks;
+    BwdPiece *pieces;
+    BwdCtrl *ctrl;
+    int32_t *flags;       // [max_slots] pieces of the row summed so far
+    float *part;          // [max_slots][2][bs][d] running partials (dK, dV)
+    int64_t max_pieces, max_slots;
+    int32_t *tile_counter;
+    __nv_bfloat16 *dq, *dk, *dv;
+    int32_t *status;
+};
+
+cudaError_t launch_bwd_delta(const BwdGeom &g, const BwdParams &p, cudaStream_t st);
+cudaError_t launch_bwd_index(const BwdGeom &g, const BwdParams &p, cudaStream_t st);
+cudaError_t launch_bwd_plan(const BwdGeom &g, const BwdParams &p, cudaStream_t st);
+cudaError_t launch_bwd_fill(const BwdGeom &g, const BwdParams &p, cudaStream_t st);
+cudaError_t launch_bwd_dq(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tdo,
+                          const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
+cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq_rows,
+                            const CUtensorMap &tdo_rows, const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
+size_t bwd_dq_smem_bytes(const BwdGeom &g);
+size_t bwd_dkdv_smem_bytes();
+
+// ---------------------------------------------------------------------------------------
 // Decode
 // ---------------------------------------------------------------------------------------
 struct DecGeom {
