@@ -391,6 +391,29 @@ def run_gpu(args, rank, world, local_rank):
                 ts.append(e0.elapsed_time(e1))
             return float(np.mean(ts))
 
+        # Backward of the selected attention on the same workload (d 128, bs 64): dq, dk, dv from the
+        # forward's out / lse and a seeded dout; 2.5x the forward's effective flops (five products
+        # of the kept pairs instead of two).
+        bwd_line = None
+        if pc.d == 128 and pc.bs == 64:
+            g_out = torch.randn(out.shape, generator=torch.Generator(device=dev).manual_seed(5), device=dev,
+                                dtype=torch.float32).to(torch.bfloat16)
+            bdq, bdk, bdv = torch.empty_like(P["q"]), torch.empty_like(P["k"]), torch.empty_like(P["v"])
+            bws = torch.empty(sfa.bwd_workspace_size(pc.batch, pc.max_sq, pc.max_sk, pc.total_q, pc.Hq, pc.Hkv, pc.d,
+                                                     pc.topk, pc.bs), dtype=torch.uint8, device=dev)
+
+            def run_bwd():
+                sfa.bwd(P["q"], P["k"], P["v"], out, g_out, lse, P["cu_q"], P["sel"], pc.bs, cu_seqlens_k=P["cu_k"],
+                        max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, causal=bool(pc.causal),
+                        window=(pc.wl, pc.wr), dq=bdq, dk=bdk, dv=bdv, workspace=bws, status=status)
+
+            b_ms = max_over_ranks([timed(run_bwd)], world, dev)[0]
+            bflops = 2.5 * flops
+            bwd_line = {"workload": "the prefill workload, seeded dout; dq, dk, dv", "ms": round(b_ms, 4),
+                        "effective_tflops": round(bflops / (b_ms * 1e-3) / 1e12, 2),
+                        "frac": round(bflops / (b_ms * 1e-3) / 1e12 / tf_burst, 4),
+                        "peak_source": f"{peak_kind} bf16 burst", "launches": 7,
+                        "flops_note": "2.5x the forward's effective flops (S, dP, dQ, dK, dV over the kept pairs)"}
         w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
         m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
         mix_bytes = 4 * pc.total_q * pc.Hq * pc.d * 2 + 3 * pc.total_q * pc.Hq * 4
@@ -403,6 +426,8 @@ def run_gpu(args, rank, world, local_rank):
                               "ms": round(m_ms, 4), "gbs": round(mix_bytes / (m_ms * 1e-3) / 1e9, 1),
                               "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
         }
+        if bwd_line is not None:
+            extras["backward"] = bwd_line
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
 

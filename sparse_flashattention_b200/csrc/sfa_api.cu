@@ -623,6 +623,7 @@ int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const 
         !encode_rows(tqr, q, d, (int64_t)total_q * Hq) || !encode_rows(tdor, dout, d, (int64_t)total_q * Hq))
         return SFA_ERR_CUDA;
     BwdParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
     p.out = static_cast<const __nv_bfloat16 *>(out);
     p.dout = static_cast<const __nv_bfloat16 *>(dout);
     p.lse = lse;

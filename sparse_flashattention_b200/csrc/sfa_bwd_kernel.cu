@@ -13,8 +13,9 @@
 //
 // bwd_dkdv_kernel (block-major, one CTA per SM, persistent): a piece is up to kBwdPieceChunks
 //   chunks of one (sequence, kv head, key block) row's token list.  K and V of the block stay in
-//   shared memory; each chunk's Q and dO rows (Tq tokens x G heads) are gathered four rows per TMA
-//   tile::gather4 copy into 128-byte-swizzled tiles.  Per chunk: S = Q K^T and dP = dO V^T (TMEM,
+//   shared memory; each chunk's Q and dO rows (Tq tokens x G heads) are gathered by two warps with
+//   coalesced 16-byte cp.async copies into 128-byte-swizzled tiles (a TMA gather4 copy per four
+//   rows measured several times slower: the copy engine, not the bytes, was the limit).  Per chunk: S = Q K^T and dP = dO V^T (TMEM,
 //   double-buffered); the softmax warps write P and dS (bf16) into shared memory; then
 //   dV^T += dO^T P and dK^T += Q^T dS, with the gathered tiles read MN-major as the A operand
 //   (M = d = 128) and P / dS MN-major as B.  The accumulators live in TMEM across the piece; the
@@ -378,8 +379,10 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     mbar_arrive(&meta->p_full[jg & 1]);
                     continue;
                 }
+                // Branch-free masking (the rows of a warp differ in what they keep): a row that did not
+                // select the block gets exponent -inf, a key outside the row's window too; 2^-inf = 0.
                 const int kb = s * BS;
-                const bool inner = kb >= lo && kb + BS - 1 <= hi;
+                const float sl = selected ? p.scale_log2 : 0.f, bias = selected ? -lse2 : -INFINITY;
 #pragma unroll
                 for (int hf = 0; hf < BS / 32; ++hf) {  // 32 keys at a time; dS half hf -> columns [16 hf, 16 hf + 16)
                     uint32_t sr[32], dr[32], packed[16];
@@ -388,11 +391,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const int c0 = hf * 32 + 2 * e, c1 = c0 + 1;
-                        const bool k0v = selected && (inner || (kb + c0 >= lo && kb + c0 <= hi));
-                        const bool k1v = selected && (inner || (kb + c1 >= lo && kb + c1 <= hi));
-                        const float p0 = k0v ? ex2(fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -lse2)) : 0.f;
-                        const float p1 = k1v ? ex2(fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -lse2)) : 0.f;
+                        const int c0 = kb + hf * 32 + 2 * e;
+                        float y0 = fmaf(__uint_as_float(sr[2 * e]), sl, bias);
+                        float y1 = fmaf(__uint_as_float(sr[2 * e + 1]), sl, bias);
+                        y0 = ((c0 >= lo) & (c0 <= hi)) ? y0 : -INFINITY;
+                        y1 = ((c0 + 1 >= lo) & (c0 + 1 <= hi)) ? y1 : -INFINITY;
+                        const float p0 = ex2(y0), p1 = ex2(y1);
                         packed[e] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * e]) - dlt),
                                                 p1 * (__uint_as_float(dr[2 * e + 1]) - dlt));
                     }
@@ -458,7 +462,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 // =========================================================================================
 // dK, dV
 // =========================================================================================
-constexpr int kKvThreads = 192;  // warp 0 loads, 1 MMA, 2..5 softmax / epilogue
+constexpr int kKvThreads = 224;  // warp 0 control + gather, 1 MMA, 2..5 softmax / epilogue, 6 gather
+constexpr int kGatherLanes = 64;  // warps 0 and 6: each copies 64 of a chunk's 128 rows
 
 template <int D, int BS>
 struct KvCfg {
@@ -540,16 +545,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     uint8_t *sP = smem + C::kOffP, *sDS = smem + C::kOffDS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    // Rows of a chunk past its tokens are never loaded; they must hold finite values (they meet
-    // P = dS = 0 in the transposed products), so the gather tiles start out zeroed.
-    for (int e = threadIdx.x; e < 4 * C::kTileBytes / 16; e += kKvThreads)
-        reinterpret_cast<uint4 *>(smem)[e] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&meta->meta_full[s], 1);
-            mbar_init(&meta->meta_empty[s], 6);  // producer, MMA thread, 4 softmax warps
-            mbar_init(&meta->qd_full[s], 1);
+            mbar_init(&meta->meta_empty[s], 7);  // warp 0, MMA thread, 4 softmax warps, warp 6
+            mbar_init(&meta->qd_full[s], kGatherLanes);  // one cp.async arrival per gathering lane
             mbar_init(&meta->qd_empty[s], 1);
             mbar_init(&meta->s_full[s], 1);
             mbar_init(&meta->p_full[s], 128);
@@ -575,11 +575,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     volatile int *abort_flag = &meta->abort_flag;
     const int npieces_total = p.ctrl->npieces;
 
-    if (warp == 0) {
+    if (warp == 0 || warp == 6) {
         // ------------------------------------------------------------------ loads
-        if (lane == 0) {
-            tma_prefetch_desc(&tmqr);
-            tma_prefetch_desc(&tmdor);
+        // Warp 0 lane 0 takes the next piece, publishes it and TMA-loads the block's K and V; warps 0
+        // and 6 gather each chunk's Q and dO rows (row r = token * G + head) with 16-byte cp.async
+        // copies into the 128-byte-swizzled tiles, eight lanes per 128-byte row segment (coalesced);
+        // rows past the chunk's tokens are zero-filled (they meet P = dS = 0).  Each lane's copies
+        // arrive on the stage's barrier when they land.
+        const int half = warp == 0 ? 0 : 1;
+        if (warp == 0 && lane == 0) {
             tma_prefetch_desc(&tmk);
             tma_prefetch_desc(&tmv);
         }
@@ -587,88 +591,94 @@ __global__ void __launch_bounds__(kKvThreads, 1)
         bool ok = true;
         while (ok) {
             const int m = kp & 1;
-            if (kp >= 2) ok = warp_all_ok(mbar_wait(&meta->meta_empty[m], ((kp >> 1) - 1) & 1, abort_flag, p.status));
-            if (!ok) break;
-            int piece = 0;
-            if (lane == 0) piece = atomicAdd(&p.ctrl->counter, 1);
-            piece = __shfl_sync(0xffffffffu, piece, 0);
             PieceInfo &pi = meta->info[m];
-            if (piece >= npieces_total) {
+            if (warp == 0) {
+                if (kp >= 2) ok = warp_all_ok(mbar_wait(&meta->meta_empty[m], ((kp >> 1) - 1) & 1, abort_flag, p.status));
+                if (!ok) break;
+                int piece = 0;
+                if (lane == 0) piece = atomicAdd(&p.ctrl->counter, 1);
+                piece = __shfl_sync(0xffffffffu, piece, 0);
+                if (piece >= npieces_total) {
+                    if (lane == 0) {
+                        pi.done = 1;
+                        mbar_arrive(&meta->meta_full[m]);
+                    }
+                    break;
+                }
                 if (lane == 0) {
-                    pi.done = 1;
+                    const BwdPiece pc = p.pieces[piece];
+                    const int s = pc.row % p.nblk_max, bh = pc.row / p.nblk_max;
+                    const int hk = bh % p.Hkv, b = bh / p.Hkv;
+                    const int q0 = __ldg(&p.cu_q[b]), k0 = __ldg(&p.cu_k[b]);
+                    pi.done = 0;
+                    pi.ntok = pc.ntok;
+                    pi.tok_begin = pc.tok_begin;
+                    pi.idx = pc.idx;
+                    pi.npieces = pc.npieces;
+                    pi.slot = pc.slot;
+                    pi.hk = hk;
+                    pi.s = s;
+                    pi.q0 = q0;
+                    pi.sq = __ldg(&p.cu_q[b + 1]) - q0;
+                    pi.k0 = k0;
+                    pi.sk = __ldg(&p.cu_k[b + 1]) - k0;
+                    pi.rowoff = p.rowoff[pc.row];
                     mbar_arrive(&meta->meta_full[m]);
+                    // K and V of the block, once the previous piece's MMAs are done with them.
+                    if (kp >= 1) ok = mbar_wait(&meta->kv_empty, (kp - 1) & 1, abort_flag, p.status);
+                    if (ok) {
+                        mbar_arrive_expect_tx(&meta->kv_full, 2u * (uint32_t)C::kKVBytes);
+                        for (int c = 0; c < D / 64; ++c) {
+                            tma_load_3d(&tmk, &meta->kv_full, sK + c * (BS * 128), c * 64, hk, k0 + s * BS);
+                            tma_load_3d(&tmv, &meta->kv_full, sV + c * (BS * 128), c * 64, hk, k0 + s * BS);
+                        }
+                        ++kv_issued;
+                    }
                 }
-                break;
+                ok = warp_all_ok(ok);
+                if (!ok) break;
+            } else {
+                ok = warp_all_ok(mbar_wait(&meta->meta_full[m], (kp >> 1) & 1, abort_flag, p.status));
+                if (!ok) break;
+                if (pi.done) break;
             }
-            const BwdPiece pc = p.pieces[piece];
-            const int s = pc.row % p.nblk_max, bh = pc.row / p.nblk_max;
-            const int hk = bh % p.Hkv, b = bh / p.Hkv;
-            const int q0 = __ldg(&p.cu_q[b]), k0 = __ldg(&p.cu_k[b]);
-            const int rowoff = p.rowoff[pc.row];
-            if (lane == 0) {
-                pi.done = 0;
-                pi.ntok = pc.ntok;
-                pi.tok_begin = pc.tok_begin;
-                pi.idx = pc.idx;
-                pi.npieces = pc.npieces;
-                pi.slot = pc.slot;
-                pi.hk = hk;
-                pi.s = s;
-                pi.q0 = q0;
-                pi.sq = __ldg(&p.cu_q[b + 1]) - q0;
-                pi.k0 = k0;
-                pi.sk = __ldg(&p.cu_k[b + 1]) - k0;
-                pi.rowoff = rowoff;
-                mbar_arrive(&meta->meta_full[m]);
-            }
-            // K and V of the block, once the previous piece's MMAs are done with them.
-            if (kp >= 1) ok = warp_all_ok(mbar_wait(&meta->kv_empty, (kp - 1) & 1, abort_flag, p.status));
-            if (!ok) break;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&meta->kv_full, 2u * (uint32_t)C::kKVBytes);
-                for (int c = 0; c < D / 64; ++c) {
-                    tma_load_3d(&tmk, &meta->kv_full, sK + c * (BS * 128), c * 64, hk, k0 + s * BS);
-                    tma_load_3d(&tmv, &meta->kv_full, sV + c * (BS * 128), c * 64, hk, k0 + s * BS);
-                }
-            }
-            ++kv_issued;
-            const int nch = (pc.ntok + p.Tq - 1) / p.Tq;
-            const int32_t *toks = p.toks + rowoff + pc.tok_begin;
+            __syncwarp();
+            const int ntok = pi.ntok, q0 = pi.q0, hk = pi.hk;
+            const int32_t *toks = p.toks + pi.rowoff + pi.tok_begin;
+            const int nch = (ntok + p.Tq - 1) / p.Tq;
+            const int sub = lane >> 3, piece16 = lane & 7;  // row within a group of 4, 16-byte piece of it
             for (int c = 0; c < nch; ++c) {
                 const int st = cg & 1;
                 if (cg >= 2) ok = warp_all_ok(mbar_wait(&meta->qd_empty[st], ((cg >> 1) - 1) & 1, abort_flag, p.status));
                 if (!ok) break;
-                const int ntc = min(p.Tq, pc.ntok - c * p.Tq), rows = ntc * p.G, n4 = (rows + 3) >> 2;
-                if (lane == 0) mbar_arrive_expect_tx(&meta->qd_full[st], (uint32_t)n4 * 512u * (D / 64) * 2u);
-                __syncwarp();
-                for (int g4 = lane; g4 < n4; g4 += 32) {
-                    int gr[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int rr = min(4 * g4 + e, rows - 1);  // a short last group repeats its last row
-                        const int tt = rr / p.G, gg = rr - tt * p.G;
-                        gr[e] = (q0 + toks[c * p.Tq + tt]) * p.Hq + hk * p.G + gg;
-                    }
+                const int ntc = min(p.Tq, ntok - c * p.Tq), rows = ntc * p.G;
+                const uint32_t qbase = smem_u32(sQ + st * C::kTileBytes), dbase = smem_u32(sDO + st * C::kTileBytes);
+#pragma unroll 4
+                for (int i = 0; i < 16; ++i) {  // 16 groups of 4 rows = this warp's 64 rows
+                    const int rr = half * 64 + i * 4 + sub;
+                    const bool live = rr < rows;
+                    const int tt = live ? rr / p.G : 0, gg = live ? rr - tt * p.G : 0;
+                    const int64_t grow = live ? ((int64_t)(q0 + toks[c * p.Tq + tt]) * p.Hq + hk * p.G + gg) : 0;
+                    const __nv_bfloat16 *qs = p.q + grow * D + piece16 * 8;
+                    const __nv_bfloat16 *ds = p.dout + grow * D + piece16 * 8;
+                    const uint32_t so = (uint32_t)(rr * 128 + ((piece16 ^ (rr & 7)) << 4));
 #pragma unroll
                     for (int cc = 0; cc < D / 64; ++cc) {
-                        const int so = st * C::kTileBytes + cc * (128 * 128) + g4 * 512;
-                        tma_gather4(&tmqr, &meta->qd_full[st], sQ + so, cc * 64, gr[0], gr[1], gr[2], gr[3]);
-                        tma_gather4(&tmdor, &meta->qd_full[st], sDO + so, cc * 64, gr[0], gr[1], gr[2], gr[3]);
+                        cp_async16(qbase + cc * (128 * 128) + so, qs + cc * 64, live ? 16u : 0u);
+                        cp_async16(dbase + cc * (128 * 128) + so, ds + cc * 64, live ? 16u : 0u);
                     }
                 }
+                cp_async_mbar_arrive(&meta->qd_full[st]);
                 ++cg;
             }
             if (!ok) break;
+            __syncwarp();
             if (lane == 0) mbar_arrive(&meta->meta_empty[m]);
             ++kp;
         }
-        if (*abort_flag && lane == 0) {  // let every copy this CTA started land
-            if (kv_issued > 0) mbar_drain(&meta->kv_full, (uint32_t)((kv_issued - 1) & 1));
-            for (int st = 0; st < 2; ++st) {
-                const int c = cg > st ? (cg - st + 1) / 2 : 0;
-                if (c > 0) mbar_drain(&meta->qd_full[st], (c - 1) & 1);
-            }
-        }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies have all landed
+        if (*abort_flag && warp == 0 && lane == 0 && kv_issued > 0)
+            mbar_drain(&meta->kv_full, (uint32_t)((kv_issued - 1) & 1));
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer
         if (lane == 0) {
@@ -706,6 +716,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     if (ns < nch && ns <= np + 1) {
                         const int cg = cg0 + ns, b = cg & 1;
                         if (mbar_try_wait(smem_u32(&meta->qd_full[b]), (cg >> 1) & 1)) {
+                            fence_proxy_async_smem();  // the rows came through cp.async (generic proxy)
                             tc_fence_after();
                             const uint32_t tS = tmem + b * BS, tDP = tmem + C::kColDP + b * BS;
 #pragma unroll
@@ -816,11 +827,13 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     tmem_ld32(tDP + hf * 32, dr);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
+                    for (int e = 0; e < 16; ++e) {  // branch-free masking: exponent -inf outside the row's keys
                         const int c0 = kb + hf * 32 + 2 * e;
-                        const float p0 = (c0 >= lo && c0 <= hi) ? ex2(fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -lse2)) : 0.f;
-                        const float p1 =
-                            (c0 + 1 >= lo && c0 + 1 <= hi) ? ex2(fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -lse2)) : 0.f;
+                        float y0 = fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -lse2);
+                        float y1 = fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -lse2);
+                        y0 = ((c0 >= lo) & (c0 <= hi)) ? y0 : -INFINITY;
+                        y1 = ((c0 + 1 >= lo) & (c0 + 1 <= hi)) ? y1 : -INFINITY;
+                        const float p0 = ex2(y0), p1 = ex2(y1);
                         pk[e] = pack_bf16x2(p0, p1);
                         dk[e] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * e]) - dlt), p1 * (__uint_as_float(dr[2 * e + 1]) - dlt));
                     }

@@ -140,7 +140,7 @@ struct BwdGeom {
 };
 
 struct BwdParams {
-    const __nv_bfloat16 *out, *dout;
+    const __nv_bfloat16 *q, *out, *dout;  // q and dout: the dK/dV kernel gathers their rows
     const float *lse;     // (Hq, total_q), natural log
     const int32_t *cu_q, *cu_k;
     const int32_t *sel_c, *cnt, *ucnt, *uni;
