@@ -325,10 +325,10 @@ int bwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     g.R = (int)R;
     g.words = (int)words;
     const int64_t per_piece = (int64_t)kBwdPieceChunks * g.f.Tq;
-    // A row of c tokens makes ceil(c / per_piece) pieces; only rows of more than per_piece tokens
-    // need a running partial.
+    // A row of c tokens makes ceil(c / per_piece) <= c / per_piece + 1 pieces; the rows of more than
+    // per_piece tokens (at most total_sel / (per_piece + 1) of them) need one partial slot per piece.
     g.max_pieces = total_sel / per_piece + std::min(R, total_sel) + 1;
-    g.max_slots = total_sel / (per_piece + 1) + 1;
+    g.max_slots = total_sel / per_piece + total_sel / (per_piece + 1) + 2;
     size_t off = align_up(g.f.off_tilectr + 8);
     g.off_delta = off;
     off = align_up(off + (size_t)total_q * Hq * 4);

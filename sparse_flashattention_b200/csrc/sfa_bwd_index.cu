@@ -6,8 +6,8 @@
 //   index  inverts the canonical selections: for each (sequence, kv head, key block) row a bitmap
 //          over the sequence's tokens that selected the block, and the row's token count.
 //   plan   one CTA: exclusive scans of the counts give each row's offset in the token-list array;
-//          rows are cut into pieces of at most kBwdPieceChunks chunks of Tq tokens; rows longer
-//          than one piece get a running-partial slot.
+//          rows are cut into pieces of at most kBwdPieceChunks chunks of Tq tokens; a row longer
+//          than one piece gets one partial slot per piece.
 //   fill   one warp per row: the bitmap, compacted, is the row's ascending token list; a block of a
 //          sequence that no token selected gets dK = dV = 0 here (no other kernel touches it).
 #include "sfa_device.cuh"
@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(1024) bwd_plan_kernel(BwdParams p)
         const int r = base + threadIdx.x;
         const int c = r < p.R ? p.rowcnt[r] : 0;
         const int np = (c + per_piece - 1) / per_piece;
-        const int multi = np > 1 ? 1 : 0;
+        const int multi = np > 1 ? np : 0;  // partial slots the row needs
         int ec, ep, es;
         const int tc = scan1024(c, scratch, ec);
         const int tp = scan1024(np, scratch, ep);
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(1024) bwd_plan_kernel(BwdParams p)
             p.rowoff[r] = (int32_t)(tok_base + ec);
             const int64_t first = piece_base + ep;
             const int slot = multi ? (int)(slot_base + es) : -1;
-            if (first + np > p.max_pieces || slot >= p.max_slots) {
+            if (first + np > p.max_pieces || slot + multi > p.max_slots) {
                 overflow = true;  // cannot happen for lists the prep kernel wrote (the bounds are exact maxima)
             } else {
                 for (int k = 0; k < np; ++k) {

@@ -7,8 +7,8 @@
 //
 // bwd_dq_kernel (query-major, one CTA per SM, persistent): the forward's tiles (Tq tokens x G heads
 //   = 128 rows of one kv head) walk the ascending union of their rows' blocks.  Per block the MMA
-//   thread issues S = Q K^T and dP = dO V^T into double-buffered TMEM, four softmax warps turn
-//   them into dS (bf16, written over the block's S columns), and dQ += dS K accumulates in TMEM
+//   thread issues S = Q K^T and dP = dO V^T into double-buffered TMEM, eight softmax warps (two per
+//   row, 32 keys each) turn them into dS (bf16, written over the block's S columns), and dQ += dS K accumulates in TMEM
 //   (A operand from TMEM, K read MN-major).  TMEM: 2 x S, 2 x dP, dQ = 384 of 512 columns.
 //
 // bwd_dkdv_kernel (block-major, one CTA per SM, persistent): a piece is up to kBwdPieceChunks
@@ -16,12 +16,13 @@
 //   shared memory; each chunk's Q and dO rows (Tq tokens x G heads) are gathered by two warps with
 //   coalesced 16-byte cp.async copies into 128-byte-swizzled tiles (a TMA gather4 copy per four
 //   rows measured several times slower: the copy engine, not the bytes, was the limit).  Per chunk: S = Q K^T and dP = dO V^T (TMEM,
-//   double-buffered); the softmax warps write P and dS (bf16) into shared memory; then
+//   double-buffered); eight softmax warps (two per row) write P and dS (bf16) into shared memory,
+//   each row's token and (lse, D) read one chunk ahead from arrays the fill kernel wrote; then
 //   dV^T += dO^T P and dK^T += Q^T dS, with the gathered tiles read MN-major as the A operand
 //   (M = d = 128) and P / dS MN-major as B.  The accumulators live in TMEM across the piece; the
-//   epilogue writes bf16 dK / dV, or, for a row cut into several pieces, adds the row's fp32
-//   running partial in piece order (piece i waits until pieces 0..i-1 are in it), so the sums do
-//   not depend on timing.
+//   epilogue writes bf16 dK / dV, or, for a row cut into several pieces, writes an fp32 partial and
+//   counts the piece done; the piece that completes the count sums the row's partials in piece
+//   order, so the sums do not depend on timing and no piece waits for another.
 //
 // Every wait is bounded (sfa_device.cuh); on a timeout the CTA records SFA_DEV_TIMEOUT, lets its
 // copies and MMAs land, frees TMEM and exits.
@@ -36,8 +37,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 // =========================================================================================
 // dQ
 // =========================================================================================
-constexpr int kDqThreads = 224;  // warp 0 producer, 1 MMA, 2..5 softmax / epilogue, 6 tile fetch
-constexpr int kDqStages = 3;     // K/V ring depth
+// warp 0 producer, 1 MMA, 2..9 softmax / epilogue (two warps per TMEM lane quadrant, one per half
+// of a block's keys and of dQ's columns), 10 tile fetch
+constexpr int kDqThreads = 352;
+constexpr int kDqFetchWarp = 10;
+// K and V rings: K is held until its block's dQ product, V only until dP, so K gets the deeper ring
+// (a K load is issued when the dQ product of the block kDqKStages back is done).
+constexpr int kDqKStages = 5;
+constexpr int kDqVStages = 3;
 
 template <int D, int BS>
 struct DqCfg {
@@ -45,14 +52,15 @@ struct DqCfg {
     static constexpr int kKVBytes = BS * D * 2;     // one K (or V) block
     static constexpr int kOffDO = kTileBytes;
     static constexpr int kOffK = 2 * kTileBytes;
-    static constexpr int kOffV = kOffK + kDqStages * kKVBytes;
-    static constexpr int kOffMeta = kOffV + kDqStages * kKVBytes;
+    static constexpr int kOffV = kOffK + kDqKStages * kKVBytes;
+    static constexpr int kOffMeta = kOffV + kDqVStages * kKVBytes;
     static constexpr int kTmemCols = 512;
     static constexpr int kColDP = 2 * BS;
     static constexpr int kColDQ = 4 * BS;
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
     static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, true);
     static_assert(kColDQ + D <= kTmemCols, "TMEM columns");
+    static_assert(BS == 64, "two softmax warps per row, 32 keys each");
 };
 
 struct DqTile {
@@ -61,7 +69,8 @@ struct DqTile {
 
 struct DqMeta {
     uint64_t q_full, q_empty;
-    uint64_t kv_full[kDqStages], kv_empty[kDqStages];
+    uint64_t k_full[kDqKStages], k_empty[kDqKStages];
+    uint64_t v_full[kDqVStages], v_empty[kDqVStages];
     uint64_t s_full[2], p_full[2], dq_done[2];
     uint64_t o_free;
     uint64_t meta_full[2], meta_empty[2];
@@ -95,18 +104,22 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     if (threadIdx.x == 0) {
         mbar_init(&meta->q_full, 1);
         mbar_init(&meta->q_empty, 1);
-        for (int s = 0; s < kDqStages; ++s) {
-            mbar_init(&meta->kv_full[s], 1);
-            mbar_init(&meta->kv_empty[s], 1);
+        for (int s = 0; s < kDqKStages; ++s) {
+            mbar_init(&meta->k_full[s], 1);
+            mbar_init(&meta->k_empty[s], 1);
+        }
+        for (int s = 0; s < kDqVStages; ++s) {
+            mbar_init(&meta->v_full[s], 1);
+            mbar_init(&meta->v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&meta->s_full[s], 1);
-            mbar_init(&meta->p_full[s], 128);
+            mbar_init(&meta->p_full[s], 256);
             mbar_init(&meta->dq_done[s], 1);
             mbar_init(&meta->meta_full[s], 32);
-            mbar_init(&meta->meta_empty[s], 6);  // producer, MMA thread, 4 softmax warps
+            mbar_init(&meta->meta_empty[s], 10);  // producer, MMA thread, 8 softmax warps
         }
-        mbar_init(&meta->o_free, 128);
+        mbar_init(&meta->o_free, 256);
         mbar_init(&meta->drain, 1);
         meta->abort_flag = 0;
         fence_mbar_init();
@@ -127,7 +140,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         tma_prefetch_desc(&tmv);
     }
 
-    if (warp == 6) {
+    if (warp == kDqFetchWarp) {
         // ------------------------------------------------------------------ tile fetch
         int k = 0;
         bool ok = true;
@@ -175,7 +188,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
         }
     } else if (warp == 0) {
         // ------------------------------------------------------------------ producer
-        int kv_st = 0, kv_ph = 0, nkv = 0, q_phases = 0;
+        int k_st = 0, k_ph = 0, nk = 0, v_st = 0, v_ph = 0, nv = 0, q_phases = 0;
         if (lane == 0) {
             int k = 0;
             bool ok = true;
@@ -197,21 +210,30 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     }
                 q_phases = k + 1;
                 for (int u = 0; ok && u < n; ++u) {
-                    const int st = kv_st;
-                    if (nkv >= kDqStages && !mbar_wait(&meta->kv_empty[st], kv_ph ^ 1, abort_flag, p.status)) {
+                    const int row = k0 + uni[u] * BS;
+                    if (nk >= kDqKStages && !mbar_wait(&meta->k_empty[k_st], k_ph ^ 1, abort_flag, p.status)) {
                         ok = false;
                         break;
                     }
-                    const int row = k0 + uni[u] * BS;
-                    mbar_arrive_expect_tx(&meta->kv_full[st], 2u * (uint32_t)C::kKVBytes);
-                    for (int c = 0; c < D / 64; ++c) {
-                        tma_load_3d(&tmk, &meta->kv_full[st], sK + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
-                        tma_load_3d(&tmv, &meta->kv_full[st], sV + st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                    mbar_arrive_expect_tx(&meta->k_full[k_st], (uint32_t)C::kKVBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(&tmk, &meta->k_full[k_st], sK + k_st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                    ++nk;
+                    if (++k_st == kDqKStages) {
+                        k_st = 0;
+                        k_ph ^= 1;
                     }
-                    ++nkv;
-                    if (++kv_st == kDqStages) {
-                        kv_st = 0;
-                        kv_ph ^= 1;
+                    if (nv >= kDqVStages && !mbar_wait(&meta->v_empty[v_st], v_ph ^ 1, abort_flag, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&meta->v_full[v_st], (uint32_t)C::kKVBytes);
+                    for (int c = 0; c < D / 64; ++c)
+                        tma_load_3d(&tmv, &meta->v_full[v_st], sV + v_st * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
+                    ++nv;
+                    if (++v_st == kDqVStages) {
+                        v_st = 0;
+                        v_ph ^= 1;
                     }
                 }
                 if (!ok) break;
@@ -220,9 +242,13 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             }
             if (*abort_flag) {  // let every copy this CTA started land
                 if (q_phases > 0) mbar_drain(&meta->q_full, (q_phases - 1) & 1);
-                for (int st = 0; st < kDqStages; ++st) {
-                    const int c = nkv > st ? (nkv - st + kDqStages - 1) / kDqStages : 0;
-                    if (c > 0) mbar_drain(&meta->kv_full[st], (c - 1) & 1);
+                for (int st = 0; st < kDqKStages; ++st) {
+                    const int c = nk > st ? (nk - st + kDqKStages - 1) / kDqKStages : 0;
+                    if (c > 0) mbar_drain(&meta->k_full[st], (c - 1) & 1);
+                }
+                for (int st = 0; st < kDqVStages; ++st) {
+                    const int c = nv > st ? (nv - st + kDqVStages - 1) / kDqVStages : 0;
+                    if (c > 0) mbar_drain(&meta->v_full[st], (c - 1) & 1);
                 }
             }
         }
@@ -235,7 +261,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16, 1024);
             const uint64_t dKmn0 = sdesc_sw128(smem_u32(sK), BS * 128, 1024);  // K as the MN-major B of dS K
             int k = 0, jg0 = 0;
-            int s_st = 0, s_ph = 0, p_st = 0, p_ph = 0;
+            int sk_st = 0, sk_ph = 0, sv_st = 0, sv_ph = 0, qk_st = 0, qk_ph = 0;  // K/V stages of the next S/dP, K of the next dQ
             bool ok = true;
             while (ok) {
                 const int m = k & 1;
@@ -256,35 +282,41 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 while (ok && np < n) {
                     bool progressed = false;
                     if (ns < n && ns <= np + 1) {
-                        const int jg = jg0 + ns, st = s_st;
-                        if (mbar_try_wait(smem_u32(&meta->kv_full[st]), s_ph)) {
+                        const int jg = jg0 + ns;
+                        if (mbar_try_wait(smem_u32(&meta->k_full[sk_st]), sk_ph) &&
+                            mbar_try_wait(smem_u32(&meta->v_full[sv_st]), sv_ph)) {
                             tc_fence_after();
                             const uint32_t tS = tmem + (jg & 1) * BS, tDP = tmem + C::kColDP + (jg & 1) * BS;
-                            const uint32_t kvo = (uint32_t)st * C::kKVBytes;
+                            const uint32_t ko = (uint32_t)sk_st * C::kKVBytes, vo = (uint32_t)sv_st * C::kKVBytes;
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
                                 const uint64_t ao = (uint64_t)(((ks >> 2) * (128 * 128) + (ks & 3) * 32) >> 4);
-                                const uint64_t bo = (uint64_t)((kvo + (ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
+                                const uint64_t bo = (uint64_t)((ko + (ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
                                 umma_bf16(tS, dQd + ao, dK0 + bo, C::kIdescS, ks > 0 ? 1u : 0u);
                             }
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
                                 const uint64_t ao = (uint64_t)(((ks >> 2) * (128 * 128) + (ks & 3) * 32) >> 4);
-                                const uint64_t bo = (uint64_t)((kvo + (ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
+                                const uint64_t bo = (uint64_t)((vo + (ks >> 2) * (BS * 128) + (ks & 3) * 32) >> 4);
                                 umma_bf16(tDP, dDOd + ao, dV0 + bo, C::kIdescS, ks > 0 ? 1u : 0u);
                             }
                             umma_commit(&meta->s_full[jg & 1]);
+                            umma_commit(&meta->v_empty[sv_st]);  // V is done once dP is
                             ++ns;
-                            if (++s_st == kDqStages) {
-                                s_st = 0;
-                                s_ph ^= 1;
+                            if (++sk_st == kDqKStages) {
+                                sk_st = 0;
+                                sk_ph ^= 1;
+                            }
+                            if (++sv_st == kDqVStages) {
+                                sv_st = 0;
+                                sv_ph ^= 1;
                             }
                             if (ns == n) umma_commit(&meta->q_empty);
                             progressed = true;
                         }
                     }
                     if (np < ns) {
-                        const int ig = jg0 + np, st = p_st;
+                        const int ig = jg0 + np, st = qk_st;
                         if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
                             (ofree || mbar_try_wait(smem_u32(&meta->o_free), (k - 1) & 1))) {
                             ofree = true;
@@ -295,11 +327,11 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                                                  dKmn0 + (uint64_t)((st * C::kKVBytes + ks * 16 * 128) >> 4), C::kIdescDQ,
                                                  (np > 0 || ks > 0) ? 1u : 0u);
                             umma_commit(&meta->dq_done[ig & 1]);
-                            umma_commit(&meta->kv_empty[st]);
+                            umma_commit(&meta->k_empty[st]);
                             ++np;
-                            if (++p_st == kDqStages) {
-                                p_st = 0;
-                                p_ph ^= 1;
+                            if (++qk_st == kDqKStages) {
+                                qk_st = 0;
+                                qk_ph ^= 1;
                             }
                             progressed = true;
                         }
@@ -329,6 +361,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
     } else {
         // ------------------------------------------------------------------ softmax + epilogue
         const int quad = warp & 3;
+        const int hs = (warp - 2) >> 2;  // which half of the keys (and of dQ's columns) this warp takes
         const int r = quad * 32 + lane;
         const int tok = r / p.G, g = r - tok * p.G;
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -372,8 +405,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     uint32_t zero[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) zero[e] = 0u;
-#pragma unroll
-                    for (int hf = 0; hf < BS / 32; ++hf) tmem_st16(tS + hf * 16, zero);
+                    tmem_st16(tS + hs * 16, zero);
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(&meta->p_full[jg & 1]);
@@ -383,15 +415,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 // select the block gets exponent -inf, a key outside the row's window too; 2^-inf = 0.
                 const int kb = s * BS;
                 const float sl = selected ? p.scale_log2 : 0.f, bias = selected ? -lse2 : -INFINITY;
-#pragma unroll
-                for (int hf = 0; hf < BS / 32; ++hf) {  // 32 keys at a time; dS half hf -> columns [16 hf, 16 hf + 16)
+                {  // this warp's 32 keys; dS of keys [32 hs, 32 hs + 32) -> columns [16 hs, 16 hs + 16)
                     uint32_t sr[32], dr[32], packed[16];
-                    tmem_ld32(tS + hf * 32, sr);
-                    tmem_ld32(tDP + hf * 32, dr);
+                    tmem_ld32(tS + hs * 32, sr);
+                    tmem_ld32(tDP + hs * 32, dr);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const int c0 = kb + hf * 32 + 2 * e;
+                        const int c0 = kb + hs * 32 + 2 * e;
                         float y0 = fmaf(__uint_as_float(sr[2 * e]), sl, bias);
                         float y1 = fmaf(__uint_as_float(sr[2 * e + 1]), sl, bias);
                         y0 = ((c0 >= lo) & (c0 <= hi)) ? y0 : -INFINITY;
@@ -400,7 +431,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                         packed[e] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * e]) - dlt),
                                                 p1 * (__uint_as_float(dr[2 * e + 1]) - dlt));
                     }
-                    tmem_st16(tS + hf * 16, packed);
+                    tmem_st16(tS + hs * 16, packed);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -416,7 +447,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             }
             __nv_bfloat16 *qrow = p.dq + (t * p.Hq + h) * D;
 #pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = hs * (D / 64); c < (hs + 1) * (D / 64); ++c) {  // this warp's half of the columns
                 uint32_t o[32];
                 if (n > 0) {
                     tmem_ld32(lane_base + C::kColDQ + c * 32, o);
@@ -462,12 +493,16 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 // =========================================================================================
 // dK, dV
 // =========================================================================================
-constexpr int kKvThreads = 224;  // warp 0 control + gather, 1 MMA, 2..5 softmax / epilogue, 6 gather
-constexpr int kGatherLanes = 64;  // warps 0 and 6: each copies 64 of a chunk's 128 rows
+// warp 0 control + gather, 1 MMA, 2..9 softmax / epilogue (two warps per TMEM lane quadrant, one
+// per half of the block's keys), 10 gather
+constexpr int kKvThreads = 352;
+constexpr int kKvGatherWarp2 = 10;
+constexpr int kGatherLanes = 64;  // warps 0 and 10: each copies 64 of a chunk's 128 rows
 
 template <int D, int BS>
 struct KvCfg {
     static_assert(D == 128, "the transposed products take d as the MMA's M dimension (128)");
+    static_assert(BS == 64, "two softmax warps per row, 32 keys each");
     static constexpr int kTileBytes = 128 * D * 2;  // 128 gathered rows of Q (or dO)
     static constexpr int kKVBytes = BS * D * 2;
     static constexpr int kPBytes = 128 * BS * 2;    // P (or dS): 128 rows x BS keys, bf16
@@ -498,39 +533,9 @@ struct KvMeta {
     uint64_t acc_full, acc_free, epi_bar, drain;
     uint32_t tmem_base;
     int abort_flag;
+    int last_flag;  // the epilogue's piece finished its row last
     PieceInfo info[2];
 };
-
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t *ptr)
-{
-    int v;
-    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(int32_t *ptr, int v)
-{
-    asm volatile("st.release.gpu.global.s32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
-}
-
-// Wait until *flag >= target (another CTA's piece of the same row is in the running partial).
-__device__ bool wait_flag(const int32_t *flag, int target, volatile int *abort_flag, int32_t *status)
-{
-    uint64_t t0 = 0;
-    int spins = 0;
-    while (ld_acquire_gpu(flag) < target) {
-        if (*abort_flag) return false;
-        if (spins++ == 0) {
-            t0 = global_timer_ns();
-        } else if ((spins & 255) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1;
-            if (status) atomicOr(status, SFA_DEV_TIMEOUT);
-            return false;
-        }
-        __nanosleep(128);
-    }
-    return true;
-}
 
 template <int D, int BS>
 __global__ void __launch_bounds__(kKvThreads, 1)
@@ -548,18 +553,18 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&meta->meta_full[s], 1);
-            mbar_init(&meta->meta_empty[s], 7);  // warp 0, MMA thread, 4 softmax warps, warp 6
+            mbar_init(&meta->meta_empty[s], 11);  // warp 0, MMA thread, 8 softmax warps, warp 10
             mbar_init(&meta->qd_full[s], kGatherLanes);  // one cp.async arrival per gathering lane
             mbar_init(&meta->qd_empty[s], 1);
             mbar_init(&meta->s_full[s], 1);
-            mbar_init(&meta->p_full[s], 128);
+            mbar_init(&meta->p_full[s], 256);
             mbar_init(&meta->p_free[s], 1);
         }
         mbar_init(&meta->kv_full, 1);
         mbar_init(&meta->kv_empty, 1);
         mbar_init(&meta->acc_full, 1);
-        mbar_init(&meta->acc_free, 128);
-        mbar_init(&meta->epi_bar, 128);
+        mbar_init(&meta->acc_free, 256);
+        mbar_init(&meta->epi_bar, 256);
         mbar_init(&meta->drain, 1);
         meta->abort_flag = 0;
         fence_mbar_init();
@@ -575,10 +580,10 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     volatile int *abort_flag = &meta->abort_flag;
     const int npieces_total = p.ctrl->npieces;
 
-    if (warp == 0 || warp == 6) {
+    if (warp == 0 || warp == kKvGatherWarp2) {
         // ------------------------------------------------------------------ loads
         // Warp 0 lane 0 takes the next piece, publishes it and TMA-loads the block's K and V; warps 0
-        // and 6 gather each chunk's Q and dO rows (row r = token * G + head) with 16-byte cp.async
+        // and 10 gather each chunk's Q and dO rows (row r = token * G + head) with 16-byte cp.async
         // copies into the 128-byte-swizzled tiles, eight lanes per 128-byte row segment (coalesced);
         // rows past the chunk's tokens are zero-filled (they meet P = dS = 0).  Each lane's copies
         // arrive on the stage's barrier when they land.
@@ -653,12 +658,18 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 if (!ok) break;
                 const int ntc = min(p.Tq, ntok - c * p.Tq), rows = ntc * p.G;
                 const uint32_t qbase = smem_u32(sQ + st * C::kTileBytes), dbase = smem_u32(sDO + st * C::kTileBytes);
-#pragma unroll 4
+                int tokv[16];  // the tokens of this lane's 16 rows, loaded together (one latency, not 16)
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int rr = half * 64 + i * 4 + sub;
+                    tokv[i] = rr < rows ? toks[c * p.Tq + rr / p.G] : 0;
+                }
+#pragma unroll
                 for (int i = 0; i < 16; ++i) {  // 16 groups of 4 rows = this warp's 64 rows
                     const int rr = half * 64 + i * 4 + sub;
                     const bool live = rr < rows;
                     const int tt = live ? rr / p.G : 0, gg = live ? rr - tt * p.G : 0;
-                    const int64_t grow = live ? ((int64_t)(q0 + toks[c * p.Tq + tt]) * p.Hq + hk * p.G + gg) : 0;
+                    const int64_t grow = live ? ((int64_t)(q0 + tokv[i]) * p.Hq + hk * p.G + gg) : 0;
                     const __nv_bfloat16 *qs = p.q + grow * D + piece16 * 8;
                     const __nv_bfloat16 *ds = p.dout + grow * D + piece16 * 8;
                     const uint32_t so = (uint32_t)(rr * 128 + ((piece16 ^ (rr & 7)) << 4));
@@ -785,6 +796,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     } else {
         // ------------------------------------------------------------------ softmax + epilogue
         const int quad = warp & 3;
+        const int hs = (warp - 2) >> 2;  // which half of the block's keys this warp takes
         const int r = quad * 32 + lane;  // a chunk row in the softmax, a d index in the epilogue
         const int tl = r / p.G, g = r - tl * p.G;
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -799,20 +811,25 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const int nch = (pi.ntok + p.Tq - 1) / p.Tq;
             const int kb = pi.s * BS, delta_k = pi.sk - pi.sq;
             const int32_t *toks = p.toks + pi.rowoff + pi.tok_begin;
-            const int h = pi.hk * p.G + g;
+            const int64_t hrow = (int64_t)(pi.hk * p.G + g) * p.total_q + pi.q0;
+            // The row's token two chunks ahead and its lse and D one chunk ahead of use, so neither
+            // the token lookup nor the two loads that depend on it wait on the critical path.
+            auto tok_of = [&](int c) { return (c < nch && tl < min(p.Tq, pi.ntok - c * p.Tq)) ? toks[c * p.Tq + tl] : -1; };
+            int i1 = tok_of(0), i2 = tok_of(1);
+            float lse1 = i1 >= 0 ? p.lse[hrow + i1] : 0.f, dlt1 = i1 >= 0 ? p.delta[hrow + i1] : 0.f;
             for (int c = 0; c < nch; ++c) {
                 const int cg = cg0 + c, b = cg & 1;
-                const int ntc = min(p.Tq, pi.ntok - c * p.Tq);
-                const bool valid = tl < ntc;
-                const int i = valid ? toks[c * p.Tq + tl] : 0;
-                const int64_t t = (int64_t)pi.q0 + i;
-                const float lse2 = valid ? p.lse[(int64_t)h * p.total_q + t] * kLog2e : 0.f;
-                const float dlt = valid ? p.delta[(int64_t)h * p.total_q + t] : 0.f;
+                const int i = i1;
+                const float lse2 = lse1 * kLog2e, dlt = dlt1;
+                i1 = i2;
+                i2 = tok_of(c + 2);
+                lse1 = i1 >= 0 ? p.lse[hrow + i1] : 0.f;
+                dlt1 = i1 >= 0 ? p.delta[hrow + i1] : 0.f;
                 int lo = 0, hi = pi.sk - 1;
                 if (p.wl >= 0) lo = max(lo, i + delta_k - p.wl);
                 if (p.causal) hi = min(hi, i + delta_k);
                 if (p.wr >= 0) hi = min(hi, i + delta_k + p.wr);
-                if (!valid) hi = -1;  // keeps nothing
+                if (i < 0) hi = -1;  // a row past the chunk's tokens keeps nothing
                 ok = warp_all_ok(mbar_wait(&meta->s_full[b], (cg >> 1) & 1, abort_flag, p.status));
                 if (ok && cg >= 2) ok = warp_all_ok(mbar_wait(&meta->p_free[b], ((cg >> 1) - 1) & 1, abort_flag, p.status));
                 if (!ok) break;
@@ -820,15 +837,14 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 const uint32_t tS = lane_base + b * BS, tDP = lane_base + C::kColDP + b * BS;
                 uint8_t *prow = sP + b * C::kPBytes + r * 128;
                 uint8_t *dsrow = sDS + b * C::kPBytes + r * 128;
-#pragma unroll
-                for (int hf = 0; hf < BS / 32; ++hf) {
+                {
                     uint32_t sr[32], dr[32], pk[16], dk[16];
-                    tmem_ld32(tS + hf * 32, sr);
-                    tmem_ld32(tDP + hf * 32, dr);
+                    tmem_ld32(tS + hs * 32, sr);
+                    tmem_ld32(tDP + hs * 32, dr);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {  // branch-free masking: exponent -inf outside the row's keys
-                        const int c0 = kb + hf * 32 + 2 * e;
+                        const int c0 = kb + hs * 32 + 2 * e;
                         float y0 = fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -lse2);
                         float y1 = fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -lse2);
                         y0 = ((c0 >= lo) & (c0 <= hi)) ? y0 : -INFINITY;
@@ -840,7 +856,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     // 16-byte pieces (8 keys) of the row, 128-byte swizzle: piece x at (x ^ (row & 7)) * 16.
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
-                        const int piece = hf * 4 + x, so = ((piece ^ (r & 7)) << 4);
+                        const int piece = hs * 4 + x, so = ((piece ^ (r & 7)) << 4);
                         *reinterpret_cast<uint4 *>(prow + so) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
                         *reinterpret_cast<uint4 *>(dsrow + so) = make_uint4(dk[4 * x], dk[4 * x + 1], dk[4 * x + 2], dk[4 * x + 3]);
                     }
@@ -850,58 +866,67 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 mbar_arrive(&meta->p_full[b]);
             }
             if (!ok) break;
-            // ------------------------------------------------------------ epilogue (thread = d index r)
+            // ------------------------------------------------------------ epilogue (thread = d index r, keys
+            // [32 hs, 32 hs + 32))
             ok = warp_all_ok(mbar_wait(&meta->acc_full, kp & 1, abort_flag, p.status));
             if (!ok) break;
             tc_fence_after();
-            float dv[BS], dkk[BS];
-#pragma unroll
-            for (int hf = 0; hf < BS / 32; ++hf) {
+            constexpr int HK = BS / 2;
+            float dv[HK], dkk[HK];
+            {
                 uint32_t a[32], bq[32];
-                tmem_ld32(lane_base + C::kColDV + hf * 32, a);
-                tmem_ld32(lane_base + C::kColDK + hf * 32, bq);
+                tmem_ld32(lane_base + C::kColDV + hs * HK, a);
+                tmem_ld32(lane_base + C::kColDK + hs * HK, bq);
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    dv[hf * 32 + e] = __uint_as_float(a[e]);
-                    dkk[hf * 32 + e] = __uint_as_float(bq[e]) * p.scale;
+                for (int e = 0; e < HK; ++e) {
+                    dv[e] = __uint_as_float(a[e]);
+                    dkk[e] = __uint_as_float(bq[e]) * p.scale;
                 }
             }
             tc_fence_before();
             mbar_arrive(&meta->acc_free);  // the accumulators are in registers now
             const int nk = min(BS, pi.sk - kb);
+            const int e0 = hs * HK;
             bool last = true;
             if (pi.npieces > 1) {
-                float *pv = p.part + (size_t)pi.slot * 2 * BS * D, *pkk = pv + BS * D;
-                if (pi.idx > 0) {
-                    ok = warp_all_ok(wait_flag(p.flags + pi.slot, pi.idx, abort_flag, p.status));
-                    if (!ok) break;
+                // Write this piece's partial; the piece whose count arrival is the row's last sums all of
+                // the row's partials in piece order (this one's included, read back) and writes dK / dV.
+                constexpr size_t kSlot = (size_t)2 * BS * D;
+                float *mine = p.part + (size_t)(pi.slot + pi.idx) * kSlot;
 #pragma unroll
-                    for (int e = 0; e < BS; ++e) {
-                        dv[e] += pv[e * D + r];
-                        dkk[e] += pkk[e * D + r];
-                    }
+                for (int e = 0; e < HK; ++e) {
+                    mine[(e0 + e) * D + r] = dv[e];
+                    mine[BS * D + (e0 + e) * D + r] = dkk[e];
                 }
-                last = pi.idx == pi.npieces - 1;
-                if (!last) {
-#pragma unroll
-                    for (int e = 0; e < BS; ++e) {
-                        pv[e * D + r] = dv[e];
-                        pkk[e * D + r] = dkk[e];
-                    }
+                __threadfence();
+                ok = group_sync(&meta->epi_bar, epi_uses, abort_flag, p.status);
+                if (!ok) break;
+                if (r == 0 && hs == 0) meta->last_flag = atomicAdd(p.flags + pi.slot, 1) == pi.npieces - 1 ? 1 : 0;
+                ok = group_sync(&meta->epi_bar, epi_uses, abort_flag, p.status);
+                if (!ok) break;
+                last = meta->last_flag != 0;
+                if (last) {
                     __threadfence();
-                    ok = group_sync(&meta->epi_bar, epi_uses, abort_flag, p.status);
-                    if (!ok) break;
-                    if (r == 0) st_release_gpu(p.flags + pi.slot, pi.idx + 1);
+#pragma unroll
+                    for (int e = 0; e < HK; ++e) dv[e] = dkk[e] = 0.f;
+                    for (int j = 0; j < pi.npieces; ++j) {
+                        const float *pj = p.part + (size_t)(pi.slot + j) * kSlot;
+#pragma unroll
+                        for (int e = 0; e < HK; ++e) {
+                            dv[e] += __ldcg(pj + (e0 + e) * D + r);
+                            dkk[e] += __ldcg(pj + BS * D + (e0 + e) * D + r);
+                        }
+                    }
                 }
             }
             if (last) {
-                __nv_bfloat16 *dvo = p.dv + ((int64_t)(pi.k0 + kb) * p.Hkv + pi.hk) * D + r;
-                __nv_bfloat16 *dko = p.dk + ((int64_t)(pi.k0 + kb) * p.Hkv + pi.hk) * D + r;
+                __nv_bfloat16 *dvo = p.dv + ((int64_t)(pi.k0 + kb + e0) * p.Hkv + pi.hk) * D + r;
+                __nv_bfloat16 *dko = p.dk + ((int64_t)(pi.k0 + kb + e0) * p.Hkv + pi.hk) * D + r;
                 const int64_t stride = (int64_t)p.Hkv * D;
 #pragma unroll
-                for (int e = 0; e < BS; ++e)
-                    if (e < nk) {
+                for (int e = 0; e < HK; ++e)
+                    if (e0 + e < nk) {
                         dvo[e * stride] = __float2bfloat16_rn(dv[e]);
                         dko[e * stride] = __float2bfloat16_rn(dkk[e]);
                     }

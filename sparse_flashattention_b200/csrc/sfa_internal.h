@@ -111,8 +111,9 @@ struct FwdAttendParams {
 // dQ runs query-major over the forward's tiles and unions (the prep kernel's canonical lists);
 // dK / dV run block-major: for every (sequence, kv head, key block) "row" the ascending list of
 // the sequence's tokens that selected the block, cut into pieces of at most kBwdPieceChunks
-// chunks of Tq tokens.  A row longer than one piece is summed piece by piece in handout order
-// through an fp32 running partial, so the result does not depend on timing.
+// chunks of Tq tokens.  Each piece of a row longer than one piece writes an fp32 partial; the
+// piece that finishes last sums the row's partials in piece order, so the result does not depend
+// on timing and no piece waits for another.
 constexpr int kBwdPieceChunks = 16;
 
 struct BwdPiece {
@@ -120,7 +121,7 @@ struct BwdPiece {
     int tok_begin;  // first entry of the row's token list this piece takes
     int ntok;       // entries it takes
     int idx, npieces;
-    int slot;       // running-partial slot of the row (-1: a one-piece row)
+    int slot;       // first of the row's npieces partial slots (-1: a one-piece row)
     int pad[2];
 };
 
@@ -152,8 +153,8 @@ struct BwdParams {
     int32_t *rowcnt, *rowoff, *toks;
     BwdPiece *pieces;
     BwdCtrl *ctrl;
-    int32_t *flags;       // [max_slots] pieces of the row summed so far
-    float *part;          // [max_slots][2][bs][d] running partials (dK, dV)
+    int32_t *flags;       // [max_slots], at a row's first slot: its pieces finished so far
+    float *part;          // [max_slots][2][bs][d] partials (dK, dV) of the pieces of multi-piece rows
     int64_t max_pieces, max_slots;
     int32_t *tile_counter;
     __nv_bfloat16 *dq, *dk, *dv;
