@@ -158,3 +158,33 @@ def gated_combine(branches):
         term = np.asarray(g, np.float64)[..., None] * of
         out = term if out is None else out + term
     return out
+
+
+def kv_append(k_cache, v_cache, block_table, cache_seqlens, k_new, v_new):
+    """In-place KV-cache append as flash_attn_with_kvcache documents it (flash-attention-npu page,
+    "FlashAttention v2" API docstrings): when k / v are given, k_cache / v_cache are updated in place
+    with them, the new rows of sequence b going to logical positions cache_seqlens[b],
+    cache_seqlens[b] + 1, ...; a paged cache (num_pages, page, Hkv, d) maps logical position j of
+    sequence b to page block_table[b, j // page], row j % page.  cache_seqlens itself is left as is
+    (the caller tracks lengths).  k_new / v_new: (B, seqlen_new, Hkv, d).  Positions past the block
+    table, or whose page id is outside [0, num_pages), are not written (counted in `bad`, the
+    reading this build takes where the docstring only asks the caller to size the cache).
+    Returns (k_cache, v_cache, bad) as new arrays; the inputs are not modified."""
+    kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+    num_pages, page = kc.shape[0], kc.shape[1]
+    B, S = k_new.shape[0], k_new.shape[1]
+    bad = 0
+    for b in range(B):
+        for j in range(S):
+            pos = int(cache_seqlens[b]) + j
+            blk = pos // page
+            if blk >= block_table.shape[1]:
+                bad += 1
+                continue
+            pg = int(block_table[b, blk])
+            if not 0 <= pg < num_pages:
+                bad += 1
+                continue
+            kc[pg, pos % page] = k_new[b, j]
+            vc[pg, pos % page] = v_new[b, j]
+    return kc, vc, bad

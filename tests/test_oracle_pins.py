@@ -342,3 +342,30 @@ def test_gated_combine_worked_example_and_gates():
     np.testing.assert_array_equal(oracle.gated_combine([(bits, one), (other, zero)]),
                                   W.bf16_bits_to_f32(bits).astype(np.float64))
     assert not oracle.gated_combine([(bits, zero), (other, zero)]).any()
+
+
+def test_kv_append_worked_example():
+    """oracle.kv_append against the hand-worked positions in tests/golden/kv_append_example.txt."""
+    import oracle
+    rows = [tuple(int(x) for x in ln.split()) for ln in open(os.path.join(GOLDEN, "kv_append_example.txt"))
+            if ln.strip() and not ln.startswith("#")]
+    kc = np.full((6, 2, 1, 1), -1.0)
+    vc = np.full((6, 2, 1, 1), -2.0)
+    bt = np.array([[4, 1, 5], [0, 3, 2]], np.int32)
+    lens = np.array([3, 0], np.int32)
+    kn = np.array([[10.0, 11.0], [20.0, 21.0]]).reshape(2, 2, 1, 1)
+    k2, v2, bad = oracle.kv_append(kc, vc, bt, lens, kn, kn + 100)
+    assert bad == 0
+    want_k = kc.copy()
+    want_v = vc.copy()
+    for pg, row, val in rows:
+        want_k[pg, row] = val
+        want_v[pg, row] = val + 100
+    np.testing.assert_array_equal(k2, want_k)
+    np.testing.assert_array_equal(v2, want_v)
+    # cache_seqlens [5, 0]: position 5 of sequence 0 -> block 2 -> page 5, row 1; position 6 -> block 3,
+    # past the 3-entry block table: not written, counted.
+    k3, _, bad3 = oracle.kv_append(kc, vc, bt, np.array([5, 0], np.int32), kn, kn)
+    assert bad3 == 1
+    assert k3[5, 1, 0, 0] == 10.0 and k3[0, 0, 0, 0] == 20.0 and k3[0, 1, 0, 0] == 21.0
+    assert (k3 != kc).sum() == 3
