@@ -414,6 +414,20 @@ def run_gpu(args, rank, world, local_rank):
                         "frac": round(bflops / (b_ms * 1e-3) / 1e12 / tf_burst, 4),
                         "peak_source": f"{peak_kind} bf16 burst", "launches": 7,
                         "flops_note": "2.5x the forward's effective flops (S, dP, dQ, dK, dV over the kept pairs)"}
+        # In-place KV-cache append on the decode workload's cache: one new token per sequence written at
+        # position L - 1 (the decode query's own position); bytes = the new rows read + written.
+        akn = torch.randn((dc.B, 1, dc.Hkv, dc.d), device=dev).to(torch.bfloat16)
+        akv = torch.randn((dc.B, 1, dc.Hkv, dc.d), device=dev).to(torch.bfloat16)
+        apos = (D["cache_seqlens"] - 1).to(torch.int32)
+
+        def run_append():
+            sfa.kv_append(akn, akv, D["k_cache"], D["v_cache"], D["block_table"], apos, status=status)
+
+        a_ms = max_over_ranks([timed(run_append)], world, dev)[0]
+        a_bytes = 2 * 2 * dc.B * dc.Hkv * dc.d * 2
+        append_line = {"workload": f"B {dc.B}, 1 new token, Hkv {dc.Hkv}, d {dc.d}, page {dc.page}",
+                       "us": round(a_ms * 1e3, 2), "gbs": round(a_bytes / (a_ms * 1e-3) / 1e9, 1), "launches": 1,
+                       "note": "launch-latency bound (256 KB moved)"}
         w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
         m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
         mix_bytes = 4 * pc.total_q * pc.Hq * pc.d * 2 + 3 * pc.total_q * pc.Hq * 4
@@ -428,6 +442,7 @@ def run_gpu(args, rank, world, local_rank):
         }
         if bwd_line is not None:
             extras["backward"] = bwd_line
+        extras["kv_append"] = append_line
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
 

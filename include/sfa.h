@@ -241,6 +241,18 @@ int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
                        int B, int Hq, int Hkv, int d, int window_left, float scale, int num_splits,
                        int32_t *status_dev, void *out, float *lse, sfa_stream_t stream);
 
+/* In-place append of new keys / values to the paged cache, as the k / v arguments of
+ * flash_attn_with_kvcache (flash-attention-npu docstrings): row j of sequence b goes to logical
+ * position cache_seqlens[b] + j, i.e. page block_table[b][pos / page_size], row pos % page_size.
+ *   k_new, v_new  bf16 (B, seqlen_new, Hkv, d);  k_cache, v_cache  bf16 (num_pages, page_size, Hkv, d)
+ * cache_seqlens is read, not updated: a decode over the appended cache passes cache_seqlens +
+ * seqlen_new.  A position past the block table (SFA_DEV_BAD_SEQLEN) or whose page id is outside
+ * [0, num_pages) (SFA_DEV_BAD_PAGE) is not written.  d a multiple of 8; 16-byte aligned tensors.
+ * One kernel (none when B or seqlen_new is 0). */
+int sfa_kv_append(const void *k_new, const void *v_new, int seqlen_new, void *k_cache, void *v_cache,
+                  const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
+                  const int32_t *cache_seqlens, int B, int Hkv, int d, int32_t *status_dev, sfa_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------
  * NSA branches beside the selected attention (the "Relaxed-System-Lab/Flash-Sparse-Attention"
  * project page, quick-start: window_size alongside block_size / topk; the Flash-Sparse-Attention
@@ -280,7 +292,7 @@ const char *sfa_status_string(int status);
 
 /* Number of kernel launches the last successful call on this host thread made (prefill: 1,
  * or 6 when the call uses the block-major schedule; decode: 1 with at most 6 splits, else 2,
- * plus 1 when topk_tok > 2048; a stage: its own count; window branch, gated mix: 1; backward: 7). */
+ * plus 1 when topk_tok > 2048; a stage: its own count; window branch, gated mix, KV append: 1; backward: 7). */
 int sfa_last_launch_count(void);
 
 #ifdef __cplusplus

@@ -59,6 +59,7 @@ def _load():
         "sfa_window_fwd_workspace_size": (Z, []),
         "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P, F, P, Z, P, P, P, P]),
         "sfa_gated_combine": (I, [P, P, P, P, P, P, I, I, I, P, P]),
+        "sfa_kv_append": (I, [P, P, I, P, P, P, I, I, I, P, I, I, I, P, P]),
         "sfa_bwd_workspace_size": (Z, [I, I, I, I, I, I, I, I, I]),
         "sfa_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, I, I, I, I, I, F, P, Z, P, P, P, P, P]),
         "sfa_status_string": (ctypes.c_char_p, [I]),
@@ -191,6 +192,28 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.T
                       _stream(stream))
     _check(rc)
     return out, lse
+
+
+def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              block_table: torch.Tensor, cache_seqlens: torch.Tensor, status: Optional[torch.Tensor] = None,
+              stream=None) -> None:
+    """In-place paged KV-cache append (sfa_kv_append): k_new / v_new (B, seqlen_new, Hkv, d) bf16 go to
+    logical positions cache_seqlens[b] + j of k_cache / v_cache (num_pages, page, Hkv, d).
+    cache_seqlens is not updated."""
+    for t, name in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, name, torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    if k_new.shape != v_new.shape or k_cache.shape != v_cache.shape:
+        raise ValueError("k / v shapes differ")
+    B, S, Hkv, d = k_new.shape
+    num_pages, page, hk2, d2 = k_cache.shape
+    if (hk2, d2) != (Hkv, d) or block_table.shape[0] != B or cache_seqlens.numel() != B:
+        raise ValueError("inconsistent shapes")
+    rc = _lib.sfa_kv_append(_ptr(k_new), _ptr(v_new), S, _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                            block_table.shape[1], num_pages, page, _ptr(cache_seqlens), B, Hkv, d, _ptr(status),
+                            _stream(stream))
+    _check(rc)
 
 
 def bwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, topk, block_size) -> int:

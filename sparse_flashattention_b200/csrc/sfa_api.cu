@@ -678,6 +678,37 @@ int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const 
     return SFA_OK;
 }
 
+int sfa_kv_append(const void *k_new, const void *v_new, int seqlen_new, void *k_cache, void *v_cache,
+                  const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
+                  const int32_t *cache_seqlens, int B, int Hkv, int d, int32_t *status_dev, sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    if (B < 0 || seqlen_new < 0 || Hkv <= 0 || d <= 0 || max_pages_per_seq < 0 || num_pages < 0 || page_size <= 0)
+        return SFA_ERR_INVALID_ARG;
+    if (d % 8 != 0) return SFA_ERR_UNSUPPORTED;
+    if (B == 0 || seqlen_new == 0) return SFA_OK;
+    if (!k_new || !v_new || !k_cache || !v_cache || !block_table || !cache_seqlens) return SFA_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
+    KvAppendParams p{};
+    p.k_new = static_cast<const __nv_bfloat16 *>(k_new);
+    p.v_new = static_cast<const __nv_bfloat16 *>(v_new);
+    p.k_cache = static_cast<__nv_bfloat16 *>(k_cache);
+    p.v_cache = static_cast<__nv_bfloat16 *>(v_cache);
+    p.bt = block_table;
+    p.seqlens = cache_seqlens;
+    p.B = B;
+    p.S = seqlen_new;
+    p.Hkv = Hkv;
+    p.d = d;
+    p.max_pages = max_pages_per_seq;
+    p.num_pages = num_pages;
+    p.page = page_size;
+    p.status = status_dev;
+    if (launch_kv_append(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SFA_ERR_CUDA;
+    g_last_launches = 1;
+    return SFA_OK;
+}
+
 int sfa_decode_num_splits(int B, int Hq, int Hkv, int d, int topk_tok, int num_splits)
 {
     DecGeom g;

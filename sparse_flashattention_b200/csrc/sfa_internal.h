@@ -259,6 +259,16 @@ struct CombineParams {
 };
 cudaError_t launch_gated_combine(const CombineParams &p, int d, cudaStream_t st);
 
+// In-place paged KV-cache append.
+struct KvAppendParams {
+    const __nv_bfloat16 *k_new, *v_new;  // (B, S, Hkv, d)
+    __nv_bfloat16 *k_cache, *v_cache;    // (num_pages, page, Hkv, d)
+    const int32_t *bt, *seqlens;         // (B, max_pages), (B)
+    int B, S, Hkv, d, max_pages, num_pages, page;
+    int32_t *status;
+};
+cudaError_t launch_kv_append(const KvAppendParams &p, cudaStream_t st);
+
 cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStream_t st);
 cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaStream_t st);
 cudaError_t launch_decode_combine(const DecGeom &g, const DecCombineParams &p, cudaStream_t st);
