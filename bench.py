@@ -46,10 +46,10 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 # was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
     "fwd_attend_pipe_kernel": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
-                               "sha256": "c0bfe6e5fd6809d644e486b85999b49ba7c92229e2cc744a83dc0cf192bbb7ad",
+                               "sha256": "10f0e66608a4e6f8d69d43cdd26fdced9e371c831cdb471584e4eeaa4551f42f",
                                "bytes": 136768256},
     "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
-                            "sha256": "0b3c75fd09b59df6d32629609ae9f9caec91a4576e50ef43e1aba16360f25f22",
+                            "sha256": "f66cc7e500f8e87bb265a44ebe4d5b524a6afb4afdfc89cc189a2957ae14d2ce",
                             "bytes": 274462976},
 }
 
