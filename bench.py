@@ -440,9 +440,7 @@ def run_gpu(args, rank, world, local_rank):
                               "ms": round(m_ms, 4), "gbs": round(mix_bytes / (m_ms * 1e-3) / 1e9, 1),
                               "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
         }
-        if bwd_line is not None:
-            extras["backward"] = bwd_line
-        extras["kv_append"] = append_line
+        extras = {"nsa_branches": extras, "backward": bwd_line, "kv_append": append_line}
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
 
@@ -568,7 +566,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="sfa", choices=["sfa", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-extras", action="store_true", help="skip the NSA window-branch and gated-mix lines")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the lines beside the step: NSA window branch, gated mix, backward, KV append")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode-small"],
@@ -646,7 +645,9 @@ def main():
     if r["e2e"]:
         line["e2e"] = r["e2e"]
     if r["extras"]:
-        line["nsa_branches"] = r["extras"]
+        for key, val in r["extras"].items():  # nsa_branches, backward, kv_append: beside the timed step
+            if val is not None:
+                line[key] = val
     if world == 1 and not args.no_cpu_baseline:
         v, n, thr, secs = cpu_oracle_rate(pc, args.cpu_seconds)
         line["cpu_baseline"] = {"value": round(v, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
