@@ -102,3 +102,53 @@ def test_decode_split_heuristic(lib):
     s = lib.sfa_decode_num_splits(32, 32, 8, 128, 2048, 0)
     assert 1 <= s <= 16
     assert lib.sfa_decode_num_splits(1, 8, 8, 128, 100, 0) == 1
+
+
+def _bwd(lib, **over):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, dout=FAKE, lse=FAKE, cu_q=FAKE, cu_k=None, batch=1, max_sq=128,
+             max_sk=128, total_q=128, total_k=128, Hq=4, Hkv=1, d=128, sel=FAKE, topk=4, bs=64, causal=1, wl=-1,
+             wr=-1, scale=0.0, ws=FAKE, ws_bytes=0, status=None, dq=FAKE, dk=FAKE, dv=FAKE, stream=None)
+    a.update(over)
+    lib.sfa_bwd.restype = I
+    lib.sfa_bwd.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, I, I, I, I, I, F, P, Z, P, P, P, P, P]
+    return lib.sfa_bwd(*a.values())
+
+
+def test_bwd_host_validation(lib):
+    """Backward: sizes outside this build (d != 128, block_size != 64) and bad arguments are rejected
+    on the host; the workspace grows with the token bitmaps and the token lists."""
+    lib.sfa_bwd_workspace_size.restype = Z
+    lib.sfa_bwd_workspace_size.argtypes = [I] * 9
+    base = lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 128, 4, 64)
+    assert base > 0
+    assert lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 64, 4, 64) == 0    # d 64
+    assert lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 128, 4, 32) == 0   # block 32
+    assert lib.sfa_bwd_workspace_size(1, 0, 0, 0, 4, 1, 128, 4, 64) == 0         # no query
+    assert lib.sfa_bwd_workspace_size(1, 4096, 4096, 4096, 4, 1, 128, 4, 64) > \
+        lib.sfa_bwd_workspace_size(1, 1024, 4096, 1024, 4, 1, 128, 4, 64) > base
+    assert _bwd(lib, d=64) == 2                   # SFA_ERR_UNSUPPORTED
+    assert _bwd(lib, bs=32) == 2
+    assert _bwd(lib, Hq=6, Hkv=4) == 1            # SFA_ERR_INVALID_ARG
+    assert _bwd(lib, dout=None) == 1
+    assert _bwd(lib, dk=None) == 1
+    assert _bwd(lib, wl=-3) == 1
+    assert _bwd(lib, ws_bytes=16) == 3            # SFA_ERR_WORKSPACE_TOO_SMALL
+    assert _bwd(lib, q=ctypes.c_void_p((1 << 20) + 8)) == 1  # misaligned
+
+
+def test_kv_append_host_validation(lib):
+    lib.sfa_kv_append.restype = I
+    lib.sfa_kv_append.argtypes = [P, P, I, P, P, P, I, I, I, P, I, I, I, P, P]
+
+    def call(**over):
+        a = dict(kn=FAKE, vn=FAKE, S=1, kc=FAKE, vc=FAKE, bt=FAKE, max_pages=4, num_pages=8, page=16, lens=FAKE,
+                 B=2, Hkv=2, d=128, status=None, stream=None)
+        a.update(over)
+        return lib.sfa_kv_append(*a.values())
+
+    assert call(d=12) == 2        # not a multiple of 8
+    assert call(B=0) == 0         # nothing to append: no launch
+    assert call(S=0) == 0
+    assert call(page=0) == 1
+    assert call(bt=None) == 1
+    assert call(kc=ctypes.c_void_p((1 << 20) + 4)) == 1
