@@ -188,3 +188,71 @@ def kv_append(k_cache, v_cache, block_table, cache_seqlens, k_new, v_new):
             kc[pg, pos % page] = k_new[b, j]
             vc[pg, pos % page] = v_new[b, j]
     return kc, vc, bad
+
+
+# ---------------------------------------------------------------------------------------------------
+# Index producer for the decode: a Lightning-Indexer-style scan ("Sparse FlashAttention" on Ascend,
+# ggplus blog post, section "那个叫Lightning Indexer的家伙": the indexer scores the current query
+# against every key with FP8-quantized dot products and keeps the top-k token indices, which then
+# crop K and V for the sparse attention; its cost is one O(L) pass over the keys).
+# ---------------------------------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_round(x):
+    """Round float values to the FP8 E4M3 format (1 sign, 4 exponent bits with bias 7, 3 mantissa
+    bits; largest finite 448, smallest subnormal 2^-9, no infinities): round to nearest, ties to an
+    even mantissa, magnitudes past 448 saturated to 448.  Returns float64 values of the format."""
+    x = np.asarray(x, np.float64)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    # exponent of the format's spacing at |a|: 2^(e - 3) for normals (e >= -6), 2^-9 below 2^-6
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    q = 2.0 ** (e - 3)
+    r = np.round(a / q) * q  # numpy rounds halves to even
+    return np.sign(x) * np.minimum(r, E4M3_MAX)
+
+
+def index_topk(q, k_cache, block_table, cache_seqlens, Hkv, topk, n_local=0):
+    """Top-k token positions per (sequence, kv head) for the paged top-k decode.
+
+    Readings where the page is silent (each stated in the design notes):
+      * the group's G query heads share one selection (one list per kv head, as the decode takes it),
+        scored by the sum of their dot products: score_j = sum_g e4m3(q_g) . e4m3(k_j);
+      * FP8 is E4M3 with round-to-nearest-even and saturation, no scale factors (N(0,1) data fit);
+      * every cache position j < cache_seqlens[b] is a candidate, the last n_local positions are kept
+        whatever their score, the rest are the highest scores, a tie going to the lower position;
+      * the result is a set: ascending positions, -1 padded when fewer than topk exist.
+    The scores are exact: the group's summed query values (G values of the format, magnitudes from 2^-9
+    to G * 448) need at most 24 significant bits, a product with a key value of the format at most 28,
+    and every partial sum of the d products stays within 53 bits, so float64 computes them without
+    rounding, in any order.
+
+    q: (B, Hq, d) bf16 bits (uint16) or floats; k_cache: (num_pages, page, Hkv, d) likewise.
+    Returns (sel int32 (B, Hkv, topk), scores: list over b of float64 (Hkv, L_b))."""
+    def f(a):
+        a = np.asarray(a)
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64) if a.dtype == np.uint16 else \
+            a.astype(np.float64)
+    qf, kf = e4m3_round(f(q)), e4m3_round(f(k_cache))
+    B, Hq, d = qf.shape
+    G = Hq // Hkv
+    page = kf.shape[1]
+    sel = np.full((B, Hkv, topk), -1, np.int32)
+    scores = []
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        pos = np.arange(L)
+        rows = kf[block_table[b, pos // page], pos % page]  # (L, Hkv, d): logical order
+        sb = np.zeros((Hkv, L), np.float64)
+        for hk in range(Hkv):
+            qs = qf[b, hk * G:(hk + 1) * G].sum(axis=0)      # exact: G values of 4 significant bits
+            sb[hk] = rows[:, hk, :] @ qs
+            nl = min(n_local, L, topk)
+            keep = list(range(L - nl, L))
+            rest = [j for j in sorted(range(L - nl), key=lambda j: (-sb[hk, j], j))][:topk - nl]
+            chosen = np.sort(np.array(keep + rest, np.int64))
+            sel[b, hk, :chosen.size] = chosen
+        scores.append(sb)
+    return sel, scores
