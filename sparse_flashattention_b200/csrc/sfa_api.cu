@@ -611,16 +611,17 @@ int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const 
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) || !aligned16(dq))
         return SFA_ERR_INVALID_ARG;
     if (total_k == 0) return SFA_ERR_UNSUPPORTED;
+    // The dQ kernel keeps two copies of a tile's block union in shared memory beside its rings.
+    if (bwd_dq_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
     uint8_t *w = static_cast<uint8_t *>(workspace);
     if (cudaMemsetAsync(w + g.off_zero, 0, g.zero_bytes, st) != cudaSuccess) return SFA_ERR_CUDA;
     rc = fwd_prep_impl(g.f, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
                        status_dev, st);
     if (rc != SFA_OK) return rc;
-    CUtensorMap tq, tdo, tk, tv, tqr, tdor;
+    CUtensorMap tq, tdo, tk, tv;
     if (!encode_3d(tq, q, d, Hq, total_q, g.f.G, g.f.Tq) || !encode_3d(tdo, dout, d, Hq, total_q, g.f.G, g.f.Tq) ||
-        !encode_3d(tk, k, d, Hkv, total_k, 1, block_size) || !encode_3d(tv, v, d, Hkv, total_k, 1, block_size) ||
-        !encode_rows(tqr, q, d, (int64_t)total_q * Hq) || !encode_rows(tdor, dout, d, (int64_t)total_q * Hq))
+        !encode_3d(tk, k, d, Hkv, total_k, 1, block_size) || !encode_3d(tv, v, d, Hkv, total_k, 1, block_size))
         return SFA_ERR_CUDA;
     BwdParams p{};
     p.q = static_cast<const __nv_bfloat16 *>(q);
@@ -672,7 +673,7 @@ int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const 
     if (launch_bwd_delta(g, p, st) != cudaSuccess || launch_bwd_index(g, p, st) != cudaSuccess ||
         launch_bwd_plan(g, p, st) != cudaSuccess || launch_bwd_fill(g, p, st) != cudaSuccess ||
         launch_bwd_dq(g, p, tq, tdo, tk, tv, st) != cudaSuccess ||
-        launch_bwd_dkdv(g, p, tqr, tdor, tk, tv, st) != cudaSuccess)
+        launch_bwd_dkdv(g, p, tk, tv, st) != cudaSuccess)
         return SFA_ERR_CUDA;
     g_last_launches = 7;
     return SFA_OK;

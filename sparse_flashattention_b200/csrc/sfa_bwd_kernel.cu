@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
             const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16, 1024);
             const uint64_t dKmn0 = sdesc_sw128(smem_u32(sK), BS * 128, 1024);  // K as the MN-major B of dS K
             int k = 0, jg0 = 0;
-            int sk_st = 0, sk_ph = 0, sv_st = 0, sv_ph = 0, qk_st = 0, qk_ph = 0;  // K/V stages of the next S/dP, K of the next dQ
+            int sk_st = 0, sk_ph = 0, sv_st = 0, sv_ph = 0, qk_st = 0;  // K/V stages of the next S/dP, K stage of the next dQ
             bool ok = true;
             while (ok) {
                 const int m = k & 1;
@@ -329,10 +329,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                             umma_commit(&meta->dq_done[ig & 1]);
                             umma_commit(&meta->k_empty[st]);
                             ++np;
-                            if (++qk_st == kDqKStages) {
-                                qk_st = 0;
-                                qk_ph ^= 1;
-                            }
+                            if (++qk_st == kDqKStages) qk_st = 0;
                             progressed = true;
                         }
                     }
@@ -539,8 +536,7 @@ struct KvMeta {
 
 template <int D, int BS>
 __global__ void __launch_bounds__(kKvThreads, 1)
-    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmqr, const __grid_constant__ CUtensorMap tmdor,
-                    const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv, const BwdParams p)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv, const BwdParams p)
 {
     using C = KvCfg<D, BS>;
     extern __shared__ uint8_t kv_smem_raw[];
@@ -986,15 +982,15 @@ cudaError_t launch_bwd_dq(const BwdGeom &g, const BwdParams &p, const CUtensorMa
     return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq_rows,
-                            const CUtensorMap &tdo_rows, const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
+cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
+                            cudaStream_t st)
 {
     (void)g;
     static int configured = 0;
     const size_t smem = bwd_dkdv_smem_bytes();
     cudaError_t e = set_smem(bwd_dkdv_kernel<128, 64>, smem, configured);
     if (e != cudaSuccess) return e;
-    bwd_dkdv_kernel<128, 64><<<sm_count(), kKvThreads, smem, st>>>(tq_rows, tdo_rows, tk, tv, p);
+    bwd_dkdv_kernel<128, 64><<<sm_count(), kKvThreads, smem, st>>>(tk, tv, p);
     return cudaGetLastError();
 }
 

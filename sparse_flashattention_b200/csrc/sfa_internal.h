@@ -167,8 +167,8 @@ cudaError_t launch_bwd_plan(const BwdGeom &g, const BwdParams &p, cudaStream_t s
 cudaError_t launch_bwd_fill(const BwdGeom &g, const BwdParams &p, cudaStream_t st);
 cudaError_t launch_bwd_dq(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tdo,
                           const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
-cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq_rows,
-                            const CUtensorMap &tdo_rows, const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st);
+cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
+                            cudaStream_t st);
 size_t bwd_dq_smem_bytes(const BwdGeom &g);
 size_t bwd_dkdv_smem_bytes();
 

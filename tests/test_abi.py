@@ -134,6 +134,11 @@ def test_bwd_host_validation(lib):
     assert _bwd(lib, wl=-3) == 1
     assert _bwd(lib, ws_bytes=16) == 3            # SFA_ERR_WORKSPACE_TOO_SMALL
     assert _bwd(lib, q=ctypes.c_void_p((1 << 20) + 8)) == 1  # misaligned
+    # G 1 (128 tokens per tile) with topk 128 over 8192 blocks: a tile's union of up to 8192 blocks
+    # (two copies, 64 KB) does not fit beside the dQ kernel's rings
+    big = dict(Hq=1, Hkv=1, topk=128, max_sq=1 << 19, max_sk=1 << 19, total_q=1 << 19, total_k=1 << 19,
+               ws_bytes=1 << 62)
+    assert _bwd(lib, **big) == 2
 
 
 def test_kv_append_host_validation(lib):
