@@ -223,14 +223,16 @@ def index_topk(q, k_cache, block_table, cache_seqlens, Hkv, topk, n_local=0):
       * FP8 is E4M3 with round-to-nearest-even and saturation, no scale factors (N(0,1) data fit);
       * every cache position j < cache_seqlens[b] is a candidate, the last n_local positions are kept
         whatever their score, the rest are the highest scores, a tie going to the lower position;
-      * the result is a set: ascending positions, -1 padded when fewer than topk exist.
+      * the result is a set: ascending positions, -1 padded when fewer than topk exist;
+      * a position whose page id is outside [0, num_pages) is no candidate (counted in `bad`), as the
+        decode drops such tokens.
     The scores are exact: the group's summed query values (G values of the format, magnitudes from 2^-9
     to G * 448) need at most 24 significant bits, a product with a key value of the format at most 28,
     and every partial sum of the d products stays within 53 bits, so float64 computes them without
     rounding, in any order.
 
     q: (B, Hq, d) bf16 bits (uint16) or floats; k_cache: (num_pages, page, Hkv, d) likewise.
-    Returns (sel int32 (B, Hkv, topk), scores: list over b of float64 (Hkv, L_b))."""
+    Returns (sel int32 (B, Hkv, topk), scores: list over b of float64 (Hkv, L_b), bad)."""
     def f(a):
         a = np.asarray(a)
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64) if a.dtype == np.uint16 else \
@@ -241,18 +243,23 @@ def index_topk(q, k_cache, block_table, cache_seqlens, Hkv, topk, n_local=0):
     page = kf.shape[1]
     sel = np.full((B, Hkv, topk), -1, np.int32)
     scores = []
+    bad = 0
+    num_pages = kf.shape[0]
     for b in range(B):
         L = int(cache_seqlens[b])
         pos = np.arange(L)
-        rows = kf[block_table[b, pos // page], pos % page]  # (L, Hkv, d): logical order
+        pg = block_table[b, pos // page]
+        ok = (pg >= 0) & (pg < num_pages)
+        bad += int((~ok).sum())
+        rows = kf[np.where(ok, pg, 0), pos % page]  # (L, Hkv, d): logical order
         sb = np.zeros((Hkv, L), np.float64)
         for hk in range(Hkv):
-            qs = qf[b, hk * G:(hk + 1) * G].sum(axis=0)      # exact: G values of 4 significant bits
+            qs = qf[b, hk * G:(hk + 1) * G].sum(axis=0)      # exact: G values of the format
             sb[hk] = rows[:, hk, :] @ qs
             nl = min(n_local, L, topk)
-            keep = list(range(L - nl, L))
-            rest = [j for j in sorted(range(L - nl), key=lambda j: (-sb[hk, j], j))][:topk - nl]
+            keep = [j for j in range(L - nl, L) if ok[j]]
+            rest = [j for j in sorted(range(L - nl), key=lambda j: (-sb[hk, j], j)) if ok[j]][:topk - nl]
             chosen = np.sort(np.array(keep + rest, np.int64))
             sel[b, hk, :chosen.size] = chosen
         scores.append(sb)
-    return sel, scores
+    return sel, scores, bad
