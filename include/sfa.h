@@ -241,6 +241,24 @@ int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
                        int B, int Hq, int Hkv, int d, int window_left, float scale, int num_splits,
                        int32_t *status_dev, void *out, float *lse, sfa_stream_t stream);
 
+/* Index producer for the decode (Lightning-Indexer style: the "Sparse FlashAttention" post on Ascend,
+ * section "那个叫Lightning Indexer的家伙" — the current query scored against every key with FP8
+ * dot products, the top-k positions kept).  Per (sequence b, kv head): score_j = sum over the G query
+ * heads of the group of e4m3(q_h) . e4m3(k_j) for every cache position j < cache_seqlens[b]
+ * (E4M3: round to nearest even, saturated at +-448, no scale factors), computed exactly; the last
+ * n_local positions are always kept, the others by descending score, a tie to the lower position.
+ *   q          bf16 (B, Hq, d);  k_cache bf16 (num_pages, page_size, Hkv, d);  block_table as sfa_decode
+ *   sel_out    int32 (B, Hkv, topk): ascending positions, -1 padded — the sel_tok_idx of sfa_decode
+ *   workspace  sfa_index_topk_workspace_size() bytes (one 64-bit key per position)
+ * Positions whose page id is outside [0, num_pages) are no candidates (SFA_DEV_BAD_PAGE); a length
+ * past the block table is cut to it (SFA_DEV_BAD_SEQLEN).  d in {64, 128}; max_pages_per_seq *
+ * page_size <= 2^20.  One kernel, one CTA per (sequence, kv head). */
+size_t sfa_index_topk_workspace_size(int B, int Hkv, int max_pages_per_seq, int page_size);
+int sfa_index_topk(const void *q, const void *k_cache, const int32_t *block_table, int max_pages_per_seq,
+                   int num_pages, int page_size, const int32_t *cache_seqlens, int B, int Hq, int Hkv, int d, int topk,
+                   int n_local, void *workspace, size_t workspace_bytes, int32_t *status_dev, int32_t *sel_out,
+                   sfa_stream_t stream);
+
 /* In-place append of new keys / values to the paged cache, as the k / v arguments of
  * flash_attn_with_kvcache (flash-attention-npu docstrings): row j of sequence b goes to logical
  * position cache_seqlens[b] + j, i.e. page block_table[b][pos / page_size], row pos % page_size.
@@ -292,7 +310,7 @@ const char *sfa_status_string(int status);
 
 /* Number of kernel launches the last successful call on this host thread made (prefill: 1,
  * or 6 when the call uses the block-major schedule; decode: 1 with at most 6 splits, else 2,
- * plus 1 when topk_tok > 2048; a stage: its own count; window branch, gated mix, KV append: 1; backward: 7). */
+ * plus 1 when topk_tok > 2048; a stage: its own count; window branch, gated mix, KV append, index top-k: 1; backward: 7). */
 int sfa_last_launch_count(void);
 
 #ifdef __cplusplus

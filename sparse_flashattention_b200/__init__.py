@@ -60,6 +60,8 @@ def _load():
         "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P, F, P, Z, P, P, P, P]),
         "sfa_gated_combine": (I, [P, P, P, P, P, P, I, I, I, P, P]),
         "sfa_kv_append": (I, [P, P, I, P, P, P, I, I, I, P, I, I, I, P, P]),
+        "sfa_index_topk_workspace_size": (Z, [I, I, I, I]),
+        "sfa_index_topk": (I, [P, P, P, I, I, I, P, I, I, I, I, I, I, P, Z, P, P, P]),
         "sfa_bwd_workspace_size": (Z, [I, I, I, I, I, I, I, I, I]),
         "sfa_bwd": (I, [P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, I, I, I, I, I, F, P, Z, P, P, P, P, P]),
         "sfa_status_string": (ctypes.c_char_p, [I]),
@@ -192,6 +194,30 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.T
                       _stream(stream))
     _check(rc)
     return out, lse
+
+
+def index_topk(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,
+               topk: int, *, n_local: int = 0, out: Optional[torch.Tensor] = None,
+               workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """Decode index producer (sfa_index_topk): per (sequence, kv head) the top-k cache positions by exact
+    FP8 (E4M3) dot products of the group's query heads with every key, the last n_local always kept.
+    Returns int32 (B, Hkv, topk), ascending, -1 padded — the sel_tok_idx argument of decode."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    B, Hq, d = q.shape
+    num_pages, page, Hkv, d2 = k_cache.shape
+    if d2 != d or block_table.shape[0] != B or cache_seqlens.numel() != B:
+        raise ValueError("inconsistent shapes")
+    out = torch.empty((B, Hkv, topk), dtype=torch.int32, device=q.device) if out is None else out
+    ws = _workspace(workspace, int(_lib.sfa_index_topk_workspace_size(B, Hkv, block_table.shape[1], page)), q.device)
+    rc = _lib.sfa_index_topk(_ptr(q), _ptr(k_cache), _ptr(block_table), block_table.shape[1], num_pages, page,
+                             _ptr(cache_seqlens), B, Hq, Hkv, d, int(topk), int(n_local), _ptr(ws),
+                             ws.numel() * ws.element_size(), _ptr(status), _ptr(out), _stream(stream))
+    _check(rc)
+    return out
 
 
 def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

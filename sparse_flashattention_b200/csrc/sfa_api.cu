@@ -679,6 +679,53 @@ int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const 
     return SFA_OK;
 }
 
+size_t sfa_index_topk_workspace_size(int B, int Hkv, int max_pages_per_seq, int page_size)
+{
+    if (B <= 0 || Hkv <= 0 || max_pages_per_seq <= 0 || page_size <= 0) return 0;
+    return (size_t)B * Hkv * max_pages_per_seq * page_size * 8;
+}
+
+int sfa_index_topk(const void *q, const void *k_cache, const int32_t *block_table, int max_pages_per_seq,
+                   int num_pages, int page_size, const int32_t *cache_seqlens, int B, int Hq, int Hkv, int d, int topk,
+                   int n_local, void *workspace, size_t workspace_bytes, int32_t *status_dev, int32_t *sel_out,
+                   sfa_stream_t stream)
+{
+    g_last_launches = 0;
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || topk <= 0 || n_local < 0 || max_pages_per_seq < 0 || num_pages < 0 ||
+        page_size <= 0)
+        return SFA_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return SFA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return SFA_ERR_UNSUPPORTED;
+    if ((int64_t)max_pages_per_seq * page_size > (1 << 20) || topk > (1 << 20)) return SFA_ERR_UNSUPPORTED;
+    if (B == 0) return SFA_OK;
+    if (!q || !k_cache || !block_table || !cache_seqlens || !sel_out || !workspace) return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache)) return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < sfa_index_topk_workspace_size(B, Hkv, max_pages_per_seq, page_size))
+        return SFA_ERR_WORKSPACE_TOO_SMALL;
+    IndexParams p{};
+    p.q = static_cast<const __nv_bfloat16 *>(q);
+    p.kc = static_cast<const __nv_bfloat16 *>(k_cache);
+    p.bt = block_table;
+    p.seqlens = cache_seqlens;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.G = Hq / Hkv;
+    p.d = d;
+    p.max_pages = max_pages_per_seq;
+    p.num_pages = num_pages;
+    p.page = page_size;
+    p.topk = topk;
+    p.n_local = n_local;
+    p.max_len = (int64_t)max_pages_per_seq * page_size;
+    p.keys = static_cast<unsigned long long *>(workspace);
+    p.sel = sel_out;
+    p.status = status_dev;
+    if (launch_index_topk(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SFA_ERR_CUDA;
+    g_last_launches = 1;
+    return SFA_OK;
+}
+
 int sfa_kv_append(const void *k_new, const void *v_new, int seqlen_new, void *k_cache, void *v_cache,
                   const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
                   const int32_t *cache_seqlens, int B, int Hkv, int d, int32_t *status_dev, sfa_stream_t stream)

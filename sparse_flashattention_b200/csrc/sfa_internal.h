@@ -259,6 +259,18 @@ struct CombineParams {
 };
 cudaError_t launch_gated_combine(const CombineParams &p, int d, cudaStream_t st);
 
+// Decode index producer (exact FP8 scores, top-k positions per (sequence, kv head)).
+struct IndexParams {
+    const __nv_bfloat16 *q, *kc;  // (B, Hq, d), (num_pages, page, Hkv, d)
+    const int32_t *bt, *seqlens;  // (B, max_pages), (B)
+    int B, Hq, Hkv, G, d, max_pages, num_pages, page, topk, n_local;
+    int64_t max_len;              // max_pages * page: the key array's stride per (sequence, kv head)
+    unsigned long long *keys;     // workspace [B * Hkv][max_len]
+    int32_t *sel;                 // (B, Hkv, topk)
+    int32_t *status;
+};
+cudaError_t launch_index_topk(const IndexParams &p, cudaStream_t st);
+
 // In-place paged KV-cache append.
 struct KvAppendParams {
     const __nv_bfloat16 *k_new, *v_new;  // (B, S, Hkv, d)

@@ -157,3 +157,27 @@ def test_kv_append_host_validation(lib):
     assert call(page=0) == 1
     assert call(bt=None) == 1
     assert call(kc=ctypes.c_void_p((1 << 20) + 4)) == 1
+
+
+def test_index_topk_host_validation(lib):
+    lib.sfa_index_topk_workspace_size.restype = Z
+    lib.sfa_index_topk_workspace_size.argtypes = [I] * 4
+    assert lib.sfa_index_topk_workspace_size(2, 4, 8, 16) == 2 * 4 * 8 * 16 * 8
+    assert lib.sfa_index_topk_workspace_size(0, 4, 8, 16) == 0
+    lib.sfa_index_topk.restype = I
+    lib.sfa_index_topk.argtypes = [P, P, P, I, I, I, P, I, I, I, I, I, I, P, Z, P, P, P]
+
+    def call(**over):
+        a = dict(q=FAKE, kc=FAKE, bt=FAKE, max_pages=8, num_pages=16, page=16, lens=FAKE, B=2, Hq=8, Hkv=4, d=128,
+                 topk=32, n_local=0, ws=FAKE, ws_bytes=1 << 20, status=None, out=FAKE, stream=None)
+        a.update(over)
+        return lib.sfa_index_topk(*a.values())
+
+    assert call(d=96) == 2                 # SFA_ERR_UNSUPPORTED
+    assert call(Hq=6) == 1                 # Hq % Hkv
+    assert call(topk=0) == 1
+    assert call(n_local=-1) == 1
+    assert call(out=None) == 1
+    assert call(ws_bytes=8) == 3           # SFA_ERR_WORKSPACE_TOO_SMALL
+    assert call(max_pages=1 << 16, page=32) == 2  # more than 2^20 positions per sequence
+    assert call(B=0) == 0
