@@ -428,6 +428,28 @@ def run_gpu(args, rank, world, local_rank):
         append_line = {"workload": f"B {dc.B}, 1 new token, Hkv {dc.Hkv}, d {dc.d}, page {dc.page}",
                        "us": round(a_ms * 1e3, 2), "gbs": round(a_bytes / (a_ms * 1e-3) / 1e9, 1), "launches": 1,
                        "note": "launch-latency bound (256 KB moved)"}
+        # Decode index producer (exact FP8 scores over every cached key, top-k positions) on the decode
+        # workload: topk = its selection size, the last 128 positions forced as in its recipe.  Bytes = the
+        # K rows it scans.  Guarded so a failure here only marks this line.
+        try:
+            itopk = int(dc.sel.shape[2])
+            isel = torch.empty((dc.B, dc.Hkv, itopk), dtype=torch.int32, device=dev)
+            istatus = torch.zeros(1, dtype=torch.int32, device=dev)
+            iws = torch.empty(sfa.index_topk_workspace_size(dc.B, dc.Hkv, D["block_table"].shape[1], dc.page)
+                              if hasattr(sfa, "index_topk_workspace_size") else 1, dtype=torch.uint8, device=dev)
+
+            def run_index():
+                sfa.index_topk(D["q"], D["k_cache"], D["block_table"], D["cache_seqlens"], itopk, n_local=128,
+                               out=isel, workspace=iws, status=istatus)
+
+            i_ms = max_over_ranks([timed(run_index)], world, dev)[0]
+            i_bytes = int(np.asarray(dc.cache_seqlens, np.int64).sum()) * dc.Hkv * dc.d * 2
+            index_line = {"workload": f"decode workload, topk {itopk} (last 128 forced), every cached key scored",
+                          "ms": round(i_ms, 4), "gbs": round(i_bytes / (i_ms * 1e-3) / 1e9, 1),
+                          "frac": round(i_bytes / (i_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind,
+                          "launches": 1, "status": int(istatus.item())}
+        except Exception as exc:  # noqa: BLE001 - reported in the line, the rest of the bench goes on
+            index_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
         m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
         mix_bytes = 4 * pc.total_q * pc.Hq * pc.d * 2 + 3 * pc.total_q * pc.Hq * 4
@@ -440,7 +462,8 @@ def run_gpu(args, rank, world, local_rank):
                               "ms": round(m_ms, 4), "gbs": round(mix_bytes / (m_ms * 1e-3) / 1e9, 1),
                               "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
         }
-        extras = {"nsa_branches": extras, "backward": bwd_line, "kv_append": append_line}
+        extras = {"nsa_branches": extras, "backward": bwd_line, "kv_append": append_line,
+                  "index_topk": index_line}
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
 

@@ -196,6 +196,10 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.T
     return out, lse
 
 
+def index_topk_workspace_size(B, Hkv, max_pages_per_seq, page_size) -> int:
+    return int(_lib.sfa_index_topk_workspace_size(B, Hkv, max_pages_per_seq, page_size))
+
+
 def index_topk(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,
                topk: int, *, n_local: int = 0, out: Optional[torch.Tensor] = None,
                workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
