@@ -321,7 +321,7 @@ def test_decode_index_and_bad_ids(oracle_lib):
 
 
 def test_workload_kept_pairs_closed_form():
-    """The NSA recipe's kept-pair count (closed form) equals the survey figure for the tiny workload."""
+    """The NSA recipe's kept-pair count (closed form) equals the figures stated with the workloads."""
     assert W.kept_pairs_nsa([256], 32, 4) == 22656
     assert W.kept_pairs_nsa([8192, 4096, 2048, 2048], 64, 16) == 14295040
     assert W.kept_pairs_nsa([65536, 32768], 64, 16) == 96583680
