@@ -181,3 +181,37 @@ def test_index_topk_host_validation(lib):
     assert call(ws_bytes=8) == 3           # SFA_ERR_WORKSPACE_TOO_SMALL
     assert call(max_pages=1 << 16, page=32) == 2  # more than 2^20 positions per sequence
     assert call(B=0) == 0
+
+
+def test_window_and_gated_combine_host_validation(lib):
+    lib.sfa_window_fwd.restype = I
+    lib.sfa_window_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P, F, P, Z, P, P, P, P]
+
+    def win(**over):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, cu_q=FAKE, cu_k=None, batch=1, max_sq=128, max_sk=128, total_q=128,
+                 total_k=128, Hq=4, Hkv=1, d=128, causal=1, wl=512, wr=0, wlh=None, wrh=None, scale=0.0, ws=FAKE,
+                 ws_bytes=256, status=None, out=FAKE, lse=FAKE, stream=None)
+        a.update(over)
+        return lib.sfa_window_fwd(*a.values())
+
+    assert win(d=96) == 2
+    assert win(wl=-2) == 1
+    assert win(causal=2) == 1
+    assert win(out=None) == 1
+    assert win(ws_bytes=4) == 3
+    assert win(total_q=0) == 0
+
+    lib.sfa_gated_combine.restype = I
+    lib.sfa_gated_combine.argtypes = [P, P, P, P, P, P, I, I, I, P, P]
+
+    def mix(**over):
+        a = dict(o1=FAKE, g1=FAKE, o2=None, g2=None, o3=None, g3=None, total_q=16, Hq=4, d=128, out=FAKE,
+                 stream=None)
+        a.update(over)
+        return lib.sfa_gated_combine(*a.values())
+
+    assert mix(d=96) == 2
+    assert mix(o1=None) == 1                      # no branch left
+    assert mix(o1=ctypes.c_void_p((1 << 20) + 2)) == 1
+    assert mix(out=None) == 1
+    assert mix(total_q=0) == 0
