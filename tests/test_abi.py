@@ -199,7 +199,8 @@ def test_window_and_gated_combine_host_validation(lib):
     assert win(causal=2) == 1
     assert win(out=None) == 1
     assert win(ws_bytes=4) == 3
-    assert win(total_q=0) == 0
+    assert win(total_q=0, total_k=0) == 0     # nothing to compute
+    assert win(total_q=0) == 1                # k lengths must match q's when cu_seqlens_k is NULL
 
     lib.sfa_gated_combine.restype = I
     lib.sfa_gated_combine.argtypes = [P, P, P, P, P, P, I, I, I, P, P]
