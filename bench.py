@@ -590,7 +590,8 @@ def main():
     ap.add_argument("--impl", default="sfa", choices=["sfa", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the lines beside the step: NSA window branch, gated mix, backward, KV append")
+                    help="skip the lines beside the step: NSA window branch, gated mix, backward, KV append, "
+                         "index top-k")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode-small"],

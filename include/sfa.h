@@ -77,7 +77,8 @@ enum {
 /* Supported in this build: bf16 inputs; d in {64, 128}; prefill block_size in {32, 64},
  * 1 <= topk <= 128, G = Hq/Hkv <= 128, ceil(max_seqlen_k / block_size) <= 65536;
  * decode G <= 16, page_size >= 1, 1 <= topk_tok <= 65536, max_pages_per_seq*page_size
- * <= 2^20.  Anything else returns SFA_ERR_UNSUPPORTED. */
+ * <= 2^20; backward d = 128 and block_size = 64; KV append d a multiple of 8; index top-k
+ * max_pages_per_seq*page_size <= 2^20.  Anything else returns SFA_ERR_UNSUPPORTED. */
 
 /* ----------------------------------------------------------------------------------------
  * Prefill
