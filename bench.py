@@ -41,9 +41,8 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant kernel of
-# each stage, from one `ncu --set full` capture (profiles/fwd_attend_pipe_kernel_nsa_varlen_16k.md and
-# profiles/decode_split_kernel_paged_topk_decode.md).  A figure holds only for the kernel sources it
-# was taken on: the digest of those files must match, else the bench reports null.
+# each stage, from one `ncu` capture of that kernel on its workload.  A figure holds only for the
+# kernel sources it was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
     "fwd_attend_pipe_kernel": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
                                "sha256": "10f0e66608a4e6f8d69d43cdd26fdced9e371c831cdb471584e4eeaa4551f42f",
@@ -229,7 +228,6 @@ def run_gpu(args, rank, world, local_rank):
     import torch.distributed as dist
 
     import sparse_flashattention_b200 as sfa
-    from tests.parity import upload_decode, upload_prefill
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -239,7 +237,7 @@ def run_gpu(args, rank, world, local_rank):
         pc = W.small_config(2)
     else:
         pc = {1: W.config1, 2: W.config2, 3: W.config3, 4: W.config4}[args.prefill_config]()
-    P = upload_prefill(pc, dev)
+    P = W.upload_prefill(pc, dev)
     flops = prefill_flops(pc)
     # Profiling aids: 'prefill' skips the 9.7 GB decode cache (a tiny decode case stands in);
     # 'decode-small' runs the decode shape with shorter caches (about 1.3 GB) for ncu captures.
@@ -249,7 +247,7 @@ def run_gpu(args, rank, world, local_rank):
         dc = W.make_decode(5, 32, 32, 8, 128, 256, 4096, 16384, 2048, 128, parallel_values=True)
     else:
         dc = W.config5(parallel_values=True)
-    D = upload_decode(dc, dev)
+    D = W.upload_decode(dc, dev)
     gbytes = decode_bytes(dc)
 
     stream = torch.cuda.current_stream()

@@ -227,12 +227,17 @@ int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache,
  * counterpart to this call: it exists for callers such as serving engines whose device memory
  * pool is fixed before serving and forbids later allocation, or plugin hooks that receive only
  * input and output pointers.  Same arguments, semantics and kernels as sfa_decode, without the
- * workspace: the scratch lives in a static device array of 8 MiB that every GPU loading this
- * library keeps until the process exits.
+ * workspace: the scratch lives in a static device array of 8 MiB that a GPU keeps, once it holds
+ * it, until the process exits.
  *   - Returns SFA_ERR_WORKSPACE_TOO_SMALL when sfa_decode_workspace_size() of these arguments
  *     exceeds 8 MiB (nothing is launched).  It calls no allocation routine of any kind.
+ *   - q (and every other tensor) must live on the current device; a q on another device, or a
+ *     pointer the runtime does not know as device memory, returns SFA_ERR_INVALID_ARG.
  *   - The first call on each device looks the array's address up on that device (with it
- *     current); make that first call before any stream capture.
+ *     current).  With CUDA's lazy module loading (the default since CUDA 12.2) that lookup is
+ *     also when the module is loaded onto the device and its 8 MiB are reserved, so the first
+ *     call can fail if the device is out of memory.  Make that first call during start-up: before
+ *     a memory pool is sized to take the rest of the device, and before any stream capture.
  *   - Every call on a device shares the one array, and each call rewrites every byte it reads
  *     from it, so nothing carries over between calls; two calls that overlap on the GPU
  *     (other streams, other host threads) race on it and give undefined results. */

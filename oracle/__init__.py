@@ -217,7 +217,7 @@ def e4m3_round(x):
 def index_topk(q, k_cache, block_table, cache_seqlens, Hkv, topk, n_local=0):
     """Top-k token positions per (sequence, kv head) for the paged top-k decode.
 
-    Readings where the page is silent (each stated in the design notes):
+    Readings taken where the page is silent:
       * the group's G query heads share one selection (one list per kv head, as the decode takes it),
         scored by the sum of their dot products: score_j = sum_g e4m3(q_g) . e4m3(k_j);
       * FP8 is E4M3 with round-to-nearest-even and saturation, no scale factors (N(0,1) data fit);

@@ -352,3 +352,30 @@ def kept_pairs_nsa(seqlens, bs, topk):
         b = p // bs
         tot += int(((np.minimum(topk, b + 1) - 1) * bs + (p % bs + 1)).sum())
     return tot
+
+
+# ---------------------------------------------------------------------------------------------
+# Device upload of a case (torch is imported only here: the generators above need numpy alone)
+# ---------------------------------------------------------------------------------------------
+def dev_tensor(a, dtype=None, device="cuda"):
+    """A numpy array as a torch tensor on `device`; `dtype` reinterprets the bits (bf16 from uint16)."""
+    import torch
+    x = torch.from_numpy(np.ascontiguousarray(a))
+    if dtype is not None:
+        x = x.view(dtype)
+    return x.to(device)
+
+
+def upload_prefill(c, device="cuda"):
+    import torch
+    return dict(q=dev_tensor(c.q, torch.bfloat16, device), k=dev_tensor(c.k, torch.bfloat16, device),
+                v=dev_tensor(c.v, torch.bfloat16, device), cu_q=dev_tensor(c.cu_q, None, device),
+                cu_k=dev_tensor(c.cu_k, None, device), sel=dev_tensor(c.sel, None, device))
+
+
+def upload_decode(c, device="cuda"):
+    import torch
+    return dict(q=dev_tensor(c.q, torch.bfloat16, device), k_cache=dev_tensor(c.k_cache, torch.bfloat16, device),
+                v_cache=dev_tensor(c.v_cache, torch.bfloat16, device),
+                block_table=dev_tensor(c.block_table, None, device),
+                cache_seqlens=dev_tensor(c.cache_seqlens, None, device), sel=dev_tensor(c.sel, None, device))

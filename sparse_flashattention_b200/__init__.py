@@ -12,6 +12,7 @@ there is no CPU or PyTorch fallback, and importing fails loudly if the library i
 from __future__ import annotations
 
 import ctypes
+import functools
 import math
 import os
 from typing import Optional, Tuple
@@ -89,6 +90,29 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream) -> ctypes.c_void_p:
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _first_cuda_tensor(args, kwargs):
+    for a in list(args) + list(kwargs.values()):
+        items = a if isinstance(a, (list, tuple)) else [a]
+        for x in items:
+            for y in (x if isinstance(x, (list, tuple)) else [x]):
+                if isinstance(y, torch.Tensor) and y.is_cuda:
+                    return y
+    return None
+
+
+def _on_tensor_device(fn):
+    """Run a call with the device of its first CUDA tensor current: the library launches on the
+    current device and the default stream is that device's current stream."""
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        t = _first_cuda_tensor(args, kwargs)
+        if t is None or t.device == torch.device("cuda", torch.cuda.current_device()):
+            return fn(*args, **kwargs)
+        with torch.cuda.device(t.device):
+            return fn(*args, **kwargs)
+    return wrapper
 
 
 def _need(t: torch.Tensor, name: str, dtype, ndim: int):
@@ -171,6 +195,7 @@ def _workspace(ws, nbytes, device):
     return ws
 
 
+@_on_tensor_device
 def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor, sel_idx: torch.Tensor,
         block_size: int, *, cu_seqlens_k: Optional[torch.Tensor] = None, max_seqlen_q: Optional[int] = None,
         max_seqlen_k: Optional[int] = None, causal: bool = True, window: Tuple[int, int] = (-1, -1),
@@ -200,6 +225,7 @@ def index_topk_workspace_size(B, Hkv, max_pages_per_seq, page_size) -> int:
     return int(_lib.sfa_index_topk_workspace_size(B, Hkv, max_pages_per_seq, page_size))
 
 
+@_on_tensor_device
 def index_topk(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor, cache_seqlens: torch.Tensor,
                topk: int, *, n_local: int = 0, out: Optional[torch.Tensor] = None,
                workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
@@ -224,6 +250,7 @@ def index_topk(q: torch.Tensor, k_cache: torch.Tensor, block_table: torch.Tensor
     return out
 
 
+@_on_tensor_device
 def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
               block_table: torch.Tensor, cache_seqlens: torch.Tensor, status: Optional[torch.Tensor] = None,
               stream=None) -> None:
@@ -251,6 +278,7 @@ def bwd_workspace_size(batch, max_seqlen_q, max_seqlen_k, total_q, Hq, Hkv, d, t
                                            block_size))
 
 
+@_on_tensor_device
 def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, dout: torch.Tensor,
         lse: torch.Tensor, cu_seqlens_q: torch.Tensor, sel_idx: torch.Tensor, block_size: int, *,
         cu_seqlens_k: Optional[torch.Tensor] = None, max_seqlen_q: Optional[int] = None,
@@ -281,6 +309,7 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor, do
     return dq, dk, dv
 
 
+@_on_tensor_device
 def window_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: torch.Tensor, *,
                cu_seqlens_k: Optional[torch.Tensor] = None, max_seqlen_q: Optional[int] = None,
                max_seqlen_k: Optional[int] = None, causal: bool = True, window: Tuple[int, int] = (-1, -1),
@@ -311,6 +340,7 @@ def window_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens_q: 
     return out, lse
 
 
+@_on_tensor_device
 def gated_combine(branches, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Gated mix (sfa_gated_combine): out = sum over (o, g) in branches of g[..., None] * o, for up to
     three (o, g) pairs in the order (compressed, selected, window); None entries are left out.
@@ -340,6 +370,7 @@ def gated_combine(branches, out: Optional[torch.Tensor] = None, stream=None) -> 
     return out
 
 
+@_on_tensor_device
 def fwd_prep(cu_seqlens_q, sel_idx, *, Hq: int, d: int, block_size: int, cu_seqlens_k=None, max_seqlen_q=None,
              max_seqlen_k=None, causal=True, window=(-1, -1), workspace=None, status=None, stream=None):
     """Stage 1 (sfa_fwd_prep).  Returns (workspace, sel_c, cnt): sel_c (total_q, Hkv, topk) and
@@ -367,6 +398,7 @@ def fwd_prep(cu_seqlens_q, sel_idx, *, Hq: int, d: int, block_size: int, cu_seql
     return ws, sel_c, cnt
 
 
+@_on_tensor_device
 def fwd_attend(q, k, v, cu_seqlens_q, workspace, *, topk: int, block_size: int, cu_seqlens_k=None,
                max_seqlen_q=None, max_seqlen_k=None, causal=True, window=(-1, -1), scale=None, out=None, lse=None,
                status=None, stream=None):
@@ -413,6 +445,7 @@ def _dec_checks(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx):
     return B, Hq, d, num_pages, page, Hkv
 
 
+@_on_tensor_device
 def decode(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx, *, window_left: int = -1, scale=None,
            num_splits: int = 0, out=None, lse=None, workspace=None, status=None, stream=None):
     """Paged top-k decode (sfa_decode): q (B, Hq, d); caches (num_pages, page, Hkv, d);
@@ -432,6 +465,7 @@ def decode(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx, *, wind
     return out, lse
 
 
+@_on_tensor_device
 def decode_prep(cache_seqlens, sel_tok_idx, *, Hq: int, d: int, max_pages_per_seq: int, page_size: int,
                 window_left=-1, num_splits=0, workspace=None, status=None, stream=None):
     """Stage 1 (sfa_decode_prep).  Returns (workspace, tok_c, cnt) with int32 views into the
@@ -454,6 +488,7 @@ def decode_prep(cache_seqlens, sel_tok_idx, *, Hq: int, d: int, max_pages_per_se
     return ws, tok_c, cnt
 
 
+@_on_tensor_device
 def decode_attend(q, k_cache, v_cache, block_table, workspace, *, topk_tok: int, scale=None, num_splits=0, out=None,
                   lse=None, status=None, stream=None):
     """sfa_decode_attend: the split kernel (and, beyond six splits, the combine kernel) on the
@@ -469,6 +504,7 @@ def decode_attend(q, k_cache, v_cache, block_table, workspace, *, topk_tok: int,
     return out, lse
 
 
+@_on_tensor_device
 def decode_noalloc(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx, *, window_left: int = -1,
                    scale=None, num_splits: int = 0, out=None, lse=None, status=None, stream=None):
     """sfa_decode_noalloc: the same decode without a workspace, for callers that may not

@@ -942,15 +942,6 @@ __global__ void __launch_bounds__(kKvThreads, 1)
     }
 }
 
-template <typename K>
-cudaError_t set_smem(K kern, size_t bytes, int &configured)
-{
-    if ((int)bytes <= configured) return cudaSuccess;
-    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess) configured = (int)bytes;
-    return e;
-}
-
 int sm_count()
 {
     int dev = 0, n = 148;
@@ -973,9 +964,8 @@ size_t bwd_dkdv_smem_bytes()
 cudaError_t launch_bwd_dq(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tdo,
                           const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
 {
-    static int configured = 0;
     const size_t smem = bwd_dq_smem_bytes(g);
-    cudaError_t e = set_smem(bwd_dq_kernel<128, 64>, smem, configured);
+    cudaError_t e = ensure_smem_for(bwd_dq_kernel<128, 64>, smem);
     if (e != cudaSuccess) return e;
     const int grid = std::max(1, std::min(p.tiles, sm_count()));
     bwd_dq_kernel<128, 64><<<grid, kDqThreads, smem, st>>>(tq, tdo, tk, tv, p);
@@ -986,9 +976,8 @@ cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensor
                             cudaStream_t st)
 {
     (void)g;
-    static int configured = 0;
     const size_t smem = bwd_dkdv_smem_bytes();
-    cudaError_t e = set_smem(bwd_dkdv_kernel<128, 64>, smem, configured);
+    cudaError_t e = ensure_smem_for(bwd_dkdv_kernel<128, 64>, smem);
     if (e != cudaSuccess) return e;
     bwd_dkdv_kernel<128, 64><<<sm_count(), kKvThreads, smem, st>>>(tk, tv, p);
     return cudaGetLastError();

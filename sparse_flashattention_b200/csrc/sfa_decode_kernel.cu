@@ -457,13 +457,8 @@ template <int D>
 cudaError_t launch_split_t(const DecGeom &g, const DecSplitParams &p, cudaStream_t st)
 {
     const size_t smem = DecCfg<D>::kBytes;
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e =
-            cudaFuncSetAttribute(decode_split_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    const cudaError_t e = ensure_smem_for(decode_split_kernel<D>, smem);
+    if (e != cudaSuccess) return e;
     const int cps = (g.S + kDecWarps - 1) / kDecWarps;
     decode_split_kernel<D><<<g.B * g.Hkv * cps, kDecThreads, smem, st>>>(p);
     return cudaGetLastError();

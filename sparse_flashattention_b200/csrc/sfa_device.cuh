@@ -321,38 +321,6 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
-// 2^x on the FMA/ALU pipes (the MUFU unit that ex2.approx uses is shared by the whole SM and
-// is the softmax's bottleneck).  Range reduction: x = j + f with j = round(x), obtained by adding
-// 1.5*2^23 so the adder rounds j into the low mantissa bits, and f in [-1/2, 1/2].  2^f is a
-// degree-3 polynomial whose coefficients were fitted for relative error on [-1/2, 1/2] (max
-// 1.2e-4 evaluated in float32, below the 2^-9 rounding of the bf16 probabilities it feeds);
-// 2^j is added to the exponent field.  Valid for x <= 8; x < -126 (and -inf) gives exactly 0.
-constexpr float kExp2C0 = 0.99994075298f;
-constexpr float kExp2C1 = 0.69341576099f;
-constexpr float kExp2C2 = 0.24250595272f;
-constexpr float kExp2C3 = 0.05431177467f;
-
-__device__ __forceinline__ float ex2_fma(float x)
-{
-    const float xc = fmaxf(x, -126.f);
-    const float t = __fadd_rn(xc, 12582912.f);
-    const float j = __fsub_rn(t, 12582912.f);
-    const float f = __fsub_rn(xc, j);
-    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, kExp2C0);
-    const int ji = __float_as_int(t) - 0x4B400000;
-    const float r = __int_as_float(__float_as_int(p) + (ji << 23));
-    return x < -126.f ? 0.f : r;
-}
-
-// Which of a row's exponentials go to the FMA pipes instead of MUFU.  Measured on the prefill
-// kernels the softmax is issue-bound rather than MUFU-bound, so none do for now; the helper and
-// its error bound stay for rows of wider blocks.
-constexpr int kExpOnFmaEvery = 0;  // 0: none; n: element c when c % n == n - 1
-__device__ __forceinline__ constexpr bool exp_on_fma(int c)
-{
-    return kExpOnFmaEvery > 0 && (c % (kExpOnFmaEvery > 0 ? kExpOnFmaEvery : 1)) == kExpOnFmaEvery - 1;
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {
     float d;
@@ -406,8 +374,8 @@ __device__ __forceinline__ float scores_to_p(const float (&x)[BS], float sc, flo
 #pragma unroll
     for (int c = 0; c < BS; c += 2) {
         const float2 y = ffma2(make_float2(x[c], x[c + 1]), sc2, b2);
-        const float p0 = exp_on_fma(c) ? ex2_fma(y.x) : ex2(y.x);
-        const float p1 = exp_on_fma(c + 1) ? ex2_fma(y.y) : ex2(y.y);
+        const float p0 = ex2(y.x);
+        const float p1 = ex2(y.y);
         acc[(c >> 1) & 3] = fadd2(acc[(c >> 1) & 3], make_float2(p0, p1));
         packed[c / 2] = pack_bf16x2(p0, p1);
     }

@@ -491,13 +491,8 @@ cudaError_t launch_inv_t(const FwdGeom &g, const FwdAttendParams &p, const CUten
                          const CUtensorMap &tv, cudaStream_t st)
 {
     const size_t smem = inv_smem_bytes<D, BS>();
-    static bool configured = false;
-    if (!configured) {
-        cudaError_t e =
-            cudaFuncSetAttribute(fwd_attend_inv_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    const cudaError_t e = ensure_smem_for(fwd_attend_inv_kernel<D, BS>, smem);
+    if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const cudaError_t le =

@@ -468,13 +468,8 @@ cudaError_t launch_t(const FwdGeom &g, const FwdAttendParams &p, const CUtensorM
                      const CUtensorMap &tv, cudaStream_t st)
 {
     const size_t smem = smem_bytes_for<D, BS>(g);
-    static int configured = 0;
-    if ((int)smem > configured) {
-        cudaError_t e =
-            cudaFuncSetAttribute(fwd_attend_kernel<D, BS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = (int)smem;
-    }
+    const cudaError_t e = ensure_smem_for(fwd_attend_kernel<D, BS>, smem);
+    if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = g.tiles < 2 * sms ? g.tiles : 2 * sms;

@@ -704,13 +704,8 @@ cudaError_t launch_pipe_t(const FwdAttendParams &p, const CUtensorMap &tq, const
                           cudaStream_t st)
 {
     const size_t smem = 1024 + pipe_layout<D, BS>(MODE, p.umax, p.Tq, p.topk, p.nblk_max).bytes;
-    static int configured = 0;
-    if ((int)smem > configured) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_attend_pipe_kernel<D, BS, MODE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        configured = (int)smem;
-    }
+    const cudaError_t e = ensure_smem_for(fwd_attend_pipe_kernel<D, BS, MODE>, smem);
+    if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = p.tiles < 2 * sms ? p.tiles : 2 * sms;

@@ -208,6 +208,16 @@ struct DecCombineParams {
     float *lse;
 };
 
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` on the current device.  The
+// limit is a per-device attribute, so the value already set is remembered per (kernel, device)
+// under a lock; a launch on another device (or from another host thread) sets it there too.
+cudaError_t ensure_smem(const void *kernel, size_t bytes);
+template <typename K>
+inline cudaError_t ensure_smem_for(K *kernel, size_t bytes)
+{
+    return ensure_smem(reinterpret_cast<const void *>(kernel), bytes);
+}
+
 // Launchers (return the launch's cudaError_t).
 // Kernel launch on `st`; with pdl the kernel may start while the previous kernel in the stream is
 // finishing (it must call grid_dep_wait() before reading that kernel's results).

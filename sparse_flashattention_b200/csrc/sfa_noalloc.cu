@@ -24,11 +24,20 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch on the current device, looked up once per device.
-int scratch_for_current_device(void **out)
+// Device address of the scratch on the device that holds `q`, which must be the current device:
+// the kernels run on the current device and read the array there, so a call whose tensors live on
+// another GPU is refused rather than pointed at the wrong GPU's array.  Looked up once per device.
+int scratch_for_device_of(const void *q, void **out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SFA_ERR_CUDA;
+    cudaPointerAttributes attr{};
+    if (cudaPointerGetAttributes(&attr, q) != cudaSuccess) {
+        (void)cudaGetLastError();  // clear the error a non-device pointer leaves behind
+        return SFA_ERR_INVALID_ARG;
+    }
+    if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged) return SFA_ERR_INVALID_ARG;
+    if (attr.device != dev) return SFA_ERR_INVALID_ARG;
     std::lock_guard<std::mutex> lock(g_mu);
     if (!g_scratch_ptr[dev]) {
         void *p = nullptr;
@@ -49,8 +58,9 @@ extern "C" int sfa_decode_noalloc(const void *q, const void *k_cache, const void
 {
     const size_t need = sfa_decode_workspace_size(B, Hq, Hkv, d, topk_tok, num_splits);
     if (need > kNoAllocScratchBytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (!q) return SFA_ERR_INVALID_ARG;
     void *scratch = nullptr;
-    const int rc = scratch_for_current_device(&scratch);
+    const int rc = scratch_for_device_of(q, &scratch);
     if (rc != SFA_OK) return rc;
     return sfa_decode(q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, cache_seqlens,
                       sel_tok_idx, topk_tok, B, Hq, Hkv, d, window_left, scale, num_splits, scratch,

@@ -317,11 +317,9 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
 {
     const size_t words = (size_t)(g.nblk_max + 31) / 32;
     const size_t smem = words * 4 + (size_t)g.Tq * g.topk * 4 + (size_t)g.topk * kPrepThreads * 4;
-    static int configured_bytes = 0;
-    if ((int)smem > 48 * 1024 && (int)smem > configured_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(fwd_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+        const cudaError_t e = ensure_smem_for(fwd_prep_kernel, smem);
         if (e != cudaSuccess) return e;
-        configured_bytes = (int)smem;
     }
     fwd_prep_kernel<<<g.tiles, kPrepThreads, smem, st>>>(p);
     return cudaGetLastError();
@@ -341,12 +339,9 @@ cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cuda
 cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStream_t st)
 {
     const size_t smem = (size_t)((p.max_len + 31) / 32) * 4;
-    static int configured_bytes = 0;
-    if ((int)smem > 48 * 1024 && (int)smem > configured_bytes) {
-        cudaError_t e =
-            cudaFuncSetAttribute(decode_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+        const cudaError_t e = ensure_smem_for(decode_prep_kernel, smem);
         if (e != cudaSuccess) return e;
-        configured_bytes = (int)smem;
     }
     decode_prep_kernel<<<g.B * g.Hkv, kDecPrepThreads, smem, st>>>(p);
     return cudaGetLastError();

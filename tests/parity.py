@@ -7,28 +7,11 @@ no kept key must be exactly 0 with lse exactly -inf; canonical index sets bit-ex
 import numpy as np
 import torch
 
+from sfa_workloads import dev_tensor, upload_decode, upload_prefill  # noqa: F401 (re-exported)
+
 OUT_ATOL = 2e-2
 OUT_RTOL = 2e-2
 LSE_ATOL = 1e-3
-
-
-def dev_tensor(a, dtype=None, device="cuda"):
-    x = torch.from_numpy(np.ascontiguousarray(a))
-    if dtype is not None:
-        x = x.view(dtype)
-    return x.to(device)
-
-
-def upload_prefill(c, device="cuda"):
-    return dict(q=dev_tensor(c.q, torch.bfloat16, device), k=dev_tensor(c.k, torch.bfloat16, device),
-                v=dev_tensor(c.v, torch.bfloat16, device), cu_q=dev_tensor(c.cu_q, None, device),
-                cu_k=dev_tensor(c.cu_k, None, device), sel=dev_tensor(c.sel, None, device))
-
-
-def upload_decode(c, device="cuda"):
-    return dict(q=dev_tensor(c.q, torch.bfloat16, device), k_cache=dev_tensor(c.k_cache, torch.bfloat16, device),
-                v_cache=dev_tensor(c.v_cache, torch.bfloat16, device), block_table=dev_tensor(c.block_table, None, device),
-                cache_seqlens=dev_tensor(c.cache_seqlens, None, device), sel=dev_tensor(c.sel, None, device))
 
 
 def run_fwd(sfa, c, d=None, status=None, sel=None, **kw):

@@ -1,22 +1,20 @@
 """GPU parity of the prefill backward (sfa_bwd) against the fp64 oracle (oracle.bwd), through the C ABI.
 
-The forward's out / lse come from sfa_fwd on the same inputs; dout is seeded.  Tolerance, from the
-arithmetic of the kernels: P and dS enter the tensor cores as bf16 (unit roundoff 2^-8), and
-D = rowsum(dO o O) is taken, as the FlashAttentionScoreGrad case study prescribes, from the forward's
-output — bf16 here — while the oracle sums p dP exactly.  Each gradient element therefore carries an
-error of a few 2^-8 times the size of the terms it sums; where those terms cancel (a row with two
-keys, a key that few rows keep) the element is small and the error is not.  The check, per tensor:
-  - every element: |gpu - ref| <= 2e-2 |ref| + 8e-2 rms(ref)
-  - 99.9 % of the elements: |gpu - ref| - 2e-2 |ref| <= 1.5e-2 rms(ref)
-  - relative Frobenius error below 1e-2.
-(Measured on B200: worst element 4.2 % of rms, 99.9th percentile 0.5 %, Frobenius 0.25 %; a wrong
-sign, a dropped term or a misplaced row is an O(1) Frobenius error.)"""
+The forward's out / lse come from sfa_fwd on the same inputs; dout is seeded.  Every element of dq,
+dk and dv must lie within its own error bound, derived from the kernels' arithmetic in
+tests/bwd_bound.py: the exactly known effect of the bf16 forward output on D = rowsum(dO o O) and of
+the forward's lse error, carried with their signs; six standard deviations of the independent bf16
+roundings of P and dS over the element's own terms; fp32 accumulation; bf16 rounding of the result.
+There is no tensor-wide term: a wrong value on a key that few rows keep is judged against that key's
+own terms.  An element with no terms must be exactly 0.
+"""
 import dataclasses
 
 import numpy as np
 import pytest
 
 import sfa_workloads as W
+from tests import bwd_bound as BB
 from tests.parity import upload_prefill, dev_tensor
 
 torch = pytest.importorskip("torch")
@@ -31,30 +29,27 @@ def sfa():
     return m
 
 
-def assert_grad_close(gpu, ref, what):
-    g = gpu.float().cpu().numpy().astype(np.float64)
-    ref = np.asarray(ref, np.float64)
-    assert g.shape == ref.shape, (what, g.shape, ref.shape)
-    assert np.isfinite(g).all(), f"{what}: non-finite values"
-    if ref.size == 0:
-        return
-    rms = float(np.sqrt(np.mean(ref * ref)))
-    excess = np.abs(g - ref) - 2e-2 * np.abs(ref)
-    worst = np.unravel_index(np.argmax(excess), excess.shape)
-    assert excess.max() <= 8e-2 * rms, \
-        f"{what}: excess {excess.max():.4g} (rms {rms:.4g}) at {worst}: gpu {g[worst]} ref {ref[worst]}"
-    p999 = np.percentile(np.maximum(excess, 0), 99.9)
-    assert p999 <= 1.5e-2 * rms, f"{what}: 99.9th percentile excess {p999:.4g} (rms {rms:.4g})"
-    rel = np.linalg.norm(g - ref) / max(np.linalg.norm(ref), 1e-30)
-    assert rel < 1e-2, f"{what}: relative Frobenius error {rel:.4g}"
-
-
-def _run(sfa, c, dd, dout, status=None):
+def _run(sfa, c, dd, dout, status=None, with_fwd=False):
     kw = dict(cu_seqlens_k=dd["cu_k"], max_seqlen_q=c.max_sq, max_seqlen_k=c.max_sk, causal=bool(c.causal),
               window=(c.wl, c.wr))
     out, lse = sfa.fwd(dd["q"], dd["k"], dd["v"], dd["cu_q"], dd["sel"], c.bs, **kw)
     dq, dk, dv = sfa.bwd(dd["q"], dd["k"], dd["v"], out, dout, lse, dd["cu_q"], dd["sel"], c.bs, status=status, **kw)
-    return dq, dk, dv
+    return (dq, dk, dv, out, lse) if with_fwd else (dq, dk, dv)
+
+
+def check_grads(oracle_lib, c, dout_bits, grads, out, lse, ref=None):
+    """Every element of dq, dk, dv within its derived bound (tests/bwd_bound.py)."""
+    rq, rk, rv, bad = oracle_lib.bwd(c, dout_bits) if ref is None else ref
+    assert bad == 0
+    ro, rl, _ = oracle_lib.fwd(c)
+    sel_c, _, _ = oracle_lib.fwd_index(c)
+    og = out.float().cpu().numpy().astype(np.float64)
+    lg = lse.cpu().numpy().astype(np.float64)
+    bq, bk, bv = BB.bwd_bounds(c, BB._f(dout_bits), og, lg, ro, rl, sel_c, chunk=128)
+    dq, dk, dv = (x.float().cpu().numpy().astype(np.float64) for x in grads)
+    BB.assert_within_bound(dq, rq, bq, "dq")
+    BB.assert_within_bound(dk, rk, bk, "dk", add_rounding=True)
+    BB.assert_within_bound(dv, rv, bv, "dv", add_rounding=True)
 
 
 BWD_CASES = {
@@ -77,15 +72,27 @@ def test_bwd_parity(sfa, oracle_lib, name):
     dout_bits = W.f32_to_bf16_bits(rng.standard_normal((c.total_q, c.Hq, c.d), dtype=np.float32))
     dd = upload_prefill(c)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dq, dk, dv = _run(sfa, c, dd, dev_tensor(dout_bits, torch.bfloat16), status)
+    dq, dk, dv, out, lse = _run(sfa, c, dd, dev_tensor(dout_bits, torch.bfloat16), status, with_fwd=True)
     assert sfa.last_launch_count() == 7
     torch.cuda.synchronize()
     assert int(status.item()) == 0
-    rq, rk, rv, bad = oracle_lib.bwd(c, dout_bits)
-    assert bad == 0
-    assert_grad_close(dq, rq, "dq")
-    assert_grad_close(dk, rk, "dk")
-    assert_grad_close(dv, rv, "dv")
+    check_grads(oracle_lib, c, dout_bits, (dq, dk, dv), out, lse)
+
+
+def test_bwd_full_length_sequence(sfa, oracle_lib):
+    """The backward at the length the benchmark runs it: one 8192-token NSA sequence, Hq 4 / Hkv 1
+    (G 4, 32 tokens per chunk), d 128, block 64, top-16 with init 1 / local 2.  Block 0 is selected
+    by all 8192 tokens, so its (block, kv head) row is cut into the largest number of pieces the
+    piece scheme makes (16), summed in piece order.  Every element of dq, dk and dv is checked."""
+    c = W.make_nsa_prefill(26, [8192], 4, 1, 128, 64, 16, 1, 2)
+    rng = np.random.default_rng(9)
+    dout_bits = W.f32_to_bf16_bits(rng.standard_normal((c.total_q, c.Hq, c.d), dtype=np.float32))
+    dd = upload_prefill(c)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dk, dv, out, lse = _run(sfa, c, dd, dev_tensor(dout_bits, torch.bfloat16), status, with_fwd=True)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    check_grads(oracle_lib, c, dout_bits, (dq, dk, dv), out, lse)
 
 
 def test_bwd_deterministic_and_empty_rows(sfa, oracle_lib):
@@ -100,16 +107,13 @@ def test_bwd_deterministic_and_empty_rows(sfa, oracle_lib):
     dout_bits = W.f32_to_bf16_bits(rng.standard_normal((c.total_q, c.Hq, c.d), dtype=np.float32))
     dd = upload_prefill(c)
     dout = dev_tensor(dout_bits, torch.bfloat16)
-    a = _run(sfa, c, dd, dout)
-    b = _run(sfa, c, dd, dout)
+    a = _run(sfa, c, dd, dout, with_fwd=True)
+    b = _run(sfa, c, dd, dout, with_fwd=True)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
     dq = a[0]
     assert (dq[5:40] == 0).all() and (dq[1510] == 0).all()
-    rq, rk, rv, _ = oracle_lib.bwd(c, dout_bits)
-    assert_grad_close(a[0], rq, "dq")
-    assert_grad_close(a[1], rk, "dk")
-    assert_grad_close(a[2], rv, "dv")
+    check_grads(oracle_lib, c, dout_bits, a[:3], a[3], a[4])
 
 
 def test_bwd_no_queries_zero_key_grads(sfa):
