@@ -3,19 +3,20 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sfa|reference]
 
 One step = one pass of the whole hot path on seeded synthetic inputs already resident in
-HBM: the varlen NSA prefill workload (lengths [8192, 4096, 2048, 2048], Hq16/Hkv4, d128,
-block 64, top-16 with init 1 / local 2; sfa_fwd_prep + sfa_fwd_attend) followed by the paged
-top-k decode workload (B32, Hq32/Hkv8, d128, L ~ U[16384, 131072], page 256, 2048 tokens per
-(sequence, kv head); sfa_decode, which deduplicates the selections inside its split kernel).
-L2 is flushed (256 MiB write)
-before every step, outside the kernel events.
+HBM: the whole public sfa_fwd call on the long-context NSA prefill workload (lengths
+[65536, 32768], Hq = Hkv = 4, d128, block 64, top-16 with init 1 / local 2: the largest
+single-GPU configuration, which also runs the block-major schedule and its partial merge),
+followed by the whole sfa_decode call on the paged top-k decode workload (B32, Hq32/Hkv8,
+d128, L ~ U[16384, 131072], page 256, 2048 tokens per (sequence, kv head)).  L2 is flushed
+(256 MiB write) before every step, outside the kernel events.
 
-The JSON line's value is prefill effective TFLOP/s (4*d flops per kept query-key pair per
-query head) from CUDA events around the two prefill stages; the decode figure (gathered
-K+V bytes per second) is reported beside it.  Under torchrun each rank runs its own
-instance of the workload (independent problems, no collective; weak scaling) and the time is
-the max over ranks.  --impl reference times the fp64 CPU oracle on a bounded sample of the
-same workload instead.
+The JSON line's value is the prefill's effective TFLOP/s (4*d flops per kept query-key pair
+per query head, the pairs counted exactly from the selections); the decode figure (gathered
+K+V bytes per second) is reported beside it.  The other prefill configurations (tiny, varlen
+NSA, dense window) are timed beside the step under "prefill_configs", each as its whole
+public call.  Under torchrun each rank runs its own instance of the workload (independent
+problems, no collective; weak scaling) and the time is the max over ranks.  --impl reference
+times the fp64 CPU oracle on a bounded sample of the same workload instead.
 """
 from __future__ import annotations
 
@@ -36,7 +37,13 @@ if ROOT not in sys.path:
 import sfa_workloads as W  # noqa: E402
 
 METRIC = "sparse-attn fwd effective TFLOP/s & decode gathered-KV GB/s, 1×B200"
-PREFILL_NAME = "nsa_varlen_16k: lens [8192,4096,2048,2048], Hq16/Hkv4, d128, bs64, topk16 (init1, local2)"
+PREFILL_NAMES = {
+    1: "tiny_256_d64: 1 x 256 tokens, Hq4/Hkv1, d64, bs32, topk4 (block 0 + own block)",
+    2: "nsa_varlen_16k: lens [8192,4096,2048,2048], Hq16/Hkv4, d128, bs64, topk16 (init1, local2)",
+    3: "dense_window_1k_4k: B2, sq1024/sk4096, Hq32/Hkv8, d128, causal, window (1024,0), all 17 touched blocks",
+    4: "nsa_long_96k: lens [65536,32768], Hq4/Hkv4, d128, bs64, topk16 (init1, local2)",
+}
+PREFILL_CONFIGS = {1: W.config1, 2: W.config2, 3: W.config3, 4: W.config4}
 DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], page256, 2048 tok/(b,hk)"
 
 
@@ -44,12 +51,11 @@ DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], p
 # each stage, from one `ncu` capture of that kernel on its workload.  A figure holds only for the
 # kernel sources it was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
-    "fwd_attend_pipe_kernel": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
-                               "sha256": "10f0e66608a4e6f8d69d43cdd26fdced9e371c831cdb471584e4eeaa4551f42f",
-                               "bytes": 136768256},
+    "prefill_c4": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_fwd_inv_kernel.cu", "sfa_prep.cu", "sfa_device.cuh"],
+                   "sha256": None, "bytes": None},
+    "prefill_c2": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"], "sha256": None, "bytes": None},
     "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
-                            "sha256": "f66cc7e500f8e87bb265a44ebe4d5b524a6afb4afdfc89cc189a2957ae14d2ce",
-                            "bytes": 274462976},
+                            "sha256": None, "bytes": None},
 }
 
 
@@ -63,7 +69,9 @@ def source_digest(files):
 
 
 def kernel_traffic(kernel):
-    t = TRAFFIC[kernel]
+    t = TRAFFIC.get(kernel)
+    if not t or t["sha256"] is None:
+        return None
     return t["bytes"] if source_digest(t["files"]) == t["sha256"] else None
 
 
@@ -75,26 +83,46 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def prefill_flops(c):
-    """4*d flops per kept (query, key) pair per query head.  NSA workloads: closed form of the
-    recipe; others (the dense window workload): count from the canonical index sets on the host."""
-    if c.causal and c.wl < 0 and c.wr < 0 and np.array_equal(c.cu_q, c.cu_k):
-        pairs = W.kept_pairs_nsa(np.diff(c.cu_q).tolist(), c.bs, c.topk)
-        return 4.0 * c.d * c.Hq * pairs
-    pairs = 0
+def kept_per_token(c):
+    """Kept keys of every (query token, kv head), int64 (total_q, Hkv): the keys of every distinct
+    block id of the token's selection that is a block of its sequence, inside the causal / window
+    mask.  Counted on the host from the selection as given (duplicates, -1 and out-of-range ids
+    dropped)."""
+    out = np.zeros((c.total_q, c.Hkv), np.int64)
     for b in range(c.batch):
-        sq, sk = int(c.cu_q[b + 1] - c.cu_q[b]), int(c.cu_k[b + 1] - c.cu_k[b])
-        i = np.arange(sq)
-        hi = np.full(sq, sk - 1)
-        lo = np.zeros(sq, dtype=np.int64)
+        q0, q1 = int(c.cu_q[b]), int(c.cu_q[b + 1])
+        sq, sk = q1 - q0, int(c.cu_k[b + 1] - c.cu_k[b])
+        if sq == 0:
+            continue
+        nblk = (sk + c.bs - 1) // c.bs
+        i = np.arange(sq, dtype=np.int64)
+        lo = np.zeros(sq, np.int64)
+        hi = np.full(sq, sk - 1, np.int64)
         if c.causal:
             hi = np.minimum(hi, i + sk - sq)
         if c.wr >= 0:
             hi = np.minimum(hi, i + sk - sq + c.wr)
         if c.wl >= 0:
             lo = np.maximum(lo, i + sk - sq - c.wl)
-        pairs += int(np.clip(hi - lo + 1, 0, None).sum())  # every block selected (dense limit)
-    return 4.0 * c.d * c.Hq * pairs
+        s = np.sort(np.asarray(c.sel[q0:q1], np.int64), axis=2)
+        keep = (s >= 0) & (s < nblk)
+        keep[..., 1:] &= s[..., 1:] != s[..., :-1]
+        bl = s * c.bs
+        bh = np.minimum(bl + c.bs, sk) - 1
+        n = np.minimum(bh, hi[:, None, None]) - np.maximum(bl, lo[:, None, None]) + 1
+        out[q0:q1] = np.where(keep, np.clip(n, 0, None), 0).sum(axis=2)
+    return out
+
+
+def kept_pairs(c):
+    """Kept (query token, key) pairs summed over (token, kv head)."""
+    return int(kept_per_token(c).sum())
+
+
+def prefill_flops(c):
+    """4*d flops per kept (query, key) pair per query head; the G query heads of a kv head share its
+    selection, so each (token, kv head) pair count is taken G times."""
+    return 4.0 * c.d * (c.Hq // c.Hkv) * kept_pairs(c)
 
 
 def decode_bytes(c):
@@ -198,14 +226,12 @@ def cpu_oracle_rate(c, seconds, seed=0):
     import oracle
 
     rng = np.random.default_rng(seed)
-    seqlens = np.diff(c.cu_q)
-    pos = np.concatenate([np.arange(L) for L in seqlens])
-    b = pos // c.bs
-    kept = (np.minimum(c.topk, b + 1) - 1) * c.bs + pos % c.bs + 1  # kept keys per token
+    kept = kept_per_token(c)  # (total_q, Hkv)
+    G = c.Hq // c.Hkv
 
     def run(n):
         rows = np.sort(rng.choice(c.total_q * c.Hq, size=n, replace=False)).astype(np.int64)
-        flops = 4.0 * c.d * kept[rows // c.Hq].sum()
+        flops = 4.0 * c.d * kept[rows // c.Hq, (rows % c.Hq) // G].sum()
         t0 = time.perf_counter()
         oracle.fwd(c, rows=rows)
         return flops, time.perf_counter() - t0, n
@@ -236,7 +262,7 @@ def run_gpu(args, rank, world, local_rank):
     if args.part == "decode-small":
         pc = W.small_config(2)
     else:
-        pc = {1: W.config1, 2: W.config2, 3: W.config3, 4: W.config4}[args.prefill_config]()
+        pc = PREFILL_CONFIGS[args.prefill_config]()
     P = W.upload_prefill(pc, dev)
     flops = prefill_flops(pc)
     # Profiling aids: 'prefill' skips the 9.7 GB decode cache (a tiny decode case stands in);
@@ -252,54 +278,42 @@ def run_gpu(args, rank, world, local_rank):
 
     stream = torch.cuda.current_stream()
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    out = torch.empty_like(P["q"])
-    lse = torch.empty((pc.Hq, pc.total_q), dtype=torch.float32, device=dev)
     dout = torch.empty_like(D["q"])
     dlse = torch.empty((dc.B, dc.Hq), dtype=torch.float32, device=dev)
-    ws_bytes = sfa.fwd_workspace_size(pc.batch, pc.max_sq, pc.max_sk, pc.total_q, pc.Hq, pc.Hkv, pc.d, pc.topk, pc.bs)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     dws = torch.empty(sfa.decode_workspace_size(dc.B, dc.Hq, dc.Hkv, dc.d, dc.topk, 0), dtype=torch.uint8,
                       device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     launches = [0]
-    # When the call needs no block-major plan, sfa_fwd is one kernel that canonicalizes the
-    # selections itself; time that whole call.  Otherwise time the prep and attention stages.
-    sfa.fwd(P["q"], P["k"], P["v"], P["cu_q"], P["sel"], pc.bs, cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq,
-            max_seqlen_k=pc.max_sk, causal=bool(pc.causal), window=(pc.wl, pc.wr), out=out, lse=lse, workspace=ws,
-            status=status)
-    fused = sfa.last_launch_count() == 1
 
-    def prefill_prep():  # staged path only (the block-major schedule needs the prep kernel's plan)
-        if fused:
-            return
-        sfa.fwd_prep(P["cu_q"], P["sel"], Hq=pc.Hq, d=pc.d, block_size=pc.bs, cu_seqlens_k=P["cu_k"],
-                     max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, causal=bool(pc.causal), window=(pc.wl, pc.wr),
-                     workspace=ws, status=status)
-        launches[0] += sfa.last_launch_count()
+    def prefill_call(c, T):
+        """The public sfa_fwd call on one uploaded prefill case, with its own outputs and workspace."""
+        o = torch.empty_like(T["q"])
+        l = torch.empty((c.Hq, c.total_q), dtype=torch.float32, device=dev)
+        w = torch.empty(max(1, sfa.fwd_workspace_size(c.batch, c.max_sq, c.max_sk, c.total_q, c.Hq, c.Hkv, c.d,
+                                                      c.topk, c.bs)), dtype=torch.uint8, device=dev)
 
-    def prefill_attend():
-        if fused:  # the whole public call: one kernel canonicalizes the selections and attends
-            sfa.fwd(P["q"], P["k"], P["v"], P["cu_q"], P["sel"], pc.bs, cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq,
-                    max_seqlen_k=pc.max_sk, causal=bool(pc.causal), window=(pc.wl, pc.wr), out=out, lse=lse,
-                    workspace=ws, status=status)
+        def run():
+            sfa.fwd(T["q"], T["k"], T["v"], T["cu_q"], T["sel"], c.bs, cu_seqlens_k=T["cu_k"], max_seqlen_q=c.max_sq,
+                    max_seqlen_k=c.max_sk, causal=bool(c.causal), window=(c.wl, c.wr), out=o, lse=l, workspace=w,
+                    status=status)
             launches[0] += sfa.last_launch_count()
-            return
-        sfa.fwd_attend(P["q"], P["k"], P["v"], P["cu_q"], ws, topk=pc.topk, block_size=pc.bs,
-                       cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, causal=bool(pc.causal),
-                       window=(pc.wl, pc.wr), out=out, lse=lse, status=status)
-        launches[0] += sfa.last_launch_count()
+        run.out, run.lse, run.ws = o, l, w
+        return run
 
-    def decode_prep():  # selections this short are deduplicated inside the split kernel: no stage
-        pass
+    prefill = prefill_call(pc, P)
+    out, lse, ws = prefill.out, prefill.lse, prefill.ws
+    prefill()
+    prefill_launches = sfa.last_launch_count()
 
-    def decode_attend():
+    def decode_call():
         sfa.decode(D["q"], D["k_cache"], D["v_cache"], D["block_table"], D["cache_seqlens"], D["sel"], out=dout,
                    lse=dlse, workspace=dws, status=status)
         launches[0] += sfa.last_launch_count()
 
-    stages = [prefill_prep, prefill_attend, decode_prep, decode_attend]
+    # one step: the whole public prefill call on the headline workload, then the whole decode call
+    stages = [prefill, decode_call]
     if args.part == "prefill":
-        stages = [prefill_prep, prefill_attend, lambda: None, lambda: None]
+        stages = [prefill, lambda: None]
     K, Wm = args.steps, args.warmup
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
 
@@ -341,14 +355,12 @@ def run_gpu(args, rank, world, local_rank):
     stage_ms = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(len(stages))] for i in range(K)])
     region_ms = t_start.elapsed_time(t_end)
     mean = stage_ms.mean(axis=0)
-    region_ms, pp_ms, pa_ms, dp_ms, da_ms = max_over_ranks([region_ms, *mean.tolist()], world, dev)
-    prefill_ms = pp_ms + pa_ms
-    decode_ms = dp_ms + da_ms
+    region_ms, prefill_ms, decode_ms = max_over_ranks([region_ms, *mean.tolist()], world, dev)
     step_ms = prefill_ms + decode_ms
     value = job_rate(world, flops, prefill_ms) / 1e12
-    attend_tflops = job_rate(1, flops, pa_ms) / 1e12
+    attend_tflops = job_rate(1, flops, prefill_ms) / 1e12
     dec_gbs = job_rate(world, gbytes, decode_ms) / 1e9
-    dec_attend_gbs = job_rate(1, gbytes, da_ms) / 1e9
+    dec_attend_gbs = dec_gbs / world
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
 
@@ -357,24 +369,6 @@ def run_gpu(args, rank, world, local_rank):
     # prefill workload's tensors; L2 flushed before every repetition, CUDA events on the stream.
     extras = None
     if not args.no_extras and args.part != "decode-small":
-        wl = 512
-        seq = np.diff(pc.cu_q).tolist()
-        wpairs = sum(int(np.minimum(np.arange(L) + 1, wl + 1).sum()) for L in seq)
-        wflops = 4.0 * pc.d * pc.Hq * wpairs
-        wws = torch.empty(256, dtype=torch.uint8, device=dev)
-        wout = torch.empty_like(out)
-        wlse = torch.empty_like(lse)
-        gates = [torch.rand((pc.total_q, pc.Hq), dtype=torch.float32, device=dev) for _ in range(3)]
-        mix = torch.empty_like(out)
-
-        def run_window():
-            sfa.window_fwd(P["q"], P["k"], P["v"], P["cu_q"], cu_seqlens_k=P["cu_k"], max_seqlen_q=pc.max_sq,
-                           max_seqlen_k=pc.max_sk, causal=True, window=(wl, 0), out=wout, lse=wlse, workspace=wws,
-                           status=status)
-
-        def run_mix():
-            sfa.gated_combine([(out, gates[0]), (wout, gates[1]), (P["q"], gates[2])], out=mix)
-
         def timed(fn, reps=10):
             for _ in range(3):
                 fn()
@@ -389,25 +383,70 @@ def run_gpu(args, rank, world, local_rank):
                 ts.append(e0.elapsed_time(e1))
             return float(np.mean(ts))
 
+        # ---- the other prefill configurations, each its whole public call (parity cases beside the step)
+        cfg_lines = {}
+        for n in sorted(PREFILL_CONFIGS):
+            if n == args.prefill_config:
+                continue
+            xc = PREFILL_CONFIGS[n]()
+            xT = W.upload_prefill(xc, dev)
+            xrun = prefill_call(xc, xT)
+            xrun()
+            xl = sfa.last_launch_count()
+            xf = prefill_flops(xc)
+            x_ms = max_over_ranks([timed(xrun, reps=20)], world, dev)[0]
+            tfl = xf / (x_ms * 1e-3) / 1e12
+            cfg_lines[str(n)] = {"workload": PREFILL_NAMES[n], "ms": round(x_ms, 4),
+                                 "effective_gflop": round(xf / 1e9, 3), "effective_tflops": round(tfl, 2),
+                                 "frac": round(tfl / tf_burst, 4), "launches": xl,
+                                 "peak_source": f"{peak_kind} bf16 burst"}
+            del xT, xrun
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item())} in the prefill configuration runs")
+        # the NSA branches and the backward run on the varlen NSA workload (configuration 2)
+        bc = pc if args.prefill_config == 2 else W.config2()
+        BP = P if args.prefill_config == 2 else W.upload_prefill(bc, dev)
+        brun = prefill_call(bc, BP)
+        brun()
+        b_out, b_lse = brun.out, brun.lse
+        b_flops = prefill_flops(bc)
+        wl = 512
+        seq = np.diff(bc.cu_q).tolist()
+        wpairs = sum(int(np.minimum(np.arange(L) + 1, wl + 1).sum()) for L in seq)
+        wflops = 4.0 * bc.d * bc.Hq * wpairs
+        wws = torch.empty(256, dtype=torch.uint8, device=dev)
+        wout = torch.empty_like(b_out)
+        wlse = torch.empty_like(b_lse)
+        gates = [torch.rand((bc.total_q, bc.Hq), dtype=torch.float32, device=dev) for _ in range(3)]
+        mix = torch.empty_like(b_out)
+
+        def run_window():
+            sfa.window_fwd(BP["q"], BP["k"], BP["v"], BP["cu_q"], cu_seqlens_k=BP["cu_k"], max_seqlen_q=bc.max_sq,
+                           max_seqlen_k=bc.max_sk, causal=True, window=(wl, 0), out=wout, lse=wlse, workspace=wws,
+                           status=status)
+
+        def run_mix():
+            sfa.gated_combine([(b_out, gates[0]), (wout, gates[1]), (BP["q"], gates[2])], out=mix)
+
         # Backward of the selected attention on the same workload (d 128, bs 64): dq, dk, dv from the
         # forward's out / lse and a seeded dout; 2.5x the forward's effective flops (five products
         # of the kept pairs instead of two).
         bwd_line = None
-        if pc.d == 128 and pc.bs == 64:
-            g_out = torch.randn(out.shape, generator=torch.Generator(device=dev).manual_seed(5), device=dev,
+        if bc.d == 128 and bc.bs == 64:
+            g_out = torch.randn(b_out.shape, generator=torch.Generator(device=dev).manual_seed(5), device=dev,
                                 dtype=torch.float32).to(torch.bfloat16)
-            bdq, bdk, bdv = torch.empty_like(P["q"]), torch.empty_like(P["k"]), torch.empty_like(P["v"])
-            bws = torch.empty(sfa.bwd_workspace_size(pc.batch, pc.max_sq, pc.max_sk, pc.total_q, pc.Hq, pc.Hkv, pc.d,
-                                                     pc.topk, pc.bs), dtype=torch.uint8, device=dev)
+            bdq, bdk, bdv = torch.empty_like(BP["q"]), torch.empty_like(BP["k"]), torch.empty_like(BP["v"])
+            bws = torch.empty(sfa.bwd_workspace_size(bc.batch, bc.max_sq, bc.max_sk, bc.total_q, bc.Hq, bc.Hkv, bc.d,
+                                                     bc.topk, bc.bs), dtype=torch.uint8, device=dev)
 
             def run_bwd():
-                sfa.bwd(P["q"], P["k"], P["v"], out, g_out, lse, P["cu_q"], P["sel"], pc.bs, cu_seqlens_k=P["cu_k"],
-                        max_seqlen_q=pc.max_sq, max_seqlen_k=pc.max_sk, causal=bool(pc.causal),
-                        window=(pc.wl, pc.wr), dq=bdq, dk=bdk, dv=bdv, workspace=bws, status=status)
+                sfa.bwd(BP["q"], BP["k"], BP["v"], b_out, g_out, b_lse, BP["cu_q"], BP["sel"], bc.bs, cu_seqlens_k=BP["cu_k"],
+                        max_seqlen_q=bc.max_sq, max_seqlen_k=bc.max_sk, causal=bool(bc.causal),
+                        window=(bc.wl, bc.wr), dq=bdq, dk=bdk, dv=bdv, workspace=bws, status=status)
 
             b_ms = max_over_ranks([timed(run_bwd)], world, dev)[0]
-            bflops = 2.5 * flops
-            bwd_line = {"workload": "the prefill workload, seeded dout; dq, dk, dv", "ms": round(b_ms, 4),
+            bflops = 2.5 * b_flops
+            bwd_line = {"workload": PREFILL_NAMES[2] + "; seeded dout; dq, dk, dv", "ms": round(b_ms, 4),
                         "effective_tflops": round(bflops / (b_ms * 1e-3) / 1e12, 2),
                         "frac": round(bflops / (b_ms * 1e-3) / 1e12 / tf_burst, 4),
                         "peak_source": f"{peak_kind} bf16 burst", "launches": 7,
@@ -450,7 +489,7 @@ def run_gpu(args, rank, world, local_rank):
             index_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
         m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
-        mix_bytes = 4 * pc.total_q * pc.Hq * pc.d * 2 + 3 * pc.total_q * pc.Hq * 4
+        mix_bytes = 4 * bc.total_q * bc.Hq * bc.d * 2 + 3 * bc.total_q * bc.Hq * 4
         extras = {
             "window_branch": {"workload": "the prefill workload's q/k/v, causal, window (512, 0), no selection",
                               "ms": round(w_ms, 4), "effective_tflops": round(wflops / (w_ms * 1e-3) / 1e12, 2),
@@ -461,7 +500,7 @@ def run_gpu(args, rank, world, local_rank):
                               "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
         }
         extras = {"nsa_branches": extras, "backward": bwd_line, "kv_append": append_line,
-                  "index_topk": index_line}
+                  "index_topk": index_line, "prefill_configs": cfg_lines}
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
 
@@ -570,13 +609,13 @@ def run_gpu(args, rank, world, local_rank):
                        "copies of neighbouring steps overlapping the compute on separate streams (two device "
                        "buffer sets); the decode KV cache is resident state, its per-step inputs are q, "
                        "block_table, cache_seqlens, sel_tok_idx"}
-    return dict(value=value, fused=fused, prefill_ms=prefill_ms, prep_ms=pp_ms, attend_ms=pa_ms, decode_ms=decode_ms,
-                dprep_ms=dp_ms, dattend_ms=da_ms, step_ms=step_ms, region_ms=region_ms, attend_tflops=attend_tflops,
+    return dict(value=value, prefill_launches=prefill_launches, prefill_ms=prefill_ms, decode_ms=decode_ms,
+                step_ms=step_ms, region_ms=region_ms, attend_tflops=attend_tflops,
                 dec_gbs=dec_gbs, dec_attend_gbs=dec_attend_gbs, flops=flops, gbytes=gbytes, clocks=clocks,
                 launches=n_launch, e2e=e2e, extras=extras, hbm=hbm, tf_burst=tf_burst, tf_sust=tf_sust,
                 peak_kind=peak_kind,
                 pc=pc, dc=dc,
-                traffic=args.traffic if args.traffic is not None else kernel_traffic("fwd_attend_pipe_kernel"),
+                traffic=args.traffic if args.traffic is not None else kernel_traffic(f"prefill_c{args.prefill_config}"),
                 dec_traffic=kernel_traffic("decode_split_kernel"))
 
 
@@ -594,8 +633,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode-small"],
                     help="'prefill' times only the prefill stages (a small decode case stands in); for profiling")
-    ap.add_argument("--prefill-config", type=int, default=2, choices=[1, 2, 3, 4],
-                    help="prefill workload (default 2, the varlen NSA one the metric is quoted on)")
+    ap.add_argument("--prefill-config", type=int, default=4, choices=[1, 2, 3, 4],
+                    help="headline prefill workload (default 4, the largest single-GPU configuration); the "
+                         "others are timed beside it")
     ap.add_argument("--traffic", type=int, default=None,
                     help="dram bytes (read+write) per attend launch from an ncu capture of this kernel version")
     args = ap.parse_args()
@@ -637,26 +677,25 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q/k/v, seeded NSA block selection; seeded paged decode inputs)",
-        "config": {"workload": PREFILL_NAME, "decode_workload": DECODE_NAME, "parallelism": f"independent x{world}",
+        "config": {"workload": PREFILL_NAMES[args.prefill_config] if args.part != "decode-small" else "small",
+                   "decode_workload": DECODE_NAME, "parallelism": f"independent x{world}",
                    "l2": "flushed by a 256 MiB write before every step (outside the kernel events)",
                    "timing": "CUDA events per stage on the launch stream, mean over steps, max over ranks"},
-        "prefill": {"ms": round(r["prefill_ms"], 4), "prep_ms": round(r["prep_ms"], 4),
-                    "attend_ms": round(r["attend_ms"], 4), "effective_gflop": round(r["flops"] / 1e9, 2)},
+        "prefill": {"ms": round(r["prefill_ms"], 4), "effective_gflop": round(r["flops"] / 1e9, 2),
+                    "launches": r["prefill_launches"]},
         "decode": {"value": round(r["dec_gbs"], 1), "unit": "GB/s", "ms": round(r["decode_ms"], 4),
-                   "prep_ms": round(r["dprep_ms"], 4), "attend_ms": round(r["dattend_ms"], 4),
                    "gathered_bytes": int(r["gbytes"]),
                    "roofline": {"bound": "hbm", "achieved": round(r["dec_attend_gbs"], 1), "peak": r["hbm"],
                                 "unit": "GB/s", "frac": round(r["dec_attend_gbs"] / r["hbm"], 4),
                                 "traffic": r["dec_traffic"], "traffic_unit": "B per decode_split_kernel launch",
-                                "kernel": "decode_split_kernel (sfa_decode: one launch, splits merged in the CTA)",
+                                "kernel": "sfa_decode whole call = one decode_split_kernel launch (splits merged "
+                                          "in the CTA)",
                                 "peak_source": r["peak_kind"]}},
         "roofline": {"bound": "tensor", "achieved": round(r["attend_tflops"], 2), "peak": r["tf_burst"],
                      "unit": "TFLOP/s", "frac": round(r["attend_tflops"] / r["tf_burst"], 4),
-                     "traffic": r["traffic"], "traffic_unit": "B per fwd_attend_pipe_kernel launch",
-                     "kernel": ("fwd_attend_pipe_kernel (the whole sfa_fwd call: one launch canonicalizes the "
-                                "selections and attends)") if r["fused"] else
-                               ("fwd_attend_pipe_kernel (the sfa_fwd_attend stage, which launches only this kernel "
-                                "on this workload)"),
+                     "traffic": r["traffic"], "traffic_unit": "B (dram read + write) per sfa_fwd call",
+                     "kernel": f"sfa_fwd whole call ({r['prefill_launches']} kernel launches; achieved = the "
+                               f"call's effective flops / the call's duration)",
                      "peak_source": f"{r['peak_kind']} bf16 burst",
                      "frac_of_sustained": round(r["attend_tflops"] / r["tf_sust"], 4) if r["tf_sust"] else None},
         "gpu_launches": r["launches"],
@@ -683,7 +722,7 @@ def main_reference(args, rank, world):
     """The CPU oracle, as it stands, on a bounded sample of the prefill workload per step."""
     if rank != 0:
         return
-    pc = W.config2()
+    pc = PREFILL_CONFIGS[args.prefill_config]()
     import oracle
     oracle.build()
     steps, warm = args.steps, args.warmup
@@ -700,7 +739,8 @@ def main_reference(args, rank, world):
     line = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": steps,
             "warmup": warm, "ms_per_step": round(1e3 * total_t / steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": PREFILL_NAME}, "impl": "reference",
+            "config": {"workload": PREFILL_NAMES[args.prefill_config], "decode_workload": DECODE_NAME},
+            "impl": "reference",
             "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                              "sample": f"{rows_tot} random (token, head) rows over {steps} steps"},
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

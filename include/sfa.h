@@ -77,7 +77,7 @@ enum {
 /* Supported in this build: bf16 inputs; d in {64, 128}; prefill block_size in {32, 64},
  * 1 <= topk <= 128, G = Hq/Hkv <= 128, ceil(max_seqlen_k / block_size) <= 65536;
  * decode G <= 16, page_size >= 1, 1 <= topk_tok <= 65536, max_pages_per_seq*page_size
- * <= 2^20; backward d = 128 and block_size = 64; KV append d a multiple of 8; index top-k
+ * <= 2^20; backward the forward's d and block_size; KV append d a multiple of 8; index top-k
  * max_pages_per_seq*page_size <= 2^20.  Anything else returns SFA_ERR_UNSUPPORTED. */
 
 /* ----------------------------------------------------------------------------------------
@@ -158,7 +158,8 @@ size_t sfa_bwd_workspace_size(int batch, int max_seqlen_q, int max_seqlen_k, int
  *   dout  bf16 (total_q, Hq, d), the gradient of the loss with respect to out
  * Outputs (written in full; the caller owns them): dq bf16 (total_q, Hq, d), dk and dv bf16
  * (total_k, Hkv, d).  A key no row keeps gets dk = dv = 0; a row that keeps no key gets dq = 0.
- * This build: d = 128, block_size = 64 (else SFA_ERR_UNSUPPORTED).  Deterministic: the sums run
+ * Sizes as sfa_fwd (d in {64, 128}, block_size in {32, 64}), and a tile's block union must fit the
+ * dQ kernel's shared memory (else SFA_ERR_UNSUPPORTED).  Deterministic: the sums run
  * in a fixed order whatever the timing.  Seven kernels and one memset on `stream`; status bits as
  * sfa_fwd (SFA_DEV_BAD_SEQLEN also when a token of a sequence is past max_seqlen_q). */
 int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const void *dout,

@@ -335,7 +335,6 @@ int bwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
 {
     int rc = fwd_geometry(batch, max_sq, max_sk, total_q, Hq, Hkv, d, topk, bs, g.f);
     if (rc != SFA_OK) return rc;
-    if (d != 128 || bs != 64) return SFA_ERR_UNSUPPORTED;
     g.f.inv = 0;  // the backward walks the query tiles; no block-major forward schedule
     const int64_t total_sel = (int64_t)total_q * Hkv * topk;
     if ((int64_t)total_q * Hq >= (1ll << 31) || total_sel >= (1ll << 31)) return SFA_ERR_UNSUPPORTED;
@@ -632,7 +631,7 @@ int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const 
         return SFA_ERR_INVALID_ARG;
     if (total_k == 0) return SFA_ERR_UNSUPPORTED;
     // The dQ kernel keeps two copies of a tile's block union in shared memory beside its rings.
-    if (bwd_dq_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
+    if (bwd_dq_smem_bytes(g) > 227 * 1024 || bwd_dkdv_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
     uint8_t *w = static_cast<uint8_t *>(workspace);
     if (cudaMemsetAsync(w + g.off_zero, 0, g.zero_bytes, st) != cudaSuccess) return SFA_ERR_CUDA;

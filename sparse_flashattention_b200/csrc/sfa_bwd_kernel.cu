@@ -60,7 +60,8 @@ struct DqCfg {
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
     static constexpr uint32_t kIdescDQ = idesc_bf16_f32(128, D, true);
     static_assert(kColDQ + D <= kTmemCols, "TMEM columns");
-    static_assert(BS == 64, "two softmax warps per row, 32 keys each");
+    static_assert(BS == 32 || BS == 64, "two softmax warps per row, BS / 2 keys each");
+    static_assert(D == 64 || D == 128, "head dimension");
 };
 
 struct DqTile {
@@ -398,11 +399,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t tS = lane_base + (jg & 1) * BS, tDP = lane_base + C::kColDP + (jg & 1) * BS;
+                constexpr int KH = BS / 2;  // keys of this warp's half of the block
                 if (!__any_sync(full, selected)) {  // dS = 0 for all 32 rows: dQ unchanged
-                    uint32_t zero[16];
+                    uint32_t zero[KH / 2];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) zero[e] = 0u;
-                    tmem_st16(tS + hs * 16, zero);
+                    for (int e = 0; e < KH / 2; ++e) zero[e] = 0u;
+                    tmem_st_cols<KH / 2>(tS + hs * (KH / 2), zero);
                     tmem_wait_st();
                     tc_fence_before();
                     mbar_arrive(&meta->p_full[jg & 1]);
@@ -412,14 +414,14 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 // select the block gets exponent -inf, a key outside the row's window too; 2^-inf = 0.
                 const int kb = s * BS;
                 const float sl = selected ? p.scale_log2 : 0.f, bias = selected ? -lse2 : -INFINITY;
-                {  // this warp's 32 keys; dS of keys [32 hs, 32 hs + 32) -> columns [16 hs, 16 hs + 16)
-                    uint32_t sr[32], dr[32], packed[16];
-                    tmem_ld32(tS + hs * 32, sr);
-                    tmem_ld32(tDP + hs * 32, dr);
+                {  // this warp's KH keys; dS of keys [KH hs, KH hs + KH) -> columns [KH/2 hs, KH/2 hs + KH/2)
+                    uint32_t sr[KH], dr[KH], packed[KH / 2];
+                    tmem_ld_cols<KH>(tS + hs * KH, sr);
+                    tmem_ld_cols<KH>(tDP + hs * KH, dr);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c0 = kb + hs * 32 + 2 * e;
+                    for (int e = 0; e < KH / 2; ++e) {
+                        const int c0 = kb + hs * KH + 2 * e;
                         float y0 = fmaf(__uint_as_float(sr[2 * e]), sl, bias);
                         float y1 = fmaf(__uint_as_float(sr[2 * e + 1]), sl, bias);
                         y0 = ((c0 >= lo) & (c0 <= hi)) ? y0 : -INFINITY;
@@ -428,7 +430,7 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                         packed[e] = pack_bf16x2(p0 * (__uint_as_float(dr[2 * e]) - dlt),
                                                 p1 * (__uint_as_float(dr[2 * e + 1]) - dlt));
                     }
-                    tmem_st16(tS + hs * 16, packed);
+                    tmem_st_cols<KH / 2>(tS + hs * (KH / 2), packed);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -496,13 +498,19 @@ constexpr int kKvThreads = 352;
 constexpr int kKvGatherWarp2 = 10;
 constexpr int kGatherLanes = 64;  // warps 0 and 10: each copies 64 of a chunk's 128 rows
 
+// The transposed products dV^T += dO^T P and dK^T += Q^T dS take d as the MMA's M dimension (128
+// rows of TMEM).  With d = 64 the A descriptor's second 64-row half reads the first one again: the
+// products run at M = 128 and TMEM lanes 64..127 hold a copy that the epilogue ignores.  Their N
+// dimension (keys) is 64: a block of 32 keys keeps 64-key rows in its P and dS tiles, keys 32..63
+// written as zero, so the same 128-byte-swizzled layout serves both block sizes.
 template <int D, int BS>
 struct KvCfg {
-    static_assert(D == 128, "the transposed products take d as the MMA's M dimension (128)");
-    static_assert(BS == 64, "two softmax warps per row, 32 keys each");
+    static_assert(D == 64 || D == 128, "head dimension");
+    static_assert(BS == 32 || BS == 64, "two softmax warps per row, BS / 2 keys each");
+    static constexpr int kNT = 64;                  // N of the transposed products
     static constexpr int kTileBytes = 128 * D * 2;  // 128 gathered rows of Q (or dO)
     static constexpr int kKVBytes = BS * D * 2;
-    static constexpr int kPBytes = 128 * BS * 2;    // P (or dS): 128 rows x BS keys, bf16
+    static constexpr int kPBytes = 128 * kNT * 2;   // P (or dS): 128 rows x 64 keys, bf16
     static constexpr int kOffQ = 0;                 // [2] stages
     static constexpr int kOffDO = 2 * kTileBytes;   // [2]
     static constexpr int kOffK = 4 * kTileBytes;
@@ -513,9 +521,11 @@ struct KvCfg {
     static constexpr int kTmemCols = 512;
     static constexpr int kColDP = 2 * BS;
     static constexpr int kColDV = 4 * BS;
-    static constexpr int kColDK = 5 * BS;
+    static constexpr int kColDK = kColDV + kNT;
+    static constexpr uint32_t kALbo = D == 128 ? 128 * 128 : 0;  // M-halves of the transposed A operand
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
-    static constexpr uint32_t kIdescT = idesc_bf16_f32_ab(128, BS, true, true);
+    static constexpr uint32_t kIdescT = idesc_bf16_f32_ab(128, kNT, true, true);
+    static_assert(kColDK + kNT <= kTmemCols, "TMEM columns");
 };
 
 struct PieceInfo {
@@ -693,8 +703,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             for (int b = 0; b < 2; ++b) {
                 dQ[b] = sdesc_sw128(smem_u32(sQ + b * C::kTileBytes), 16, 1024);
                 dDO[b] = sdesc_sw128(smem_u32(sDO + b * C::kTileBytes), 16, 1024);
-                dQt[b] = sdesc_sw128(smem_u32(sQ + b * C::kTileBytes), 128 * 128, 1024);   // M = d, MN-major
-                dDOt[b] = sdesc_sw128(smem_u32(sDO + b * C::kTileBytes), 128 * 128, 1024);
+                dQt[b] = sdesc_sw128(smem_u32(sQ + b * C::kTileBytes), C::kALbo, 1024);   // M = d, MN-major
+                dDOt[b] = sdesc_sw128(smem_u32(sDO + b * C::kTileBytes), C::kALbo, 1024);
                 dP[b] = sdesc_sw128(smem_u32(sP + b * C::kPBytes), C::kPBytes, 1024);     // N = keys, MN-major
                 dDS[b] = sdesc_sw128(smem_u32(sDS + b * C::kPBytes), C::kPBytes, 1024);
             }
@@ -833,14 +843,15 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 const uint32_t tS = lane_base + b * BS, tDP = lane_base + C::kColDP + b * BS;
                 uint8_t *prow = sP + b * C::kPBytes + r * 128;
                 uint8_t *dsrow = sDS + b * C::kPBytes + r * 128;
+                constexpr int KH = BS / 2;  // keys of this warp's half of the block
                 {
-                    uint32_t sr[32], dr[32], pk[16], dk[16];
-                    tmem_ld32(tS + hs * 32, sr);
-                    tmem_ld32(tDP + hs * 32, dr);
+                    uint32_t sr[KH], dr[KH], pk[KH / 2], dk[KH / 2];
+                    tmem_ld_cols<KH>(tS + hs * KH, sr);
+                    tmem_ld_cols<KH>(tDP + hs * KH, dr);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {  // branch-free masking: exponent -inf outside the row's keys
-                        const int c0 = kb + hs * 32 + 2 * e;
+                    for (int e = 0; e < KH / 2; ++e) {  // branch-free masking: exponent -inf outside the row's keys
+                        const int c0 = kb + hs * KH + 2 * e;
                         float y0 = fmaf(__uint_as_float(sr[2 * e]), p.scale_log2, -lse2);
                         float y1 = fmaf(__uint_as_float(sr[2 * e + 1]), p.scale_log2, -lse2);
                         y0 = ((c0 >= lo) & (c0 <= hi)) ? y0 : -INFINITY;
@@ -851,10 +862,18 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     }
                     // 16-byte pieces (8 keys) of the row, 128-byte swizzle: piece x at (x ^ (row & 7)) * 16.
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const int piece = hs * 4 + x, so = ((piece ^ (r & 7)) << 4);
+                    for (int x = 0; x < KH / 8; ++x) {
+                        const int piece = hs * (KH / 8) + x, so = ((piece ^ (r & 7)) << 4);
                         *reinterpret_cast<uint4 *>(prow + so) = make_uint4(pk[4 * x], pk[4 * x + 1], pk[4 * x + 2], pk[4 * x + 3]);
                         *reinterpret_cast<uint4 *>(dsrow + so) = make_uint4(dk[4 * x], dk[4 * x + 1], dk[4 * x + 2], dk[4 * x + 3]);
+                    }
+                    if constexpr (BS < C::kNT) {  // keys BS..63 of the 64-key row are zero
+#pragma unroll
+                        for (int x = 0; x < (C::kNT - BS) / 16; ++x) {
+                            const int piece = BS / 8 + hs * ((C::kNT - BS) / 16) + x, so = ((piece ^ (r & 7)) << 4);
+                            *reinterpret_cast<uint4 *>(prow + so) = make_uint4(0u, 0u, 0u, 0u);
+                            *reinterpret_cast<uint4 *>(dsrow + so) = make_uint4(0u, 0u, 0u, 0u);
+                        }
                     }
                 }
                 fence_proxy_async_smem();
@@ -869,10 +888,11 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             tc_fence_after();
             constexpr int HK = BS / 2;
             float dv[HK], dkk[HK];
+            const bool dvalid = r < D;  // with d = 64, lanes 64..127 hold the ignored copy
             {
-                uint32_t a[32], bq[32];
-                tmem_ld32(lane_base + C::kColDV + hs * HK, a);
-                tmem_ld32(lane_base + C::kColDK + hs * HK, bq);
+                uint32_t a[HK], bq[HK];
+                tmem_ld_cols<HK>(lane_base + C::kColDV + hs * HK, a);
+                tmem_ld_cols<HK>(lane_base + C::kColDK + hs * HK, bq);
                 tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < HK; ++e) {
@@ -890,11 +910,12 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 // the row's partials in piece order (this one's included, read back) and writes dK / dV.
                 constexpr size_t kSlot = (size_t)2 * BS * D;
                 float *mine = p.part + (size_t)(pi.slot + pi.idx) * kSlot;
+                if (dvalid)
 #pragma unroll
-                for (int e = 0; e < HK; ++e) {
-                    mine[(e0 + e) * D + r] = dv[e];
-                    mine[BS * D + (e0 + e) * D + r] = dkk[e];
-                }
+                    for (int e = 0; e < HK; ++e) {
+                        mine[(e0 + e) * D + r] = dv[e];
+                        mine[BS * D + (e0 + e) * D + r] = dkk[e];
+                    }
                 __threadfence();
                 ok = group_sync(&meta->epi_bar, epi_uses, abort_flag, p.status);
                 if (!ok) break;
@@ -902,7 +923,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                 ok = group_sync(&meta->epi_bar, epi_uses, abort_flag, p.status);
                 if (!ok) break;
                 last = meta->last_flag != 0;
-                if (last) {
+                if (last && dvalid) {
                     __threadfence();
 #pragma unroll
                     for (int e = 0; e < HK; ++e) dv[e] = dkk[e] = 0.f;
@@ -916,7 +937,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     }
                 }
             }
-            if (last) {
+            if (last && dvalid) {
                 __nv_bfloat16 *dvo = p.dv + ((int64_t)(pi.k0 + kb + e0) * p.Hkv + pi.hk) * D + r;
                 __nv_bfloat16 *dko = p.dk + ((int64_t)(pi.k0 + kb + e0) * p.Hkv + pi.hk) * D + r;
                 const int64_t stride = (int64_t)p.Hkv * D;
@@ -949,38 +970,68 @@ int sm_count()
     return n > 0 ? n : 148;
 }
 
+
+template <int D, int BS>
+size_t dq_smem_t(const BwdGeom &g)
+{
+    return 1024 + dq_union_offset<D, BS>() + (size_t)2 * g.f.umax * 4;
+}
+
+template <int D, int BS>
+size_t dkdv_smem_t()
+{
+    return 1024 + KvCfg<D, BS>::kOffMeta + sizeof(KvMeta);
+}
+
+template <int D, int BS>
+cudaError_t launch_dq_t(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tdo,
+                        const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
+{
+    const size_t smem = dq_smem_t<D, BS>(g);
+    cudaError_t e = ensure_smem_for(bwd_dq_kernel<D, BS>, smem);
+    if (e != cudaSuccess) return e;
+    const int grid = std::max(1, std::min(p.tiles, sm_count()));
+    bwd_dq_kernel<D, BS><<<grid, kDqThreads, smem, st>>>(tq, tdo, tk, tv, p);
+    return cudaGetLastError();
+}
+
+template <int D, int BS>
+cudaError_t launch_dkdv_t(const BwdParams &p, const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
+{
+    const size_t smem = dkdv_smem_t<D, BS>();
+    cudaError_t e = ensure_smem_for(bwd_dkdv_kernel<D, BS>, smem);
+    if (e != cudaSuccess) return e;
+    bwd_dkdv_kernel<D, BS><<<sm_count(), kKvThreads, smem, st>>>(tk, tv, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t bwd_dq_smem_bytes(const BwdGeom &g)
 {
-    return 1024 + dq_union_offset<128, 64>() + (size_t)2 * g.f.umax * 4;
+    if (g.f.d == 64) return g.f.bs == 32 ? dq_smem_t<64, 32>(g) : dq_smem_t<64, 64>(g);
+    return g.f.bs == 32 ? dq_smem_t<128, 32>(g) : dq_smem_t<128, 64>(g);
 }
 
-size_t bwd_dkdv_smem_bytes()
+size_t bwd_dkdv_smem_bytes(const BwdGeom &g)
 {
-    return 1024 + KvCfg<128, 64>::kOffMeta + sizeof(KvMeta);
+    if (g.f.d == 64) return g.f.bs == 32 ? dkdv_smem_t<64, 32>() : dkdv_smem_t<64, 64>();
+    return g.f.bs == 32 ? dkdv_smem_t<128, 32>() : dkdv_smem_t<128, 64>();
 }
 
 cudaError_t launch_bwd_dq(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tq, const CUtensorMap &tdo,
                           const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t st)
 {
-    const size_t smem = bwd_dq_smem_bytes(g);
-    cudaError_t e = ensure_smem_for(bwd_dq_kernel<128, 64>, smem);
-    if (e != cudaSuccess) return e;
-    const int grid = std::max(1, std::min(p.tiles, sm_count()));
-    bwd_dq_kernel<128, 64><<<grid, kDqThreads, smem, st>>>(tq, tdo, tk, tv, p);
-    return cudaGetLastError();
+    if (g.f.d == 64)
+        return g.f.bs == 32 ? launch_dq_t<64, 32>(g, p, tq, tdo, tk, tv, st) : launch_dq_t<64, 64>(g, p, tq, tdo, tk, tv, st);
+    return g.f.bs == 32 ? launch_dq_t<128, 32>(g, p, tq, tdo, tk, tv, st) : launch_dq_t<128, 64>(g, p, tq, tdo, tk, tv, st);
 }
 
 cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
                             cudaStream_t st)
 {
-    (void)g;
-    const size_t smem = bwd_dkdv_smem_bytes();
-    cudaError_t e = ensure_smem_for(bwd_dkdv_kernel<128, 64>, smem);
-    if (e != cudaSuccess) return e;
-    bwd_dkdv_kernel<128, 64><<<sm_count(), kKvThreads, smem, st>>>(tk, tv, p);
-    return cudaGetLastError();
+    if (g.f.d == 64) return g.f.bs == 32 ? launch_dkdv_t<64, 32>(p, tk, tv, st) : launch_dkdv_t<64, 64>(p, tk, tv, st);
+    return g.f.bs == 32 ? launch_dkdv_t<128, 32>(p, tk, tv, st) : launch_dkdv_t<128, 64>(p, tk, tv, st);
 }
 
 }  // namespace sfa

@@ -38,6 +38,8 @@ struct InvCfg {
     static constexpr int kOffK = kLoadStages * kQBytes;            // K[kLoadStages]
     static constexpr int kOffV = kOffK + kLoadStages * kKVBytes;   // V[kLoadStages]
     static constexpr int kOffMeta = kOffV + kLoadStages * kKVBytes;
+    static constexpr int kOffStage = kOffMeta + 4608;  // 8 softmax warps x 2 KB epilogue staging
+    static constexpr int kStageBytes = 8 * 2048;
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
     static constexpr int kTmemCols = 512;  // S/P of group w at w*BS, O of group w at 128 + w*D
@@ -54,6 +56,42 @@ struct InvMeta {
     int abort_flag;
     InvItem slot[kItemSlots];
 };
+
+// Rows [r0, r0 + 64) of an item's Q tile (row r = token * G + head; rows >= `rows` zero-filled) into
+// the 128-byte-swizzled K-major tile at qt: chunk k of a row's 64-element half c lands at
+// c * 16 KB + r * 128 + ((k ^ (r & 7)) << 4).  Lane l first finds the source rows r0 + l and
+// r0 + 32 + l (one division and one shared-memory read each); then the lanes take consecutive
+// 16-byte chunks of 32 / (D / 8) consecutive rows, each row's address broadcast from the lane that
+// found it, so every copy instruction reads whole rows from global memory (coalesced) and fills
+// whole 128-byte shared-memory lines.
+template <int D>
+__device__ __forceinline__ void gather_q_rows(const FwdAttendParams &p, const InvItem *item, int hk, int rows, int r0,
+                                              uint32_t qt, int lane)
+{
+    constexpr int kChunks = D / 8;               // 16-byte chunks per row
+    constexpr int kRowsPerIter = 32 / kChunks;   // rows one warp instruction covers
+    const __nv_bfloat16 *src_row[2];
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+        const int r = r0 + 32 * h2 + lane;
+        const bool live = r < rows;
+        const int tk = live ? r / p.G : 0, gg = live ? r - tk * p.G : 0;
+        src_row[h2] = p.q + ((int64_t)(live ? (item->tok[tk] >> 7) : 0) * p.Hq + hk * p.G + gg) * D;
+    }
+    const int cc = lane % kChunks, c = cc >> 3, k = cc & 7;
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+        for (int i = 0; i < 32 / kRowsPerIter; ++i) {
+            const int rl = i * kRowsPerIter + lane / kChunks;  // row within this half of 32
+            const int r = r0 + 32 * h2 + rl;
+            const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(
+                __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(src_row[h2]), rl));
+            cp_async16(qt + c * (128 * 128) + r * 128 + ((k ^ (r & 7)) << 4), src + c * 64 + k * 8,
+                       r < rows ? 16u : 0u);
+        }
+    }
+}
 
 template <int D, int BS>
 __global__ void __launch_bounds__(kInvThreadsAttn, 1)
@@ -151,29 +189,14 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 issued[sl]++;
             }
             // Q rows 0..63 of the item's tokens (row r = token * G + head) into the 128-byte-swizzled
-            // K-major tile the MMA reads: 16-byte cp.async copies, lane l taking rows l and l+32 (rows
-            // past the item are zero-filled; warp 10 copies rows 64..127).  Each lane's copies land on
-            // q_full through its own arrival.
+            // K-major tile the MMA reads (rows past the item are zero-filled; warp 10 copies rows
+            // 64..127).  16-byte cp.async copies with the lanes spread along the rows, so one warp
+            // instruction moves whole rows (coalesced).  Each lane's copies land on q_full through its
+            // own arrival.
             if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
-            {
-                const int rows = rec.w * p.G;
-                const uint32_t qt = smem_u32(sQ + sl * C::kQBytes);
-#pragma unroll 1
-                for (int r = lane; r < 64; r += 32) {
-                    const bool live = r < rows;
-                    const int tk = live ? r / p.G : 0, gg = live ? r - tk * p.G : 0;
-                    const __nv_bfloat16 *src =
-                        p.q + ((int64_t)(live ? (item->tok[tk] >> 7) : 0) * p.Hq + hk * p.G + gg) * D;
-#pragma unroll
-                    for (int c = 0; c < D / 64; ++c)
-#pragma unroll
-                        for (int k = 0; k < 8; ++k)
-                            cp_async16(qt + c * (128 * 128) + r * 128 + ((k ^ (r & 7)) << 4), src + c * 64 + k * 8,
-                                       live ? 16u : 0u);
-                }
-                cp_async_mbar_arrive(&meta->q_full[sl]);
-            }
+            gather_q_rows<D>(p, item, hk, rec.w * p.G, 0, smem_u32(sQ + sl * C::kQBytes), lane);
+            cp_async_mbar_arrive(&meta->q_full[sl]);
             // Item j+4 goes into the slot item j-4 used, once its softmax group is done with it.
             if (j + kFetchAhead >= kItemSlots)
                 ok = warp_all_ok(mbar_wait(&meta->item_free[(j + kFetchAhead) % kItemSlots],
@@ -277,20 +300,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             const int hk = rec.x % p.Hkv;
             if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
-            const int rows = rec.w * p.G;
-            const uint32_t qt = smem_u32(sQ + sl * C::kQBytes);
-#pragma unroll 1
-            for (int r = 64 + lane; r < 128; r += 32) {
-                const bool live = r < rows;
-                const int tk = live ? r / p.G : 0, gg = live ? r - tk * p.G : 0;
-                const __nv_bfloat16 *src = p.q + ((int64_t)(live ? (item->tok[tk] >> 7) : 0) * p.Hq + hk * p.G + gg) * D;
-#pragma unroll
-                for (int c = 0; c < D / 64; ++c)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        cp_async16(qt + c * (128 * 128) + r * 128 + ((k ^ (r & 7)) << 4), src + c * 64 + k * 8,
-                                   live ? 16u : 0u);
-            }
+            gather_q_rows<D>(p, item, hk, rec.w * p.G, 64, smem_u32(sQ + sl * C::kQBytes), lane);
             cp_async_mbar_arrive(&meta->q_full[sl]);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies have all landed
@@ -302,6 +312,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         const uint32_t tS = lane_base + grp * BS;
         const uint32_t tO = lane_base + 128 + grp * D;
+        uint4 *stg = reinterpret_cast<uint4 *>(smem + C::kOffStage) + (warp - 2) * 128;  // 32 rows x 64 bytes
         bool ok = true;
         for (int j = grp; ok; j += 2) {
             const uint32_t ph = (j >> 1) & 1;
@@ -368,19 +379,37 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             const int h = hk * p.G + gg;
             const int64_t pslot = (t * p.Hq + h) * p.topk + kslot;
             const float inv = l > 0.f ? 1.f / l : 0.f;
+            // The warp's 32 rows go out 32 columns (64 bytes of bf16) at a time through its staging
+            // buffer: each lane writes its row's four 16-byte segments, then lane l stores segment
+            // l % 4 of row 8i + l / 4, so one store instruction writes whole 64-byte row pieces.
+            // Segment j of row r sits at (j + r / 2) % 4, which keeps both sides bank-conflict free.
+            int64_t ps_i[4];
+            bool vr_i[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int rr = 8 * i + (lane >> 2);
+                ps_i[i] = __shfl_sync(0xffffffffu, (long long)pslot, rr);
+                vr_i[i] = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
+            }
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];
                 tmem_ld32(tO + c * 32, o);
                 tmem_wait_ld();
-                if (valid) {
-                    uint32_t wv[16];
+                uint32_t wv[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.po + pslot * D + c * 32);
+                for (int e = 0; e < 16; ++e)
+                    wv[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+                __syncwarp();  // the previous chunk's segments have been read out
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+                for (int e = 0; e < 4; ++e)
+                    stg[lane * 4 + ((e + (lane >> 1)) & 3)] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int rr = 8 * i + (lane >> 2), seg = lane & 3;
+                    const uint4 v = stg[rr * 4 + ((seg + (rr >> 1)) & 3)];
+                    if (vr_i[i]) reinterpret_cast<uint4 *>(p.po + ps_i[i] * D + c * 32)[seg] = v;
                 }
             }
             tc_fence_before();
@@ -402,78 +431,104 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
 // Merge of the block-major partials, one warp per (token, kv head) whose tile went block-major:
 // for each of the G heads, M = max m_k, L = sum l_k 2^(m_k - M), out = sum (l_k 2^(m_k - M) / L) o_k,
 // lse = (M + log2 L) ln 2.  Lanes cover the head dimension in 16-byte chunks and split the
-// partials between them, so every lane keeps several independent loads in flight.
+// partials between them; each lane loads a batch of its partials at once (independent loads in
+// flight), folds them into a running max / sum / weighted chunk, and the lanes sharing a chunk
+// combine at the end.  The partials are read once, with streaming loads (they are not reused).
 constexpr int kMergeWarps = 8;
+constexpr int kMergeBatch = 8;  // partials each lane loads before folding them in
 
 template <int D>
 __global__ void __launch_bounds__(32 * kMergeWarps) fwd_merge_kernel(const FwdAttendParams p)
 {
     constexpr int kChunks = D / 8;       // 16-byte chunks of a row
     constexpr int kSplit = 32 / kChunks; // lanes sharing a chunk, each over every kSplit-th partial
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     grid_dep_wait();
-    const int64_t u = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
-    if (u >= (int64_t)p.total_q * p.Hkv) return;
+    // One CTA per query tile (the tile numbering of the other prefill kernels); only the tiles the
+    // plan sent block-major (ucnt = -1) have partials to merge.
+    const int tile = blockIdx.x;
     if (__ldcg(&p.ctrl->item_total) == 0) return;  // every row was written by the query-major kernel
-    const int cnt = p.cnt[u];
-    if (cnt == 0) return;  // written by the query-major kernel
-    const int64_t t = u / p.Hkv;
-    const int hk = (int)(u - t * p.Hkv);
-    int lo = 0, hi = p.batch - 1;
-    while (lo < hi) {  // batch entry of token t
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.cu_q[mid] <= t) lo = mid;
-        else hi = mid - 1;
-    }
-    const int b = lo;
-    const int qt = (int)(t - p.cu_q[b]) / p.Tq;
-    if (p.ucnt[((p.nqt - 1 - qt) * p.batch + b) * p.Hkv + hk] >= 0) return;  // query-major tile
-
+    if (__ldcg(&p.ucnt[tile]) != -1) return;
+    const int hk = tile % p.Hkv;
+    const int rest = tile / p.Hkv;
+    const int b = rest % p.batch;
+    const int qt = p.nqt - 1 - rest / p.batch;
+    const int q0 = p.cu_q[b], sq = p.cu_q[b + 1] - q0;
+    const int tok0 = qt * p.Tq;
+    const int ntok = min(p.Tq, sq - tok0);
+    if (ntok <= 0) return;
+    const int nrows = ntok * p.G;
+    // the selection counts of this warp's rows (row e = warp + kMergeWarps * i, i = lane), read at once
+    const int e_l = warp + kMergeWarps * lane;
+    const int cnt_l = e_l < nrows ? __ldg(&p.cnt[((int64_t)q0 + tok0 + e_l / p.G) * p.Hkv + hk]) : 0;
     const int c = lane % kChunks, kq = lane / kChunks;
-    for (int g = 0; g < p.G; ++g) {
+    for (int i = 0; warp + kMergeWarps * i < nrows; ++i) {
+        const int e = warp + kMergeWarps * i;
+        const int cnt = __shfl_sync(0xffffffffu, cnt_l, i);
+        if (cnt == 0) continue;  // a row that keeps no key: written by the query-major kernel
+        const int tt = e / p.G, g = e - tt * p.G;
+        const int64_t t = (int64_t)q0 + tok0 + tt;
         const int h = hk * p.G + g;
         const int64_t base = (t * p.Hq + h) * p.topk;
-        float M = -INFINITY;
-        for (int k = lane; k < cnt; k += 32) {
-            const float2 ml = __ldcg(&p.pml[base + k]);
-            if (ml.y > 0.f) M = fmaxf(M, ml.x);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-        float L = 0.f;
-        for (int k = lane; k < cnt; k += 32) {
-            const float2 ml = __ldcg(&p.pml[base + k]);
-            if (ml.y > 0.f) L += ml.y * ex2(ml.x - M);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-        const float invL = L > 0.f ? 1.f / L : 0.f;
-        float acc[8];
+        // Lane (kq, c) merges partials kq, kq + kSplit, ... of chunk c: a batch of their (m, l) and
+        // 16-byte chunks is loaded at once, then folded into a running (max, sum, weighted chunk).
+        float Mx = -INFINITY, Ls = 0.f, acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-#pragma unroll 4
-        for (int k = kq; k < cnt; k += kSplit) {
-            const float2 ml = __ldcg(&p.pml[base + k]);
-            const uint4 v = __ldcg(reinterpret_cast<const uint4 *>(p.po + (base + k) * D) + c);
-            const float w = ml.y > 0.f ? ml.y * ex2(ml.x - M) * invL : 0.f;
-            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+        for (int k0 = kq; k0 < cnt; k0 += kSplit * kMergeBatch) {
+            float2 ml[kMergeBatch];
+            uint4 v[kMergeBatch];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vv[e]));
-                acc[2 * e] += w * f.x;
-                acc[2 * e + 1] += w * f.y;
+            for (int i = 0; i < kMergeBatch; ++i) {
+                const int k = k0 + i * kSplit;
+                ml[i] = k < cnt ? __ldcs(&p.pml[base + k]) : make_float2(-INFINITY, 0.f);
+                v[i] = k < cnt ? __ldcs(reinterpret_cast<const uint4 *>(p.po + (base + k) * D) + c)
+                               : make_uint4(0u, 0u, 0u, 0u);
+            }
+            float bm = Mx;
+#pragma unroll
+            for (int i = 0; i < kMergeBatch; ++i)
+                if (ml[i].y > 0.f) bm = fmaxf(bm, ml[i].x);
+            if (bm == -INFINITY) continue;
+            const float f = Mx == -INFINITY ? 0.f : ex2(Mx - bm);
+            Ls *= f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] *= f;
+            Mx = bm;
+#pragma unroll
+            for (int i = 0; i < kMergeBatch; ++i) {
+                const float w = ml[i].y > 0.f ? ml[i].y * ex2(ml[i].x - bm) : 0.f;
+                Ls += w;
+                const uint32_t vv[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vv[e]));
+                    acc[2 * e] = fmaf(w, x.x, acc[2 * e]);
+                    acc[2 * e + 1] = fmaf(w, x.y, acc[2 * e + 1]);
+                }
             }
         }
+        // combine the kSplit lanes of each chunk (lanes c, c + kChunks, ...)
+        float M = Mx;
 #pragma unroll
-        for (int o = kChunks; o < 32; o <<= 1)
+        for (int o = kChunks; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float f = Mx == -INFINITY ? 0.f : ex2(Mx - M);
+        float L = Ls * f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] *= f;
+#pragma unroll
+        for (int o = kChunks; o < 32; o <<= 1) {
+            L += __shfl_xor_sync(0xffffffffu, L, o);
 #pragma unroll
             for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+        }
+        const float invL = L > 0.f ? 1.f / L : 0.f;
         if (kq == 0) {
             uint4 w4;
-            w4.x = pack_bf16x2(acc[0], acc[1]);
-            w4.y = pack_bf16x2(acc[2], acc[3]);
-            w4.z = pack_bf16x2(acc[4], acc[5]);
-            w4.w = pack_bf16x2(acc[6], acc[7]);
+            w4.x = pack_bf16x2(acc[0] * invL, acc[1] * invL);
+            w4.y = pack_bf16x2(acc[2] * invL, acc[3] * invL);
+            w4.z = pack_bf16x2(acc[4] * invL, acc[5] * invL);
+            w4.w = pack_bf16x2(acc[6] * invL, acc[7] * invL);
             reinterpret_cast<uint4 *>(p.out + (t * p.Hq + h) * D)[c] = w4;
         }
         if (lane == 0) p.lse[(int64_t)h * p.total_q + t] = L > 0.f ? (M + log2f(L)) * kLn2i : -INFINITY;
@@ -483,7 +538,8 @@ __global__ void __launch_bounds__(32 * kMergeWarps) fwd_merge_kernel(const FwdAt
 template <int D, int BS>
 size_t inv_smem_bytes()
 {
-    return 1024 + InvCfg<D, BS>::kOffMeta + sizeof(InvMeta);
+    static_assert(sizeof(InvMeta) <= 4608, "InvMeta must fit below the staging buffers");
+    return 1024 + InvCfg<D, BS>::kOffStage + InvCfg<D, BS>::kStageBytes;
 }
 
 template <int D, int BS>
@@ -511,8 +567,7 @@ size_t fwd_attend_inv_smem_bytes(const FwdGeom &g)
 
 cudaError_t launch_fwd_merge(const FwdGeom &g, const FwdAttendParams &p, cudaStream_t st)
 {
-    const int64_t units = (int64_t)g.total_q * g.Hkv;
-    const unsigned grid = (unsigned)((units + kMergeWarps - 1) / kMergeWarps);
+    const unsigned grid = (unsigned)g.tiles;
     if (g.d == 64) return launch_kernel(fwd_merge_kernel<64>, dim3(grid), dim3(32 * kMergeWarps), 0, st, true, p);
     return launch_kernel(fwd_merge_kernel<128>, dim3(grid), dim3(32 * kMergeWarps), 0, st, true, p);
 }

@@ -4,7 +4,7 @@
 // attention; one O(L) pass over the keys).
 //
 // One CTA of 1024 threads per (sequence, kv head):
-//   1. the group's G query rows rounded to FP8 E4M3 and summed per dimension (exact in fp64);
+//   1. the group's G query rows rounded to FP8 E4M3 and summed per dimension (exact in fp32);
 //   2. every cache position's key row (through the block table) rounded to E4M3 and dotted with that
 //      sum in fp64, D/8 lanes per row, 8 elements each.  Every product and partial sum is exact (the
 //      format's values have 4 significant bits and span 2^-9 .. 448), so the score does not depend on
@@ -27,6 +27,7 @@ namespace {
 
 constexpr int kIdxThreads = 1024;
 constexpr int kIdxBins = 4096;  // 12-bit digits
+constexpr int kIdxBtMax = 4096; // block-table entries of a sequence kept in shared memory
 
 // x rounded to FP8 E4M3 (round to nearest even, saturated at +-448) and back to float.  Both halves of
 // the pair carry x, so the result does not depend on which half a conversion fills.
@@ -37,6 +38,17 @@ __device__ __forceinline__ float e4m3_round_trip(float x)
     uint32_t r;
     asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
     return __half2float(__ushort_as_half((unsigned short)(r & 0xffffu)));
+}
+
+// Two values at once: (lo, hi) rounded to E4M3 as above, returned as floats (one conversion each way
+// for the pair; the E4M3 values are exact in f16 and in f32).
+__device__ __forceinline__ float2 e4m3_round_trip2(float lo, float hi)
+{
+    uint16_t h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+    uint32_t r;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(h));
+    return __half22float2(*reinterpret_cast<const __half2 *>(&r));
 }
 
 // Order-preserving key of a finite score (larger score, larger key); -0 and +0 tie.  Keys of finite
@@ -81,6 +93,7 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_topk_kernel(IndexParams 
 {
     __shared__ double qs[D];
     __shared__ unsigned int hist[kIdxBins];
+    __shared__ int bt_s[kIdxBtMax];
     __shared__ int scratch[32];
     __shared__ int s_digit, s_above;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -96,46 +109,71 @@ __global__ void __launch_bounds__(kIdxThreads, 1) index_topk_kernel(IndexParams 
     unsigned long long *keys = p.keys + (int64_t)blockIdx.x * p.max_len;
     int32_t *out = p.sel + (int64_t)blockIdx.x * p.topk;
 
-    // 1. the group's summed E4M3 query
+    // 1. the group's summed E4M3 query (exact in fp64), and the sequence's block-table row when it
+    // fits in shared memory
     for (int c = tid; c < D; c += kIdxThreads) {
         double a = 0.0;
         for (int g = 0; g < p.G; ++g)
             a += (double)e4m3_round_trip(__bfloat162float(p.q[((int64_t)b * p.Hq + hk * p.G + g) * D + c]));
         qs[c] = a;
     }
+    const int32_t *bt_g = p.bt + (int64_t)b * p.max_pages;
+    const bool bt_smem = p.max_pages <= kIdxBtMax;
+    if (bt_smem)
+        for (int i = tid; i < p.max_pages; i += kIdxThreads) bt_s[i] = __ldg(&bt_g[i]);
     for (int i = tid; i < kIdxBins; i += kIdxThreads) hist[i] = 0u;
     __syncthreads();
 
-    // 2. scores -> keys, and the histogram of their top digit
+    // 2. scores -> keys, and the histogram of their top digit.  A lane group of D/8 lanes scores a row;
+    // each group takes kRowsPerGroup rows at a time, their loads issued before any arithmetic.
+    // score = sum over the row of e4m3(k) * qsum in fp64: every product and partial sum is exact (see
+    // above), so the order of the sum does not matter.
     constexpr int kLanesPerRow = D / 8;
     constexpr int kRowsPerWarp = 32 / kLanesPerRow;
+    constexpr int kRowsPerGroup = 4;
+    constexpr int64_t kStep = (int64_t)(kIdxThreads / 32) * kRowsPerWarp * kRowsPerGroup;
     const int sub = lane / kLanesPerRow, part = lane % kLanesPerRow;
     double qv[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) qv[e] = qs[part * 8 + e];
-    for (int64_t j0 = (int64_t)warp * kRowsPerWarp; j0 < L; j0 += (int64_t)(kIdxThreads / 32) * kRowsPerWarp) {
-        const int64_t j = j0 + sub;
-        const bool in = j < L;
-        const int pg = in ? __ldg(&p.bt[(int64_t)b * p.max_pages + j / p.page]) : -1;
-        const bool okp = in && pg >= 0 && pg < p.num_pages;
-        double acc = 0.0;
-        if (okp) {
-            const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(
-                p.kc + (((int64_t)pg * p.page + j % p.page) * p.Hkv + hk) * D + part * 8));
-            const __nv_bfloat16 *v = reinterpret_cast<const __nv_bfloat16 *>(&raw);
+    bool bad_page = false;
+    for (int64_t j0 = (int64_t)warp * kRowsPerWarp * kRowsPerGroup; j0 < L; j0 += kStep) {
+        uint4 raw[kRowsPerGroup];
+        bool okp[kRowsPerGroup];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc = fma((double)e4m3_round_trip(__bfloat162float(v[e])), qv[e], acc);
+        for (int u = 0; u < kRowsPerGroup; ++u) {
+            const int64_t j = j0 + u * kRowsPerWarp + sub;
+            const bool in = j < L;
+            const int pi = in ? (int)(j / p.page) : 0;
+            const int pg = in ? (bt_smem ? bt_s[pi] : __ldg(&bt_g[pi])) : -1;
+            okp[u] = in && pg >= 0 && pg < p.num_pages;
+            raw[u] = okp[u] ? __ldg(reinterpret_cast<const uint4 *>(
+                                  p.kc + (((int64_t)pg * p.page + (j - (int64_t)pi * p.page)) * p.Hkv + hk) * D + part * 8))
+                            : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
-        for (int o = kLanesPerRow / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (part == 0 && in) {
-            const unsigned long long key = (okp && j < Lc) ? order_key(acc) : 0ull;
-            keys[j] = key;
-            if (key) atomicAdd(&hist[key >> 52], 1u);
-            if (!okp && p.status) atomicOr(p.status, SFA_DEV_BAD_PAGE);
+        for (int u = 0; u < kRowsPerGroup; ++u) {
+            const int64_t j = j0 + u * kRowsPerWarp + sub;
+            const __nv_bfloat162 *v = reinterpret_cast<const __nv_bfloat162 *>(&raw[u]);
+            double acc = 0.0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = __bfloat1622float2(v[e]);
+                const float2 k8 = e4m3_round_trip2(x.x, x.y);
+                acc = fma((double)k8.x, qv[2 * e], acc);
+                acc = fma((double)k8.y, qv[2 * e + 1], acc);
+            }
+#pragma unroll
+            for (int o = kLanesPerRow / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+            if (part == 0 && j < L) {
+                const unsigned long long key = (okp[u] && j < Lc) ? order_key(acc) : 0ull;
+                keys[j] = key;
+                if (key) atomicAdd(&hist[key >> 52], 1u);
+                bad_page |= !okp[u];
+            }
         }
     }
-    __syncthreads();
+    if (__syncthreads_or(bad_page) && tid == 0 && p.status) atomicOr(p.status, SFA_DEV_BAD_PAGE);
 
     // 3. the k-th largest key T; `remaining` = how many keys equal to T the result takes
     int cand = 0;

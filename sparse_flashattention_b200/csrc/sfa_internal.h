@@ -170,7 +170,7 @@ cudaError_t launch_bwd_dq(const BwdGeom &g, const BwdParams &p, const CUtensorMa
 cudaError_t launch_bwd_dkdv(const BwdGeom &g, const BwdParams &p, const CUtensorMap &tk, const CUtensorMap &tv,
                             cudaStream_t st);
 size_t bwd_dq_smem_bytes(const BwdGeom &g);
-size_t bwd_dkdv_smem_bytes();
+size_t bwd_dkdv_smem_bytes(const BwdGeom &g);
 
 // ---------------------------------------------------------------------------------------
 // Decode

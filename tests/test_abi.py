@@ -121,13 +121,14 @@ def test_bwd_host_validation(lib):
     lib.sfa_bwd_workspace_size.argtypes = [I] * 9
     base = lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 128, 4, 64)
     assert base > 0
-    assert lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 64, 4, 64) == 0    # d 64
-    assert lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 128, 4, 32) == 0   # block 32
+    assert lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 64, 4, 64) > 0     # d 64
+    assert lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 128, 4, 32) > 0    # block 32
+    assert lib.sfa_bwd_workspace_size(1, 128, 128, 128, 4, 1, 96, 4, 64) == 0    # d 96: unsupported
     assert lib.sfa_bwd_workspace_size(1, 0, 0, 0, 4, 1, 128, 4, 64) == 0         # no query
     assert lib.sfa_bwd_workspace_size(1, 4096, 4096, 4096, 4, 1, 128, 4, 64) > \
         lib.sfa_bwd_workspace_size(1, 1024, 4096, 1024, 4, 1, 128, 4, 64) > base
-    assert _bwd(lib, d=64) == 2                   # SFA_ERR_UNSUPPORTED
-    assert _bwd(lib, bs=32) == 2
+    assert _bwd(lib, d=96) == 2                   # SFA_ERR_UNSUPPORTED
+    assert _bwd(lib, bs=48) == 2
     assert _bwd(lib, Hq=6, Hkv=4) == 1            # SFA_ERR_INVALID_ARG
     assert _bwd(lib, dout=None) == 1
     assert _bwd(lib, dk=None) == 1

@@ -62,6 +62,14 @@ BWD_CASES = {
     "window_g1": lambda: W.make_window_prefill(23, 2, 150, 260, 2, 2, 128, 64, 100, 20, causal=0),
     # causal window, sq < sk (bottom-right), G 2.
     "window_g2": lambda: W.make_window_prefill(24, 1, 200, 640, 4, 2, 128, 64, 256, 0, causal=1),
+    # the tiny configuration's shape: d 64, block 32, G 4, top-4 with block 0 and the own block forced
+    "tiny_d64_bs32": lambda: W.config1(),
+    # d 128, block 32: 35 chunks of 32 tokens select block 0 (a row of three pieces)
+    "nsa_d128_bs32": lambda: W.make_nsa_prefill(41, [1100, 130], 8, 2, 128, 32, 8, 1, 2),
+    # d 64, block 64, G 1 (128 tokens per chunk)
+    "nsa_d64_bs64_g1": lambda: W.make_nsa_prefill(42, [900, 77], 4, 4, 64, 64, 6, 1, 2),
+    # d 64, block 32, G 3, causal window with sq < sk
+    "window_d64_bs32_g3": lambda: W.make_window_prefill(43, 1, 300, 500, 6, 2, 64, 32, 100, 0, causal=1),
 }
 
 
@@ -131,10 +139,13 @@ def test_bwd_no_queries_zero_key_grads(sfa):
 
 
 def test_bwd_unsupported_shapes_rejected(sfa):
-    """d = 64 or block_size = 32 are outside the backward of this build: an error, no launch."""
-    q = torch.zeros((8, 2, 64), dtype=torch.bfloat16, device="cuda")
+    """A head dimension outside {64, 128} or a block size outside {32, 64}: an error, no launch."""
     cu = torch.tensor([0, 8], dtype=torch.int32, device="cuda")
     sel = torch.zeros((8, 2, 1), dtype=torch.int32, device="cuda")
     lse = torch.zeros((2, 8), dtype=torch.float32, device="cuda")
+    q = torch.zeros((8, 2, 96), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(sfa.SfaError):
         sfa.bwd(q, q, q, q, q, lse, cu, sel, 64)
+    q = torch.zeros((8, 2, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(sfa.SfaError):
+        sfa.bwd(q, q, q, q, q, lse, cu, sel, 16)
