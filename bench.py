@@ -487,6 +487,27 @@ def run_gpu(args, rank, world, local_rank):
                           "launches": 1, "status": int(istatus.item())}
         except Exception as exc:  # noqa: BLE001 - reported in the line, the rest of the bench goes on
             index_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        # FP8 E4M3 caches (the decode workload quantized per (sequence, kv head) on the device): the same
+        # gathered rows at one byte per value.
+        try:
+            fk, fv, fkd, fvd = W.quantize_cache_e4m3_device(dc, D)
+            f_out = torch.empty_like(dout)
+            f_lse = torch.empty_like(dlse)
+
+            def run_fp8():
+                sfa.decode_fp8(D["q"], fk, fv, D["block_table"], D["cache_seqlens"], D["sel"], k_descale=fkd,
+                               v_descale=fvd, out=f_out, lse=f_lse, workspace=dws, status=status)
+
+            f_ms = max_over_ranks([timed(run_fp8, reps=20)], world, dev)[0]
+            f_bytes = gbytes // 2
+            fp8_line = {"workload": DECODE_NAME + ", caches E4M3 + per (sequence, kv head) descales",
+                        "ms": round(f_ms, 4), "gathered_bytes": int(f_bytes),
+                        "gbs": round(f_bytes / (f_ms * 1e-3) / 1e9, 1),
+                        "frac": round(f_bytes / (f_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind,
+                        "speedup_vs_bf16_cache": round(decode_ms / f_ms, 3), "launches": 1}
+            del fk, fv
+        except Exception as exc:  # noqa: BLE001 - reported in the line, the rest of the bench goes on
+            fp8_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
         m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
         mix_bytes = 4 * bc.total_q * bc.Hq * bc.d * 2 + 3 * bc.total_q * bc.Hq * 4
@@ -500,7 +521,7 @@ def run_gpu(args, rank, world, local_rank):
                               "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
         }
         extras = {"nsa_branches": extras, "backward": bwd_line, "kv_append": append_line,
-                  "index_topk": index_line, "prefill_configs": cfg_lines}
+                  "index_topk": index_line, "prefill_configs": cfg_lines, "decode_fp8": fp8_line}
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
 

@@ -224,6 +224,21 @@ int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache,
                       void *workspace, size_t workspace_bytes, int32_t *status_dev,
                       void *out, float *lse, sfa_stream_t stream);
 
+/* Paged top-k decode over FP8 caches: k_cache and v_cache hold FP8 E4M3 codes (1 byte per value,
+ * (num_pages, page_size, Hkv, d), 16-byte aligned) and the cached value of sequence b, kv head h is
+ * code * k_descale[b * Hkv + h] (keys) or code * v_descale[b * Hkv + h] (values): the descale
+ * convention of the FlashAttention-3 docstrings (flash-attention-npu page, k_descale / v_descale of
+ * shape (batch, kv heads)); FP8 caches are in the Flash-Sparse-Attention README feature list ("Fused
+ * Quant").  k_descale / v_descale: fp32 device arrays (B, Hkv), or NULL for 1.  Every other argument,
+ * the workspace (sfa_decode_workspace_size), the semantics, the launches and the status bits are
+ * sfa_decode's; q, out and lse stay bf16 / fp32.  The E4M3 values are exact in bf16, so the kernel
+ * computes with the cached values themselves: half the bytes per gathered row. */
+int sfa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const float *k_descale,
+                   const float *v_descale, const int32_t *block_table, int max_pages_per_seq, int num_pages,
+                   int page_size, const int32_t *cache_seqlens, const int32_t *sel_tok_idx, int topk_tok, int B,
+                   int Hq, int Hkv, int d, int window_left, float scale, int num_splits, void *workspace,
+                   size_t workspace_bytes, int32_t *status_dev, void *out, float *lse, sfa_stream_t stream);
+
 /* Paged top-k decode for callers that cannot allocate device memory.  The pages have no
  * counterpart to this call: it exists for callers such as serving engines whose device memory
  * pool is fixed before serving and forbids later allocation, or plugin hooks that receive only

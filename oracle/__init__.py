@@ -263,3 +263,59 @@ def index_topk(q, k_cache, block_table, cache_seqlens, Hkv, topk, n_local=0):
             sel[b, hk, :chosen.size] = chosen
         scores.append(sb)
     return sel, scores, bad
+
+
+def e4m3_decode(codes):
+    """Values of FP8 E4M3 codes (uint8) as float64, from the format's definition: sign bit 7,
+    exponent field E = bits 6..3 (bias 7), mantissa field M = bits 2..0; E = 0 gives M * 2^-9
+    (subnormals), otherwise (1 + M / 8) * 2^(E - 7); E = 15 with M = 7 is not a number."""
+    c = np.asarray(codes, np.uint8).astype(np.int64)
+    s = np.where((c >> 7) & 1, -1.0, 1.0)
+    E = (c >> 3) & 15
+    M = c & 7
+    mag = np.where(E == 0, M * 2.0 ** -9, (1.0 + M / 8.0) * np.exp2(E - 7.0))
+    return np.where((E == 15) & (M == 7), np.nan, s * mag)
+
+
+def decode_fp8(case, sel=None):
+    """Paged top-k decode over FP8 caches, in float64: the attention of decode() with every cached
+    value equal to e4m3_decode(code) * descale of its (sequence, kv head) (the k_descale / v_descale
+    arguments of the FlashAttention-3 docstrings, per batch entry and kv head).  The key set per
+    (sequence, kv head) is decode()'s: distinct positions p of the selection with 0 <= p < L (and
+    p >= L - 1 - window_left when a window is given) whose page id is inside the cache.
+    Returns (out (B, Hq, d), lse (B, Hq), bad = [bad token ids, bad pages])."""
+    sel = np.asarray(case.sel if sel is None else sel)
+    q = (np.asarray(case.q, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    kc, vc = case.k_cache, case.v_cache  # codes; only the gathered rows are decoded
+    B, Hq, d = q.shape
+    Hkv, page, num_pages = case.Hkv, case.page, kc.shape[0]
+    G = Hq // Hkv
+    scale = case.scale if case.scale > 0 else 1.0 / np.sqrt(d)
+    out = np.zeros((B, Hq, d))
+    lse = np.full((B, Hq), -np.inf)
+    bad = np.zeros(2, np.int64)
+    for b in range(B):
+        L = int(case.cache_seqlens[b])
+        for hk in range(Hkv):
+            ids = sel[b, hk]
+            bad[0] += int(((ids != -1) & ((ids < 0) | (ids >= L))).sum())
+            pos = np.unique(ids[(ids >= 0) & (ids < L)])
+            if case.wl >= 0:
+                pos = pos[pos >= L - 1 - case.wl]
+            pg = case.block_table[b, pos // page]
+            okp = (pg >= 0) & (pg < num_pages)
+            bad[1] += int((~okp).sum())
+            pos, pg = pos[okp], pg[okp]
+            if pos.size == 0:
+                continue
+            K = e4m3_decode(kc[pg, pos % page, hk]) * float(case.k_descale[b, hk])
+            V = e4m3_decode(vc[pg, pos % page, hk]) * float(case.v_descale[b, hk])
+            for g in range(G):
+                h = hk * G + g
+                s = scale * (K @ q[b, h])
+                m = s.max()
+                w = np.exp(s - m)
+                Z = w.sum()
+                out[b, h] = (w @ V) / Z
+                lse[b, h] = m + np.log(Z)
+    return out, lse, bad

@@ -44,6 +44,27 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
+def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round finite float32 values to FP8 E4M3 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+    bits; largest finite 448, no infinities): round to nearest, ties to even, magnitudes past 448
+    saturated to 448; return uint8 codes.  Input preparation for FP8 caches."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    sign = np.signbit(x).astype(np.uint8)
+    a = np.minimum(np.abs(x), 448.0)
+    e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)                 # below 2^-6 the spacing stays 2^-9 (subnormals)
+    q = np.exp2(e - 3.0)
+    r = np.round(a / q)                     # multiples of the spacing, halves to even
+    # r is in [0, 16]; 16 means the next binade (exponent e + 1, mantissa 0)
+    up = r >= 16
+    e = np.where(up, e + 1, e)
+    r = np.where(up, 8.0, r)
+    normal = r >= 8                         # 1.mmm x 2^e
+    E = np.where(normal, e + 7, 0).astype(np.int64)
+    M = np.where(normal, r - 8, r).astype(np.int64)  # subnormal: r = mmm (value r * 2^-9)
+    return ((sign.astype(np.int64) << 7) | (E << 3) | M).astype(np.uint8)
+
+
 def _normal_bf16(rng: np.random.Generator, shape) -> np.ndarray:
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
@@ -196,6 +217,10 @@ class DecodeCase:
     page: int
     wl: int = -1
     scale: float = 0.0
+    # FP8 caches: k_cache / v_cache hold E4M3 codes (uint8) and a cached value is code * descale of its
+    # (sequence, kv head); None for bf16 caches.
+    k_descale: Optional[np.ndarray] = None   # float32 (B, Hkv)
+    v_descale: Optional[np.ndarray] = None
 
     @property
     def B(self):
@@ -300,6 +325,28 @@ def make_decode(seed: int, B, Hq, Hkv, d, page, len_lo, len_hi, topk_tok, n_last
 # The five named workloads and their oracle-sized variants.
 # ---------------------------------------------------------------------------------------------
 
+def make_decode_fp8(seed: int, B, Hq, Hkv, d, page, len_lo, len_hi, topk_tok, n_last, name="decode_fp8",
+                    parallel_values=False, max_len=None) -> DecodeCase:
+    """The paged decode inputs of make_decode with the caches stored as FP8 E4M3: per (sequence, kv
+    head) a descale = max |value| of the sequence's cached rows / 448 (float32), and every cached
+    value of that sequence stored as e4m3(value / descale)."""
+    c = make_decode(seed, B, Hq, Hkv, d, page, len_lo, len_hi, topk_tok, n_last, name=name,
+                    parallel_values=parallel_values, max_len=max_len)
+    kq = np.zeros(c.k_cache.shape, np.uint8)
+    vq = np.zeros(c.v_cache.shape, np.uint8)
+    kd = np.ones((B, Hkv), np.float32)
+    vd = np.ones((B, Hkv), np.float32)
+    for b in range(B):
+        pages = c.block_table[b][c.block_table[b] >= 0]
+        for h in range(Hkv):
+            for src, dst, ds in ((c.k_cache, kq, kd), (c.v_cache, vq, vd)):
+                vals = bf16_bits_to_f32(src[pages, :, h, :])
+                amax = float(np.abs(vals).max()) if vals.size else 0.0
+                ds[b, h] = np.float32(amax / 448.0) if amax > 0 else np.float32(1.0)
+                dst[pages, :, h, :] = f32_to_e4m3_bits(vals / ds[b, h])
+    return dataclasses.replace(c, k_cache=kq, v_cache=vq, k_descale=kd, v_descale=vd)
+
+
 def config1():
     """Tiny selected attention: 1 x 256 tokens, Hq4/Hkv1, d64, bs32, topk4 (block 0 + own block forced)."""
     return make_nsa_prefill(1, [256], 4, 1, 64, 32, 4, init_blocks=1, local_blocks=1, name="tiny_256_d64")
@@ -379,3 +426,26 @@ def upload_decode(c, device="cuda"):
                 v_cache=dev_tensor(c.v_cache, torch.bfloat16, device),
                 block_table=dev_tensor(c.block_table, None, device),
                 cache_seqlens=dev_tensor(c.cache_seqlens, None, device), sel=dev_tensor(c.sel, None, device))
+
+
+def quantize_cache_e4m3_device(c, d):
+    """FP8 E4M3 codes (uint8) and descales (B, Hkv) of an uploaded bf16 paged cache, made on the device
+    with torch for workloads too large to quantize on the host: per (sequence, kv head) descale =
+    max |value| / 448, codes = round-to-nearest-even E4M3 of value / descale (make_decode_fp8's recipe).
+    Returns (k_codes, v_codes, k_descale, v_descale) device tensors."""
+    import torch
+    kq = torch.empty(d["k_cache"].shape, dtype=torch.uint8, device=d["k_cache"].device)
+    vq = torch.empty_like(kq)
+    kd = torch.ones((c.B, c.Hkv), dtype=torch.float32, device=kq.device)
+    vd = torch.ones_like(kd)
+    bt = c.block_table
+    for b in range(c.B):
+        pages = torch.as_tensor(bt[b][bt[b] >= 0], device=kq.device, dtype=torch.long)
+        for src, dst, ds in ((d["k_cache"], kq, kd), (d["v_cache"], vq, vd)):
+            vals = src.index_select(0, pages).float()           # (pages, page, Hkv, d)
+            amax = vals.abs().amax(dim=(0, 1, 3))                # (Hkv,)
+            sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+            ds[b] = sc
+            codes = (vals / sc.view(1, 1, -1, 1)).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+            dst.index_copy_(0, pages, codes)
+    return kq, vq, kd, vd

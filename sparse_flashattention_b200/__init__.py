@@ -21,7 +21,7 @@ import torch
 
 __all__ = ["SfaError", "lib_path", "fwd", "fwd_prep", "fwd_attend", "fwd_workspace_size", "window_fwd",
            "gated_combine", "decode", "decode_prep",
-           "decode_attend", "decode_noalloc", "decode_workspace_size", "decode_num_splits", "last_launch_count",
+           "decode_attend", "decode_noalloc", "decode_fp8", "decode_workspace_size", "decode_num_splits", "last_launch_count",
            "DEV_BAD_INDEX", "DEV_BAD_PAGE", "DEV_TIMEOUT"]
 
 DEV_BAD_INDEX, DEV_BAD_PAGE, DEV_TIMEOUT = 1, 2, 4
@@ -57,6 +57,7 @@ def _load():
         "sfa_decode_prep": (I, [P, P, I, I, I, I, I, I, I, I, I, P, Z, P, P]),
         "sfa_decode_attend": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]),
         "sfa_decode_noalloc": (I, [P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, F, I, P, P, P, P]),
+        "sfa_decode_fp8": (I, [P, P, P, P, P, P, I, I, I, P, P, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]),
         "sfa_window_fwd_workspace_size": (Z, []),
         "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P, F, P, Z, P, P, P, P]),
         "sfa_gated_combine": (I, [P, P, P, P, P, P, I, I, I, P, P]),
@@ -427,10 +428,10 @@ def decode_workspace_size(B, Hq, Hkv, d, topk_tok, num_splits=0) -> int:
     return int(_lib.sfa_decode_workspace_size(B, Hq, Hkv, d, topk_tok, num_splits))
 
 
-def _dec_checks(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx):
+def _dec_checks(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx, cache_dtype=torch.bfloat16):
     _need(q, "q", torch.bfloat16, 3)
-    _need(k_cache, "k_cache", torch.bfloat16, 4)
-    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", cache_dtype, 4)
+    _need(v_cache, "v_cache", cache_dtype, 4)
     _need(block_table, "block_table", torch.int32, 2)
     if cache_seqlens is not None:
         _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
@@ -461,6 +462,33 @@ def decode(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx, *, wind
                          page, _ptr(cache_seqlens), _ptr(sel_tok_idx), topk, B, Hq, Hkv, d, int(window_left),
                          _scale(scale), int(num_splits), _ptr(ws), ws.numel() * ws.element_size(), _ptr(status),
                          _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+@_on_tensor_device
+def decode_fp8(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx, *, k_descale=None, v_descale=None,
+               window_left: int = -1, scale=None, num_splits: int = 0, out=None, lse=None, workspace=None,
+               status=None, stream=None):
+    """Paged top-k decode over FP8 caches (sfa_decode_fp8): k_cache / v_cache hold E4M3 codes as uint8
+    (num_pages, page, Hkv, d); k_descale / v_descale fp32 (B, Hkv) or None (1).  Otherwise as decode()."""
+    B, Hq, d, num_pages, page, Hkv = _dec_checks(q, k_cache, v_cache, block_table, cache_seqlens, sel_tok_idx,
+                                                 cache_dtype=torch.uint8)
+    for name, t in (("k_descale", k_descale), ("v_descale", v_descale)):
+        if t is not None:
+            _need(t, name, torch.float32, 2)
+            if tuple(t.shape) != (B, Hkv):
+                raise ValueError(f"{name} must have shape (B, Hkv)")
+    topk = sel_tok_idx.shape[2]
+    nbytes = decode_workspace_size(B, Hq, Hkv, d, topk, num_splits)
+    ws = _workspace(workspace, nbytes, q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    rc = _lib.sfa_decode_fp8(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_descale), _ptr(v_descale),
+                             _ptr(block_table), block_table.shape[1], num_pages, page, _ptr(cache_seqlens),
+                             _ptr(sel_tok_idx), topk, B, Hq, Hkv, d, int(window_left), _scale(scale), int(num_splits),
+                             _ptr(ws), ws.numel() * ws.element_size(), _ptr(status), _ptr(out), _ptr(lse),
+                             _stream(stream))
     _check(rc)
     return out, lse
 

@@ -447,7 +447,8 @@ int dec_prep_impl(const DecGeom &g, const int32_t *seqlens, const int32_t *sel, 
 // canonical sets from the workspace.
 int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void *vc, const int32_t *bt, int max_pages,
                     int num_pages, int page, const int32_t *seqlens, const int32_t *sel, int wl, bool fused,
-                    float scale, void *ws, int32_t *status, void *out, float *lse, cudaStream_t st)
+                    float scale, void *ws, int32_t *status, void *out, float *lse, cudaStream_t st,
+                    bool fp8 = false, const float *kd = nullptr, const float *vd = nullptr)
 {
     if ((int64_t)num_pages * page * g.Hkv > (int64_t)INT32_MAX) return SFA_ERR_UNSUPPORTED;
     uint8_t *w = static_cast<uint8_t *>(ws);
@@ -480,6 +481,9 @@ int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void 
     p.plse = reinterpret_cast<float *>(w + g.off_plse);
     p.out_direct = static_cast<__nv_bfloat16 *>(out);
     p.lse_direct = lse;
+    p.fp8 = fp8 ? 1 : 0;
+    p.kd = kd;
+    p.vd = vd;
     p.status = status;
     if (launch_decode_split(g, p, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (g.S <= decode_split_warps_per_block()) return SFA_OK;  // combined inside the split kernel
@@ -491,6 +495,45 @@ int dec_attend_impl(const DecGeom &g, const void *q, const void *kc, const void 
     c.out = static_cast<__nv_bfloat16 *>(out);
     c.lse = lse;
     return launch_decode_combine(g, c, st) == cudaSuccess ? SFA_OK : SFA_ERR_CUDA;
+}
+
+}  // namespace
+
+namespace {
+
+// sfa_decode and sfa_decode_fp8: fp8 caches hold E4M3 codes with descales kd / vd (B, Hkv) or nullptr.
+int decode_impl(const void *q, const void *k_cache, const void *v_cache, const int32_t *block_table,
+                int max_pages_per_seq, int num_pages, int page_size, const int32_t *cache_seqlens,
+                const int32_t *sel_tok_idx, int topk_tok, int B, int Hq, int Hkv, int d, int window_left, float scale,
+                int num_splits, void *workspace, size_t workspace_bytes, int32_t *status_dev, void *out, float *lse,
+                sfa_stream_t stream, bool fp8, const float *kd, const float *vd)
+{
+    g_last_launches = 0;
+    DecGeom g;
+    int rc = dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g);
+    if (rc != SFA_OK) return rc;
+    if (page_size <= 0 || max_pages_per_seq <= 0 || num_pages < 0 || window_left < -1) return SFA_ERR_INVALID_ARG;
+    if (B == 0) return SFA_OK;
+    if (!q || !k_cache || !v_cache || !block_table || !cache_seqlens || !sel_tok_idx || !workspace || !out || !lse)
+        return SFA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
+    if (fp8 && ((kd && (reinterpret_cast<uintptr_t>(kd) & 3u)) || (vd && (reinterpret_cast<uintptr_t>(vd) & 3u))))
+        return SFA_ERR_INVALID_ARG;
+    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    // Selections of up to decode_fused_max_topk() positions are deduplicated inside the split
+    // kernel; longer ones go through the prep kernel first.
+    const bool fused = topk_tok <= decode_fused_max_topk();
+    if (!fused) {
+        rc = dec_prep_impl(g, cache_seqlens, sel_tok_idx, max_pages_per_seq, page_size, window_left, workspace,
+                           status_dev, stream);
+        if (rc != SFA_OK) return rc;
+    } else if ((int64_t)max_pages_per_seq * page_size > (1 << 20)) {
+        return SFA_ERR_UNSUPPORTED;
+    }
+    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, cache_seqlens,
+                         sel_tok_idx, window_left, fused, scale, workspace, status_dev, out, lse, stream, fp8, kd, vd);
+    if (rc == SFA_OK) g_last_launches = (fused ? 0 : 1) + (g.S <= decode_split_warps_per_block() ? 1 : 2);
+    return rc;
 }
 
 }  // namespace
@@ -845,30 +888,20 @@ int sfa_decode(const void *q, const void *k_cache, const void *v_cache, const in
                int num_splits, void *workspace, size_t workspace_bytes, int32_t *status_dev, void *out, float *lse,
                sfa_stream_t stream)
 {
-    g_last_launches = 0;
-    DecGeom g;
-    int rc = dec_geometry(B, Hq, Hkv, d, topk_tok, num_splits, g);
-    if (rc != SFA_OK) return rc;
-    if (page_size <= 0 || max_pages_per_seq <= 0 || num_pages < 0 || window_left < -1) return SFA_ERR_INVALID_ARG;
-    if (B == 0) return SFA_OK;
-    if (!q || !k_cache || !v_cache || !block_table || !cache_seqlens || !sel_tok_idx || !workspace || !out || !lse)
-        return SFA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
-    if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
-    // Selections of up to decode_fused_max_topk() positions are deduplicated inside the split
-    // kernel; longer ones go through the prep kernel first.
-    const bool fused = topk_tok <= decode_fused_max_topk();
-    if (!fused) {
-        rc = dec_prep_impl(g, cache_seqlens, sel_tok_idx, max_pages_per_seq, page_size, window_left, workspace,
-                           status_dev, stream);
-        if (rc != SFA_OK) return rc;
-    } else if ((int64_t)max_pages_per_seq * page_size > (1 << 20)) {
-        return SFA_ERR_UNSUPPORTED;
-    }
-    rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, cache_seqlens,
-                         sel_tok_idx, window_left, fused, scale, workspace, status_dev, out, lse, stream);
-    if (rc == SFA_OK) g_last_launches = (fused ? 0 : 1) + (g.S <= decode_split_warps_per_block() ? 1 : 2);
-    return rc;
+    return decode_impl(q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, cache_seqlens,
+                       sel_tok_idx, topk_tok, B, Hq, Hkv, d, window_left, scale, num_splits, workspace, workspace_bytes,
+                       status_dev, out, lse, stream, false, nullptr, nullptr);
+}
+
+int sfa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, const float *k_descale,
+                   const float *v_descale, const int32_t *block_table, int max_pages_per_seq, int num_pages,
+                   int page_size, const int32_t *cache_seqlens, const int32_t *sel_tok_idx, int topk_tok, int B,
+                   int Hq, int Hkv, int d, int window_left, float scale, int num_splits, void *workspace,
+                   size_t workspace_bytes, int32_t *status_dev, void *out, float *lse, sfa_stream_t stream)
+{
+    return decode_impl(q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, cache_seqlens,
+                       sel_tok_idx, topk_tok, B, Hq, Hkv, d, window_left, scale, num_splits, workspace, workspace_bytes,
+                       status_dev, out, lse, stream, true, k_descale, v_descale);
 }
 
 size_t sfa_window_fwd_workspace_size(void)

@@ -20,6 +20,8 @@
 // flash-attention-npu flash_attn_with_kvcache docstring; split-KV for decode load balance is
 // listed in the Flash-Sparse-Attention README).  A split with no token has lse_s = -inf and
 // weight 0; a row with no token at all outputs 0 and lse = -inf.
+#include <cuda_fp16.h>
+
 #include "sfa_device.cuh"
 
 namespace sfa {
@@ -180,7 +182,42 @@ __device__ int dedupe_positions(const int32_t *sel, int topk, int L, int wl, uin
     return n;
 }
 
+// FP8 caches (F8): a warp's ring keeps the same size, split into one bf16 K/V tile pair (the layout
+// the MMA code reads, at the start of the ring) and two landing stages of E4M3 rows (D bytes each,
+// unswizzled) behind it; each stage is converted into the bf16 tiles before its products.  E4M3
+// values are exact in bf16, so the products see the cached values themselves; the per (sequence, kv
+// head) descales multiply the score scale (k) and the normalised output (v).
 template <int D>
+struct DecF8 {
+    static constexpr int kRowBytes = D;                        // E4M3 row
+    static constexpr int kChunks = D / 16;                     // 16-byte chunks per row
+    static constexpr int kTileBytes = kStageTok * kRowBytes;
+    static constexpr int kStageBytes = 2 * kTileBytes;         // K then V
+    static constexpr int kOffLanding = DecCfg<D>::kStageBytes;  // behind the bf16 tile pair
+    static_assert(kOffLanding + kDecStages * kStageBytes == DecCfg<D>::kWarpRing, "ring size");
+};
+
+// 16 E4M3 values (one 16-byte chunk, lowest byte first) to 16 bf16 values (two 16-byte chunks).
+__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 in, uint4 &lo, uint4 &hi)
+{
+    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
+    uint32_t r[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const uint16_t pair = (uint16_t)(w[i] >> (16 * hh));
+            uint32_t h2;
+            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(pair));
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&h2));
+            r[2 * i + hh] = pack_bf16x2(f.x, f.y);
+        }
+    }
+    lo = make_uint4(r[0], r[1], r[2], r[3]);
+    hi = make_uint4(r[4], r[5], r[6], r[7]);
+}
+
+template <int D, bool F8>
 __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSplitParams p)
 {
     using C = DecCfg<D>;
@@ -192,6 +229,8 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
     const int bh = blockIdx.x / cps;                     // b * Hkv + hk
     const int split = (blockIdx.x - bh * cps) * kDecWarps + warp;
     const int hk = bh % p.Hkv, b = bh / p.Hkv;
+    const float k_ds = F8 && p.kd ? __ldg(&p.kd[bh]) : 1.f, v_ds = F8 && p.vd ? __ldg(&p.vd[bh]) : 1.f;
+    const float scale_log2 = p.scale_log2 * k_ds;  // the k descale scales every score of this (b, kv head)
     // The sequence's block-table row into shared memory when it fits (read while the selection is
     // deduplicated), so a token's physical row is found without a dependent global load.
     int *bt_s = reinterpret_cast<int *>(dsm + C::kOffBt);
@@ -272,17 +311,35 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
         __syncwarp();
         const int nst = (wn + kStageTok - 1) / kStageTok;
         auto load_stage = [&](int stage, int s) {
-            const uint32_t kdst = ring + stage * C::kStageBytes;
-            const uint32_t vdst = kdst + C::kTileBytes;
-            const int c = lane % C::kChunks;
+            if constexpr (F8) {
+                using F = DecF8<D>;
+                const uint32_t kdst = ring + F::kOffLanding + stage * F::kStageBytes;
+                const uint32_t vdst = kdst + F::kTileBytes;
+                const uint8_t *kc8 = reinterpret_cast<const uint8_t *>(p.kc);
+                const uint8_t *vc8 = reinterpret_cast<const uint8_t *>(p.vc);
+                const int c = lane % F::kChunks;
 #pragma unroll
-            for (int tt = lane / C::kChunks; tt < kStageTok; tt += 32 / C::kChunks) {
-                const int e = s * kStageTok + tt;
-                const int ro = e < wn ? rowoff[e] : -1;
-                const int64_t off = ro >= 0 ? (int64_t)ro * D + c * 8 : 0;
-                const uint32_t nbytes = ro >= 0 ? 16u : 0u;
-                cp_async16(kdst + swz<D>(tt, c), p.kc + off, nbytes);
-                cp_async16(vdst + swz<D>(tt, c), p.vc + off, nbytes);
+                for (int tt = lane / F::kChunks; tt < kStageTok; tt += 32 / F::kChunks) {
+                    const int e = s * kStageTok + tt;
+                    const int ro = e < wn ? rowoff[e] : -1;
+                    const int64_t off = ro >= 0 ? (int64_t)ro * D + c * 16 : 0;
+                    const uint32_t nbytes = ro >= 0 ? 16u : 0u;
+                    cp_async16(kdst + tt * D + c * 16, kc8 + off, nbytes);
+                    cp_async16(vdst + tt * D + c * 16, vc8 + off, nbytes);
+                }
+            } else {
+                const uint32_t kdst = ring + stage * C::kStageBytes;
+                const uint32_t vdst = kdst + C::kTileBytes;
+                const int c = lane % C::kChunks;
+#pragma unroll
+                for (int tt = lane / C::kChunks; tt < kStageTok; tt += 32 / C::kChunks) {
+                    const int e = s * kStageTok + tt;
+                    const int ro = e < wn ? rowoff[e] : -1;
+                    const int64_t off = ro >= 0 ? (int64_t)ro * D + c * 8 : 0;
+                    const uint32_t nbytes = ro >= 0 ? 16u : 0u;
+                    cp_async16(kdst + swz<D>(tt, c), p.kc + off, nbytes);
+                    cp_async16(vdst + swz<D>(tt, c), p.vc + off, nbytes);
+                }
             }
         };
 #pragma unroll
@@ -298,7 +355,26 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
                 if (nxt < nst) load_stage(nxt % kDecStages, nxt);
                 cp_async_commit();
             }
-            const uint32_t kt = ring + (it % kDecStages) * C::kStageBytes;
+            uint32_t kt = ring + (it % kDecStages) * C::kStageBytes;
+            if constexpr (F8) {
+                // this stage's E4M3 rows into the bf16 tile pair (swizzled as the MMA code reads it)
+                using F = DecF8<D>;
+                const uint8_t *land = dsm + (ring - smem_u32(dsm)) + F::kOffLanding + (it % kDecStages) * F::kStageBytes;
+                uint8_t *tiles = dsm + (ring - smem_u32(dsm));
+#pragma unroll
+                for (int e = lane; e < 2 * kStageTok * F::kChunks; e += 32) {
+                    const int kv = e / (kStageTok * F::kChunks), rem = e - kv * (kStageTok * F::kChunks);
+                    const int tt = rem / F::kChunks, c = rem - tt * F::kChunks;
+                    const uint4 in = *reinterpret_cast<const uint4 *>(land + kv * F::kTileBytes + tt * D + c * 16);
+                    uint4 lo, hi;
+                    e4m3x16_to_bf16(in, lo, hi);
+                    uint8_t *tile = tiles + kv * C::kTileBytes;
+                    *reinterpret_cast<uint4 *>(tile + swz<D>(tt, 2 * c)) = lo;
+                    *reinterpret_cast<uint4 *>(tile + swz<D>(tt, 2 * c + 1)) = hi;
+                }
+                __syncwarp();
+                kt = ring;
+            }
             const uint32_t vt = kt + C::kTileBytes;
             const int mi = lane >> 3;
 
@@ -332,7 +408,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
                 float mx = fmaxf(fmaxf(sv[h][0], sv[h][1]), fmaxf(sv[h][2], sv[h][3]));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
                 mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-                const float m_blk = mx * p.scale_log2;
+                const float m_blk = mx * scale_log2;
                 if (m_blk > m_r[h] + kRescaleLog2d) {  // uniform across the 4 lanes of a row
                     const float f = m_r[h] == -INFINITY ? 0.f : ex2(m_r[h] - m_blk);
                     m_r[h] = m_blk;
@@ -347,7 +423,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
                 float sum = 0.f;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    pr[h][u] = ex2(fmaf(sv[h][u], p.scale_log2, -m_use));
+                    pr[h][u] = ex2(fmaf(sv[h][u], scale_log2, -m_use));
                     sum += pr[h][u];
                 }
                 l_r[h] += sum;
@@ -387,7 +463,7 @@ __global__ void __launch_bounds__(kDecThreads) decode_split_kernel(const DecSpli
         if (active && row < p.G) {
             const int hq = hk * p.G + row;
             const int64_t slot = ((int64_t)b * p.Hq + hq) * p.S + split;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float inv = l > 0.f ? v_ds / l : 0.f;  // the v descale scales the output
             float *dst = (cta_combine ? po_s + row * D : p.po + slot * D) + 2 * (lane & 3);
 #pragma unroll
             for (int nt = 0; nt < D / 8; ++nt)
@@ -453,14 +529,14 @@ __global__ void decode_combine_kernel(const DecCombineParams p)
     if (threadIdx.x == 0) p.lse[row] = lse;
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_split_t(const DecGeom &g, const DecSplitParams &p, cudaStream_t st)
 {
     const size_t smem = DecCfg<D>::kBytes;
-    const cudaError_t e = ensure_smem_for(decode_split_kernel<D>, smem);
+    const cudaError_t e = ensure_smem_for(decode_split_kernel<D, F8>, smem);
     if (e != cudaSuccess) return e;
     const int cps = (g.S + kDecWarps - 1) / kDecWarps;
-    decode_split_kernel<D><<<g.B * g.Hkv * cps, kDecThreads, smem, st>>>(p);
+    decode_split_kernel<D, F8><<<g.B * g.Hkv * cps, kDecThreads, smem, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -485,7 +561,8 @@ int decode_fused_max_topk()
 
 cudaError_t launch_decode_split(const DecGeom &g, const DecSplitParams &p, cudaStream_t st)
 {
-    return g.d == 64 ? launch_split_t<64>(g, p, st) : launch_split_t<128>(g, p, st);
+    if (p.fp8) return g.d == 64 ? launch_split_t<64, true>(g, p, st) : launch_split_t<128, true>(g, p, st);
+    return g.d == 64 ? launch_split_t<64, false>(g, p, st) : launch_split_t<128, false>(g, p, st);
 }
 
 cudaError_t launch_decode_combine(const DecGeom &g, const DecCombineParams &p, cudaStream_t st)

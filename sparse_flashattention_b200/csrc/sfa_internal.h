@@ -194,6 +194,8 @@ struct DecSplitParams {
     int fused, wl;
     int B, max_pages, num_pages, page, Hq, Hkv, G, topk, S;  // CTA c of (b, kv head) runs splits 6c..6c+5
     int page_shift;  // log2(page) when page is a power of two, else -1
+    int fp8;         // caches hold E4M3 codes (1 byte per value); kd / vd: descales (B, Hkv) or nullptr (1)
+    const float *kd, *vd;
     float scale_log2;
     float *po, *plse;  // partial outputs (B, Hq, S, d) and natural-log lse (B, Hq, S)
     __nv_bfloat16 *out_direct;  // S <= 4: the CTA combines its splits and writes out / lse itself
