@@ -231,6 +231,7 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     pl.W = g.W;
     pl.nblk_max = g.nblk_max;
     pl.cu_q = cu_q;
+    pl.cu_k = p.cu_k;
     pl.items = reinterpret_cast<InvItem *>(w + g.off_items);
     pl.ctrl = reinterpret_cast<InvCtrl *>(w + g.off_ctrl);
     if (launch_fwd_plan(g, pl, st) != cudaSuccess) return SFA_ERR_CUDA;

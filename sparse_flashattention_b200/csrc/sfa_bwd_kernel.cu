@@ -284,8 +284,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     bool progressed = false;
                     if (ns < n && ns <= np + 1) {
                         const int jg = jg0 + ns;
-                        if (mbar_try_wait(smem_u32(&meta->k_full[sk_st]), sk_ph) &&
-                            mbar_try_wait(smem_u32(&meta->v_full[sv_st]), sv_ph)) {
+                        if (mbar_test(smem_u32(&meta->k_full[sk_st]), sk_ph) &&
+                            mbar_test(smem_u32(&meta->v_full[sv_st]), sv_ph)) {
                             tc_fence_after();
                             const uint32_t tS = tmem + (jg & 1) * BS, tDP = tmem + C::kColDP + (jg & 1) * BS;
                             const uint32_t ko = (uint32_t)sk_st * C::kKVBytes, vo = (uint32_t)sv_st * C::kKVBytes;
@@ -318,8 +318,8 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                     }
                     if (np < ns) {
                         const int ig = jg0 + np, st = qk_st;
-                        if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
-                            (ofree || mbar_try_wait(smem_u32(&meta->o_free), (k - 1) & 1))) {
+                        if (mbar_test(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
+                            (ofree || mbar_test(smem_u32(&meta->o_free), (k - 1) & 1))) {
                             ofree = true;
                             tc_fence_after();
 #pragma unroll
@@ -732,7 +732,7 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     bool progressed = false;
                     if (ns < nch && ns <= np + 1) {
                         const int cg = cg0 + ns, b = cg & 1;
-                        if (mbar_try_wait(smem_u32(&meta->qd_full[b]), (cg >> 1) & 1)) {
+                        if (mbar_test(smem_u32(&meta->qd_full[b]), (cg >> 1) & 1)) {
                             fence_proxy_async_smem();  // the rows came through cp.async (generic proxy)
                             tc_fence_after();
                             const uint32_t tS = tmem + b * BS, tDP = tmem + C::kColDP + b * BS;
@@ -755,8 +755,8 @@ __global__ void __launch_bounds__(kKvThreads, 1)
                     }
                     if (np < ns) {
                         const int cg = cg0 + np, b = cg & 1;
-                        if (mbar_try_wait(smem_u32(&meta->p_full[b]), (cg >> 1) & 1) &&
-                            (accfree || mbar_try_wait(smem_u32(&meta->acc_free), (kp - 1) & 1))) {
+                        if (mbar_test(smem_u32(&meta->p_full[b]), (cg >> 1) & 1) &&
+                            (accfree || mbar_test(smem_u32(&meta->acc_free), (kp - 1) & 1))) {
                             accfree = true;
                             tc_fence_after();
 #pragma unroll

@@ -64,6 +64,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.  Loops that poll several barriers in turn
+// (the MMA-issuing threads) use this: try_wait may suspend the thread while its phase is pending, up
+// to a system-dependent time limit, and meanwhile work behind another barrier that is ready waits.
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false when the CTA's
 // abort flag is (or becomes) set or the time limit passes; the latter sets the flag and
 // records SFA_DEV_TIMEOUT.

@@ -23,8 +23,8 @@ namespace sfa {
 
 namespace {
 
-constexpr int kInvThreadsAttn = 352;  // warp 0 producer, warp 1 MMA, warps 2-5 and 6-9: two softmax groups,
-                                      // warp 10: second half of each item's Q-row gather
+constexpr int kInvThreadsAttn = 384;  // warp 0 producer, warp 1 MMA, warps 2-5 and 6-9: two softmax groups,
+                                      // warps 11 and 10: the first and second half of each item's Q-row gather
 constexpr float kLn2i = 0.6931471805599453f;
 constexpr int kItemSlots = 8;   // item j lives in slot j % 8; softmax group j % 2 handles it
 constexpr int kFetchAhead = 4;  // item records are fetched this many items ahead
@@ -180,7 +180,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->kv_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
             if (lane == 0) {
-                const int row = __ldg(&p.cu_k[b]) + rec.y * BS;
+                const int row = rec.z + rec.y * BS;  // the sequence's first K row comes with the record
                 mbar_arrive_expect_tx(&meta->kv_full[sl], 2u * (uint32_t)C::kKVBytes);
                 for (int c = 0; c < D / 64; ++c) {
                     tma_load_3d(&tmk, &meta->kv_full[sl], sK + sl * C::kKVBytes + c * (BS * 128), c * 64, hk, row);
@@ -188,15 +188,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 }
                 issued[sl]++;
             }
-            // Q rows 0..63 of the item's tokens (row r = token * G + head) into the 128-byte-swizzled
-            // K-major tile the MMA reads (rows past the item are zero-filled; warp 10 copies rows
-            // 64..127).  16-byte cp.async copies with the lanes spread along the rows, so one warp
-            // instruction moves whole rows (coalesced).  Each lane's copies land on q_full through its
-            // own arrival.
-            if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
-            if (!ok) break;
-            gather_q_rows<D>(p, item, hk, rec.w * p.G, 0, smem_u32(sQ + sl * C::kQBytes), lane);
-            cp_async_mbar_arrive(&meta->q_full[sl]);
+            // (the item's Q rows are gathered by warps 11 and 10)
             // Item j+4 goes into the slot item j-4 used, once its softmax group is done with it.
             if (j + kFetchAhead >= kItemSlots)
                 ok = warp_all_ok(mbar_wait(&meta->item_free[(j + kFetchAhead) % kItemSlots],
@@ -205,7 +197,6 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             if (lane == 0) fetch(j + kFetchAhead);
             __syncwarp();
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's Q copies have all landed
         if (*abort_flag && lane == 0) {
             for (int sl = 0; sl < kLoadStages; ++sl)
                 if (issued[sl] > 0) mbar_drain(&meta->kv_full[sl], (issued[sl] - 1) & 1);
@@ -226,12 +217,12 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 if (!end_seen && ns <= np + 1) {
                     const int it = ns % kItemSlots, sl = ns % kLoadStages, sb = ns & 1;
                     const uint32_t ph = (ns / kLoadStages) & 1;
-                    if (mbar_try_wait(smem_u32(&meta->item_full[it]), (ns / kItemSlots) & 1)) {
+                    if (mbar_test(smem_u32(&meta->item_full[it]), (ns / kItemSlots) & 1)) {
                         if (meta->slot[it].rec.w < 0) {
                             end_seen = true;
                             progressed = true;
-                        } else if (mbar_try_wait(smem_u32(&meta->q_full[sl]), ph) &&
-                                   mbar_try_wait(smem_u32(&meta->kv_full[sl]), ph)) {
+                        } else if (mbar_test(smem_u32(&meta->q_full[sl]), ph) &&
+                                   mbar_test(smem_u32(&meta->kv_full[sl]), ph)) {
                             tc_fence_after();
                             const uint32_t tS = tmem + sb * BS;
 #pragma unroll
@@ -251,8 +242,8 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 }
                 if (np < ns) {
                     const int w = np & 1;
-                    if (mbar_try_wait(smem_u32(&meta->p_full[w]), (np >> 1) & 1) &&
-                        (np < 2 || mbar_try_wait(smem_u32(&meta->o_free[w]), ((np >> 1) - 1) & 1))) {
+                    if (mbar_test(smem_u32(&meta->p_full[w]), (np >> 1) & 1) &&
+                        (np < 2 || mbar_test(smem_u32(&meta->o_free[w]), ((np >> 1) - 1) & 1))) {
                         tc_fence_after();
                         const uint32_t tO = tmem + 128 + w * D;
                         const int vs = np % kLoadStages;
@@ -284,10 +275,14 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 mbar_drain(&meta->drain, 0);
             }
         }
-    } else if (warp == 10) {
-        // ---------------------------------------------------------------- Q-row gather, rows 64..127
-        // Follows the producer's item sequence: the item's slot stays valid until its softmax group
-        // frees it, which needs this warp's copies (q_full) first.
+    } else if (warp >= 10) {
+        // ---------------------------------------------------------------- Q-row gather
+        // Warp 11 copies rows 0..63 of each item's Q tile (row r = token * G + head) into the
+        // 128-byte-swizzled K-major tile the MMA reads, warp 10 rows 64..127; rows past the item are
+        // zero-filled.  Each lane's copies land on q_full through its own arrival.  Both follow the
+        // producer's item sequence: the item's slot stays valid until its softmax group frees it,
+        // which needs these copies (q_full) first.
+        const int r0 = warp == 11 ? 0 : 64;
         bool ok = true;
         for (int j = 0; ok; ++j) {
             const int sl = j % kLoadStages, it = j % kItemSlots;
@@ -300,7 +295,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             const int hk = rec.x % p.Hkv;
             if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->q_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
-            gather_q_rows<D>(p, item, hk, rec.w * p.G, 64, smem_u32(sQ + sl * C::kQBytes), lane);
+            gather_q_rows<D>(p, item, hk, rec.w * p.G, r0, smem_u32(sQ + sl * C::kQBytes), lane);
             cp_async_mbar_arrive(&meta->q_full[sl]);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");  // this lane's copies have all landed
@@ -391,11 +386,8 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 ps_i[i] = __shfl_sync(0xffffffffu, (long long)pslot, rr);
                 vr_i[i] = __shfl_sync(0xffffffffu, valid ? 1 : 0, rr) != 0;
             }
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tO + c * 32, o);
-                tmem_wait_ld();
+            // one 32-column chunk c of the row: pack, stage, store
+            auto put_chunk = [&](int c, const uint32_t(&o)[32]) {
                 uint32_t wv[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
@@ -411,6 +403,15 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                     const uint4 v = stg[rr * 4 + ((seg + (rr >> 1)) & 3)];
                     if (vr_i[i]) reinterpret_cast<uint4 *>(p.po + ps_i[i] * D + c * 32)[seg] = v;
                 }
+            };
+#pragma unroll 1
+            for (int c = 0; c < D / 32; c += 2) {  // two chunks per TMEM wait
+                uint32_t oa[32], ob[32];
+                tmem_ld32(tO + c * 32, oa);
+                tmem_ld32(tO + (c + 1) * 32, ob);
+                tmem_wait_ld();
+                put_chunk(c, oa);
+                put_chunk(c + 1, ob);
             }
             tc_fence_before();
             mbar_arrive(&meta->o_free[grp]);

@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         bool progressed = false;
                         if (ns < nU && ns <= np + 1) {
                             const int jg = jbase + ns, st = jg % kStages;
-                            if (mbar_try_wait(smem_u32(&meta->k_full[st]), (jg / kStages) & 1)) {
+                            if (mbar_test(smem_u32(&meta->k_full[st]), (jg / kStages) & 1)) {
                                 tc_fence_after();
                                 const uint32_t tS = tmem + (jg & 1) * BS;
 #pragma unroll
@@ -245,8 +245,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                         }
                         if (np < ns) {
                             const int ig = jbase + np, st = ig % kStages;
-                            if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
-                                mbar_try_wait(smem_u32(&meta->v_full[st]), (ig / kStages) & 1)) {
+                            if (mbar_test(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
+                                mbar_test(smem_u32(&meta->v_full[st]), (ig / kStages) & 1)) {
                                 tc_fence_after();
 #pragma unroll
                                 for (int ks = 0; ks < BS / 16; ++ks) {

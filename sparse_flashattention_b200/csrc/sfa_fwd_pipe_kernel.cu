@@ -422,7 +422,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
                     bool progressed = false;
                     if (ns < n && ns <= np + 1) {
                         const int jg = jg0 + ns, st = s_st;
-                        if (mbar_try_wait(smem_u32(&meta->k_full[st]), s_ph)) {
+                        if (mbar_test(smem_u32(&meta->k_full[st]), s_ph)) {
                             tc_fence_after();
                             const uint32_t tS = tmem + (jg & 1) * BS;
                             const uint64_t dK = dK0 + (uint64_t)((st * C::kKVBytes) >> 4);
@@ -444,9 +444,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
                     }
                     if (np < ns) {
                         const int ig = jg0 + np, st = p_st;
-                        if (mbar_try_wait(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
-                            mbar_try_wait(smem_u32(&meta->v_full[st]), p_ph) &&
-                            (ofree || mbar_try_wait(smem_u32(&meta->o_free), (k - 1) & 1))) {
+                        if (mbar_test(smem_u32(&meta->p_full[ig & 1]), (ig >> 1) & 1) &&
+                            mbar_test(smem_u32(&meta->v_full[st]), p_ph) &&
+                            (ofree || mbar_test(smem_u32(&meta->o_free), (k - 1) & 1))) {
                             ofree = true;
                             tc_fence_after();
                             const uint64_t dV = dV0 + (uint64_t)((st * C::kKVBytes) >> 4);

@@ -48,7 +48,7 @@ struct GroupStat {
 
 // One block-major item as stored in the workspace and copied whole into shared memory.
 struct InvItem {
-    int4 rec;      // {b * Hkv + hk, block, 0, tokens}; tokens < 0 marks the end of the work
+    int4 rec;      // {b * Hkv + hk, block, first K row of the sequence, tokens}; tokens < 0 ends the work
     int tok[128];  // (token << 7) | position of the block in the token's canonical list
 };
 
@@ -70,7 +70,7 @@ struct FwdPlanParams {
     const int32_t *gcount;
     int32_t *gfirst;
     int batch, Hkv, Tq, nqt, W, nblk_max;
-    const int32_t *cu_q;
+    const int32_t *cu_q, *cu_k;
     InvItem *items;
     InvCtrl *ctrl;
 };

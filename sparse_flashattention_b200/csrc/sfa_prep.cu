@@ -233,12 +233,13 @@ __global__ void __launch_bounds__(kInvThreads) fwd_plan_kernel(FwdPlanParams p)
     if (threadIdx.x == 0) item_base = atomicAdd(&p.ctrl->item_total, nitems);
     __syncthreads();
     int32_t *gfirst = p.gfirst + (int64_t)g * p.nblk_max;
+    const int k0 = p.cu_k[b];
     for (int s = threadIdx.x; s < p.nblk_max; s += kInvThreads) {
         const int c = count[s];
         const int i0 = item_base + first[s];
         gfirst[s] = i0;
         for (int i = 0; i * p.Tq < c; ++i)
-            p.items[i0 + i].rec = make_int4(b * p.Hkv + hk, s, 0, min(p.Tq, c - i * p.Tq));
+            p.items[i0 + i].rec = make_int4(b * p.Hkv + hk, s, k0, min(p.Tq, c - i * p.Tq));
     }
 }
 
