@@ -29,6 +29,7 @@ constexpr float kLn2i = 0.6931471805599453f;
 constexpr int kItemSlots = 8;   // item j lives in slot j % 8; softmax group j % 2 handles it
 constexpr int kFetchAhead = 4;  // item records are fetched this many items ahead
 constexpr int kLoadStages = 3;  // Q and K/V buffers: item j uses buffer j % 3
+constexpr int kInvCuCache = 255;  // sequences whose cu_seqlens entries are kept in shared memory
 
 template <int D, int BS>
 struct InvCfg {
@@ -40,6 +41,7 @@ struct InvCfg {
     static constexpr int kOffMeta = kOffV + kLoadStages * kKVBytes;
     static constexpr int kOffStage = kOffMeta + 4608;  // 8 softmax warps x 2 KB epilogue staging
     static constexpr int kStageBytes = 8 * 2048;
+    static constexpr int kOffCu = kOffStage + kStageBytes;  // cu_seqlens_q, cu_seqlens_k
     static constexpr uint32_t kIdescS = idesc_bf16_f32(128, BS, false);
     static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
     static constexpr int kTmemCols = 512;  // S/P of group w at w*BS, O of group w at 128 + w*D
@@ -132,6 +134,14 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
         tmem_alloc(&meta->tmem_base, C::kTmemCols);
         tmem_relinquish();
     }
+    // cu_seqlens_q / _k in shared memory (batches of up to kInvCuCache sequences), so an item's sequence
+    // bounds cost no dependent global load on the softmax groups' path
+    int *s_cu = reinterpret_cast<int *>(smem + C::kOffCu);
+    if (p.batch <= kInvCuCache)
+        for (int i = threadIdx.x; i <= p.batch; i += blockDim.x) {
+            s_cu[i] = __ldg(&p.cu_q[i]);
+            s_cu[kInvCuCache + 1 + i] = __ldg(&p.cu_k[i]);
+        }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -317,8 +327,11 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             const int4 rec = meta->slot[it].rec;
             if (rec.w < 0) break;
             const int hk = rec.x % p.Hkv, b = rec.x / p.Hkv, s = rec.y, n = rec.w;
-            const int q0 = __ldg(&p.cu_q[b]), sq = __ldg(&p.cu_q[b + 1]) - q0;
-            const int sk = __ldg(&p.cu_k[b + 1]) - __ldg(&p.cu_k[b]);
+            const bool cached = p.batch <= kInvCuCache;
+            const int q0 = cached ? s_cu[b] : __ldg(&p.cu_q[b]);
+            const int sq = (cached ? s_cu[b + 1] : __ldg(&p.cu_q[b + 1])) - q0;
+            const int sk = cached ? s_cu[kInvCuCache + 1 + b + 1] - s_cu[kInvCuCache + 1 + b]
+                                  : __ldg(&p.cu_k[b + 1]) - __ldg(&p.cu_k[b]);
             const int tok = r / p.G, gg = r - tok * p.G;
             const bool valid = tok < n;
             int64_t t = 0;
@@ -410,11 +423,13 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
                 tmem_ld32(tO + c * 32, oa);
                 tmem_ld32(tO + (c + 1) * 32, ob);
                 tmem_wait_ld();
+                if (c + 2 >= D / 32) {  // O is in registers: the group's next P.V may overwrite it
+                    tc_fence_before();
+                    mbar_arrive(&meta->o_free[grp]);
+                }
                 put_chunk(c, oa);
                 put_chunk(c + 1, ob);
             }
-            tc_fence_before();
-            mbar_arrive(&meta->o_free[grp]);
             if (valid) p.pml[pslot] = make_float2(m, l);
 
             mbar_arrive(&meta->item_free[it]);
@@ -540,7 +555,7 @@ template <int D, int BS>
 size_t inv_smem_bytes()
 {
     static_assert(sizeof(InvMeta) <= 4608, "InvMeta must fit below the staging buffers");
-    return 1024 + InvCfg<D, BS>::kOffStage + InvCfg<D, BS>::kStageBytes;
+    return 1024 + InvCfg<D, BS>::kOffCu + 2 * (kInvCuCache + 1) * 4;
 }
 
 template <int D, int BS>
