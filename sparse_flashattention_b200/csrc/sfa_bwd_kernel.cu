@@ -657,32 +657,37 @@ __global__ void __launch_bounds__(kKvThreads, 1)
             const int ntok = pi.ntok, q0 = pi.q0, hk = pi.hk;
             const int32_t *toks = p.toks + pi.rowoff + pi.tok_begin;
             const int nch = (ntok + p.Tq - 1) / p.Tq;
-            const int sub = lane >> 3, piece16 = lane & 7;  // row within a group of 4, 16-byte piece of it
+            // Lane l resolves rows half*64 + l and half*64 + 32 + l of each chunk (one token lookup and
+            // one division each); the copies then run along whole rows, D/8 lanes per row, each row's
+            // global row index broadcast from the lane that resolved it.
+            constexpr int kChunks = D / 8;              // 16-byte pieces per row
+            constexpr int kRowsPerIter = 32 / kChunks;  // rows one copy instruction covers
+            const int cl = lane % kChunks, chalf = cl >> 3, k8 = cl & 7;
             for (int c = 0; c < nch; ++c) {
                 const int st = cg & 1;
                 if (cg >= 2) ok = warp_all_ok(mbar_wait(&meta->qd_empty[st], ((cg >> 1) - 1) & 1, abort_flag, p.status));
                 if (!ok) break;
                 const int ntc = min(p.Tq, ntok - c * p.Tq), rows = ntc * p.G;
                 const uint32_t qbase = smem_u32(sQ + st * C::kTileBytes), dbase = smem_u32(sDO + st * C::kTileBytes);
-                int tokv[16];  // the tokens of this lane's 16 rows, loaded together (one latency, not 16)
+                long long grow2[2];  // global (token, head) rows of this lane's two rows, -1 past the chunk
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int rr = half * 64 + i * 4 + sub;
-                    tokv[i] = rr < rows ? toks[c * p.Tq + rr / p.G] : 0;
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int rr = half * 64 + 32 * h2 + lane;
+                    const int tt = rr / p.G, gg = rr - tt * p.G;
+                    grow2[h2] = rr < rows ? ((long long)(q0 + toks[c * p.Tq + tt]) * p.Hq + hk * p.G + gg) : -1ll;
                 }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {  // 16 groups of 4 rows = this warp's 64 rows
-                    const int rr = half * 64 + i * 4 + sub;
-                    const bool live = rr < rows;
-                    const int tt = live ? rr / p.G : 0, gg = live ? rr - tt * p.G : 0;
-                    const int64_t grow = live ? ((int64_t)(q0 + tokv[i]) * p.Hq + hk * p.G + gg) : 0;
-                    const __nv_bfloat16 *qs = p.q + grow * D + piece16 * 8;
-                    const __nv_bfloat16 *ds = p.dout + grow * D + piece16 * 8;
-                    const uint32_t so = (uint32_t)(rr * 128 + ((piece16 ^ (rr & 7)) << 4));
+                for (int h2 = 0; h2 < 2; ++h2) {
 #pragma unroll
-                    for (int cc = 0; cc < D / 64; ++cc) {
-                        cp_async16(qbase + cc * (128 * 128) + so, qs + cc * 64, live ? 16u : 0u);
-                        cp_async16(dbase + cc * (128 * 128) + so, ds + cc * 64, live ? 16u : 0u);
+                    for (int i = 0; i < 32 / kRowsPerIter; ++i) {
+                        const int rl = i * kRowsPerIter + lane / kChunks;  // row within this half of 32
+                        const int rr = half * 64 + 32 * h2 + rl;
+                        const long long g = __shfl_sync(0xffffffffu, grow2[h2], rl);
+                        const bool live = g >= 0;
+                        const int64_t off = live ? (int64_t)g * D + cl * 8 : 0;
+                        const uint32_t so = (uint32_t)(chalf * (128 * 128) + rr * 128 + ((k8 ^ (rr & 7)) << 4));
+                        cp_async16(qbase + so, p.q + off, live ? 16u : 0u);
+                        cp_async16(dbase + so, p.dout + off, live ? 16u : 0u);
                     }
                 }
                 cp_async_mbar_arrive(&meta->qd_full[st]);
