@@ -86,9 +86,10 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     g.W = g.Tq * 64;
     g.nwin = (max_sq + g.W - 1) / g.W;
     g.groups = g.nwin * batch * Hkv;
-    // A window goes block-major only when its tiles' unions hold over 10x its selected blocks; with at
-    // most 10*topk blocks per sequence that needs most selections padded away, so the schedule (and
-    // its planning kernels) is left off.
+    // A window goes block-major when its tiles' unions hold over 4x its selected blocks (the fitted cost
+    // of a block-major row-block, its partial merge included, is about 3.7 query-major row-blocks).  With
+    // at most 10*topk blocks per sequence the schedule (and its planning kernels) is left off: the
+    // windows of such sequences reach that ratio only in their last tiles, where it did not pay.
     g.inv = (g.nblk_max <= 2048 && g.nblk_max > 10 * topk && total_q < (1 << 24) &&
              fwd_attend_inv_smem_bytes(g) <= 227 * 1024)
                 ? 1

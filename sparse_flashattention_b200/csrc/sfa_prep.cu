@@ -199,7 +199,7 @@ __device__ int block_scan_array(int *v, int n, int *scratch)
 }
 
 // Block-major plan, one CTA per (window, sequence, kv head) group.  The window stays with the
-// query-major kernel unless the union of its query tiles' blocks is over 10x its selected
+// query-major kernel unless the union of its query tiles' blocks is over 4x its selected
 // blocks (a block-major item moves several times the memory of a query-major tile per selected
 // row-block: its bf16 partial is written and read back and its Q rows are gathered).  For a
 // block-major window: mark its tiles (ucnt = -1), cut each selected block's token list into
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(kInvThreads) fwd_plan_kernel(FwdPlanParams p)
     const int t0 = w * p.W;
     if (t0 >= sq) return;
     const GroupStat st = p.gstat[g];
-    if (st.uni <= 10ull * st.useful) return;  // the query-major kernel keeps this window
+    if (st.uni <= 4ull * st.useful) return;  // the query-major kernel keeps this window
     const int nt = min(p.W, sq - t0);
     const int qt0 = t0 / p.Tq, qt1 = (t0 + nt - 1) / p.Tq;
     for (int qt = qt0 + threadIdx.x; qt <= qt1; qt += kInvThreads)

@@ -221,7 +221,7 @@ def test_launch_count_and_stages(sfa, oracle_lib, n):
 
 def _block_major_windows(c, oracle_lib):
     """How many (window, sequence, kv head) groups the prep will send to the block-major kernel:
-    the union of a window's query-tile block sets exceeds 10x the window's selected blocks."""
+    the union of a window's query-tile block sets exceeds 4x the window's selected blocks."""
     sel_c, cnt, _ = oracle_lib.fwd_index(c)
     G = c.Hq // c.Hkv
     Tq = 128 // G
@@ -237,7 +237,7 @@ def _block_major_windows(c, oracle_lib):
                     t1 = min(sq, t0 + Tq)
                     blocks = set(sel_c[q0 + t0:q0 + t1, hk].ravel().tolist()) - {-1}
                     union += len(blocks) * (t1 - t0)
-                n += union > 10 * useful
+                n += union > 4 * useful
     return n
 
 
