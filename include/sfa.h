@@ -45,6 +45,8 @@
  *     or a pipeline wait that exceeded its time limit (the kernel then stops early; its
  *     outputs are undefined).  Kernels never trap.
  *   - Calls on one workspace must not overlap in time (use one workspace per stream).
+ *   - A workspace starts on a 256-byte boundary (as cudaMalloc and the PyTorch caching
+ *     allocator return); another base is SFA_ERR_INVALID_ARG.
  */
 #ifndef SFA_H_
 #define SFA_H_

@@ -47,6 +47,12 @@ bool aligned16(const void *p)
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
 }
 
+// Workspaces: every array in one starts on a multiple of kAlign from its base.
+bool aligned256(const void *p)
+{
+    return (reinterpret_cast<uintptr_t>(p) & (kAlign - 1)) == 0;
+}
+
 // ----------------------------------------------------------------------------------------
 // Prefill geometry
 // ----------------------------------------------------------------------------------------
@@ -522,6 +528,7 @@ int decode_impl(const void *q, const void *k_cache, const void *v_cache, const i
     if (fp8 && ((kd && (reinterpret_cast<uintptr_t>(kd) & 3u)) || (vd && (reinterpret_cast<uintptr_t>(vd) & 3u))))
         return SFA_ERR_INVALID_ARG;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (g.bytes > 0 && !aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     // Selections of up to decode_fused_max_topk() positions are deduplicated inside the split
     // kernel; longer ones go through the prep kernel first.
     const bool fused = topk_tok <= decode_fused_max_topk();
@@ -575,6 +582,7 @@ int sfa_fwd_prep(const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k, int b
     if (total_q == 0 || batch == 0) return SFA_OK;
     if (!workspace) return SFA_ERR_INVALID_ARG;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (g.bytes > 0 && !aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     rc = fwd_prep_impl(g, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
                        status_dev, stream);
     if (rc == SFA_OK) g_last_launches = 1 + 2 * g.inv;
@@ -599,6 +607,7 @@ int sfa_fwd_attend(const void *q, const void *k, const void *v, const int32_t *c
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
     if (total_k == 0) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (g.bytes > 0 && !aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     rc = fwd_attend_impl(g, q, k, v, cu_seqlens_q, cu_seqlens_k, total_k, causal, window_left, window_right, scale,
                          workspace, status_dev, out, lse, stream);
     if (rc == SFA_OK) g_last_launches = 1 + 2 * g.inv;
@@ -623,6 +632,7 @@ int sfa_fwd(const void *q, const void *k, const void *v, const int32_t *cu_seqle
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return SFA_ERR_INVALID_ARG;
     if (total_k == 0) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (g.bytes > 0 && !aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     if (!fwd_pipe_fits(g, kPipePrep) && fwd_attend_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     if (!g.inv && fwd_pipe_fits(g, kPipeFused)) {
         // One launch: the attention kernel canonicalizes each tile's selections itself.
@@ -678,6 +688,7 @@ int sfa_bwd(const void *q, const void *k, const void *v, const void *out, const 
     // The dQ kernel keeps two copies of a tile's block union in shared memory beside its rings.
     if (bwd_dq_smem_bytes(g) > 227 * 1024 || bwd_dkdv_smem_bytes(g) > 227 * 1024) return SFA_ERR_UNSUPPORTED;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (g.bytes > 0 && !aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     uint8_t *w = static_cast<uint8_t *>(workspace);
     if (cudaMemsetAsync(w + g.off_zero, 0, g.zero_bytes, st) != cudaSuccess) return SFA_ERR_CUDA;
     rc = fwd_prep_impl(g.f, cu_seqlens_q, cu_seqlens_k, sel_idx, causal, window_left, window_right, workspace,
@@ -766,6 +777,7 @@ int sfa_index_topk(const void *q, const void *k_cache, const int32_t *block_tabl
     if (!aligned16(q) || !aligned16(k_cache)) return SFA_ERR_INVALID_ARG;
     if (workspace_bytes < sfa_index_topk_workspace_size(B, Hkv, max_pages_per_seq, page_size))
         return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     IndexParams p{};
     p.q = static_cast<const __nv_bfloat16 *>(q);
     p.kc = static_cast<const __nv_bfloat16 *>(k_cache);
@@ -858,6 +870,7 @@ int sfa_decode_prep(const int32_t *cache_seqlens, const int32_t *sel_tok_idx, in
     if (B == 0) return SFA_OK;
     if (!cache_seqlens || !sel_tok_idx || !workspace) return SFA_ERR_INVALID_ARG;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (g.bytes > 0 && !aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     rc = dec_prep_impl(g, cache_seqlens, sel_tok_idx, max_pages_per_seq, page_size, window_left, workspace, status_dev,
                        stream);
     if (rc == SFA_OK) g_last_launches = 1;
@@ -878,6 +891,7 @@ int sfa_decode_attend(const void *q, const void *k_cache, const void *v_cache, c
     if (!q || !k_cache || !v_cache || !block_table || !workspace || !out || !lse) return SFA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache)) return SFA_ERR_INVALID_ARG;
     if (workspace_bytes < g.bytes) return SFA_ERR_WORKSPACE_TOO_SMALL;
+    if (g.bytes > 0 && !aligned256(workspace)) return SFA_ERR_INVALID_ARG;
     rc = dec_attend_impl(g, q, k_cache, v_cache, block_table, max_pages_per_seq, num_pages, page_size, nullptr,
                          nullptr, -1, false, scale, workspace, status_dev, out, lse, stream);
     if (rc == SFA_OK) g_last_launches = g.S <= decode_split_warps_per_block() ? 1 : 2;

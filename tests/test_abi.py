@@ -67,6 +67,7 @@ def test_fwd_host_validation(lib):
     assert _fwd(lib, sel=None) == 1
     assert _fwd(lib, total_k=100) == 1           # cu_k NULL but total_k != total_q
     assert _fwd(lib, ws_bytes=need - 1) == 3     # SFA_ERR_WORKSPACE_TOO_SMALL
+    assert _fwd(lib, ws=ctypes.c_void_p((1 << 20) + 16), ws_bytes=need) == 1  # workspace off a 256-byte boundary
     assert _fwd(lib, total_q=0, total_k=0) == 0   # nothing to do: OK without launching
 
 
@@ -92,6 +93,7 @@ def test_decode_host_validation(lib):
     assert call(bt=None) == 1
     assert call(wl=-5) == 1
     assert call(ws_bytes=need - 1) == 3
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16), ws_bytes=need) == 1  # workspace off a 256-byte boundary
     assert call(B=0) == 0
 
 
@@ -134,6 +136,7 @@ def test_bwd_host_validation(lib):
     assert _bwd(lib, dk=None) == 1
     assert _bwd(lib, wl=-3) == 1
     assert _bwd(lib, ws_bytes=16) == 3            # SFA_ERR_WORKSPACE_TOO_SMALL
+    assert _bwd(lib, ws=ctypes.c_void_p((1 << 20) + 16), ws_bytes=1 << 40) == 1  # workspace off a 256-byte boundary
     assert _bwd(lib, q=ctypes.c_void_p((1 << 20) + 8)) == 1  # misaligned
     # G 1 (128 tokens per tile) with topk 128 over 8192 blocks: a tile's union of up to 8192 blocks
     # (two copies, 64 KB) does not fit beside the dQ kernel's rings
@@ -180,6 +183,7 @@ def test_index_topk_host_validation(lib):
     assert call(n_local=-1) == 1
     assert call(out=None) == 1
     assert call(ws_bytes=8) == 3           # SFA_ERR_WORKSPACE_TOO_SMALL
+    assert call(ws=ctypes.c_void_p((1 << 20) + 16)) == 1  # workspace off a 256-byte boundary
     assert call(max_pages=1 << 16, page=32) == 2  # more than 2^20 positions per sequence
     assert call(B=0) == 0
 
