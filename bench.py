@@ -45,17 +45,28 @@ PREFILL_NAMES = {
 }
 PREFILL_CONFIGS = {1: W.config1, 2: W.config2, 3: W.config3, 4: W.config4}
 DECODE_NAME = "paged_topk_decode_b32: B32, Hq32/Hkv8, d128, L~U[16384,131072], page256, 2048 tok/(b,hk)"
+# the decode cases the profiling parts put in its place
+DECODE_PART_NAMES = {"all": DECODE_NAME,
+                     "prefill": "tiny decode: B2, Hq32/Hkv8, d128, L~U[1024,2048], page256, 256 tok/(b,hk)",
+                     "decode-small": "paged_topk_decode_b32 with L~U[4096,16384]"}
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the dominant kernel of
 # each stage, from one `ncu` capture of that kernel on its workload.  A figure holds only for the
 # kernel sources it was taken on: the digest of those files must match, else the bench reports null.
 TRAFFIC = {
+    # the six kernels of one call on nsa_long_96k (prep, plan, scatter, query-major, block-major, merge)
     "prefill_c4": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_fwd_inv_kernel.cu", "sfa_prep.cu", "sfa_device.cuh"],
-                   "sha256": None, "bytes": None},
-    "prefill_c2": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"], "sha256": None, "bytes": None},
+                   "sha256": "349ed79d2885f7e457fd58c88d2fb64d0ab88ef3f492c396adbf0b39212cc580",
+                   "bytes": 4193034752},
+    # the one kernel of a call on nsa_varlen_16k (the fused query-major kernel)
+    "prefill_c2": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
+                   "sha256": "f8b1585aed8bcf23a6056420f9d897e21a56bccd284f10646aaf0fb216cf7a05",
+                   "bytes": 138302208},
+    # one launch on paged_topk_decode_b32
     "decode_split_kernel": {"files": ["sfa_decode_kernel.cu", "sfa_device.cuh"],
-                            "sha256": None, "bytes": None},
+                            "sha256": "3c37939e4121865544ad7821a99c3ea8855117df49a3588bb15bf558a99db3f4",
+                            "bytes": 271037696},
 }
 
 
@@ -261,6 +272,8 @@ def run_gpu(args, rank, world, local_rank):
 
     if args.part == "decode-small":
         pc = W.small_config(2)
+    elif args.shrink > 1:
+        pc = PREFILL_CONFIGS[args.prefill_config](shrink=args.shrink)
     else:
         pc = PREFILL_CONFIGS[args.prefill_config]()
     P = W.upload_prefill(pc, dev)
@@ -368,7 +381,8 @@ def run_gpu(args, rank, world, local_rank):
     # branch (window 512 as in the NSA module example, causal) and the three-branch gated mix, on the
     # prefill workload's tensors; L2 flushed before every repetition, CUDA events on the stream.
     extras = None
-    if not args.no_extras and args.part != "decode-small":
+    want = (lambda name: True) if args.extras is None else (lambda name: name in args.extras.split(","))
+    if not args.no_extras and (args.part != "decode-small" or args.extras is not None):
         def timed(fn, reps=10):
             for _ in range(3):
                 fn()
@@ -386,7 +400,7 @@ def run_gpu(args, rank, world, local_rank):
         # ---- the other prefill configurations, each its whole public call (parity cases beside the step)
         cfg_lines = {}
         for n in sorted(PREFILL_CONFIGS):
-            if n == args.prefill_config:
+            if n == args.prefill_config or not want("prefill_configs"):
                 continue
             xc = PREFILL_CONFIGS[n]()
             xT = W.upload_prefill(xc, dev)
@@ -432,7 +446,7 @@ def run_gpu(args, rank, world, local_rank):
         # forward's out / lse and a seeded dout; 2.5x the forward's effective flops (five products
         # of the kept pairs instead of two).
         bwd_line = None
-        if bc.d == 128 and bc.bs == 64:
+        if bc.d == 128 and bc.bs == 64 and want("backward"):
             g_out = torch.randn(b_out.shape, generator=torch.Generator(device=dev).manual_seed(5), device=dev,
                                 dtype=torch.float32).to(torch.bfloat16)
             bdq, bdk, bdv = torch.empty_like(BP["q"]), torch.empty_like(BP["k"]), torch.empty_like(BP["v"])
@@ -453,74 +467,79 @@ def run_gpu(args, rank, world, local_rank):
                         "flops_note": "2.5x the forward's effective flops (S, dP, dQ, dK, dV over the kept pairs)"}
         # In-place KV-cache append on the decode workload's cache: one new token per sequence written at
         # position L - 1 (the decode query's own position); bytes = the new rows read + written.
-        akn = torch.randn((dc.B, 1, dc.Hkv, dc.d), device=dev).to(torch.bfloat16)
-        akv = torch.randn((dc.B, 1, dc.Hkv, dc.d), device=dev).to(torch.bfloat16)
-        apos = (D["cache_seqlens"] - 1).to(torch.int32)
+        append_line = index_line = fp8_line = nsa_line = None
+        if want("kv_append"):
+            akn = torch.randn((dc.B, 1, dc.Hkv, dc.d), device=dev).to(torch.bfloat16)
+            akv = torch.randn((dc.B, 1, dc.Hkv, dc.d), device=dev).to(torch.bfloat16)
+            apos = (D["cache_seqlens"] - 1).to(torch.int32)
 
-        def run_append():
-            sfa.kv_append(akn, akv, D["k_cache"], D["v_cache"], D["block_table"], apos, status=status)
+            def run_append():
+                sfa.kv_append(akn, akv, D["k_cache"], D["v_cache"], D["block_table"], apos, status=status)
 
-        a_ms = max_over_ranks([timed(run_append)], world, dev)[0]
-        a_bytes = 2 * 2 * dc.B * dc.Hkv * dc.d * 2
-        append_line = {"workload": f"B {dc.B}, 1 new token, Hkv {dc.Hkv}, d {dc.d}, page {dc.page}",
-                       "us": round(a_ms * 1e3, 2), "gbs": round(a_bytes / (a_ms * 1e-3) / 1e9, 1), "launches": 1,
-                       "note": "launch-latency bound (256 KB moved)"}
+            a_ms = max_over_ranks([timed(run_append)], world, dev)[0]
+            a_bytes = 2 * 2 * dc.B * dc.Hkv * dc.d * 2
+            append_line = {"workload": f"B {dc.B}, 1 new token, Hkv {dc.Hkv}, d {dc.d}, page {dc.page}",
+                           "us": round(a_ms * 1e3, 2), "gbs": round(a_bytes / (a_ms * 1e-3) / 1e9, 1), "launches": 1,
+                           "note": "launch-latency bound (256 KB moved)"}
         # Decode index producer (exact FP8 scores over every cached key, top-k positions) on the decode
         # workload: topk = its selection size, the last 128 positions forced as in its recipe.  Bytes = the
         # K rows it scans.  Guarded so a failure here only marks this line.
-        try:
-            itopk = int(dc.sel.shape[2])
-            isel = torch.empty((dc.B, dc.Hkv, itopk), dtype=torch.int32, device=dev)
-            istatus = torch.zeros(1, dtype=torch.int32, device=dev)
-            iws = torch.empty(sfa.index_topk_workspace_size(dc.B, dc.Hkv, D["block_table"].shape[1], dc.page)
-                              if hasattr(sfa, "index_topk_workspace_size") else 1, dtype=torch.uint8, device=dev)
+        if want("index_topk"):
+            try:
+                itopk = int(dc.sel.shape[2])
+                isel = torch.empty((dc.B, dc.Hkv, itopk), dtype=torch.int32, device=dev)
+                istatus = torch.zeros(1, dtype=torch.int32, device=dev)
+                iws = torch.empty(sfa.index_topk_workspace_size(dc.B, dc.Hkv, D["block_table"].shape[1], dc.page)
+                                  if hasattr(sfa, "index_topk_workspace_size") else 1, dtype=torch.uint8, device=dev)
 
-            def run_index():
-                sfa.index_topk(D["q"], D["k_cache"], D["block_table"], D["cache_seqlens"], itopk, n_local=128,
-                               out=isel, workspace=iws, status=istatus)
+                def run_index():
+                    sfa.index_topk(D["q"], D["k_cache"], D["block_table"], D["cache_seqlens"], itopk, n_local=128,
+                                   out=isel, workspace=iws, status=istatus)
 
-            i_ms = max_over_ranks([timed(run_index)], world, dev)[0]
-            i_bytes = int(np.asarray(dc.cache_seqlens, np.int64).sum()) * dc.Hkv * dc.d * 2
-            index_line = {"workload": f"decode workload, topk {itopk} (last 128 forced), every cached key scored",
-                          "ms": round(i_ms, 4), "gbs": round(i_bytes / (i_ms * 1e-3) / 1e9, 1),
-                          "frac": round(i_bytes / (i_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind,
-                          "launches": 1, "status": int(istatus.item())}
-        except Exception as exc:  # noqa: BLE001 - reported in the line, the rest of the bench goes on
-            index_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+                i_ms = max_over_ranks([timed(run_index)], world, dev)[0]
+                i_bytes = int(np.asarray(dc.cache_seqlens, np.int64).sum()) * dc.Hkv * dc.d * 2
+                index_line = {"workload": f"decode workload, topk {itopk} (last 128 forced), every cached key scored",
+                              "ms": round(i_ms, 4), "gbs": round(i_bytes / (i_ms * 1e-3) / 1e9, 1),
+                              "frac": round(i_bytes / (i_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind,
+                              "launches": 1, "status": int(istatus.item())}
+            except Exception as exc:  # noqa: BLE001 - reported in the line, the rest of the bench goes on
+                index_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
         # FP8 E4M3 caches (the decode workload quantized per (sequence, kv head) on the device): the same
         # gathered rows at one byte per value.
-        try:
-            fk, fv, fkd, fvd = W.quantize_cache_e4m3_device(dc, D)
-            f_out = torch.empty_like(dout)
-            f_lse = torch.empty_like(dlse)
+        if want("decode_fp8"):
+            try:
+                fk, fv, fkd, fvd = W.quantize_cache_e4m3_device(dc, D)
+                f_out = torch.empty_like(dout)
+                f_lse = torch.empty_like(dlse)
 
-            def run_fp8():
-                sfa.decode_fp8(D["q"], fk, fv, D["block_table"], D["cache_seqlens"], D["sel"], k_descale=fkd,
-                               v_descale=fvd, out=f_out, lse=f_lse, workspace=dws, status=status)
+                def run_fp8():
+                    sfa.decode_fp8(D["q"], fk, fv, D["block_table"], D["cache_seqlens"], D["sel"], k_descale=fkd,
+                                   v_descale=fvd, out=f_out, lse=f_lse, workspace=dws, status=status)
 
-            f_ms = max_over_ranks([timed(run_fp8, reps=20)], world, dev)[0]
-            f_bytes = gbytes // 2
-            fp8_line = {"workload": DECODE_NAME + ", caches E4M3 + per (sequence, kv head) descales",
-                        "ms": round(f_ms, 4), "gathered_bytes": int(f_bytes),
-                        "gbs": round(f_bytes / (f_ms * 1e-3) / 1e9, 1),
-                        "frac": round(f_bytes / (f_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind,
-                        "speedup_vs_bf16_cache": round(decode_ms / f_ms, 3), "launches": 1}
-            del fk, fv
-        except Exception as exc:  # noqa: BLE001 - reported in the line, the rest of the bench goes on
-            fp8_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
-        w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
-        m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
-        mix_bytes = 4 * bc.total_q * bc.Hq * bc.d * 2 + 3 * bc.total_q * bc.Hq * 4
-        extras = {
-            "window_branch": {"workload": "the prefill workload's q/k/v, causal, window (512, 0), no selection",
-                              "ms": round(w_ms, 4), "effective_tflops": round(wflops / (w_ms * 1e-3) / 1e12, 2),
-                              "frac": round(wflops / (w_ms * 1e-3) / 1e12 / tf_burst, 4),
-                              "peak_source": f"{peak_kind} bf16 burst", "launches": 1},
-            "gated_combine": {"workload": "3 branches of (total_q, Hq, d) bf16 + fp32 gates -> bf16",
-                              "ms": round(m_ms, 4), "gbs": round(mix_bytes / (m_ms * 1e-3) / 1e9, 1),
-                              "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
-        }
-        extras = {"nsa_branches": extras, "backward": bwd_line, "kv_append": append_line,
+                f_ms = max_over_ranks([timed(run_fp8, reps=20)], world, dev)[0]
+                f_bytes = gbytes // 2
+                fp8_line = {"workload": DECODE_PART_NAMES[args.part] + ", caches E4M3 + per (sequence, kv head) descales",
+                            "ms": round(f_ms, 4), "gathered_bytes": int(f_bytes),
+                            "gbs": round(f_bytes / (f_ms * 1e-3) / 1e9, 1),
+                            "frac": round(f_bytes / (f_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind,
+                            "speedup_vs_bf16_cache": round(decode_ms / f_ms, 3), "launches": 1}
+                del fk, fv
+            except Exception as exc:  # noqa: BLE001 - reported in the line, the rest of the bench goes on
+                fp8_line = {"error": f"{type(exc).__name__}: {exc}"[:300]}
+        if want("nsa_branches"):
+            w_ms = max_over_ranks([timed(run_window)], world, dev)[0]
+            m_ms = max_over_ranks([timed(run_mix)], world, dev)[0]
+            mix_bytes = 4 * bc.total_q * bc.Hq * bc.d * 2 + 3 * bc.total_q * bc.Hq * 4
+            nsa_line = {
+                "window_branch": {"workload": "the prefill workload's q/k/v, causal, window (512, 0), no selection",
+                                  "ms": round(w_ms, 4), "effective_tflops": round(wflops / (w_ms * 1e-3) / 1e12, 2),
+                                  "frac": round(wflops / (w_ms * 1e-3) / 1e12 / tf_burst, 4),
+                                  "peak_source": f"{peak_kind} bf16 burst", "launches": 1},
+                "gated_combine": {"workload": "3 branches of (total_q, Hq, d) bf16 + fp32 gates -> bf16",
+                                  "ms": round(m_ms, 4), "gbs": round(mix_bytes / (m_ms * 1e-3) / 1e9, 1),
+                                  "frac": round(mix_bytes / (m_ms * 1e-3) / 1e9 / hbm, 4), "peak_source": peak_kind},
+            }
+        extras = {"nsa_branches": nsa_line, "backward": bwd_line, "kv_append": append_line,
                   "index_topk": index_line, "prefill_configs": cfg_lines, "decode_fp8": fp8_line}
         if int(status.item()) != 0:
             raise RuntimeError(f"device status {int(status.item())} in the NSA branch runs")
@@ -650,6 +669,9 @@ def main():
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the lines beside the step: NSA window branch, gated mix, backward, KV append, "
                          "index top-k")
+    ap.add_argument("--extras", default=None,
+                    help="profiling aid: comma list of the lines beside the step to run (prefill_configs, "
+                         "nsa_branches, backward, kv_append, index_topk, decode_fp8); default all")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--part", default="all", choices=["all", "prefill", "decode-small"],
@@ -657,10 +679,15 @@ def main():
     ap.add_argument("--prefill-config", type=int, default=4, choices=[1, 2, 3, 4],
                     help="headline prefill workload (default 4, the largest single-GPU configuration); the "
                          "others are timed beside it")
+    ap.add_argument("--shrink", type=int, default=1,
+                    help="profiling aid: divide the headline NSA prefill workload's lengths by this (configs 2 "
+                         "and 4); the line then names the smaller workload")
     ap.add_argument("--traffic", type=int, default=None,
                     help="dram bytes (read+write) per attend launch from an ncu capture of this kernel version")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.shrink < 1 or (args.shrink > 1 and args.prefill_config not in (2, 4)):
+        ap.error("--shrink takes a positive factor and applies to prefill configs 2 and 4")
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -698,8 +725,10 @@ def main():
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) bf16 q/k/v, seeded NSA block selection; seeded paged decode inputs)",
-        "config": {"workload": PREFILL_NAMES[args.prefill_config] if args.part != "decode-small" else "small",
-                   "decode_workload": DECODE_NAME, "parallelism": f"independent x{world}",
+        "config": {"workload": (PREFILL_NAMES[args.prefill_config] + (f", lengths / {args.shrink}" if args.shrink > 1
+                                                                       else "")) if args.part != "decode-small"
+                   else "small",
+                   "decode_workload": DECODE_PART_NAMES[args.part], "parallelism": f"independent x{world}",
                    "l2": "flushed by a 256 MiB write before every step (outside the kernel events)",
                    "timing": "CUDA events per stage on the launch stream, mean over steps, max over ranks"},
         "prefill": {"ms": round(r["prefill_ms"], 4), "effective_gflop": round(r["flops"] / 1e9, 2),

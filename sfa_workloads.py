@@ -352,9 +352,11 @@ def config1():
     return make_nsa_prefill(1, [256], 4, 1, 64, 32, 4, init_blocks=1, local_blocks=1, name="tiny_256_d64")
 
 
-def config2(parallel_values=False):
-    """Varlen NSA: lengths [8192, 4096, 2048, 2048], Hq16/Hkv4, d128, bs64, topk16, init 1, local 2."""
-    return make_nsa_prefill(2, [8192, 4096, 2048, 2048], 16, 4, 128, 64, 16, 1, 2, name="nsa_varlen_16k",
+def config2(parallel_values=False, shrink=1):
+    """Varlen NSA: lengths [8192, 4096, 2048, 2048], Hq16/Hkv4, d128, bs64, topk16, init 1, local 2.
+    shrink > 1 divides the lengths (a smaller case of the same kernels, for profiler captures)."""
+    return make_nsa_prefill(2, [n // shrink for n in (8192, 4096, 2048, 2048)], 16, 4, 128, 64, 16, 1, 2,
+                            name="nsa_varlen_16k" if shrink == 1 else f"nsa_varlen_16k/{shrink}",
                             parallel_values=parallel_values)
 
 
@@ -363,9 +365,11 @@ def config3():
     return make_window_prefill(3, 2, 1024, 4096, 32, 8, 128, 64, 1024, 0, causal=1, name="dense_window_1k_4k")
 
 
-def config4(parallel_values=False):
-    """Long context: lengths [65536, 32768], Hq=Hkv=4, d128, bs64, topk16, init 1, local 2."""
-    return make_nsa_prefill(4, [65536, 32768], 4, 4, 128, 64, 16, 1, 2, name="nsa_long_96k",
+def config4(parallel_values=False, shrink=1):
+    """Long context: lengths [65536, 32768], Hq=Hkv=4, d128, bs64, topk16, init 1, local 2.
+    shrink > 1 divides the lengths (a smaller case of the same kernels, for profiler captures)."""
+    return make_nsa_prefill(4, [n // shrink for n in (65536, 32768)], 4, 4, 128, 64, 16, 1, 2,
+                            name="nsa_long_96k" if shrink == 1 else f"nsa_long_96k/{shrink}",
                             parallel_values=parallel_values)
 
 
