@@ -168,6 +168,18 @@ class ClockSampler:
         except Exception:
             self.proc = None
 
+    def wait_first(self, limit_s=3.0):
+        """Block until nvidia-smi has written its first sample (it takes a few hundred ms to start), so a
+        short timed region still falls between samples."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while time.time() - t0 < limit_s and self.proc.poll() is None:
+            self.f.flush()
+            if os.path.getsize(self.path) > 0:
+                return
+            time.sleep(0.02)
+
     def stop(self):
         if self.proc is None:
             return None
@@ -339,17 +351,19 @@ def run_gpu(args, rank, world, local_rank):
             if i is not None:
                 ev[i][s + 1].record(stream)
 
+    # clocks: the sampler starts before the warm-up and has its first sample before the timed region
+    import tempfile
+    sampler = ClockSampler(physical_gpu_index(local_rank), os.path.join(tempfile.gettempdir(),
+                                                                        f"sfa_bench_clocks_{os.getpid()}.csv")) \
+        if rank == 0 else None
     for _ in range(Wm):
         step()
     torch.cuda.synchronize()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during warm-up")
     launches[0] = 0
-
-    import tempfile
-    sampler = ClockSampler(physical_gpu_index(local_rank), os.path.join(tempfile.gettempdir(),
-                                                                        f"sfa_bench_clocks_{os.getpid()}.csv")) \
-        if rank == 0 else None
+    if sampler:
+        sampler.wait_first()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
             const InvItem *item = &meta->slot[it];
             const int4 rec = item->rec;
             if (rec.w < 0) break;  // item j+1 is past the end too, so both groups get a marker
-            const int hk = rec.x % p.Hkv, b = rec.x / p.Hkv;
+            const int hk = rec.x % p.Hkv;
             // K/V block
             if (j >= kLoadStages) ok = warp_all_ok(mbar_wait(&meta->kv_empty[sl], ph, abort_flag, p.status));
             if (!ok) break;
@@ -454,7 +454,7 @@ constexpr int kMergeWarps = 8;
 constexpr int kMergeBatch = 8;  // partials each lane loads before folding them in
 
 template <int D>
-__global__ void __launch_bounds__(32 * kMergeWarps) fwd_merge_kernel(const FwdAttendParams p)
+__global__ void __launch_bounds__(32 * kMergeWarps, 3) fwd_merge_kernel(const FwdAttendParams p)
 {
     constexpr int kChunks = D / 8;       // 16-byte chunks of a row
     constexpr int kSplit = 32 / kChunks; // lanes sharing a chunk, each over every kSplit-th partial
