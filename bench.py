@@ -57,8 +57,8 @@ DECODE_PART_NAMES = {"all": DECODE_NAME,
 TRAFFIC = {
     # the six kernels of one call on nsa_long_96k (prep, plan, scatter, query-major, block-major, merge)
     "prefill_c4": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_fwd_inv_kernel.cu", "sfa_prep.cu", "sfa_device.cuh"],
-                   "sha256": "349ed79d2885f7e457fd58c88d2fb64d0ab88ef3f492c396adbf0b39212cc580",
-                   "bytes": 4193034752},
+                   "sha256": "baccbf83c3058d4d81ec203f53a44b001529d2b41dca806e66ddeaa100bdbbf1",
+                   "bytes": 4200355328},
     # the one kernel of a call on nsa_varlen_16k (the fused query-major kernel)
     "prefill_c2": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
                    "sha256": "f8b1585aed8bcf23a6056420f9d897e21a56bccd284f10646aaf0fb216cf7a05",
