@@ -114,16 +114,14 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
     if (g.inv) {
         const size_t gb = (size_t)g.groups * g.nblk_max;
         g.cap_items = ((int64_t)total_q * Hkv * topk + g.Tq - 1) / g.Tq + (int64_t)gb;
-        g.off_zero = off;  // ctrl, group statistics, block histograms and cursors: cleared per call
+        g.off_zero = off;  // ctrl and group statistics: cleared per call
         g.off_ctrl = off;
         off = align_up(off + sizeof(InvCtrl));
         g.off_gstat = off;
         off = align_up(off + (size_t)g.groups * sizeof(GroupStat));
-        g.off_gcount = off;
-        off = align_up(off + gb * 4);
-        g.off_gcursor = off;
-        off = align_up(off + gb * 4);
         g.zero_bytes = off - g.off_zero;
+        g.off_tcount = off;  // written whole by the prep kernel
+        off = align_up(off + (size_t)g.tiles * g.nblk_max * 4);
         g.off_gfirst = off;
         off = align_up(off + gb * 4);
         g.off_items = off;
@@ -221,7 +219,7 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     p.uni = reinterpret_cast<int32_t *>(w + g.off_union);
     p.W = g.W;
     p.gstat = g.inv ? reinterpret_cast<GroupStat *>(w + g.off_gstat) : nullptr;
-    p.gcount = g.inv ? reinterpret_cast<int32_t *>(w + g.off_gcount) : nullptr;
+    p.tcount = g.inv ? reinterpret_cast<int32_t *>(w + g.off_tcount) : nullptr;
     p.status = status;
     if (launch_fwd_prep(g, p, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
@@ -229,7 +227,7 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     FwdPlanParams pl{};
     pl.ucnt = p.ucnt;
     pl.gstat = p.gstat;
-    pl.gcount = p.gcount;
+    pl.tcount = p.tcount;
     pl.gfirst = reinterpret_cast<int32_t *>(w + g.off_gfirst);
     pl.batch = g.batch;
     pl.Hkv = g.Hkv;
@@ -248,7 +246,7 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     sc.cnt = p.cnt;
     sc.ucnt = p.ucnt;
     sc.gfirst = pl.gfirst;
-    sc.gcursor = reinterpret_cast<int32_t *>(w + g.off_gcursor);
+    sc.tcount = p.tcount;
     sc.batch = g.batch;
     sc.Hkv = g.Hkv;
     sc.topk = g.topk;

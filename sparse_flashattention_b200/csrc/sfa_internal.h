@@ -31,7 +31,7 @@ struct FwdGeom {
     int64_t cap_items;
     size_t off_sel_c, off_cnt, off_ucnt, off_union, off_tilectr;
     size_t off_zero, zero_bytes;  // the part of the workspace cleared before every prep
-    size_t off_ctrl, off_gstat, off_gcount, off_gcursor, off_gfirst, off_items, off_pml, off_po;
+    size_t off_ctrl, off_gstat, off_tcount, off_gfirst, off_items, off_pml, off_po;
     size_t bytes;
 };
 
@@ -57,17 +57,18 @@ struct FwdPrepParams {
     int32_t *tile_counter;  // cleared here (two ints) for the attend kernel
     int batch, Hkv, topk, bs, causal, wl, wr, Tq, nqt, umax, max_sq, nblk_max;
     int32_t *sel_c, *cnt, *ucnt, *uni;
-    // block-major statistics (nullptr when the schedule is off)
+    // block-major statistics (nullptr when the schedule is off): per group, and per tile the number of
+    // its tokens that selected each block ([tiles][nblk_max])
     int W;
     GroupStat *gstat;
-    int32_t *gcount;
+    int32_t *tcount;
     int32_t *status;
 };
 
 struct FwdPlanParams {
     int32_t *ucnt;
     const GroupStat *gstat;
-    const int32_t *gcount;
+    int32_t *tcount;  // per-tile counts in; for block-major windows, each tile's first list position out
     int32_t *gfirst;
     int batch, Hkv, Tq, nqt, W, nblk_max;
     const int32_t *cu_q, *cu_k;
@@ -77,7 +78,7 @@ struct FwdPlanParams {
 
 struct FwdScatterParams {
     const int32_t *cu_q, *sel_c, *cnt, *ucnt, *gfirst;
-    int32_t *gcursor;
+    const int32_t *tcount;  // each tile's first position in every block's token list
     int batch, Hkv, topk, Tq, nqt, W, nblk_max;
     InvItem *items;
 };

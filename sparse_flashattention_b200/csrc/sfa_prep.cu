@@ -70,21 +70,6 @@ __device__ int compact_bitmap(const uint32_t *bm, int words, int32_t *dst, int *
     return total;
 }
 
-// One warp-wide op on per-lane keys (-1 = no key): lanes holding the same key are counted
-// together and only the lowest of them touches shared memory.  Returns, for each lane, the
-// first value it may use (the leader's old value plus the lane's rank among equal keys).
-__device__ __forceinline__ int warp_aggregated_add(int *counters, int key)
-{
-    const int lane = threadIdx.x & 31;
-    const unsigned m = __match_any_sync(0xffffffffu, key);
-    const int leader = __ffs(m) - 1;
-    const int rank = __popc(m & ((1u << lane) - 1));
-    int base = 0;
-    if (lane == leader && key >= 0) base = atomicAdd(&counters[key], __popc(m));
-    base = __shfl_sync(0xffffffffu, base, leader);
-    return base + rank;
-}
-
 __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
 {
     extern __shared__ uint32_t prep_smem[];
@@ -111,14 +96,20 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
     }
     const int words = (p.nblk_max + 31) / 32;
     uint32_t *bm = prep_smem;
-    int *raw = reinterpret_cast<int *>(prep_smem + words);  // [Tq][topk] selections as given
-    int *lists = raw + p.Tq * p.topk;                         // [topk][kPrepThreads] canonical
+    // [Tq][rs] selections as given: an odd row stride rs keeps a warp's 32 rows on 32 banks when each
+    // thread walks its own row
+    const int rs = p.topk | 1;
+    int *raw = reinterpret_cast<int *>(prep_smem + words);
+    int *lists = raw + p.Tq * rs;                             // [topk][kPrepThreads] canonical
+    int *hist = p.tcount ? lists + p.topk * kPrepThreads : nullptr;  // [nblk_max] this tile's tokens per block
     for (int w = threadIdx.x; w < words; w += kPrepThreads) bm[w] = 0;
+    if (hist)
+        for (int s = threadIdx.x; s < p.nblk_max; s += kPrepThreads) hist[s] = 0;
     const int64_t row0 = ((int64_t)(q0 + tok0) * p.Hkv + hk) * p.topk;
     const int64_t tok_stride = (int64_t)p.Hkv * p.topk;
     for (int e = threadIdx.x; e < ntok * p.topk; e += kPrepThreads) {
         const int tt = e / p.topk;
-        raw[e] = p.sel[row0 + tt * tok_stride + (e - tt * p.topk)];
+        raw[tt * rs + (e - tt * p.topk)] = p.sel[row0 + tt * tok_stride + (e - tt * p.topk)];
     }
     __syncthreads();
 
@@ -133,7 +124,7 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
         if (p.wr >= 0) hi = min(hi, i + delta + p.wr);
         bool bad = false;
         // canonical list into column tt of lists ([slot][kPrepThreads])
-        const int *r = raw + tt * p.topk;
+        const int *r = raw + tt * rs;
         if (p.topk <= 16) n = canon_list_regs<16>(r, p.topk, nblk, p.bs, sk, lo, hi, lists + tt, kPrepThreads, bad);
         else if (p.topk <= 32) n = canon_list_regs<32>(r, p.topk, nblk, p.bs, sk, lo, hi, lists + tt, kPrepThreads, bad);
         else n = canon_list_insert(r, p.topk, nblk, p.bs, sk, lo, hi, lists + tt, kPrepThreads, bad);
@@ -142,18 +133,18 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
         if (bad && p.status) atomicOr(p.status, SFA_DEV_BAD_INDEX);
     }
     // Union bitmap: lanes that hold the same block set its bit once.  With the block-major
-    // schedule on, also count each block's selecting tokens for the window's group.
+    // schedule on, also count each block's selecting tokens of this tile (shared memory; the tile's
+    // counts then go out whole, so no counter is shared between CTAs).
     const int grp = p.gstat ? ((tok0 / p.W) * p.batch + b) * p.Hkv + hk : 0;
     {
         const int maxn = __reduce_max_sync(0xffffffffu, n);
         const int lane = threadIdx.x & 31;
-        int32_t *gc = p.gstat ? p.gcount + (int64_t)grp * p.nblk_max : nullptr;
         for (int e = 0; e < maxn; ++e) {
             const int s = e < n ? lists[e * kPrepThreads + tt] : -1;
             const unsigned m = __match_any_sync(0xffffffffu, s);
             if (s >= 0 && lane == __ffs(m) - 1) {
                 atomicOr(&bm[s >> 5], 1u << (s & 31));
-                if (gc) atomicAdd(&gc[s], __popc(m));
+                if (hist) atomicAdd(&hist[s], __popc(m));
             }
         }
         if (p.gstat) {
@@ -163,12 +154,14 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
     }
     __syncthreads();  // every thread is done reading raw
     if (tt < ntok)
-        for (int e = 0; e < p.topk; ++e) raw[tt * p.topk + e] = e < n ? lists[e * kPrepThreads + tt] : -1;
+        for (int e = 0; e < p.topk; ++e) raw[tt * rs + e] = e < n ? lists[e * kPrepThreads + tt] : -1;
     __syncthreads();
     for (int e = threadIdx.x; e < ntok * p.topk; e += kPrepThreads) {
         const int t2 = e / p.topk;
-        p.sel_c[row0 + t2 * tok_stride + (e - t2 * p.topk)] = raw[e];
+        p.sel_c[row0 + t2 * tok_stride + (e - t2 * p.topk)] = raw[t2 * rs + (e - t2 * p.topk)];
     }
+    if (hist)
+        for (int s = threadIdx.x; s < p.nblk_max; s += kPrepThreads) p.tcount[(int64_t)tile * p.nblk_max + s] = hist[s];
     const int total = compact_bitmap<kPrepThreads>(bm, (nblk + 31) / 32, p.uni + (int64_t)tile * p.umax,
                                                    scan_scratch);
     if (threadIdx.x == 0) {
@@ -180,38 +173,21 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
 
 constexpr int kInvThreads = 256;
 
-// Exclusive scan of v[0..n) in place (all threads); returns the total.
-__device__ int block_scan_array(int *v, int n, int *scratch)
-{
-    const int per = (n + kInvThreads - 1) / kInvThreads;
-    const int i0 = min(n, (int)threadIdx.x * per), i1 = min(n, i0 + per);
-    int c = 0;
-    for (int i = i0; i < i1; ++i) c += v[i];
-    int pos;
-    const int total = block_exclusive_scan<kInvThreads>(c, scratch, pos);
-    for (int i = i0; i < i1; ++i) {
-        const int x = v[i];
-        v[i] = pos;
-        pos += x;
-    }
-    __syncthreads();
-    return total;
-}
-
-// Block-major plan, one CTA per (window, sequence, kv head) group.  The window stays with the
-// query-major kernel unless the union of its query tiles' blocks is over 4x its selected
-// blocks (a block-major item moves several times the memory of a query-major tile per selected
-// row-block: its bf16 partial is written and read back and its Q rows are gathered).  For a
-// block-major window: mark its tiles (ucnt = -1), cut each selected block's token list into
-// items of at most Tq tokens, reserve them, and write their records (tokens come from the
-// scatter kernel).
+// Block-major plan, one CTA per (window, sequence, kv head) group and run of kInvThreads blocks.
+// The window stays with the query-major kernel unless the union of its query tiles' blocks is
+// over 4x its selected blocks (a block-major item moves several times the memory of a query-major
+// tile per selected row-block: its bf16 partial is written and read back and its Q rows are
+// gathered).  For a block-major window: mark its tiles (ucnt = -1); per block (one thread each)
+// add up the window's tiles' counts, leaving in each tile's place its first position in the
+// block's list; cut each block's list into items of at most Tq tokens, reserve the CTA's items,
+// and write their records (tokens come from the scatter kernel).
 __global__ void __launch_bounds__(kInvThreads) fwd_plan_kernel(FwdPlanParams p)
 {
-    extern __shared__ int plan_smem[];
     __shared__ int scan_scratch[32];
     __shared__ int item_base;
     grid_dep_wait();
     const int g = blockIdx.x;
+    const int s = blockIdx.y * kInvThreads + threadIdx.x;  // this thread's block
     const int hk = g % p.Hkv;
     const int b = (g / p.Hkv) % p.batch;
     const int w = g / (p.Hkv * p.batch);
@@ -222,32 +198,49 @@ __global__ void __launch_bounds__(kInvThreads) fwd_plan_kernel(FwdPlanParams p)
     if (st.uni <= 4ull * st.useful) return;  // the query-major kernel keeps this window
     const int nt = min(p.W, sq - t0);
     const int qt0 = t0 / p.Tq, qt1 = (t0 + nt - 1) / p.Tq;
-    for (int qt = qt0 + threadIdx.x; qt <= qt1; qt += kInvThreads)
-        p.ucnt[((p.nqt - 1 - qt) * p.batch + b) * p.Hkv + hk] = -1;
+    if (blockIdx.y == 0)
+        for (int qt = qt0 + threadIdx.x; qt <= qt1; qt += kInvThreads)
+            p.ucnt[((p.nqt - 1 - qt) * p.batch + b) * p.Hkv + hk] = -1;
 
-    const int32_t *count = p.gcount + (int64_t)g * p.nblk_max;
-    int *first = plan_smem;  // first item of each block, local to the group
-    for (int s = threadIdx.x; s < p.nblk_max; s += kInvThreads) first[s] = (count[s] + p.Tq - 1) / p.Tq;
-    __syncthreads();
-    const int nitems = block_scan_array(first, p.nblk_max, scan_scratch);
+    // The block's token count over the window's tiles, and in place of each tile's count the tile's
+    // first position in the block's list (tiles in query order; eight tiles' counts loaded at once).
+    int c = 0;
+    if (s < p.nblk_max) {
+        for (int q8 = qt0; q8 <= qt1; q8 += 8) {
+            int v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                v[i] = q8 + i <= qt1 ? p.tcount[(int64_t)(((p.nqt - 1 - (q8 + i)) * p.batch + b) * p.Hkv + hk) * p.nblk_max + s]
+                                     : 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (q8 + i <= qt1) {
+                    p.tcount[(int64_t)(((p.nqt - 1 - (q8 + i)) * p.batch + b) * p.Hkv + hk) * p.nblk_max + s] = c;
+                    c += v[i];
+                }
+        }
+    }
+    // this CTA's items: reserved together, each block's consecutive
+    int pos;
+    const int nitems = block_exclusive_scan<kInvThreads>((c + p.Tq - 1) / p.Tq, scan_scratch, pos);
     if (threadIdx.x == 0) item_base = atomicAdd(&p.ctrl->item_total, nitems);
     __syncthreads();
-    int32_t *gfirst = p.gfirst + (int64_t)g * p.nblk_max;
-    const int k0 = p.cu_k[b];
-    for (int s = threadIdx.x; s < p.nblk_max; s += kInvThreads) {
-        const int c = count[s];
-        const int i0 = item_base + first[s];
-        gfirst[s] = i0;
+    if (s < p.nblk_max) {
+        const int i0 = item_base + pos;
+        p.gfirst[(int64_t)g * p.nblk_max + s] = i0;
+        const int k0 = p.cu_k[b];
         for (int i = 0; i * p.Tq < c; ++i)
             p.items[i0 + i].rec = make_int4(b * p.Hkv + hk, s, k0, min(p.Tq, c - i * p.Tq));
     }
 }
 
 // Block-major token lists, one CTA per query tile of a block-major window: every (token, block)
-// of the tile's canonical selections takes the next position in its block's list, which names
-// the item (position / Tq) and the slot in it.
+// of the tile's canonical selections takes the next position in its block's list, counted on from
+// the tile's first position there (the plan's scan of the tiles' counts; shared-memory atomics, no
+// counter shared between CTAs), which names the item (position / Tq) and the slot in it.
 __global__ void __launch_bounds__(kPrepThreads) fwd_scatter_kernel(FwdScatterParams p)
 {
+    extern __shared__ int scatter_smem[];
     grid_dep_wait();
     const int tile = blockIdx.x;
     if (p.ucnt[tile] != -1) return;
@@ -259,18 +252,21 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_scatter_kernel(FwdScatterPar
     const int tok0 = qt * p.Tq;
     const int ntok = min(p.Tq, sq - tok0);
     const int grp = ((tok0 / p.W) * p.batch + b) * p.Hkv + hk;
-    int32_t *cursor = p.gcursor + (int64_t)grp * p.nblk_max;
-    const int32_t *first = p.gfirst + (int64_t)grp * p.nblk_max;
+    int *pos_s = scatter_smem;                // next position of each block's list for this tile
+    int *first_s = scatter_smem + p.nblk_max; // first item of each block
+    for (int s = threadIdx.x; s < p.nblk_max; s += kPrepThreads) {
+        pos_s[s] = p.tcount[(int64_t)tile * p.nblk_max + s];
+        first_s[s] = p.gfirst[(int64_t)grp * p.nblk_max + s];
+    }
+    __syncthreads();
     const int tt = threadIdx.x;
     const int64_t t = (int64_t)q0 + tok0 + tt;
     const int n = tt < ntok ? p.cnt[t * p.Hkv + hk] : 0;
     const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
-    const int maxn = __reduce_max_sync(0xffffffffu, n);
-    for (int e = 0; e < maxn; ++e) {
-        const int s = e < n ? row[e] : -1;
-        // cursor is global here; warp_aggregated_add works on any address space
-        const int pos = warp_aggregated_add(cursor, s);
-        if (s >= 0) p.items[first[s] + pos / p.Tq].tok[pos % p.Tq] = (int)(t << 7) | e;
+    for (int e = 0; e < n; ++e) {
+        const int s = row[e];
+        const int pos = atomicAdd(&pos_s[s], 1);
+        p.items[first_s[s] + pos / p.Tq].tok[pos % p.Tq] = (int)(t << 7) | e;
     }
 }
 
@@ -317,7 +313,8 @@ __global__ void __launch_bounds__(kDecPrepThreads) decode_prep_kernel(DecPrepPar
 cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream_t st)
 {
     const size_t words = (size_t)(g.nblk_max + 31) / 32;
-    const size_t smem = words * 4 + (size_t)g.Tq * g.topk * 4 + (size_t)g.topk * kPrepThreads * 4;
+    const size_t smem = words * 4 + (size_t)g.Tq * (g.topk | 1) * 4 + (size_t)g.topk * kPrepThreads * 4 +
+                        (p.tcount ? (size_t)g.nblk_max * 4 : 0);
     if (smem > 48 * 1024) {
         const cudaError_t e = ensure_smem_for(fwd_prep_kernel, smem);
         if (e != cudaSuccess) return e;
@@ -328,13 +325,18 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
 
 cudaError_t launch_fwd_plan(const FwdGeom &g, const FwdPlanParams &p, cudaStream_t st)
 {
-    const size_t smem = (size_t)g.nblk_max * 4;
-    return launch_kernel(fwd_plan_kernel, dim3(g.groups), dim3(kInvThreads), smem, st, true, p);
+    const dim3 grid(g.groups, (g.nblk_max + kInvThreads - 1) / kInvThreads);
+    return launch_kernel(fwd_plan_kernel, grid, dim3(kInvThreads), 0, st, true, p);
 }
 
 cudaError_t launch_fwd_scatter(const FwdGeom &g, const FwdScatterParams &p, cudaStream_t st)
 {
-    return launch_kernel(fwd_scatter_kernel, dim3(g.tiles), dim3(kPrepThreads), 0, st, true, p);
+    const size_t smem = (size_t)g.nblk_max * 8;
+    if (smem > 48 * 1024) {
+        const cudaError_t e = ensure_smem_for(fwd_scatter_kernel, smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_kernel(fwd_scatter_kernel, dim3(g.tiles), dim3(kPrepThreads), smem, st, true, p);
 }
 
 cudaError_t launch_decode_prep(const DecGeom &g, const DecPrepParams &p, cudaStream_t st)
