@@ -124,6 +124,12 @@ int fwd_geometry(int batch, int max_sq, int max_sk, int total_q, int Hq, int Hkv
         off = align_up(off + (size_t)g.tiles * g.nblk_max * 4);
         g.off_gfirst = off;
         off = align_up(off + gb * 4);
+        g.off_duni = off;
+        off = align_up(off + (size_t)g.tiles * kDenseMax * 4);
+        g.off_dcnt = off;
+        off = align_up(off + (size_t)g.tiles * 4);
+        g.off_dsel = off;  // dsel then dmask
+        off = align_up(off + (size_t)2 * total_q * Hkv * 4);
         g.off_items = off;
         off = align_up(off + (size_t)g.cap_items * sizeof(InvItem));
         g.off_pml = off;
@@ -213,6 +219,7 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     p.umax = g.umax;
     p.max_sq = g.max_sq;
     p.nblk_max = g.nblk_max;
+    p.total_q = g.total_q;
     p.sel_c = reinterpret_cast<int32_t *>(w + g.off_sel_c);
     p.cnt = reinterpret_cast<int32_t *>(w + g.off_cnt);
     p.ucnt = reinterpret_cast<int32_t *>(w + g.off_ucnt);
@@ -220,6 +227,11 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     p.W = g.W;
     p.gstat = g.inv ? reinterpret_cast<GroupStat *>(w + g.off_gstat) : nullptr;
     p.tcount = g.inv ? reinterpret_cast<int32_t *>(w + g.off_tcount) : nullptr;
+    // dense blocks of block-major tiles go to the pipelined query-major kernel (not the one-tile one)
+    const bool dense = g.inv && g.topk <= 32 && fwd_pipe_fits(g, kPipePrep);
+    p.duni = dense ? reinterpret_cast<int32_t *>(w + g.off_duni) : nullptr;
+    p.dcnt = dense ? reinterpret_cast<int32_t *>(w + g.off_dcnt) : nullptr;
+    p.dsel = dense ? reinterpret_cast<uint32_t *>(w + g.off_dsel) : nullptr;
     p.status = status;
     if (launch_fwd_prep(g, p, st) != cudaSuccess) return SFA_ERR_CUDA;
     if (!g.inv) return SFA_OK;
@@ -247,6 +259,7 @@ int fwd_prep_impl(const FwdGeom &g, const int32_t *cu_q, const int32_t *cu_k, co
     sc.ucnt = p.ucnt;
     sc.gfirst = pl.gfirst;
     sc.tcount = p.tcount;
+    sc.dmask = dense ? p.dsel + (size_t)g.total_q * g.Hkv : nullptr;
     sc.batch = g.batch;
     sc.Hkv = g.Hkv;
     sc.topk = g.topk;
@@ -304,6 +317,13 @@ int fwd_attend_impl(const FwdGeom &g, const void *q, const void *k, const void *
     p.bs = g.bs;
     p.max_sq = g.max_sq;
     p.nblk_max = g.nblk_max;
+    if (g.inv && g.topk <= 32 && pipe) {  // the dense blocks of block-major tiles (see the prep)
+        const uint8_t *wd = static_cast<const uint8_t *>(ws);
+        p.duni = reinterpret_cast<const int32_t *>(wd + g.off_duni);
+        p.dcnt = reinterpret_cast<const int32_t *>(wd + g.off_dcnt);
+        p.dsel = reinterpret_cast<const uint32_t *>(wd + g.off_dsel);
+        p.dmask = p.dsel + (size_t)g.total_q * g.Hkv;
+    }
     if (fused && cudaMemsetAsync(p.tile_counter, 0, 2 * sizeof(int32_t), st) != cudaSuccess) return SFA_ERR_CUDA;
     if ((pipe ? launch_fwd_attend_pipe(g, p, fused ? kPipeFused : kPipePrep, tq, tk, tv, st)
               : launch_fwd_attend(g, p, tq, tk, tv, st)) !=

@@ -476,30 +476,55 @@ __global__ void __launch_bounds__(32 * kMergeWarps, 3) fwd_merge_kernel(const Fw
     const int nrows = ntok * p.G;
     // the selection counts of this warp's rows (row e = warp + kMergeWarps * i, i = lane), read at once
     const int e_l = warp + kMergeWarps * lane;
-    const int cnt_l = e_l < nrows ? __ldg(&p.cnt[((int64_t)q0 + tok0 + e_l / p.G) * p.Hkv + hk]) : 0;
+    const int64_t tl_l = (int64_t)q0 + tok0 + e_l / p.G;
+    const int cnt_l = e_l < nrows ? __ldg(&p.cnt[tl_l * p.Hkv + hk]) : 0;
+    // entries of dense blocks (their partial is the query-major kernel's, in out / lse)
+    const uint32_t dm_l = e_l < nrows && p.dmask ? __ldg(&p.dmask[tl_l * p.Hkv + hk]) : 0u;
     const int c = lane % kChunks, kq = lane / kChunks;
     for (int i = 0; warp + kMergeWarps * i < nrows; ++i) {
         const int e = warp + kMergeWarps * i;
         const int cnt = __shfl_sync(0xffffffffu, cnt_l, i);
-        if (cnt == 0) continue;  // a row that keeps no key: written by the query-major kernel
+        const uint32_t dm = __shfl_sync(0xffffffffu, dm_l, i);
+        // a row that keeps no key, or keeps only dense blocks: the query-major kernel wrote it
+        if (cnt == __popc(dm)) continue;
         const int tt = e / p.G, g = e - tt * p.G;
         const int64_t t = (int64_t)q0 + tok0 + tt;
         const int h = hk * p.G + g;
         const int64_t base = (t * p.Hq + h) * p.topk;
         // Lane (kq, c) merges partials kq, kq + kSplit, ... of chunk c: a batch of their (m, l) and
         // 16-byte chunks is loaded at once, then folded into a running (max, sum, weighted chunk).
+        // With dense blocks, lanes kq = 0 start from the query-major partial: normalised in out, its
+        // log-sum-exp in lse (as (m, l) = (lse in base 2, 1)).
         float Mx = -INFINITY, Ls = 0.f, acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        // (its two loads go out with the first batch of partials, not ahead of them)
+        bool qdone = !(dm != 0u && kq == 0);
         for (int k0 = kq; k0 < cnt; k0 += kSplit * kMergeBatch) {
             float2 ml[kMergeBatch];
             uint4 v[kMergeBatch];
 #pragma unroll
             for (int i = 0; i < kMergeBatch; ++i) {
                 const int k = k0 + i * kSplit;
-                ml[i] = k < cnt ? __ldcs(&p.pml[base + k]) : make_float2(-INFINITY, 0.f);
-                v[i] = k < cnt ? __ldcs(reinterpret_cast<const uint4 *>(p.po + (base + k) * D) + c)
-                               : make_uint4(0u, 0u, 0u, 0u);
+                const bool use = k < cnt && !((dm >> k) & 1u);
+                ml[i] = use ? __ldcs(&p.pml[base + k]) : make_float2(-INFINITY, 0.f);
+                v[i] = use ? __ldcs(reinterpret_cast<const uint4 *>(p.po + (base + k) * D) + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+            if (!qdone) {  // the query-major partial as (m, l) = (lse in base 2, 1), normalised chunk vq
+                qdone = true;
+                const float lq = p.lse[(int64_t)h * p.total_q + t];
+                const uint4 vq = reinterpret_cast<const uint4 *>(p.out + (t * p.Hq + h) * D)[c];
+                if (lq != -INFINITY) {
+                    Mx = lq * 1.4426950408889634f;
+                    Ls = 1.f;
+                    const uint32_t vv[4] = {vq.x, vq.y, vq.z, vq.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&vv[e]));
+                        acc[2 * e] = x.x;
+                        acc[2 * e + 1] = x.y;
+                    }
+                }
             }
             float bm = Mx;
 #pragma unroll

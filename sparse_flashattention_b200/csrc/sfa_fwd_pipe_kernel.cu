@@ -57,6 +57,8 @@ struct QCfg {
 struct TileInfo {
     int done;  // no tile left: every role leaves its loop
     int nU;    // union blocks (< 0: a block-major tile, whose rows another kernel computes)
+    int dense; // a block-major tile whose dense blocks run here: the union is those blocks, a row's
+               // selection of them is a bit mask, and out / lse receive a partial the merge combines
     int b, hk, q0, sq, k0, sk, tok0, ntok;
     int blo;   // window mode: the union is blocks blo, blo+1, ..., blo+nU-1
 };
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kQThreads, 2)
             const int k0 = p.cu_k[b], sk = p.cu_k[b + 1] - k0;
             const int tok0 = qt * p.Tq;
             const int ntok = min(p.Tq, sq - tok0);
-            int nU, blo = 0;
+            int nU, blo = 0, dense = 0;
             if constexpr (WIN) {
                 // Rows' key windows [lo(i), hi(i)] move right with i, so the tile's blocks are the
                 // contiguous range from the first row's lo to the last row's hi.
@@ -292,11 +294,18 @@ __global__ void __launch_bounds__(kQThreads, 2)
                 nU = total;
             } else {
                 nU = p.ucnt[tile];
-                for (int i = lane; i < nU; i += 32) uni[i] = p.uni[(int64_t)tile * U + i];
+                if (nU < 0 && p.duni) {  // a block-major tile: its dense blocks are this kernel's
+                    nU = p.dcnt[tile];
+                    dense = 1;
+                    for (int i = lane; i < nU; i += 32) uni[i] = p.duni[(int64_t)tile * kDenseMax + i];
+                } else {
+                    for (int i = lane; i < nU; i += 32) uni[i] = p.uni[(int64_t)tile * U + i];
+                }
             }
             if (lane == 0) {
                 ti.done = 0;
                 ti.nU = nU;
+                ti.dense = dense;
                 ti.b = b;
                 ti.hk = hk;
                 ti.q0 = q0;
@@ -533,7 +542,9 @@ __global__ void __launch_bounds__(kQThreads, 2)
             const int64_t t = (int64_t)q0 + i;
             const int *mylist = s_lists + (m * p.Tq + (row_valid ? tok : 0)) * p.topk;
             const int32_t *gl = p.sel_c + (row_valid && MODE == kModePrep ? (t * p.Hkv + hk) * p.topk : 0);
-            const int mycnt = !row_valid || WIN ? 0 : FUSED ? s_cnts[m * p.Tq + tok] : p.cnt[t * p.Hkv + hk];
+            const bool dense = !WIN && !FUSED && ti.dense;
+            const uint32_t dsel = dense && row_valid ? __ldg(&p.dsel[t * p.Hkv + hk]) : 0u;
+            const int mycnt = !row_valid || WIN || dense ? 0 : FUSED ? s_cnts[m * p.Tq + tok] : p.cnt[t * p.Hkv + hk];
             int nxt = (MODE == kModePrep && mycnt > 0) ? gl[0] : -1;
             int ptr = 0;
             float m_run = -INFINITY;  // running max of s*scale*log2e
@@ -548,6 +559,8 @@ __global__ void __launch_bounds__(kQThreads, 2)
                 } else if constexpr (FUSED) {
                     selected = ptr < mycnt && mylist[ptr] == s;
                     if (selected) ++ptr;
+                } else if (dense) {
+                    selected = (dsel >> j) & 1u;
                 } else {
                     selected = nxt == s;
                     if (selected) {

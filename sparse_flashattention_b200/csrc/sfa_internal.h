@@ -20,6 +20,10 @@ namespace sfa {
 // head: Tq * G <= 128 rows, the M dimension of one tcgen05 MMA.  Tiles are numbered
 // tile = (qt_rev * batch + b) * Hkv + hk with qt = nqt - 1 - qt_rev, so the tiles deepest
 // into their sequences (the ones with the most blocks under a causal mask) start first.
+// Block-major windows: a tile's blocks that at least a quarter of its 128 rows select ("dense", at
+// most kDenseMax of them, ascending) run query-major for the tile; the rest go to block-major items.
+constexpr int kDenseMax = 32;
+
 struct FwdGeom {
     int batch, max_sq, max_sk, total_q, Hq, Hkv, d, topk, bs;
     int G, Tq, nqt, tiles, nblk_max, umax;
@@ -31,7 +35,7 @@ struct FwdGeom {
     int64_t cap_items;
     size_t off_sel_c, off_cnt, off_ucnt, off_union, off_tilectr;
     size_t off_zero, zero_bytes;  // the part of the workspace cleared before every prep
-    size_t off_ctrl, off_gstat, off_tcount, off_gfirst, off_items, off_pml, off_po;
+    size_t off_ctrl, off_gstat, off_tcount, off_gfirst, off_duni, off_dcnt, off_dsel, off_items, off_pml, off_po;
     size_t bytes;
 };
 
@@ -55,13 +59,18 @@ struct InvItem {
 struct FwdPrepParams {
     const int32_t *cu_q, *cu_k, *sel;
     int32_t *tile_counter;  // cleared here (two ints) for the attend kernel
-    int batch, Hkv, topk, bs, causal, wl, wr, Tq, nqt, umax, max_sq, nblk_max;
+    int batch, Hkv, topk, bs, causal, wl, wr, Tq, nqt, umax, max_sq, nblk_max, total_q;
     int32_t *sel_c, *cnt, *ucnt, *uni;
     // block-major statistics (nullptr when the schedule is off): per group, and per tile the number of
     // its tokens that selected each block ([tiles][nblk_max])
     int W;
     GroupStat *gstat;
     int32_t *tcount;
+    // the tile's dense blocks ([tiles][kDenseMax], count per tile) and per (token, kv head) two masks:
+    // the dense blocks it selected (bit j: the tile's dense block j) and its canonical entries that are
+    // dense (bit e: entry e), [2][total_q * Hkv]
+    int32_t *duni, *dcnt;
+    uint32_t *dsel;
     int32_t *status;
 };
 
@@ -79,6 +88,7 @@ struct FwdPlanParams {
 struct FwdScatterParams {
     const int32_t *cu_q, *sel_c, *cnt, *ucnt, *gfirst;
     const int32_t *tcount;  // each tile's first position in every block's token list
+    const uint32_t *dmask;  // per (token, kv head): canonical entries of dense blocks (not in items)
     int batch, Hkv, topk, Tq, nqt, W, nblk_max;
     InvItem *items;
 };
@@ -104,6 +114,10 @@ struct FwdAttendParams {
     InvCtrl *ctrl;
     __nv_bfloat16 *po;  // partial outputs, (total_q, Hq, topk, d) bf16, normalised
     float2 *pml;        // partial (max, sum) in the base-2 scaled domain, (total_q, Hq, topk)
+    // dense blocks of block-major tiles (the query-major kernel attends over them and leaves its result
+    // in out / lse, one more partial for the merge); nullptr when the schedule is off
+    const int32_t *duni, *dcnt;
+    const uint32_t *dsel, *dmask;
 };
 
 // ---------------------------------------------------------------------------------------

@@ -102,6 +102,7 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
     int *raw = reinterpret_cast<int *>(prep_smem + words);
     int *lists = raw + p.Tq * rs;                             // [topk][kPrepThreads] canonical
     int *hist = p.tcount ? lists + p.topk * kPrepThreads : nullptr;  // [nblk_max] this tile's tokens per block
+    uint32_t *dbm = p.duni ? reinterpret_cast<uint32_t *>(hist + p.nblk_max) : nullptr;  // [words] dense blocks
     for (int w = threadIdx.x; w < words; w += kPrepThreads) bm[w] = 0;
     if (hist)
         for (int s = threadIdx.x; s < p.nblk_max; s += kPrepThreads) hist[s] = 0;
@@ -160,8 +161,41 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_prep_kernel(FwdPrepParams p)
         const int t2 = e / p.topk;
         p.sel_c[row0 + t2 * tok_stride + (e - t2 * p.topk)] = raw[t2 * rs + (e - t2 * p.topk)];
     }
+    if (dbm) {
+        // Dense blocks: selected by at least a quarter of a full tile's rows (Tq / 4 tokens), at most
+        // kDenseMax, ascending.  They run query-major for this tile (the query-major kernel leaves that
+        // partial in out / lse), so they leave the tile's counts; each token notes which of the dense
+        // blocks it selected and which of its canonical entries they are.  (The lists region is free
+        // now and holds up to 2 * topk dense blocks: each needs Tq / 4 of the tile's Tq * topk entries.)
+        for (int w = threadIdx.x; w < words; w += kPrepThreads) dbm[w] = 0;
+        __syncthreads();
+        for (int s = threadIdx.x; s < nblk; s += kPrepThreads)
+            if (hist[s] > 0 && 4 * hist[s] >= p.Tq) atomicOr(&dbm[s >> 5], 1u << (s & 31));
+        __syncthreads();
+        const int nd = min(kDenseMax, compact_bitmap<kPrepThreads>(dbm, (nblk + 31) / 32, lists, scan_scratch));
+        for (int j = threadIdx.x; j < nd; j += kPrepThreads) {
+            hist[lists[j]] = -1 - j;
+            p.duni[(int64_t)tile * kDenseMax + j] = lists[j];
+        }
+        if (threadIdx.x == 0) p.dcnt[tile] = nd;
+        __syncthreads();
+        if (tt < ntok) {
+            uint32_t sel_bits = 0, entry_bits = 0;
+            for (int e = 0; e < n; ++e) {
+                const int v = hist[raw[tt * rs + e]];
+                if (v < 0) {
+                    sel_bits |= 1u << (-1 - v);
+                    entry_bits |= 1u << e;
+                }
+            }
+            const int64_t t = (int64_t)q0 + tok0 + tt;
+            p.dsel[t * p.Hkv + hk] = sel_bits;
+            p.dsel[(int64_t)p.total_q * p.Hkv + t * p.Hkv + hk] = entry_bits;
+        }
+    }
     if (hist)
-        for (int s = threadIdx.x; s < p.nblk_max; s += kPrepThreads) p.tcount[(int64_t)tile * p.nblk_max + s] = hist[s];
+        for (int s = threadIdx.x; s < p.nblk_max; s += kPrepThreads)
+            p.tcount[(int64_t)tile * p.nblk_max + s] = max(hist[s], 0);
     const int total = compact_bitmap<kPrepThreads>(bm, (nblk + 31) / 32, p.uni + (int64_t)tile * p.umax,
                                                    scan_scratch);
     if (threadIdx.x == 0) {
@@ -262,8 +296,10 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_scatter_kernel(FwdScatterPar
     const int tt = threadIdx.x;
     const int64_t t = (int64_t)q0 + tok0 + tt;
     const int n = tt < ntok ? p.cnt[t * p.Hkv + hk] : 0;
+    const uint32_t dense = tt < ntok && p.dmask ? p.dmask[t * p.Hkv + hk] : 0u;  // run query-major
     const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
     for (int e = 0; e < n; ++e) {
+        if ((dense >> e) & 1u) continue;
         const int s = row[e];
         const int pos = atomicAdd(&pos_s[s], 1);
         p.items[first_s[s] + pos / p.Tq].tok[pos % p.Tq] = (int)(t << 7) | e;
@@ -314,7 +350,7 @@ cudaError_t launch_fwd_prep(const FwdGeom &g, const FwdPrepParams &p, cudaStream
 {
     const size_t words = (size_t)(g.nblk_max + 31) / 32;
     const size_t smem = words * 4 + (size_t)g.Tq * (g.topk | 1) * 4 + (size_t)g.topk * kPrepThreads * 4 +
-                        (p.tcount ? (size_t)g.nblk_max * 4 : 0);
+                        (p.tcount ? (size_t)g.nblk_max * 4 : 0) + (p.duni ? words * 4 : 0);
     if (smem > 48 * 1024) {
         const cudaError_t e = ensure_smem_for(fwd_prep_kernel, smem);
         if (e != cudaSuccess) return e;
