@@ -499,16 +499,18 @@ __global__ void __launch_bounds__(32 * kMergeWarps, 3) fwd_merge_kernel(const Fw
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
         // (its two loads go out with the first batch of partials, not ahead of them)
+        // The block-major partials fill the row's first nk slots (the scatter numbers a row's entries
+        // that are not dense consecutively).
         bool qdone = !(dm != 0u && kq == 0);
-        for (int k0 = kq; k0 < cnt; k0 += kSplit * kMergeBatch) {
+        const int nk = cnt - __popc(dm);
+        for (int k0 = kq; k0 < nk; k0 += kSplit * kMergeBatch) {
             float2 ml[kMergeBatch];
             uint4 v[kMergeBatch];
 #pragma unroll
             for (int i = 0; i < kMergeBatch; ++i) {
                 const int k = k0 + i * kSplit;
-                const bool use = k < cnt && !((dm >> k) & 1u);
-                ml[i] = use ? __ldcs(&p.pml[base + k]) : make_float2(-INFINITY, 0.f);
-                v[i] = use ? __ldcs(reinterpret_cast<const uint4 *>(p.po + (base + k) * D) + c) : make_uint4(0u, 0u, 0u, 0u);
+                ml[i] = k < nk ? __ldcs(&p.pml[base + k]) : make_float2(-INFINITY, 0.f);
+                v[i] = k < nk ? __ldcs(reinterpret_cast<const uint4 *>(p.po + (base + k) * D) + c) : make_uint4(0u, 0u, 0u, 0u);
             }
             if (!qdone) {  // the query-major partial as (m, l) = (lse in base 2, 1), normalised chunk vq
                 qdone = true;

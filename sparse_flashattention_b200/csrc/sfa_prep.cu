@@ -298,11 +298,14 @@ __global__ void __launch_bounds__(kPrepThreads) fwd_scatter_kernel(FwdScatterPar
     const int n = tt < ntok ? p.cnt[t * p.Hkv + hk] : 0;
     const uint32_t dense = tt < ntok && p.dmask ? p.dmask[t * p.Hkv + hk] : 0u;  // run query-major
     const int32_t *row = p.sel_c + (t * p.Hkv + hk) * p.topk;
+    // An entry's partial goes to slot (its rank among the token's entries that are not dense), so a
+    // row's block-major partials fill the first slots of its range.
     for (int e = 0; e < n; ++e) {
         if ((dense >> e) & 1u) continue;
         const int s = row[e];
         const int pos = atomicAdd(&pos_s[s], 1);
-        p.items[first_s[s] + pos / p.Tq].tok[pos % p.Tq] = (int)(t << 7) | e;
+        const int slot = e - __popc(dense & ((1u << e) - 1u));
+        p.items[first_s[s] + pos / p.Tq].tok[pos % p.Tq] = (int)(t << 7) | slot;
     }
 }
 
