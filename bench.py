@@ -57,8 +57,8 @@ DECODE_PART_NAMES = {"all": DECODE_NAME,
 TRAFFIC = {
     # the six kernels of one call on nsa_long_96k (prep, plan, scatter, query-major, block-major, merge)
     "prefill_c4": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_fwd_inv_kernel.cu", "sfa_prep.cu", "sfa_device.cuh"],
-                   "sha256": "e3650da55d622ebf8e763520b7d476f6b1a1ca49a8fd1fd910b0f50f8aa9cbb1",
-                   "bytes": 4294524416},
+                   "sha256": "e521394bdfa170ccaf86361b5bd4927c64533d4ad89f1a2f890e31f3b52f307f",
+                   "bytes": 3969697536},
     # the one kernel of a call on nsa_varlen_16k (the fused query-major kernel)
     "prefill_c2": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],
                    "sha256": "f8b1585aed8bcf23a6056420f9d897e21a56bccd284f10646aaf0fb216cf7a05",

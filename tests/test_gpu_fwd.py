@@ -244,12 +244,15 @@ def _block_major_windows(c, oracle_lib):
 @pytest.mark.parametrize("Hq,Hkv,d,bs,topk,lens", [(16, 4, 128, 64, 6, [12000, 300]),
                                                    (2, 2, 64, 32, 6, [9000, 77]),
                                                    (8, 2, 128, 32, 8, [8000]),
-                                                   (6, 2, 64, 64, 5, [10000, 1000])])
+                                                   (6, 2, 64, 64, 5, [10000, 1000]),
+                                                   (8, 2, 64, 32, 40, [20000])])
 def test_block_major_windows(sfa, oracle_lib, Hq, Hkv, d, bs, topk, lens):
     """Long sequences with a small random top-k: late windows' query tiles select unions of
     blocks over 10x their selected work, so those windows go to the block-major kernel (items of
     one block and the tokens that selected it, bf16 partials, merge kernel) while early windows
-    stay query-major.  Every element against the oracle, ragged lengths included."""
+    stay query-major.  The blocks most of a block-major tile selects (the forced initial and local
+    ones) run query-major for the tile and join the merge as one more partial; with topk 40 (over
+    32) that split is off.  Every element against the oracle, ragged lengths included."""
     c = W.make_nsa_prefill(Hq + 7 * d + bs + topk, lens, Hq, Hkv, d, bs, topk, 1, 2)
     assert _block_major_windows(c, oracle_lib) > 0
     _full_parity(sfa, oracle_lib, c)
