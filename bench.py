@@ -57,7 +57,7 @@ DECODE_PART_NAMES = {"all": DECODE_NAME,
 TRAFFIC = {
     # the six kernels of one call on nsa_long_96k (prep, plan, scatter, query-major, block-major, merge)
     "prefill_c4": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_fwd_inv_kernel.cu", "sfa_prep.cu", "sfa_device.cuh"],
-                   "sha256": "e521394bdfa170ccaf86361b5bd4927c64533d4ad89f1a2f890e31f3b52f307f",
+                   "sha256": "2c5060e737605c2773b8d36dde669c8833f4615aad99b892c2e733003c06c81b",
                    "bytes": 3969697536},
     # the one kernel of a call on nsa_varlen_16k (the fused query-major kernel)
     "prefill_c2": {"files": ["sfa_fwd_pipe_kernel.cu", "sfa_device.cuh"],

@@ -444,12 +444,15 @@ __global__ void __launch_bounds__(kInvThreadsAttn, 1)
     }
 }
 
-// Merge of the block-major partials, one warp per (token, kv head) whose tile went block-major:
-// for each of the G heads, M = max m_k, L = sum l_k 2^(m_k - M), out = sum (l_k 2^(m_k - M) / L) o_k,
-// lse = (M + log2 L) ln 2.  Lanes cover the head dimension in 16-byte chunks and split the
+// Merge of the block-major partials, one warp per row (token, head) of a tile that went block-major:
+// M = max m_k, L = sum l_k 2^(m_k - M), out = sum (l_k 2^(m_k - M) / L) o_k, lse = (M + log2 L) ln 2
+// over the row's partials: its block-major ones (the first slots of its range) and, when the tile
+// has dense blocks, the query-major kernel's partial over them, left in out / lse (taken as
+// (m, l) = (lse in base 2, 1)).  Lanes cover the head dimension in 16-byte chunks and split the
 // partials between them; each lane loads a batch of its partials at once (independent loads in
 // flight), folds them into a running max / sum / weighted chunk, and the lanes sharing a chunk
 // combine at the end.  The partials are read once, with streaming loads (they are not reused).
+// Three CTAs per SM (80 registers): the loads in flight are what this kernel's speed rests on.
 constexpr int kMergeWarps = 8;
 constexpr int kMergeBatch = 8;  // partials each lane loads before folding them in
 
