@@ -276,7 +276,8 @@ int sfa_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
  *   workspace  sfa_index_topk_workspace_size() bytes (one 64-bit key per position)
  * Positions whose page id is outside [0, num_pages) are no candidates (SFA_DEV_BAD_PAGE); a length
  * past the block table is cut to it (SFA_DEV_BAD_SEQLEN).  d in {64, 128}; max_pages_per_seq *
- * page_size <= 2^20.  One kernel, one CTA per (sequence, kv head). */
+ * page_size <= 2^20; G = Hq / Hkv <= 1024 (the exactness bound).  Two kernels: the scores (one CTA per (sequence, kv head, run of 4096
+ * positions)), then the selection (one CTA per (sequence, kv head)). */
 size_t sfa_index_topk_workspace_size(int B, int Hkv, int max_pages_per_seq, int page_size);
 int sfa_index_topk(const void *q, const void *k_cache, const int32_t *block_table, int max_pages_per_seq,
                    int num_pages, int page_size, const int32_t *cache_seqlens, int B, int Hq, int Hkv, int d, int topk,

@@ -789,6 +789,7 @@ int sfa_index_topk(const void *q, const void *k_cache, const int32_t *block_tabl
         return SFA_ERR_INVALID_ARG;
     if (Hq % Hkv != 0) return SFA_ERR_INVALID_ARG;
     if (d != 64 && d != 128) return SFA_ERR_UNSUPPORTED;
+    if (Hq / Hkv > 1024) return SFA_ERR_UNSUPPORTED;  // past that, fp64 no longer holds the scores exactly
     if ((int64_t)max_pages_per_seq * page_size > (1 << 20) || topk > (1 << 20)) return SFA_ERR_UNSUPPORTED;
     if (B == 0) return SFA_OK;
     if (!q || !k_cache || !block_table || !cache_seqlens || !sel_out || !workspace) return SFA_ERR_INVALID_ARG;
@@ -816,7 +817,7 @@ int sfa_index_topk(const void *q, const void *k_cache, const int32_t *block_tabl
     p.sel = sel_out;
     p.status = status_dev;
     if (launch_index_topk(p, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SFA_ERR_CUDA;
-    g_last_launches = 1;
+    g_last_launches = 2;
     return SFA_OK;
 }
 

@@ -179,6 +179,7 @@ def test_index_topk_host_validation(lib):
 
     assert call(d=96) == 2                 # SFA_ERR_UNSUPPORTED
     assert call(Hq=6) == 1                 # Hq % Hkv
+    assert call(Hq=4 * 1025) == 2          # groups past 1024 query heads: scores no longer exact in fp64
     assert call(topk=0) == 1
     assert call(n_local=-1) == 1
     assert call(out=None) == 1
