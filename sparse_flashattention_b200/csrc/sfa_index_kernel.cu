@@ -168,11 +168,13 @@ __global__ void __launch_bounds__(kIdxScoreThreads, 3) index_score_kernel(IndexP
         for (int u = 0; u < kRowsPerGroup; ++u) {
             const int64_t j = j0 + u * kRowsPerWarp + sub;
             const bool in = j < c1;
-            const int pi = in ? (int)(j / p.page) : 0;
+            // positions are below 2^20: 32-bit division (a 64-bit one is a long software routine)
+            const unsigned pi = in ? (unsigned)j / (unsigned)p.page : 0u;
             const int pg = in ? __ldg(&bt_g[pi]) : -1;
             const bool ok = in && pg >= 0 && pg < p.num_pages;
+            const int row = (int)j - (int)pi * p.page;
             const __nv_bfloat16 *src =
-                ok ? p.kc + (((int64_t)pg * p.page + (j - (int64_t)pi * p.page)) * p.Hkv + hk) * D + part * 8 : p.kc;
+                ok ? p.kc + (((int64_t)pg * p.page + row) * p.Hkv + hk) * D + part * 8 : p.kc;
             cp_async16(smem_u32(&stage[(slot * kRowsPerGroup + u) * kIdxScoreThreads + tid]), src, ok ? 16u : 0u);
             m |= (uint32_t)ok << u;
             bad_page |= in && !ok;
