@@ -63,7 +63,7 @@ typedef struct CUstream_st *sfa_stream_t; /* same type as cudaStream_t */
 typedef enum sfa_status {
     SFA_OK = 0,
     SFA_ERR_INVALID_ARG = 1,         /* NULL pointer, negative size, Hq % Hkv != 0, misaligned base */
-    SFA_ERR_UNSUPPORTED = 2,         /* valid but outside this build: see the limits below */
+    SFA_ERR_UNSUPPORTED = 2,         /* valid but outside what this library supports: see the limits below */
     SFA_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the matching *_workspace_size() */
     SFA_ERR_CUDA = 4                 /* a CUDA launch or driver call failed */
 } sfa_status;
@@ -76,10 +76,10 @@ enum {
                                excess is not computed / its ids are treated as out of range */
 };
 
-/* Supported in this build: bf16 inputs; d in {64, 128}; prefill block_size in {32, 64},
+/* Supported by this library: bf16 inputs; d in {64, 128}; prefill block_size in {32, 64},
  * 1 <= topk <= 128, G = Hq/Hkv <= 128, ceil(max_seqlen_k / block_size) <= 65536;
  * decode G <= 16, page_size >= 1, 1 <= topk_tok <= 65536, max_pages_per_seq*page_size
- * <= 2^20; backward the forward's d and block_size; KV append d a multiple of 8; index top-k
+ * <= 2^20; backward the forward's d and block_size; KV append d a multiple of 8; index top-k G <= 1024,
  * max_pages_per_seq*page_size <= 2^20.  Anything else returns SFA_ERR_UNSUPPORTED. */
 
 /* ----------------------------------------------------------------------------------------

@@ -168,7 +168,7 @@ def kv_append(k_cache, v_cache, block_table, cache_seqlens, k_new, v_new):
     sequence b to page block_table[b, j // page], row j % page.  cache_seqlens itself is left as is
     (the caller tracks lengths).  k_new / v_new: (B, seqlen_new, Hkv, d).  Positions past the block
     table, or whose page id is outside [0, num_pages), are not written (counted in `bad`, the
-    reading this build takes where the docstring only asks the caller to size the cache).
+    reading taken here where the docstring only asks the caller to size the cache).
     Returns (k_cache, v_cache, bad) as new arrays; the inputs are not modified."""
     kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
     num_pages, page = kc.shape[0], kc.shape[1]

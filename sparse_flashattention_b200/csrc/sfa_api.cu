@@ -1035,7 +1035,7 @@ const char *sfa_status_string(int status)
     switch (status) {
     case SFA_OK: return "SFA_OK";
     case SFA_ERR_INVALID_ARG: return "SFA_ERR_INVALID_ARG: invalid argument";
-    case SFA_ERR_UNSUPPORTED: return "SFA_ERR_UNSUPPORTED: valid but not supported by this build";
+    case SFA_ERR_UNSUPPORTED: return "SFA_ERR_UNSUPPORTED: valid but not supported by this library";
     case SFA_ERR_WORKSPACE_TOO_SMALL: return "SFA_ERR_WORKSPACE_TOO_SMALL: workspace below the required size";
     case SFA_ERR_CUDA: return "SFA_ERR_CUDA: a CUDA launch or driver call failed";
     default: return "unknown sfa_status";
