@@ -160,24 +160,47 @@ __global__ void __launch_bounds__(kIdxScoreThreads, 3) index_score_kernel(IndexP
     bool bad_page = false;
     uint32_t okm = 0;  // bit slot * kRowsPerGroup + u: row u of the iteration held in that slot is readable
 
+    // A warp's rows of one iteration are the kGroupRows consecutive positions from a multiple of
+    // kGroupRows; when the page size is a multiple of that, they sit in one page: one block-table
+    // lookup serves them all and the rows are constant offsets from the first.
+    constexpr int kGroupRows = kRowsPerWarp * kRowsPerGroup;
+    const bool one_page = p.page % kGroupRows == 0;
+    const int64_t row_elems = (int64_t)p.Hkv * D;  // elements from one cache row to the next
     auto issue = [&](int it) {
         const int slot = it % kIdxStages;
         const int64_t j0 = j_first + (int64_t)it * kStep;
         uint32_t m = 0;
+        if (one_page) {
+            // j0 < c1 <= 2^20: 32-bit division (a 64-bit one is a long software routine)
+            const unsigned pi = (unsigned)j0 / (unsigned)p.page;
+            const int pg = __ldg(&bt_g[pi]);
+            const bool okg = pg >= 0 && pg < p.num_pages;
+            const __nv_bfloat16 *base =
+                p.kc + ((int64_t)pg * p.page + ((int)j0 - (int)pi * p.page)) * row_elems + hk * D + part * 8;
 #pragma unroll
-        for (int u = 0; u < kRowsPerGroup; ++u) {
-            const int64_t j = j0 + u * kRowsPerWarp + sub;
-            const bool in = j < c1;
-            // positions are below 2^20: 32-bit division (a 64-bit one is a long software routine)
-            const unsigned pi = in ? (unsigned)j / (unsigned)p.page : 0u;
-            const int pg = in ? __ldg(&bt_g[pi]) : -1;
-            const bool ok = in && pg >= 0 && pg < p.num_pages;
-            const int row = (int)j - (int)pi * p.page;
-            const __nv_bfloat16 *src =
-                ok ? p.kc + (((int64_t)pg * p.page + row) * p.Hkv + hk) * D + part * 8 : p.kc;
-            cp_async16(smem_u32(&stage[(slot * kRowsPerGroup + u) * kIdxScoreThreads + tid]), src, ok ? 16u : 0u);
-            m |= (uint32_t)ok << u;
-            bad_page |= in && !ok;
+            for (int u = 0; u < kRowsPerGroup; ++u) {
+                const int du = u * kRowsPerWarp + sub;
+                const bool in = j0 + du < c1;
+                const bool ok = in && okg;
+                cp_async16(smem_u32(&stage[(slot * kRowsPerGroup + u) * kIdxScoreThreads + tid]),
+                           ok ? base + du * row_elems : p.kc, ok ? 16u : 0u);
+                m |= (uint32_t)ok << u;
+                bad_page |= in && !ok;
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < kRowsPerGroup; ++u) {
+                const int64_t j = j0 + u * kRowsPerWarp + sub;
+                const bool in = j < c1;
+                const unsigned pi = in ? (unsigned)j / (unsigned)p.page : 0u;
+                const int pg = in ? __ldg(&bt_g[pi]) : -1;
+                const bool ok = in && pg >= 0 && pg < p.num_pages;
+                const int row = (int)j - (int)pi * p.page;
+                const __nv_bfloat16 *src = ok ? p.kc + ((int64_t)pg * p.page + row) * row_elems + hk * D + part * 8 : p.kc;
+                cp_async16(smem_u32(&stage[(slot * kRowsPerGroup + u) * kIdxScoreThreads + tid]), src, ok ? 16u : 0u);
+                m |= (uint32_t)ok << u;
+                bad_page |= in && !ok;
+            }
         }
         const int sh = slot * kRowsPerGroup;
         okm = (okm & ~(((1u << kRowsPerGroup) - 1u) << sh)) | (m << sh);

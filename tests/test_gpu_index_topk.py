@@ -29,6 +29,7 @@ def sfa():
     (2, 8, 2, 128, 16, 100, 900, 50, 3, "ties"),      # many exact ties
     (2, 8, 2, 128, 64, 500, 2000, 100, 4, "tiny"),    # keys mostly E4M3 subnormals (below 2^-6)
     (2, 8, 2, 64, 64, 500, 2000, 100, 4, "huge"),     # keys often past 448: saturated
+    (3, 8, 4, 128, 100, 300, 2500, 128, 8, "normal"), # page not a multiple of a warp's 8 rows
 ])
 def test_index_topk_bitwise(sfa, B, Hq, Hkv, d, page, lo, hi, topk, nl, keys):
     c = W.make_decode(200 + topk, B, Hq, Hkv, d, page, lo, hi, 8, 2)
