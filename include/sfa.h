@@ -296,6 +296,29 @@ int sfa_kv_append(const void *k_new, const void *v_new, int seqlen_new, void *k_
                   const int32_t *block_table, int max_pages_per_seq, int num_pages, int page_size,
                   const int32_t *cache_seqlens, int B, int Hkv, int d, int32_t *status_dev, sfa_stream_t stream);
 
+/* Non-paged caches with a batch index, the cache_batch_idx argument of flash_attn_with_kvcache
+ * (flash-attention-npu docstrings): k_cache / v_cache bf16 (batch_cache, seqlen_cache, Hkv, d) and
+ * cache_batch_idx int32 (B): sequence b reads and appends row j at k_cache[cache_batch_idx[b]][j].
+ * (The docstring's default, cache_batch_idx = None, is 0, 1, ..., B-1: pass that array.)  Such a
+ * cache is the paged cache of batch_cache pages of seqlen_cache rows whose block table is
+ * cache_batch_idx itself (one page per sequence), so these calls are sfa_decode / sfa_kv_append with
+ * block_table = cache_batch_idx, max_pages_per_seq = 1, num_pages = batch_cache, page_size =
+ * seqlen_cache: the same kernels, launches, workspace (sfa_decode_workspace_size), limits
+ * (seqlen_cache <= 2^20) and status bits.  An index outside [0, batch_cache) sets
+ * SFA_DEV_BAD_PAGE and drops the sequence's rows (decode: out 0, lse -inf; append: nothing
+ * written); cache_seqlens[b] (+ the new rows) past seqlen_cache sets SFA_DEV_BAD_SEQLEN and the
+ * excess is cut.  As the docstring warns, an append whose cache_batch_idx repeats an index writes
+ * the same rows from several sequences: which one lands is unspecified. */
+int sfa_decode_kvcache(const void *q, const void *k_cache, const void *v_cache, int batch_cache, int seqlen_cache,
+                       const int32_t *cache_batch_idx, const int32_t *cache_seqlens, const int32_t *sel_tok_idx,
+                       int topk_tok, int B, int Hq, int Hkv, int d, int window_left, float scale, int num_splits,
+                       void *workspace, size_t workspace_bytes, int32_t *status_dev, void *out, float *lse,
+                       sfa_stream_t stream);
+int sfa_kv_append_kvcache(const void *k_new, const void *v_new, int seqlen_new, void *k_cache, void *v_cache,
+                          int batch_cache, int seqlen_cache, const int32_t *cache_batch_idx,
+                          const int32_t *cache_seqlens, int B, int Hkv, int d, int32_t *status_dev,
+                          sfa_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------
  * NSA branches beside the selected attention (the "Relaxed-System-Lab/Flash-Sparse-Attention"
  * project page, quick-start: window_size alongside block_size / topk; the Flash-Sparse-Attention

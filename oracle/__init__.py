@@ -190,6 +190,69 @@ def kv_append(k_cache, v_cache, block_table, cache_seqlens, k_new, v_new):
     return kc, vc, bad
 
 
+
+def _bf16_f64(a):
+    a = np.asarray(a)
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64) if a.dtype == np.uint16 else \
+        a.astype(np.float64)
+
+
+def decode_kvcache(q, k_cache, v_cache, cache_seqlens, sel, cache_batch_idx, Hkv, scale, wl=-1):
+    """Top-k decode over a non-paged cache, in float64, as flash_attn_with_kvcache documents its
+    cache_batch_idx argument (flash-attention-npu page, "FlashAttention v2" API docstrings): k_cache /
+    v_cache are (batch_cache, seqlen_cache, Hkv, d) and cache_batch_idx (B,) says which of their
+    batch entries sequence b uses, so its row j is k_cache[cache_batch_idx[b], j].  For query head h
+    (kv head h // G) the kept positions are the distinct entries j >= 0 of sel[b, h // G] below
+    L = min(cache_seqlens[b], seqlen_cache) (and >= L - 1 - wl when wl >= 0); out is the softmax of
+    scale * q . k_j over them applied to the v_j, lse the natural log of its normaliser.  No kept
+    position, or an index outside [0, batch_cache): out 0, lse -inf.  Other negative or too large
+    positions are counted in `bad` and skipped.
+    q: (B, Hq, d); sel: (B, Hkv, topk).  Returns (out (B, Hq, d), lse (B, Hq), bad)."""
+    qf, kf, vf = _bf16_f64(q), _bf16_f64(k_cache), _bf16_f64(v_cache)
+    B, Hq, d = qf.shape
+    batch_cache, seqlen_cache = kf.shape[0], kf.shape[1]
+    G = Hq // Hkv
+    out = np.zeros((B, Hq, d), np.float64)
+    lse = np.full((B, Hq), -np.inf, np.float64)
+    bad = 0
+    for b in range(B):
+        L = min(int(cache_seqlens[b]), seqlen_cache)
+        c = int(cache_batch_idx[b])
+        for hk in range(Hkv):
+            row = [int(j) for j in sel[b, hk]]
+            bad += sum(1 for j in row if j != -1 and not 0 <= j < L)
+            keep = sorted({j for j in row if 0 <= j < L and (wl < 0 or j >= L - 1 - wl)})
+            if not keep or not 0 <= c < batch_cache:
+                continue
+            K, V = kf[c, keep, hk], vf[c, keep, hk]
+            for h in range(hk * G, (hk + 1) * G):
+                s_ = scale * (K @ qf[b, h])
+                m = s_.max()
+                e = np.exp(s_ - m)
+                out[b, h] = e @ V / e.sum()
+                lse[b, h] = m + np.log(e.sum())
+    return out, lse, bad
+
+
+def kv_append_kvcache(k_cache, v_cache, cache_batch_idx, cache_seqlens, k_new, v_new):
+    """In-place append to a non-paged cache (flash_attn_with_kvcache with cache_batch_idx, same
+    docstrings): row j of k_new[b] goes to k_cache[cache_batch_idx[b], cache_seqlens[b] + j].  Rows past
+    seqlen_cache, or of a sequence whose index is outside [0, batch_cache), are not written (counted in
+    `bad`).  Returns (k_cache, v_cache, bad) as new arrays."""
+    kc, vc = np.array(k_cache, copy=True), np.array(v_cache, copy=True)
+    batch_cache, seqlen_cache = kc.shape[0], kc.shape[1]
+    bad = 0
+    for b in range(k_new.shape[0]):
+        c = int(cache_batch_idx[b])
+        for j in range(k_new.shape[1]):
+            pos = int(cache_seqlens[b]) + j
+            if not (0 <= c < batch_cache and pos < seqlen_cache):
+                bad += 1
+                continue
+            kc[c, pos] = k_new[b, j]
+            vc[c, pos] = v_new[b, j]
+    return kc, vc, bad
+
 # ---------------------------------------------------------------------------------------------------
 # Index producer for the decode: a Lightning-Indexer-style scan ("Sparse FlashAttention" on Ascend,
 # ggplus blog post, section "那个叫Lightning Indexer的家伙": the indexer scores the current query

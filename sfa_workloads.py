@@ -243,6 +243,57 @@ class DecodeCase:
         return self.scale if self.scale > 0 else 1.0 / np.sqrt(self.d)
 
 
+@dataclasses.dataclass
+class KVCacheCase:
+    """Decode inputs over a non-paged cache addressed through cache_batch_idx."""
+    name: str
+    q: np.ndarray               # uint16 (B, Hq, d)
+    k_cache: np.ndarray         # uint16 (batch_cache, seqlen_cache, Hkv, d)
+    v_cache: np.ndarray
+    cache_batch_idx: np.ndarray  # int32 (B,): the cache entry of each sequence
+    cache_seqlens: np.ndarray   # int32 (B,)
+    sel: np.ndarray             # int32 (B, Hkv, topk_tok)
+    Hq: int
+    Hkv: int
+    d: int
+    wl: int = -1
+
+    @property
+    def B(self):
+        return int(self.q.shape[0])
+
+    @property
+    def softmax_scale(self):
+        return 1.0 / np.sqrt(self.d)
+
+
+def make_decode_kvcache(seed: int, B, batch_cache, seqlen_cache, Hq, Hkv, d, len_lo, len_hi, topk_tok, n_last,
+                        name="decode_kvcache") -> KVCacheCase:
+    """Non-paged decode inputs: cache_seqlens ~ U[len_lo, len_hi] (<= seqlen_cache), each sequence on
+    a distinct cache entry drawn from [0, batch_cache), selections as make_decode draws them."""
+    ss = np.random.SeedSequence(seed)
+    s_len, s_idx, s_q, s_k, s_v, s_sel = ss.spawn(6)
+    L = np.random.Generator(np.random.PCG64(s_len)).integers(len_lo, len_hi + 1, size=B).astype(np.int32)
+    idx = np.random.Generator(np.random.PCG64(s_idx)).permutation(batch_cache)[:B].astype(np.int32)
+    q = _normal_bf16(np.random.Generator(np.random.PCG64(s_q)), (B, Hq, d))
+    kc = _normal_bf16(np.random.Generator(np.random.PCG64(s_k)), (batch_cache, seqlen_cache, Hkv, d))
+    vc = _normal_bf16(np.random.Generator(np.random.PCG64(s_v)), (batch_cache, seqlen_cache, Hkv, d))
+    g_sel = np.random.Generator(np.random.PCG64(s_sel))
+    sel = np.full((B, Hkv, topk_tok), INVALID, dtype=np.int32)
+    for b in range(B):
+        Lb = int(L[b])
+        nl = min(n_last, Lb, topk_tok)
+        last = np.arange(Lb - nl, Lb, dtype=np.int32)
+        nr = min(topk_tok - nl, Lb - nl)
+        for h in range(Hkv):
+            rest = g_sel.choice(Lb - nl, size=nr, replace=False).astype(np.int32) if nr > 0 else \
+                np.zeros(0, np.int32)
+            row = np.concatenate([last, rest])
+            g_sel.shuffle(row)
+            sel[b, h, :row.size] = row
+    return KVCacheCase(name, q, kc, vc, idx, L, sel, Hq, Hkv, d)
+
+
 def _cu(lens):
     return np.concatenate([[0], np.cumsum(np.asarray(lens, dtype=np.int64))]).astype(np.int32)
 

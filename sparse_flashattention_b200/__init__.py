@@ -62,6 +62,8 @@ def _load():
         "sfa_window_fwd": (I, [P, P, P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, P, F, P, Z, P, P, P, P]),
         "sfa_gated_combine": (I, [P, P, P, P, P, P, I, I, I, P, P]),
         "sfa_kv_append": (I, [P, P, I, P, P, P, I, I, I, P, I, I, I, P, P]),
+        "sfa_decode_kvcache": (I, [P, P, P, I, I, P, P, P, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]),
+        "sfa_kv_append_kvcache": (I, [P, P, I, P, P, I, I, P, P, I, I, I, P, P]),
         "sfa_index_topk_workspace_size": (Z, [I, I, I, I]),
         "sfa_index_topk": (I, [P, P, P, I, I, I, P, I, I, I, I, I, I, P, Z, P, P, P]),
         "sfa_bwd_workspace_size": (Z, [I, I, I, I, I, I, I, I, I]),
@@ -271,6 +273,68 @@ def kv_append(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v
     rc = _lib.sfa_kv_append(_ptr(k_new), _ptr(v_new), S, _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
                             block_table.shape[1], num_pages, page, _ptr(cache_seqlens), B, Hkv, d, _ptr(status),
                             _stream(stream))
+    _check(rc)
+
+
+def _batch_idx(cache_batch_idx, B, device):
+    if cache_batch_idx is None:
+        return torch.arange(B, dtype=torch.int32, device=device)
+    _need(cache_batch_idx, "cache_batch_idx", torch.int32, 1)
+    if cache_batch_idx.numel() != B:
+        raise ValueError("cache_batch_idx must have one entry per sequence")
+    return cache_batch_idx
+
+
+@_on_tensor_device
+def decode_kvcache(q, k_cache, v_cache, cache_seqlens, sel_tok_idx, *, cache_batch_idx=None, window_left: int = -1,
+                   scale=None, num_splits: int = 0, out=None, lse=None, workspace=None, status=None, stream=None):
+    """Top-k decode over non-paged caches (sfa_decode_kvcache): k_cache / v_cache (batch_cache,
+    seqlen_cache, Hkv, d); sequence b reads row j at k_cache[cache_batch_idx[b], j] (None = 0..B-1,
+    the flash_attn_with_kvcache default).  Other arguments and the result as decode()."""
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(q, "q", torch.bfloat16, 3)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    _need(sel_tok_idx, "sel_tok_idx", torch.int32, 3)
+    if k_cache.shape != v_cache.shape:
+        raise ValueError("k_cache and v_cache must have the same shape")
+    B, Hq, d = q.shape
+    batch_cache, seqlen_cache, Hkv, dk = k_cache.shape
+    if dk != d:
+        raise ValueError("q and cache head dims differ")
+    idx = _batch_idx(cache_batch_idx, B, q.device)
+    topk = sel_tok_idx.shape[2]
+    nbytes = decode_workspace_size(B, Hq, Hkv, d, topk, num_splits)
+    ws = _workspace(workspace, nbytes, q.device)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    rc = _lib.sfa_decode_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), batch_cache, seqlen_cache, _ptr(idx),
+                                 _ptr(cache_seqlens), _ptr(sel_tok_idx), topk, B, Hq, Hkv, d, int(window_left),
+                                 _scale(scale), int(num_splits), _ptr(ws), ws.numel() * ws.element_size(),
+                                 _ptr(status), _ptr(out), _ptr(lse), _stream(stream))
+    _check(rc)
+    return out, lse
+
+
+@_on_tensor_device
+def kv_append_kvcache(k_new: torch.Tensor, v_new: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                      cache_seqlens: torch.Tensor, cache_batch_idx: Optional[torch.Tensor] = None,
+                      status: Optional[torch.Tensor] = None, stream=None) -> None:
+    """In-place append to non-paged caches (sfa_kv_append_kvcache): row j of k_new[b] goes to
+    k_cache[cache_batch_idx[b], cache_seqlens[b] + j] (None = 0..B-1).  cache_seqlens is not updated."""
+    for t, name in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, name, torch.bfloat16, 4)
+    _need(cache_seqlens, "cache_seqlens", torch.int32, 1)
+    if k_new.shape != v_new.shape or k_cache.shape != v_cache.shape:
+        raise ValueError("k / v shapes differ")
+    B, S, Hkv, d = k_new.shape
+    batch_cache, seqlen_cache, hk2, d2 = k_cache.shape
+    if (hk2, d2) != (Hkv, d) or cache_seqlens.numel() != B:
+        raise ValueError("inconsistent shapes")
+    idx = _batch_idx(cache_batch_idx, B, k_new.device)
+    rc = _lib.sfa_kv_append_kvcache(_ptr(k_new), _ptr(v_new), S, _ptr(k_cache), _ptr(v_cache), batch_cache,
+                                    seqlen_cache, _ptr(idx), _ptr(cache_seqlens), B, Hkv, d, _ptr(status),
+                                    _stream(stream))
     _check(rc)
 
 

@@ -939,6 +939,29 @@ int sfa_decode_fp8(const void *q, const void *k_cache, const void *v_cache, cons
                        status_dev, out, lse, stream, true, k_descale, v_descale);
 }
 
+// A cache of batch_cache sequences of seqlen_cache rows each is a paged cache of batch_cache pages of
+// seqlen_cache rows whose block table has one column, cache_batch_idx: row j of sequence b is then
+// k_cache[cache_batch_idx[b]][j], the non-paged indexing of flash_attn_with_kvcache.
+int sfa_decode_kvcache(const void *q, const void *k_cache, const void *v_cache, int batch_cache, int seqlen_cache,
+                       const int32_t *cache_batch_idx, const int32_t *cache_seqlens, const int32_t *sel_tok_idx,
+                       int topk_tok, int B, int Hq, int Hkv, int d, int window_left, float scale, int num_splits,
+                       void *workspace, size_t workspace_bytes, int32_t *status_dev, void *out, float *lse,
+                       sfa_stream_t stream)
+{
+    return sfa_decode(q, k_cache, v_cache, cache_batch_idx, 1, batch_cache, seqlen_cache, cache_seqlens, sel_tok_idx,
+                      topk_tok, B, Hq, Hkv, d, window_left, scale, num_splits, workspace, workspace_bytes, status_dev,
+                      out, lse, stream);
+}
+
+int sfa_kv_append_kvcache(const void *k_new, const void *v_new, int seqlen_new, void *k_cache, void *v_cache,
+                          int batch_cache, int seqlen_cache, const int32_t *cache_batch_idx,
+                          const int32_t *cache_seqlens, int B, int Hkv, int d, int32_t *status_dev,
+                          sfa_stream_t stream)
+{
+    return sfa_kv_append(k_new, v_new, seqlen_new, k_cache, v_cache, cache_batch_idx, 1, batch_cache, seqlen_cache,
+                         cache_seqlens, B, Hkv, d, status_dev, stream);
+}
+
 size_t sfa_window_fwd_workspace_size(void)
 {
     return 256;

@@ -222,3 +222,38 @@ def test_window_and_gated_combine_host_validation(lib):
     assert mix(o1=ctypes.c_void_p((1 << 20) + 2)) == 1
     assert mix(out=None) == 1
     assert mix(total_q=0) == 0
+
+
+def test_kvcache_entries_host_validation(lib):
+    """The non-paged entries are the paged ones with block_table = cache_batch_idx, one page of
+    seqlen_cache rows per cache entry: the same host checks apply."""
+    lib.sfa_decode_kvcache.restype = I
+    lib.sfa_decode_kvcache.argtypes = [P, P, P, I, I, P, P, P, I, I, I, I, I, I, F, I, P, Z, P, P, P, P]
+
+    def dec(**over):
+        a = dict(q=FAKE, kc=FAKE, vc=FAKE, batch_cache=4, seqlen_cache=1024, idx=FAKE, lens=FAKE, sel=FAKE,
+                 topk=64, B=2, Hq=8, Hkv=2, d=128, wl=-1, scale=0.0, splits=0, ws=FAKE, ws_bytes=1 << 30,
+                 status=None, out=FAKE, lse=FAKE, stream=None)
+        a.update(over)
+        return lib.sfa_decode_kvcache(*a.values())
+
+    assert dec(idx=None) == 1                          # cache_batch_idx is required
+    assert dec(seqlen_cache=0) == 1
+    assert dec(seqlen_cache=(1 << 20) + 64) == 2       # more than 2^20 rows per sequence
+    assert dec(d=96) == 2
+    assert dec(ws_bytes=8) == 3
+    assert dec(B=0) == 0
+
+    lib.sfa_kv_append_kvcache.restype = I
+    lib.sfa_kv_append_kvcache.argtypes = [P, P, I, P, P, I, I, P, P, I, I, I, P, P]
+
+    def app(**over):
+        a = dict(kn=FAKE, vn=FAKE, S=4, kc=FAKE, vc=FAKE, batch_cache=4, seqlen_cache=1024, idx=FAKE, lens=FAKE,
+                 B=2, Hkv=2, d=128, status=None, stream=None)
+        a.update(over)
+        return lib.sfa_kv_append_kvcache(*a.values())
+
+    assert app(idx=None) == 1
+    assert app(seqlen_cache=0) == 1
+    assert app(d=12) == 2
+    assert app(S=0) == 0
