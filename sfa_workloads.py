@@ -294,6 +294,27 @@ def make_decode_kvcache(seed: int, B, batch_cache, seqlen_cache, Hq, Hkv, d, len
     return KVCacheCase(name, q, kc, vc, idx, L, sel, Hq, Hkv, d)
 
 
+def kvcache_as_paged(c: KVCacheCase, page: int, seed: int) -> DecodeCase:
+    """The same logical rows as a paged cache: each sequence's rows cut into pages of `page` rows,
+    the pages placed at random physical slots.  Returns a DecodeCase for the C oracle."""
+    rng = np.random.default_rng(seed)
+    seqlen_cache = c.k_cache.shape[1]
+    npp = (seqlen_cache + page - 1) // page
+    num_pages = c.B * npp
+    perm = rng.permutation(num_pages).astype(np.int32)
+    shape = (num_pages, page) + c.k_cache.shape[2:]
+    kp, vp = np.zeros(shape, np.uint16), np.zeros(shape, np.uint16)
+    bt = perm.reshape(c.B, npp)
+    for b in range(c.B):
+        for p in range(npp):
+            rows = slice(p * page, min((p + 1) * page, seqlen_cache))
+            n = rows.stop - rows.start
+            kp[bt[b, p], :n] = c.k_cache[c.cache_batch_idx[b], rows]
+            vp[bt[b, p], :n] = c.v_cache[c.cache_batch_idx[b], rows]
+    return DecodeCase("repacked", c.q, kp, vp, bt, c.cache_seqlens, c.sel, c.Hq, c.Hkv, c.d, page, wl=c.wl,
+                        scale=c.softmax_scale)
+
+
 def _cu(lens):
     return np.concatenate([[0], np.cumsum(np.asarray(lens, dtype=np.int64))]).astype(np.int32)
 

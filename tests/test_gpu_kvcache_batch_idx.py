@@ -8,7 +8,6 @@ import pytest
 import oracle
 import sfa_workloads as W
 from tests.parity import assert_lse_close, assert_out_close, dev_tensor
-from tests.test_oracle_kvcache_pins import repack_paged
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -48,7 +47,7 @@ def test_decode_kvcache_parity(sfa, B, batch_cache, seqlen_cache, Hq, Hkv, d, lo
     assert_out_close(out, ro)
     assert_lse_close(lse, rl)
     # the same rows in pages of 64 at random places: the paged decode gives the same bits
-    pc = repack_paged(c, 64, seed=B)
+    pc = W.kvcache_as_paged(c, 64, seed=B)
     po, pl = sfa.decode(t["q"], dev_tensor(pc.k_cache, torch.bfloat16), dev_tensor(pc.v_cache, torch.bfloat16),
                         dev_tensor(pc.block_table), t["lens"], t["sel"], window_left=wl)
     assert torch.equal(out, po) and torch.equal(lse, pl)

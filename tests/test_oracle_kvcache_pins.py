@@ -12,34 +12,13 @@ import oracle
 import sfa_workloads as W
 
 
-def repack_paged(c: W.KVCacheCase, page: int, seed: int):
-    """The same logical rows as a paged cache: each sequence's rows cut into pages of `page` rows,
-    the pages placed at random physical slots.  Returns a DecodeCase for the C oracle."""
-    rng = np.random.default_rng(seed)
-    seqlen_cache = c.k_cache.shape[1]
-    npp = (seqlen_cache + page - 1) // page
-    num_pages = c.B * npp
-    perm = rng.permutation(num_pages).astype(np.int32)
-    shape = (num_pages, page) + c.k_cache.shape[2:]
-    kp, vp = np.zeros(shape, np.uint16), np.zeros(shape, np.uint16)
-    bt = perm.reshape(c.B, npp)
-    for b in range(c.B):
-        for p in range(npp):
-            rows = slice(p * page, min((p + 1) * page, seqlen_cache))
-            n = rows.stop - rows.start
-            kp[bt[b, p], :n] = c.k_cache[c.cache_batch_idx[b], rows]
-            vp[bt[b, p], :n] = c.v_cache[c.cache_batch_idx[b], rows]
-    return W.DecodeCase("repacked", c.q, kp, vp, bt, c.cache_seqlens, c.sel, c.Hq, c.Hkv, c.d, page, wl=c.wl,
-                        scale=c.softmax_scale)
-
-
 @pytest.mark.parametrize("page,wl", [(16, -1), (100, -1), (64, 50)])
 def test_decode_kvcache_equals_paged_oracle(page, wl):
     c = W.make_decode_kvcache(31 + page, 4, 7, 900, 8, 2, 64, 1, 900, 96, 8)
     c.wl = wl
     out, lse, bad = oracle.decode_kvcache(c.q, c.k_cache, c.v_cache, c.cache_seqlens, c.sel, c.cache_batch_idx,
                                           c.Hkv, c.softmax_scale, wl=wl)
-    ro, rl, rbad = oracle.decode(repack_paged(c, page, seed=page))
+    ro, rl, rbad = oracle.decode(W.kvcache_as_paged(c, page, seed=page))
     assert bad == 0 and int(rbad[0]) == 0 and int(rbad[1]) == 0
     np.testing.assert_allclose(out, ro, rtol=1e-12, atol=1e-12)
     np.testing.assert_allclose(lse, rl, rtol=1e-12, atol=1e-12)
@@ -103,7 +82,7 @@ def test_kv_append_kvcache_equals_paged_append():
     vn = rng.integers(0, 1 << 15, size=(3, 60, 2, 16)).astype(np.uint16)
     k2, v2, bad = oracle.kv_append_kvcache(c.k_cache, c.v_cache, c.cache_batch_idx, c.cache_seqlens, kn, vn)
     page = 32
-    pc = repack_paged(c, page, seed=4)
+    pc = W.kvcache_as_paged(c, page, seed=4)
     kp, vp, pbad = oracle.kv_append(pc.k_cache, pc.v_cache, pc.block_table, c.cache_seqlens, kn, vn)
     # positions 200.. of a sequence lie past the non-paged cache but inside its last page's padding (224
     # rows of pages): the paged append writes them, the non-paged one cannot; compare the rows both hold
