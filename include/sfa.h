@@ -19,6 +19,12 @@
  *               flash_attn_with_kvcache docstrings (paged cache + block_table, cache_seqlens,
  *               num_splits with 0 = automatic, softmax_lse).
  *
+ * Built around them, each documented at its declaration: the backward (sfa_bwd), the NSA
+ * sliding-window branch and gated mix (sfa_window_fwd, sfa_gated_combine), the decode over FP8
+ * caches (sfa_decode_fp8), an allocation-free decode (sfa_decode_noalloc), decode and KV append
+ * over non-paged caches addressed by cache_batch_idx (sfa_decode_kvcache, sfa_kv_append_kvcache),
+ * the paged KV append (sfa_kv_append) and the decode index producer (sfa_index_topk).
+ *
  * Semantics common to both (the plain reading of those pages):
  *   - q head h reads kv head h / (Hq/Hkv); Hq must be a multiple of Hkv.
  *   - For a query at local position i of a sequence with lengths (sq, sk), delta = sk - sq.
